@@ -1,0 +1,392 @@
+/*
+ * fp4_oracle.c — plain CPU oracle for microscaling FP4 (MXFP4 / NVFP4),
+ * the block-diagonal Hadamard rotation and the W4A4 product.
+ *
+ * TEST INFRASTRUCTURE ONLY: used by tests/, the smoke check and the CPU
+ * baseline of the benchmark.  The product path never links it.  It is
+ * deliberately slow and written step by step in the order the method is
+ * described; no blocking, vectorisation or reordering beyond that.
+ *
+ * Sources (web pages; section / equation / table):
+ *   [TransFP4]  "Portable FP4 quantization (TransFP4)", elexvx.com research:
+ *               §1.1 Eq.(1) microscaling form; §2.3 Eq.(2) orthogonal
+ *               rotation; §3.1 absmax scale + nearest rounding; §3.2 NMSE.
+ *   [Guide]     "4.5 FP8 and NVFP4/MXFP4" (inference guide): §1.1 E4M3 bit
+ *               pattern 00111000 = 1.0; §1.2 E4M3 max 448, spacing; §3.1 the
+ *               E2M1 magnitudes {0,0.5,1,1.5,2,3,4,6}; §3.3 scale formats;
+ *               §4.1 NVFP4 two-level dequantization s_tensor*s_block*q.
+ *   [Explainer] "MXFP4 quantization explainer" (AI Daily 2026-08-05), §3:
+ *               32-element blocks, scale maps the block max to the FP4 max.
+ *   [MR-GPTQ]   "FP4 quantization analysis: MXFP4 vs NVFP4" (jsqmd.com),
+ *               §3.2.3: block-diagonal Hadamard H_k, k in {16,32,64,128}.
+ *   [gpt-oss]   "gpt-oss MXFP4" article (juejin.cn), MXFP4 section: the
+ *               worked example 0.0625, 0.375, 0.078125, 0.25.
+ *
+ * Readings where the pages are silent (each one also listed in the design
+ * notes): E2M1 ties either to the even code (default) or away from zero;
+ * MXFP4 scale exponent = the smallest power of two that keeps the block
+ * max <= 6 (default) or the OCP floor rule; E8M0 bias 127; NVFP4 global
+ * scale s_g = amax/(6*448); one reciprocal per NVFP4 block, then a multiply;
+ * the rotation is the normalised Sylvester FWHT along K, stages h ascending.
+ */
+#include "fp4_oracle.h"
+
+#include <float.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* Element format E2M1 ([Guide] §3.1): 1 sign, 2 exponent, 1 mantissa bit.   */
+/* Code c (0..7) of the magnitude: exponent bits = c>>1, mantissa bit = c&1, */
+/* bias 1, exponent 0 is subnormal (0 or 0.5).  Largest value 2^2*1.5 = 6.   */
+/* ------------------------------------------------------------------------ */
+static double e2m1_magnitude(int c)
+{
+    int ebits = (c >> 1) & 3, mbit = c & 1;
+    if (ebits == 0) return 0.5 * mbit;                      /* subnormal */
+    return ldexp(1.0 + 0.5 * mbit, ebits - 1);
+}
+
+double fp4o_e2m1_decode(int code)
+{
+    double m = e2m1_magnitude(code & 7);
+    return (code & 8) ? -m : m;
+}
+
+/* Nearest-value encode of v ([TransFP4] §3.1 "nearest rounding").  |v| >= 6
+ * (including +inf) saturates to the largest code.  At an exact midpoint the
+ * tie goes to the even code (mantissa bit 0) or to the larger magnitude.
+ * The sign is copied from v, so -0 and negatives that round to 0 give 0x8. */
+int fp4o_e2m1_encode(float v, int tie)
+{
+    int sign = signbit(v) ? 8 : 0;
+    double a = fabs((double)v);
+    if (!(a < 6.0)) return sign | 7;                        /* sat / inf */
+    int lo = 0;
+    while (lo < 7 && e2m1_magnitude(lo + 1) <= a) lo++;     /* g[lo] <= a */
+    int hi = lo + 1;
+    double dlo = a - e2m1_magnitude(lo), dhi = e2m1_magnitude(hi) - a;
+    int c;
+    if (dlo < dhi) c = lo;
+    else if (dhi < dlo) c = hi;
+    else c = (tie == FP4O_TIE_AWAY) ? hi : ((lo & 1) ? hi : lo);
+    return sign | c;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Scale format E4M3, unsigned use ([Guide] §1.1-1.2): exponent 4 bits,      */
+/* bias 7, mantissa 3 bits, subnormals at exponent 0, largest finite 448     */
+/* (0x7E); 0x7F is NaN and no infinity exists.                               */
+/* ------------------------------------------------------------------------ */
+double fp4o_e4m3_decode(int byte)
+{
+    int b = byte & 0x7F;
+    if (b == 0x7F) return NAN;
+    int e = b >> 3, m = b & 7;
+    if (e == 0) return ldexp((double)m, -9);                /* m/8 * 2^-6 */
+    return ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/* Round-to-nearest-even onto the 127 finite non-negative codes, saturating
+ * at 448.  t must be >= 0 (block scales are non-negative). */
+int fp4o_e4m3_encode(float t)
+{
+    double a = (double)t;
+    if (!(a < 448.0)) return 0x7E;                          /* satfinite */
+    int best = 0;
+    double bestd = fabs(a - fp4o_e4m3_decode(0));
+    for (int c = 1; c <= 0x7E; c++) {
+        double d = fabs(a - fp4o_e4m3_decode(c));
+        if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            bestd = d;
+        }
+    }
+    return best;
+}
+
+/* E8M0: power-of-two scale 2^(byte-127) ([TransFP4] §1.1, [Guide] §3.3);
+ * 0xFF is NaN. */
+double fp4o_e8m0_decode(int byte)
+{
+    if ((byte & 0xFF) == 0xFF) return NAN;
+    return ldexp(1.0, (byte & 0xFF) - 127);
+}
+
+/* MXFP4 shared exponent of a block with largest magnitude amax.
+ * CEIL (default): the smallest e with amax <= 6 * 2^e, i.e. the block max
+ *   is mapped onto the E2M1 range without clipping ([Explainer] §3).
+ * FLOOR (option): e = floor(log2 amax) - 2 (the OCP MX rule; block values
+ *   in (6, 8) * 2^e saturate to 6).
+ * amax == 0 gives -127 (byte 0x00).  The result is clamped to [-127, 127]. */
+int fp4o_mx_scale_exponent(float amax, int rule)
+{
+    if (amax == 0.0f) return -127;
+    int p;
+    double f = frexp((double)amax, &p);                     /* amax = f*2^p */
+    (void)f;
+    int e;
+    if (rule == FP4O_MX_FLOOR) {
+        e = (p - 1) - 2;                                    /* floor(log2) = p-1 */
+    } else {
+        /* amax > 2^(p-1) >= 6*2^(p-4), so no e below p-4 can satisfy the bound:
+         * search upward from there. */
+        e = p - 4;
+        while (!((double)amax <= ldexp(6.0, e))) e++;
+    }
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block-diagonal Hadamard rotation H_k ([MR-GPTQ] §3.2.3; [TransFP4] §2.3)  */
+/* ------------------------------------------------------------------------ */
+float fp4o_hadamard_ck(int k)
+{
+    return (float)(1.0 / sqrt((double)k));
+}
+
+/* Normalised Sylvester Walsh-Hadamard transform of one chunk of k values,
+ * in place, in fp32: stages h = 1, 2, ..., k/2 replace each pair
+ * (y[j], y[j+h]) (bit h of j clear) by (y[j] + y[j+h], y[j] - y[j+h]); then
+ * every value is multiplied by c_k = RN(1/sqrt(k)).  The matrix is
+ * symmetric and orthogonal, so applying it twice returns the input up to
+ * rounding. */
+void fp4o_fwht(float *y, int k)
+{
+    for (int h = 1; h < k; h *= 2) {
+        for (int j = 0; j < k; j++) {
+            if (j & h) continue;
+            float a = y[j], b = y[j + h];
+            y[j] = a + b;
+            y[j + h] = a - b;
+        }
+    }
+    float ck = fp4o_hadamard_ck(k);
+    for (int j = 0; j < k; j++) y[j] = y[j] * ck;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantize ([TransFP4] Eq.(1): x^_i = s_g s_b Q_f(x_i / (s_g s_b)))         */
+/* ------------------------------------------------------------------------ */
+static float bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static int valid_shape(int fmt, int block, int hk, int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0) return 0;
+    if (fmt == FP4O_MXFP4 && block != 32) return 0;
+    if (fmt == FP4O_NVFP4 && block != 16) return 0;
+    if (fmt != FP4O_MXFP4 && fmt != FP4O_NVFP4) return 0;
+    if (!(hk == 0 || hk == 16 || hk == 32 || hk == 64 || hk == 128)) return 0;
+    if (cols % block) return 0;
+    if (hk && cols % hk) return 0;
+    return 1;
+}
+
+/* Row r of x as fp32, rotated when hk > 0. */
+static void load_row(const uint16_t *x, int64_t ld, int64_t r, int64_t cols,
+                     int hk, float *y)
+{
+    for (int64_t c = 0; c < cols; c++) y[c] = bf16_to_f32(x[r * ld + c]);
+    if (hk)
+        for (int64_t c = 0; c < cols; c += hk) fp4o_fwht(y + c, hk);
+}
+
+/* NVFP4 tensor scale ([Guide] §4.1: the FP32 tensor-level scale brings the
+ * tensor into the E4M3 block-scale range): s_g = amax / (6 * 448), so the
+ * largest block scale lands at the E4M3 maximum; an all-zero tensor (or a
+ * non-finite amax) gets s_g = 1. */
+static float nv_global_scale(float amax_t)
+{
+    if (amax_t > 0.0f && amax_t <= FLT_MAX) return amax_t / 2688.0f;
+    return 1.0f;
+}
+
+int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                  int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                  int gscale_given, float *gscale,
+                  uint8_t *q, uint8_t *s_logical)
+{
+    if (!valid_shape(fmt, block, hadamard_k, rows, cols) || ld < cols) return -1;
+    const int64_t nkb = cols / block;
+
+    float sg = 1.0f;
+    if (fmt == FP4O_NVFP4) {
+        if (gscale_given) {
+            sg = *gscale;
+        } else {
+            float amax_t = 0.0f;
+#pragma omp parallel
+            {
+                float *y = (float *)malloc(sizeof(float) * (size_t)(cols ? cols : 1));
+                float local = 0.0f;
+#pragma omp for schedule(static)
+                for (int64_t r = 0; r < rows; r++) {
+                    load_row(x, ld, r, cols, hadamard_k, y);
+                    for (int64_t c = 0; c < cols; c++) {
+                        float a = fabsf(y[c]);
+                        if (a > local) local = a;
+                    }
+                }
+#pragma omp critical
+                if (local > amax_t) amax_t = local;
+                free(y);
+            }
+            sg = nv_global_scale(amax_t);
+            *gscale = sg;
+        }
+    }
+
+#pragma omp parallel
+    {
+        float *y = (float *)malloc(sizeof(float) * (size_t)(cols ? cols : 1));
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < rows; r++) {
+            load_row(x, ld, r, cols, hadamard_k, y);
+            uint8_t *qrow = q + r * (cols / 2);
+            memset(qrow, 0, (size_t)(cols / 2));
+            for (int64_t kb = 0; kb < nkb; kb++) {
+                const float *blk = y + kb * block;
+                float amax_b = 0.0f;
+                for (int i = 0; i < block; i++)
+                    if (fabsf(blk[i]) > amax_b) amax_b = fabsf(blk[i]);
+
+                int codes[32];
+                uint8_t sbyte;
+                if (fmt == FP4O_MXFP4) {
+                    /* Power-of-two scale: x / 2^e is a plain exponent shift. */
+                    int e = fp4o_mx_scale_exponent(amax_b, mx_rule);
+                    sbyte = (uint8_t)(e + 127);
+                    float inv = ldexpf(1.0f, -e);
+                    for (int i = 0; i < block; i++)
+                        codes[i] = fp4o_e2m1_encode(blk[i] * inv, tie);
+                } else {
+                    /* Two-level scale: t = amax_b / (6 s_g) is stored as E4M3,
+                     * d = s_g * s_b, values are multiplied by r = 1/d. */
+                    float six_sg = 6.0f * sg;
+                    float t = amax_b / six_sg;
+                    int sb = fp4o_e4m3_encode(t);
+                    sbyte = (uint8_t)sb;
+                    float d = sg * (float)fp4o_e4m3_decode(sb);
+                    if (d == 0.0f) {
+                        for (int i = 0; i < block; i++) codes[i] = signbit(blk[i]) ? 8 : 0;
+                    } else {
+                        float rcp = 1.0f / d;
+                        if (rcp > FLT_MAX) rcp = FLT_MAX;
+                        for (int i = 0; i < block; i++)
+                            codes[i] = fp4o_e2m1_encode(blk[i] * rcp, tie);
+                    }
+                }
+                s_logical[r * nkb + kb] = sbyte;
+                for (int i = 0; i < block; i++) {
+                    int64_t c = kb * block + i;
+                    qrow[c / 2] |= (uint8_t)((codes[i] & 0xF) << ((c & 1) ? 4 : 0));
+                }
+            }
+        }
+        free(y);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dequantize ([TransFP4] Eq.(1); [Guide] §4.1 x^ = s_tensor * s_block * q)  */
+/* ------------------------------------------------------------------------ */
+int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
+                    int64_t rows, int64_t cols, int fmt, int block,
+                    int hadamard_k, float *out)
+{
+    if (!valid_shape(fmt, block, hadamard_k, rows, cols)) return -1;
+    const int64_t nkb = cols / block;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        float *o = out + r * cols;
+        for (int64_t c = 0; c < cols; c++) {
+            int code = (q[r * (cols / 2) + c / 2] >> ((c & 1) ? 4 : 0)) & 0xF;
+            float qv = (float)fp4o_e2m1_decode(code);
+            uint8_t sb = s_logical[r * nkb + c / block];
+            if (fmt == FP4O_MXFP4) {
+                o[c] = qv * (float)fp4o_e8m0_decode(sb);
+            } else {
+                float d = gscale * (float)fp4o_e4m3_decode(sb);
+                o[c] = d * qv;
+            }
+        }
+        if (hadamard_k)
+            for (int64_t c = 0; c < cols; c += hadamard_k) fp4o_fwht(o + c, hadamard_k);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Scale tile layout consumed by the block-scaled tensor-core MMA: 512-byte   */
+/* atoms of 128 rows x 4 scale columns; atoms ordered row-block major, then  */
+/* scale-column block.  Inside an atom, row r and column j sit at byte       */
+/* (r % 32) * 16 + (r / 32) * 4 + j.  Rows pad to 128, columns to 4; padding */
+/* bytes are 0.  (A hardware convention; the pages do not fix it.)           */
+/* ------------------------------------------------------------------------ */
+static int64_t atom_offset(int64_t r, int64_t kb, int64_t nkb4)
+{
+    return ((r / 128) * nkb4 + kb / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (kb % 4);
+}
+
+void fp4o_scales_to_atoms(const uint8_t *s_logical, int64_t rows, int64_t nkb,
+                          uint8_t *s_atoms)
+{
+    int64_t rows_p = (rows + 127) / 128 * 128, nkb4 = (nkb + 3) / 4;
+    memset(s_atoms, 0, (size_t)(rows_p * nkb4 * 4));
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t kb = 0; kb < nkb; kb++)
+            s_atoms[atom_offset(r, kb, nkb4)] = s_logical[r * nkb + kb];
+}
+
+void fp4o_scales_from_atoms(const uint8_t *s_atoms, int64_t rows, int64_t nkb,
+                            uint8_t *s_logical)
+{
+    int64_t nkb4 = (nkb + 3) / 4;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t kb = 0; kb < nkb; kb++)
+            s_logical[r * nkb + kb] = s_atoms[atom_offset(r, kb, nkb4)];
+}
+
+/* ------------------------------------------------------------------------ */
+/* W4A4 linear reference: C = A_hat * W_hat^T in fp64 over the dequantized   */
+/* operands ([Guide] §5: the product of quantized activations and weights).  */
+/* ------------------------------------------------------------------------ */
+void fp4o_gemm_ref(const float *a, const float *w, int64_t M, int64_t N,
+                   int64_t K, double *c, double *bound)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0, acc_abs = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double p = (double)a[m * K + k] * (double)w[n * K + k];
+                acc += p;
+                acc_abs += fabs(p);
+            }
+            c[m * N + n] = acc;
+            if (bound) bound[m * N + n] = acc_abs;
+        }
+    }
+}
+
+int fp4o_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,79 @@
+/*
+ * fp4_oracle.h — plain, slow CPU oracle for microscaling FP4 quantization
+ * and the block-scaled W4A4 product.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link
+ * or call this library; only the test-suite, the smoke check and the CPU
+ * baseline leg of the benchmark load it.  It shares no code, header, table
+ * or constant with the CUDA library under fp4_microscaling_quantization_b200/.
+ *
+ * Conventions (all functions):
+ *   - Every fp32 operation is a single IEEE-754 binary32 operation rounded to
+ *     nearest-even (the build uses -ffp-contract=off and no fast-math, so no
+ *     operation is fused or reassociated).  Subnormals are kept.
+ *   - Elements are bf16 bit patterns (uint16_t), rows x cols, row stride ld
+ *     (in elements).  The quantization / contraction axis is cols (K).
+ *   - Scales are returned in LOGICAL layout: s[row * (cols/block) + kb].
+ *     The hardware tile layout is produced by fp4o_scales_to_atoms().
+ *   - Packed elements: byte (row, j) holds element 2j in bits [3:0] and
+ *     element 2j+1 in bits [7:4]; row stride cols/2 bytes.
+ */
+#ifndef FP4_ORACLE_H
+#define FP4_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { FP4O_MXFP4 = 0, FP4O_NVFP4 = 1 };
+enum { FP4O_TIE_EVEN = 0, FP4O_TIE_AWAY = 1 };
+enum { FP4O_MX_CEIL = 0, FP4O_MX_FLOOR = 1 };
+
+/* ---- element and scale codecs ------------------------------------------- */
+int    fp4o_e2m1_encode(float v, int tie);      /* 4-bit code, sign in bit 3 */
+double fp4o_e2m1_decode(int code);
+int    fp4o_e4m3_encode(float t);               /* t >= 0, RNE, satfinite    */
+double fp4o_e4m3_decode(int byte);
+double fp4o_e8m0_decode(int byte);              /* 2^(byte-127); NaN at 0xFF */
+int    fp4o_mx_scale_exponent(float amax, int rule);  /* e in [-127, 127]    */
+
+/* ---- rotation ----------------------------------------------------------- */
+float  fp4o_hadamard_ck(int k);                 /* RN_fp32(1/sqrt(k))        */
+void   fp4o_fwht(float *y, int k);              /* in place, incl. c_k       */
+
+/* ---- quantize / dequantize --------------------------------------------- */
+/* gscale: NVFP4 only.  If gscale_given, *gscale is read as s_g; otherwise
+ * s_g is computed from the tensor and written to *gscale.  Returns 0 on
+ * success, -1 on an invalid argument. */
+int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                  int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                  int gscale_given, float *gscale,
+                  uint8_t *q, uint8_t *s_logical);
+
+/* out: rows x cols fp32.  hadamard_k > 0 applies the (self-inverse)
+ * rotation again to return to the original domain. */
+int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
+                    int64_t rows, int64_t cols, int fmt, int block,
+                    int hadamard_k, float *out);
+
+/* logical scales (rows x nkb) -> tcgen05 scale-atom layout
+ * (pad128(rows) x pad4(nkb) bytes, padding bytes 0), and back. */
+void fp4o_scales_to_atoms(const uint8_t *s_logical, int64_t rows, int64_t nkb,
+                          uint8_t *s_atoms);
+void fp4o_scales_from_atoms(const uint8_t *s_atoms, int64_t rows, int64_t nkb,
+                            uint8_t *s_logical);
+
+/* C[m][n] = sum_k a[m][k] * w[n][k] in fp64, and bound[m][n] =
+ * sum_k |a[m][k]| * |w[n][k]|.  a: M x K, w: N x K fp32 (dequantized). */
+void fp4o_gemm_ref(const float *a, const float *w, int64_t M, int64_t N,
+                   int64_t K, double *c, double *bound);
+
+/* Number of OpenMP threads the oracle's row loops use (1 without OpenMP). */
+int fp4o_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
