@@ -1,0 +1,349 @@
+#!/usr/bin/env python3
+"""Benchmark of the microscaling FP4 hot path on B200.
+
+One step = one pass of the quantization path over the heavy-tailed
+1024 x 131072 bf16 tensor (Student-t(3) with 1% outliers x20):
+MXFP4 quantize, NVFP4 quantize (tensor scale computed, i.e. the amax pass
+plus the quantize pass), MXFP4 dequantize and NVFP4 dequantize (bf16 out).
+`value` = algorithmic bytes of the step / device time of the step (GB/s).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (weak scaling): one process per GPU under torchrun, every rank
+runs the same step on its own tensor; value = all ranks' bytes / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+ROWS, COLS = 1024, 131072
+WORKLOAD = "quantize sweep 1024x131072 bf16 Student-t(3)+1% outliers x20: MXFP4 + NVFP4 quantize and dequantize"
+METRIC = "FP4 quantize GB/s (% HBM peak)"
+
+
+def step_bytes(rows=ROWS, cols=COLS):
+    """Algorithmic HBM bytes of one step (each tensor read or written once per
+    kernel pass; the NVFP4 amax pass reads x once more)."""
+    n = rows * cols
+    mx_q = n * (2 + 0.5 + 1 / 32)          # read x, write nibbles + E8M0 scales
+    nv_q = n * (2 + 2 + 0.5 + 1 / 16)      # amax read, read x, write nibbles + E4M3 scales
+    mx_d = n * (0.5 + 1 / 32 + 2)          # read nibbles + scales, write bf16
+    nv_d = n * (0.5 + 1 / 16 + 2)
+    return {"mx_quantize": mx_q, "nv_quantize": nv_q, "mx_dequantize": mx_d, "nv_dequantize": nv_d}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks -----
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.out = out
+        return False
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for row in csv.reader(io.StringIO(self.out)):
+            if len(row) < 9:
+                continue
+            try:
+                mhz.append(float(row[1]))
+                mx = float(row[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, row[5:9]):
+                if v.strip() == "Active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "samples": len(mhz), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- dist -------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, ws: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if ws == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- oracle leg --
+def oracle_sample(rows: int, seed: int = 2):
+    """Times the CPU oracle on a `rows`-row slab of the same workload."""
+    import oracle
+    from fp4_microscaling_quantization_b200 import inputs
+    x = inputs.quant_sweep(rows=rows, cols=COLS, seed=seed)
+    t0 = time.perf_counter()
+    qm, sm, _ = oracle.quantize(x, oracle.MXFP4)
+    qn, sn, gn = oracle.quantize(x, oracle.NVFP4)
+    oracle.dequantize(qm, sm, 1.0, oracle.MXFP4)
+    oracle.dequantize(qn, sn, gn, oracle.NVFP4)
+    dt = time.perf_counter() - t0
+    b = sum(step_bytes(rows, COLS).values())
+    return b / dt / 1e9, dt, oracle.num_threads()
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    rows = 16
+    times = []
+    for i in range(args.warmup + args.steps):
+        gbs, dt, cores = oracle_sample(rows)
+        if i >= args.warmup:
+            times.append(dt)
+    dt = statistics.mean(times)
+    b = sum(step_bytes(rows, COLS).values())
+    v = b / dt / 1e9
+    sample = f"{rows} of {ROWS} rows of the same workload per step (oracle, OpenMP over rows)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD + f" (oracle sample: {rows} rows)"},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our leg ----
+def run_ours(args):
+    import torch
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    import fp4_microscaling_quantization_b200 as fp4
+    from fp4_microscaling_quantization_b200 import _lib, inputs
+
+    x_np = inputs.quant_sweep(rows=args.rows, seed=2 + rank)
+    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x = x_host.to(dev)
+    rows, cols = x.shape
+    stream = torch.cuda.current_stream(dev)
+
+    qm, sm, gm = fp4.quantize(x, fp4.FP4_MXFP4)
+    qn, sn, gn = fp4.quantize(x, fp4.FP4_NVFP4)
+    dm = fp4.dequantize(qm, sm, gm, fp4.FP4_MXFP4, out_dtype=fp4.FP4_OUT_BF16)
+    dn = fp4.dequantize(qn, sn, gn, fp4.FP4_NVFP4, out_dtype=fp4.FP4_OUT_BF16)
+    torch.cuda.synchronize()
+
+    names = ["mx_quantize", "nv_quantize", "mx_dequantize", "nv_dequantize"]
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        fp4.quantize(x, fp4.FP4_MXFP4, out=(qm, sm, gm))
+        mark(1)
+        fp4.quantize(x, fp4.FP4_NVFP4, out=(qn, sn, gn))
+        mark(2)
+        fp4.dequantize(qm, sm, gm, fp4.FP4_MXFP4, out_dtype=fp4.FP4_OUT_BF16, out=dm)
+        mark(3)
+        fp4.dequantize(qn, sn, gn, fp4.FP4_NVFP4, out_dtype=fp4.FP4_OUT_BF16, out=dn)
+        mark(4)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    per = {n: 0.0 for n in names}
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    launches0 = _lib.lib().fp4_kernel_launches()
+    with ClockSampler(dev.index) as clk:
+        barrier(ws)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evsets[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+    launches = _lib.lib().fp4_kernel_launches() - launches0
+    total_ms = t0.elapsed_time(t1)
+    for ev in evsets:
+        for j, n in enumerate(names):
+            per[n] += ev[j].elapsed_time(ev[j + 1])
+    per = {n: v / args.steps for n, v in per.items()}
+    total_ms = max_over_ranks(total_ms, ws, dev)
+    ms_per_step = total_ms / args.steps
+
+    sb = step_bytes(rows, cols)
+    value = sum(sb.values()) * ws / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+
+    # dominant single-launch kernel: MXFP4 quantize is one kernel launch per call
+    dom = "mx_quantize"
+    achieved = sb[dom] / (per[dom] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "quantize_kernel<MXFP4,k=0>", "achieved": achieved, "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None,
+                "per_call_ms": per,
+                "per_call_gbs": {n: sb[n] / (per[n] * 1e-3) / 1e9 for n in names}}
+
+    # ---- end to end through the public API with host buffers ----------------
+    e2e = None
+    if not args.no_e2e:
+        outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (qm, sm, qn, sn, gn)]
+        h2d = x_host.numel() * 2
+        d2h = sum(t.numel() * t.element_size() for t in outs_host)
+        e_steps = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            x.copy_(x_host, non_blocking=True)
+            step()
+            for h, d in zip(outs_host, (qm, sm, qn, sn, gn)):
+                h.copy_(d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a0.elapsed_time(a1), ws, dev) / e_steps
+        e2e = {"value": sum(sb.values()) * ws / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    # ---- NMSE of the step's outputs (host, untimed) ------------------------------
+    idx = slice(0, 8)
+    xs = inputs.bf16_bits_to_f32(x_np[idx]).astype(np.float64)
+
+    def nmse(t):
+        y = t[idx].float().cpu().numpy().astype(np.float64)
+        return float(((xs - y) ** 2).sum() / (xs ** 2).sum())
+
+    nmse_vals = {"mxfp4": nmse(dm), "nvfp4": nmse(dn), "rows_sampled": 8}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        crow = 16
+        gbs, dt, cores = oracle_sample(crow)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"{crow} of {ROWS} rows of the same step, {dt:.1f} s"}
+
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD if rows == ROWS else WORKLOAD.replace(str(ROWS), str(rows)), "rows": rows, "cols": cols, "parallelism": f"replicas{ws}",
+                   "l2": "inputs larger than L2 (268 MB bf16 tensor), no flush",
+                   "step_bytes": sum(sb.values())},
+        "frac_of_hbm_peak": value / ws / peak,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "nmse": nmse_vals,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rows", type=int, default=ROWS, help="rows of the tensor (profiling runs use fewer)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,130 @@
+"""B200 (sm_100a) microscaling FP4: MXFP4 / NVFP4 quantization with a fused
+block-diagonal Hadamard rotation, and the block-scaled W4A4 GEMM.
+
+Python front end of the C ABI in include/fp4.h.  Tensors are torch CUDA
+tensors (device memory and the current stream come from torch); all
+arithmetic runs in libfp4.so.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_NVFP4, FP4_OUT_BF16,
+                   FP4_OUT_F32, FP4_ROUND_AWAY, FP4_ROUND_EVEN, Fp4Error)
+
+__all__ = [
+    "quantize", "dequantize", "gemm", "quantize_sizes", "gemm_workspace_size", "check_device_status",
+    "FP4_MXFP4", "FP4_NVFP4", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
+    "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "Fp4Error", "block_of",
+]
+
+
+def block_of(fmt: int) -> int:
+    return 32 if fmt == FP4_MXFP4 else 16
+
+
+def _fmt(fmt) -> int:
+    if isinstance(fmt, str):
+        return {"mxfp4": FP4_MXFP4, "nvfp4": FP4_NVFP4}[fmt.lower()]
+    return int(fmt)
+
+
+def _stream_handle(torch, device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def quantize_sizes(rows: int, cols: int, fmt) -> tuple[int, int]:
+    fmt = _fmt(fmt)
+    qb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _lib.check("fp4_quantize_sizes",
+               _lib.lib().fp4_quantize_sizes(rows, cols, fmt, block_of(fmt), ctypes.byref(qb), ctypes.byref(sb)))
+    return qb.value, sb.value
+
+
+def quantize(x, fmt, hadamard_k: int = 0, round: int = FP4_ROUND_EVEN,
+             mx_scale_rule: int = FP4_MX_SCALE_CEIL, gscale=None, out=None):
+    """Quantize a 2-D bf16 CUDA tensor along its last axis.
+
+    Returns (q, s, g): q uint8 (rows, cols/2) packed nibbles, s uint8 scales in
+    the tensor-core tile layout, g a 1-element fp32 tensor holding s_g (NVFP4;
+    for MXFP4 a tensor holding 1).  If ``gscale`` is given (NVFP4) it is used
+    as s_g instead of computing it.  ``out`` = (q, s, g) reuses buffers.
+    """
+    import torch
+
+    fmt = _fmt(fmt)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a 2-D bf16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must be contiguous along its last axis")
+    rows, cols = x.shape
+    qb, sb = quantize_sizes(rows, cols, fmt)
+    if out is None:
+        q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+        s = torch.empty((sb,), dtype=torch.uint8, device=x.device)
+        g = torch.ones((1,), dtype=torch.float32, device=x.device)
+    else:
+        q, s, g = out
+    given = gscale is not None
+    if given:
+        g.copy_(gscale.reshape(1).to(torch.float32))
+    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(given))
+    gp = g.data_ptr() if fmt == FP4_NVFP4 else None
+    _lib.check("fp4_quantize", _lib.lib().fp4_quantize(
+        x.data_ptr(), rows, cols, x.stride(0), fmt, block_of(fmt), int(hadamard_k), ctypes.byref(opts),
+        q.data_ptr(), s.data_ptr(), gp, _stream_handle(torch, x.device)))
+    return q, s, g
+
+
+def dequantize(q, s, g, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_F32, out=None):
+    """Inverse of :func:`quantize`; returns a (rows, cols) fp32 or bf16 tensor."""
+    import torch
+
+    fmt = _fmt(fmt)
+    rows, half = q.shape
+    cols = half * 2
+    dt = torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((rows, cols), dtype=dt, device=q.device)
+    gp = g.data_ptr() if fmt == FP4_NVFP4 else None
+    _lib.check("fp4_dequantize", _lib.lib().fp4_dequantize(
+        q.data_ptr(), s.data_ptr(), gp, rows, cols, fmt, block_of(fmt), int(hadamard_k), int(out_dtype),
+        out.data_ptr(), _stream_handle(torch, q.device)))
+    return out
+
+
+def gemm_workspace_size(M: int, N: int, K: int, fmt) -> int:
+    b = ctypes.c_size_t()
+    _lib.check("fp4_gemm_workspace_size",
+               _lib.lib().fp4_gemm_workspace_size(M, N, K, _fmt(fmt), ctypes.byref(b)))
+    return b.value
+
+
+def gemm(a, w, M: int, N: int, K: int, fmt, out_dtype: int = FP4_OUT_BF16, out=None, workspace=None):
+    """C = A W^T from quantized operands a = (Aq, As, gA), w = (Wq, Ws, gW)."""
+    import torch
+
+    fmt = _fmt(fmt)
+    Aq, As, gA = a
+    Wq, Ws, gW = w
+    dt = torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, N), dtype=dt, device=Aq.device)
+    need = gemm_workspace_size(M, N, K, fmt)
+    if need and workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=Aq.device)
+    wp = workspace.data_ptr() if workspace is not None else None
+    wb = workspace.numel() if workspace is not None else 0
+    _lib.check("fp4_gemm", _lib.lib().fp4_gemm(
+        Aq.data_ptr(), As.data_ptr(), gA.data_ptr(), Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(),
+        M, N, K, fmt, int(out_dtype), out.data_ptr(), out.stride(0), wp, wb,
+        _stream_handle(torch, Aq.device)))
+    return out
+
+
+def check_device_status() -> None:
+    import torch
+
+    _lib.check("fp4_check_device_status",
+               _lib.lib().fp4_check_device_status(_stream_handle(torch, torch.cuda.current_device())))

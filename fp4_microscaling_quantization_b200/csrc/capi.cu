@@ -1,0 +1,166 @@
+// capi.cu — the extern "C" boundary declared in include/fp4.h: host-side
+// validation of every argument, then stream-ordered launches.  No entry point
+// allocates or frees device memory or synchronizes the host (except
+// fp4_check_device_status, which is documented to).
+#include <math.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace fp4 {
+cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
+                            int hk, float ck, int round_away, int mx_floor, int gscale_given,
+                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
+                              int64_t cols, int fmt, int hk, float ck, int bf16out, void *out,
+                              int sms, cudaStream_t st);
+cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
+                        const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K,
+                        int fmt, int bf16out, void *C, int64_t ldc, void *ws, size_t ws_bytes,
+                        int sms, cudaStream_t st, int *timeout_flag_out);
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int sms);
+cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace fp4
+
+namespace {
+
+int sm_count()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_fmt(int fmt, int block)
+{
+    return (fmt == FP4_MXFP4 && block == 32) || (fmt == FP4_NVFP4 && block == 16);
+}
+
+bool valid_k(int k) { return k == 0 || k == 16 || k == 32 || k == 64 || k == 128; }
+
+// RN_fp32(1/sqrt(k)): the double quotient is within 2^-52 relative of the
+// exact value, far inside half an fp32 ulp, so rounding it once to fp32 gives
+// the correctly rounded constant.
+float hadamard_constant(int k) { return k ? (float)(1.0 / sqrt((double)k)) : 1.0f; }
+
+}  // namespace
+
+extern "C" {
+
+const char *fp4_status_string(fp4_status st)
+{
+    switch (st) {
+    case FP4_OK: return "FP4_OK";
+    case FP4_ERR_INVALID_ARG: return "FP4_ERR_INVALID_ARG: invalid argument";
+    case FP4_ERR_UNSUPPORTED: return "FP4_ERR_UNSUPPORTED: shape or format not supported";
+    case FP4_ERR_ALIGNMENT: return "FP4_ERR_ALIGNMENT: pointer or stride misaligned";
+    case FP4_ERR_CUDA: return "FP4_ERR_CUDA: CUDA runtime error";
+    case FP4_ERR_TIMEOUT: return "FP4_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    }
+    return "unknown fp4_status";
+}
+
+fp4_status fp4_quantize_sizes(int64_t rows, int64_t cols, int fmt, int block, size_t *q_bytes,
+                              size_t *s_bytes)
+{
+    if (rows < 0 || cols < 0 || !q_bytes || !s_bytes) return FP4_ERR_INVALID_ARG;
+    if (!valid_fmt(fmt, block)) return FP4_ERR_UNSUPPORTED;
+    if (cols % block) return FP4_ERR_UNSUPPORTED;
+    const int64_t nkb = cols / block;
+    *q_bytes = (size_t)(rows * (cols / 2));
+    *s_bytes = (size_t)(((rows + 127) / 128 * 128) * ((nkb + 3) / 4 * 4));
+    return FP4_OK;
+}
+
+fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int fmt, int block,
+                        int hadamard_k, const fp4_opts *opts, uint8_t *q, uint8_t *s, float *gscale,
+                        void *stream)
+{
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0};
+    if (opts) o = *opts;
+    if (rows < 0 || cols < 0 || ld_x < cols) return FP4_ERR_INVALID_ARG;
+    if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
+    if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR)
+        return FP4_ERR_INVALID_ARG;
+    if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    const bool empty = rows == 0 || cols == 0;
+    if (fmt == FP4_NVFP4 && !gscale) return FP4_ERR_INVALID_ARG;
+    if (!empty && (!x || !q || !s)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || (ld_x % 8) || !aligned(q, 16) || !aligned(s, 16)) return FP4_ERR_ALIGNMENT;
+    if (gscale && !aligned(gscale, 4)) return FP4_ERR_ALIGNMENT;
+    if (empty && fmt == FP4_MXFP4) return FP4_OK;
+    cudaError_t e = fp4::launch_quantize(static_cast<const uint16_t *>(x), rows, cols, ld_x, fmt,
+                                         hadamard_k, hadamard_constant(hadamard_k),
+                                         o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
+                                         o.gscale_given, q, s, gscale, sm_count(),
+                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status fp4_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
+                          int64_t cols, int fmt, int block, int hadamard_k, int out_dtype, void *out,
+                          void *stream)
+{
+    if (rows < 0 || cols < 0) return FP4_ERR_INVALID_ARG;
+    if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+    if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0) return FP4_OK;
+    if (!q || !s || !out || (fmt == FP4_NVFP4 && !gscale)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(s, 16) || !aligned(out, 16)) return FP4_ERR_ALIGNMENT;
+    cudaError_t e = fp4::launch_dequantize(q, s, gscale, rows, cols, fmt, hadamard_k,
+                                           hadamard_constant(hadamard_k), out_dtype == FP4_OUT_BF16,
+                                           out, sm_count(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes)
+{
+    if (M < 0 || N < 0 || K < 0 || !bytes) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    *bytes = fp4::gemm_workspace_bytes(M, N, K, fmt, sm_count());
+    return FP4_OK;
+}
+
+fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
+                    const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K, int fmt,
+                    int out_dtype, void *C, int64_t ldc, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+    if (K % 256) return FP4_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return FP4_OK;
+    if (!Aq || !As || !Wq || !Ws || !C) return FP4_ERR_INVALID_ARG;
+    if (fmt == FP4_NVFP4 && (!gA || !gW)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(Aq, 16) || !aligned(Wq, 16) || !aligned(As, 16) || !aligned(Ws, 16) || !aligned(C, 16))
+        return FP4_ERR_ALIGNMENT;
+    const int sms = sm_count();
+    const size_t need = fp4::gemm_workspace_bytes(M, N, K, fmt, sms);
+    if (need > 0 && (!workspace || ws_bytes < need)) return FP4_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return FP4_ERR_ALIGNMENT;
+    int bad = 0;
+    cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16,
+                                     C, ldc, workspace, ws_bytes, sms,
+                                     static_cast<cudaStream_t>(stream), &bad);
+    if (bad) return FP4_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+uint64_t fp4_kernel_launches(void) { return fp4::g_launches.load(std::memory_order_relaxed); }
+
+fp4_status fp4_check_device_status(void *stream)
+{
+    unsigned int err = 0;
+    if (fp4::read_and_clear_device_errors(static_cast<cudaStream_t>(stream), &err) != cudaSuccess)
+        return FP4_ERR_CUDA;
+    return err ? FP4_ERR_TIMEOUT : FP4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,437 @@
+// quantize.cu — HBM-streaming quantize / dequantize kernels for MXFP4 and
+// NVFP4, with the optional block-diagonal Hadamard rotation fused in.
+//
+// Method: "Portable FP4 quantization (TransFP4)" §1.1 Eq.(1)
+//   x^_i = s_g * s_b * Q_f(x_i / (s_g * s_b)),
+// absmax block scales and nearest rounding (§3.1); the NVFP4 two-level scale
+// ("4.5 FP8 and NVFP4/MXFP4" §4.1); the rotation H_k, k in {16,32,64,128},
+// computed online for activations ("FP4 quantization analysis: MXFP4 vs
+// NVFP4" §3.2.3, §3.3 fused online-rotation kernel).
+//
+// Work decomposition: one thread owns one 32-element unit of a row (one
+// MXFP4 block or two NVFP4 blocks): four 16-byte loads, the block max in
+// registers, one 16-byte store of 32 nibbles.  A Hadamard chunk of k <= 32
+// lies inside one thread; k = 64 / 128 spans 2 / 4 neighbouring lanes and
+// the last butterfly stages exchange values with shuffles.  Warps walk the
+// tensor in a grid-stride loop of 32 consecutive units, so neighbouring
+// lanes read and write neighbouring memory.
+#include "common.cuh"
+
+namespace fp4 {
+
+struct QuantArgs {
+    const uint16_t *x;
+    int64_t ld;             // row stride of x, elements
+    int64_t units_per_row;  // cols / 32
+    int64_t total_units;    // rows * units_per_row
+    int64_t nkb4;           // ceil(blocks per row / 4)
+    int64_t q_row_bytes;    // cols / 2
+    uint8_t *q;
+    uint8_t *s;
+    float *gscale;
+    float ck;               // RN(1/sqrt(k)) of the rotation
+    int round_away;         // E2M1 ties to the larger magnitude
+    int mx_floor;           // MX scale: floor rule
+    int gscale_computed;    // NVFP4: *gscale holds amax bits (set by the amax pass)
+};
+
+// Load one 32-element unit as fp32.
+FP4_DEV void load_unit(const uint16_t *x, int64_t ld, int64_t upr, int64_t u, float *v)
+{
+    int64_t row = u / upr;
+    int64_t j = u - row * upr;
+    const uint4 *p = reinterpret_cast<const uint4 *>(x + row * ld + j * 32);
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+        uint4 w = __ldg(p + c);
+        v[8 * c + 0] = bf16lo(w.x);
+        v[8 * c + 1] = bf16hi(w.x);
+        v[8 * c + 2] = bf16lo(w.y);
+        v[8 * c + 3] = bf16hi(w.y);
+        v[8 * c + 4] = bf16lo(w.z);
+        v[8 * c + 5] = bf16hi(w.z);
+        v[8 * c + 6] = bf16lo(w.w);
+        v[8 * c + 7] = bf16hi(w.w);
+    }
+}
+
+// Normalised Sylvester Walsh-Hadamard transform of every k-chunk, stages
+// h = 1, 2, ..., k/2 in ascending order: (a, b) -> (a + b, a - b) with a the
+// element whose index has bit h clear; then every value times ck.  Stages
+// with h >= 32 pair this lane with lane ^ (h / 32).
+template <int HK>
+FP4_DEV void fwht_unit(float *v, float ck, int lane)
+{
+#pragma unroll
+    for (int h = 1; h < (HK < 32 ? HK : 32); h <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            if (j & h) continue;
+            float a = v[j], b = v[j + h];
+            v[j] = __fadd_rn(a, b);
+            v[j + h] = __fsub_rn(a, b);
+        }
+    }
+#pragma unroll
+    for (int lm = 1; lm < HK / 32; lm <<= 1) {
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
+            v[j] = lower ? __fadd_rn(v[j], o) : __fsub_rn(o, v[j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; j++) v[j] = __fmul_rn(v[j], ck);
+}
+
+FP4_DEV float nv_global_from_amax(float amax)
+{
+    return (amax > 0.0f && amax <= kFltMax) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+FP4_DEV float read_global_scale(const float *g, int computed)
+{
+    float v = *g;
+    return computed ? nv_global_from_amax(v) : v;
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 tensor max |H_k x| -> *gscale (as the bits of a non-negative float;
+// integer order equals float order).  *gscale must be 0 on entry.
+template <int HK>
+__global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    float m = 0.0f;
+    for (int64_t base = warp * 32; base < a.total_units; base += nwarps * 32) {
+        const int64_t u = base + lane;
+        float v[32];
+        if (u < a.total_units) {
+            load_unit(a.x, a.ld, a.units_per_row, u, v);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; j++) v[j] = 0.0f;
+        }
+        if (HK) fwht_unit<HK>(v, a.ck, lane);
+#pragma unroll
+        for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ float red[8];
+    if (lane == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = red[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); w++) b = fmaxf(b, red[w]);
+        atomicMax(reinterpret_cast<unsigned int *>(a.gscale), __float_as_uint(b));
+    }
+}
+
+// Converts the tensor max left by amax_kernel into s_g = amax / (6 * 448)
+// (1 for an all-zero tensor).  Runs after the quantize kernel has read it.
+__global__ void finalize_gscale_kernel(float *g)
+{
+    *g = nv_global_from_amax(*g);
+}
+
+// ---------------------------------------------------------------------------
+template <int FMT, int HK>
+__global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+
+    float sg = 1.0f, six_sg = 6.0f;
+    if (FMT == FP4_NVFP4) {
+        sg = read_global_scale(a.gscale, a.gscale_computed);
+        six_sg = __fmul_rn(6.0f, sg);
+    }
+
+    for (int64_t base = warp * 32; base < a.total_units; base += nwarps * 32) {
+        const int64_t u = base + lane;
+        const bool live = u < a.total_units;
+        float v[32];
+        if (live) {
+            load_unit(a.x, a.ld, a.units_per_row, u, v);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; j++) v[j] = 0.0f;
+        }
+        if (HK) fwht_unit<HK>(v, a.ck, lane);
+        if (!live) continue;
+
+        const int64_t row = u / a.units_per_row;
+        const int64_t j = u - row * a.units_per_row;
+        if (FMT == FP4_MXFP4) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+            const int e = mx_exponent(amax, a.mx_floor);
+            const float inv = exp2i(-e);
+#pragma unroll
+            for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
+            a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)(e + 127);
+        } else {
+            uint32_t sb2 = 0;
+#pragma unroll
+            for (int b = 0; b < 2; b++) {
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[16 * b + i]));
+                const float t = __fdiv_rn(amax, six_sg);
+                const uint32_t sb = e4m3_rn(t);
+                const float d = __fmul_rn(sg, e4m3_to_f32(sb));
+                const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
+#pragma unroll
+                for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
+                sb2 |= sb << (8 * b);
+            }
+            *reinterpret_cast<uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4)) = (uint16_t)sb2;
+        }
+        uint4 out;
+        if (!a.round_away) {
+            out.x = e2m1x8_rn(v + 0);
+            out.y = e2m1x8_rn(v + 8);
+            out.z = e2m1x8_rn(v + 16);
+            out.w = e2m1x8_rn(v + 24);
+        } else {
+            out.x = e2m1x8_away(v + 0);
+            out.y = e2m1x8_away(v + 8);
+            out.z = e2m1x8_away(v + 16);
+            out.w = e2m1x8_away(v + 24);
+        }
+        *reinterpret_cast<uint4 *>(a.q + row * a.q_row_bytes + j * 16) = out;
+    }
+}
+
+// Zero the padding bytes of the scale tile layout: scale columns
+// [nkb, 4*nkb4) of real rows, and every byte of rows [rows, pad128(rows)).
+__global__ void scale_pad_kernel(uint8_t *s, int64_t rows, int64_t nkb, int64_t nkb4)
+{
+    const int64_t cpad = nkb4 * 4 - nkb;
+    const int64_t rows_p = (rows + 127) / 128 * 128;
+    const int64_t n1 = rows * cpad;
+    const int64_t n2 = (rows_p - rows) * nkb4 * 4;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n1 + n2;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r, kb;
+        if (i < n1) {
+            r = i / cpad;
+            kb = nkb + (i - r * cpad);
+        } else {
+            const int64_t t = i - n1;
+            r = rows + t / (nkb4 * 4);
+            kb = t % (nkb4 * 4);
+        }
+        s[scale_offset(r, kb, nkb4)] = 0;
+    }
+}
+
+// ---------------------------------------------------------------------------
+struct DequantArgs {
+    const uint8_t *q;
+    const uint8_t *s;
+    const float *gscale;
+    int64_t units_per_row;
+    int64_t total_units;
+    int64_t nkb4;
+    int64_t q_row_bytes;
+    int64_t cols;
+    void *out;
+    float ck;
+};
+
+template <int FMT, int HK, int BF16OUT>
+__global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const float sg = (FMT == FP4_NVFP4) ? *a.gscale : 1.0f;
+
+    for (int64_t base = warp * 32; base < a.total_units; base += nwarps * 32) {
+        const int64_t u = base + lane;
+        const bool live = u < a.total_units;
+        float v[32];
+        int64_t row = 0, j = 0;
+        if (live) {
+            row = u / a.units_per_row;
+            j = u - row * a.units_per_row;
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.q + row * a.q_row_bytes + j * 16));
+            const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+            float d0, d1;
+            if (FMT == FP4_MXFP4) {
+                const uint32_t sb = a.s[scale_offset(row, j, a.nkb4)];
+                d0 = d1 = (sb == 0xFF) ? __uint_as_float(0x7FC00000u) : exp2i((int)sb - 127);
+            } else {
+                const uint16_t sb2 = *reinterpret_cast<const uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4));
+                d0 = __fmul_rn(sg, e4m3_to_f32(sb2 & 0xFF));
+                d1 = __fmul_rn(sg, e4m3_to_f32(sb2 >> 8));
+            }
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+#pragma unroll
+                for (int b = 0; b < 4; b++) {
+                    float lo, hi;
+                    e2m1x2_to_f32((words[c] >> (8 * b)) & 0xFF, lo, hi);
+                    const float d = (c < 2) ? d0 : d1;
+                    v[8 * c + 2 * b] = __fmul_rn(d, lo);
+                    v[8 * c + 2 * b + 1] = __fmul_rn(d, hi);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; i++) v[i] = 0.0f;
+        }
+        if (HK) fwht_unit<HK>(v, a.ck, lane);
+        if (!live) continue;
+        if (BF16OUT) {
+            uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(a.out) + row * a.cols + j * 32);
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * c + 2 * i], v[8 * c + 2 * i + 1]);
+                    w[i] = *reinterpret_cast<uint32_t *>(&p);
+                }
+                o[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        } else {
+            float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + row * a.cols + j * 32);
+#pragma unroll
+            for (int c = 0; c < 8; c++) o[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers (called from capi.cu after validation).
+static int grid_for(int64_t total_units, int sms)
+{
+    const int64_t warps = (total_units + 31) / 32;
+    const int64_t blocks = (warps + 7) / 8;  // 8 warps per 256-thread block
+    const int64_t cap = (int64_t)sms * 8;
+    return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+template <int FMT>
+static cudaError_t launch_quant_fmt(const QuantArgs &a, int hk, int grid, cudaStream_t st)
+{
+    count_launches(1);
+    switch (hk) {
+    case 0: quantize_kernel<FMT, 0><<<grid, 256, 0, st>>>(a); break;
+    case 16: quantize_kernel<FMT, 16><<<grid, 256, 0, st>>>(a); break;
+    case 32: quantize_kernel<FMT, 32><<<grid, 256, 0, st>>>(a); break;
+    case 64: quantize_kernel<FMT, 64><<<grid, 256, 0, st>>>(a); break;
+    case 128: quantize_kernel<FMT, 128><<<grid, 256, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_amax(const QuantArgs &a, int hk, int grid, cudaStream_t st)
+{
+    count_launches(1);
+    switch (hk) {
+    case 0: amax_kernel<0><<<grid, 256, 0, st>>>(a); break;
+    case 16: amax_kernel<16><<<grid, 256, 0, st>>>(a); break;
+    case 32: amax_kernel<32><<<grid, 256, 0, st>>>(a); break;
+    case 64: amax_kernel<64><<<grid, 256, 0, st>>>(a); break;
+    case 128: amax_kernel<128><<<grid, 256, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
+                            int hk, float ck, int round_away, int mx_floor, int gscale_given,
+                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st)
+{
+    QuantArgs a;
+    a.x = x;
+    a.ld = ld;
+    a.units_per_row = cols / 32;
+    a.total_units = rows * (cols / 32);
+    const int64_t nkb = cols / (fmt == FP4_MXFP4 ? 32 : 16);
+    a.nkb4 = (nkb + 3) / 4;
+    a.q_row_bytes = cols / 2;
+    a.q = q;
+    a.s = s;
+    a.gscale = gscale;
+    a.ck = ck;
+    a.round_away = round_away;
+    a.mx_floor = mx_floor;
+    a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
+    const int grid = grid_for(a.total_units, sms);
+    cudaError_t err = cudaSuccess;
+    if (a.gscale_computed) {
+        if ((err = cudaMemsetAsync(gscale, 0, sizeof(float), st)) != cudaSuccess) return err;
+        if ((err = launch_amax(a, hk, grid, st)) != cudaSuccess) return err;
+    }
+    if (a.total_units > 0) {
+        err = (fmt == FP4_MXFP4) ? launch_quant_fmt<FP4_MXFP4>(a, hk, grid, st)
+                                 : launch_quant_fmt<FP4_NVFP4>(a, hk, grid, st);
+        if (err != cudaSuccess) return err;
+    }
+    if (a.gscale_computed) {
+        count_launches(1);
+        finalize_gscale_kernel<<<1, 1, 0, st>>>(gscale);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    const int64_t rows_p = (rows + 127) / 128 * 128;
+    const int64_t npad = rows * (a.nkb4 * 4 - nkb) + (rows_p - rows) * a.nkb4 * 4;
+    if (npad > 0) {
+        int g = (int)((npad + 255) / 256);
+        if (g > sms * 4) g = sms * 4;
+        count_launches(1);
+        scale_pad_kernel<<<g, 256, 0, st>>>(s, rows, nkb, a.nkb4);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+}
+
+template <int FMT, int BF>
+static cudaError_t launch_deq_fmt(const DequantArgs &a, int hk, int grid, cudaStream_t st)
+{
+    count_launches(1);
+    switch (hk) {
+    case 0: dequantize_kernel<FMT, 0, BF><<<grid, 256, 0, st>>>(a); break;
+    case 16: dequantize_kernel<FMT, 16, BF><<<grid, 256, 0, st>>>(a); break;
+    case 32: dequantize_kernel<FMT, 32, BF><<<grid, 256, 0, st>>>(a); break;
+    case 64: dequantize_kernel<FMT, 64, BF><<<grid, 256, 0, st>>>(a); break;
+    case 128: dequantize_kernel<FMT, 128, BF><<<grid, 256, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
+                              int64_t cols, int fmt, int hk, float ck, int bf16out, void *out,
+                              int sms, cudaStream_t st)
+{
+    DequantArgs a;
+    a.q = q;
+    a.s = s;
+    a.gscale = gscale;
+    a.units_per_row = cols / 32;
+    a.total_units = rows * (cols / 32);
+    const int64_t nkb = cols / (fmt == FP4_MXFP4 ? 32 : 16);
+    a.nkb4 = (nkb + 3) / 4;
+    a.q_row_bytes = cols / 2;
+    a.cols = cols;
+    a.out = out;
+    a.ck = ck;
+    if (a.total_units == 0) return cudaSuccess;
+    const int grid = grid_for(a.total_units, sms);
+    if (fmt == FP4_MXFP4)
+        return bf16out ? launch_deq_fmt<FP4_MXFP4, 1>(a, hk, grid, st) : launch_deq_fmt<FP4_MXFP4, 0>(a, hk, grid, st);
+    return bf16out ? launch_deq_fmt<FP4_NVFP4, 1>(a, hk, grid, st) : launch_deq_fmt<FP4_NVFP4, 0>(a, hk, grid, st);
+}
+
+}  // namespace fp4

@@ -1,0 +1,163 @@
+/*
+ * fp4.h — C ABI of the B200 (sm_100a) microscaling FP4 library.
+ *
+ * Formats (element E2M1 in every case):
+ *   MXFP4  32-element blocks along K, one E8M0 (power-of-two) scale per block.
+ *   NVFP4  16-element blocks along K, one unsigned E4M3 scale per block, and
+ *          one FP32 tensor-level scale s_g.
+ * Sources: "Portable FP4 quantization (TransFP4)" §1.1 Eq.(1)
+ * (x^_i = s_g s_b Q_f(x_i / (s_g s_b))) and Table 1; "4.5 FP8 and
+ * NVFP4/MXFP4" §3.1 (E2M1 magnitudes), §3.3 and §4.1 (scale formats, the
+ * two-level NVFP4 dequantization); "FP4 quantization analysis: MXFP4 vs
+ * NVFP4" §3.2.3 (block-diagonal Hadamard H_k, k in {16,32,64,128}) and §3.3
+ * (fused rotation kernel, FP4-specific operand re-layout for the GEMM).
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless the name says host.  The caller
+ *     allocates and owns every buffer; the library never allocates or frees
+ *     device memory and keeps no pointer after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous and stream-ordered; none synchronizes
+ *     the host.
+ *   - Shapes are validated on the host before any launch; an invalid call
+ *     launches nothing and returns an error code.  Errors raised by a
+ *     launch return FP4_ERR_CUDA; faults of an earlier asynchronous launch
+ *     surface on a later call or synchronization.
+ *   - Inputs must be finite.  Quantization axis = contraction axis = K, the
+ *     contiguous (column) axis of a row-major rows x cols tensor.
+ *
+ * Layouts:
+ *   Packed elements q: rows x cols/2 bytes, row stride cols/2; byte j of a
+ *     row holds element 2j in bits [3:0] and element 2j+1 in bits [7:4];
+ *     bit 3 of a nibble is the sign.
+ *   Scales s: the tile layout the block-scaled tensor-core MMA reads.
+ *     Logical scale S[r][kb] (kb = block index along K, nkb = cols/block)
+ *     lives at byte
+ *       ((r/128) * ceil(nkb/4) + kb/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + kb%4
+ *     i.e. 512-byte atoms of 128 rows x 4 scales.  Rows are padded to a
+ *     multiple of 128 and scale columns to a multiple of 4; fp4_quantize
+ *     writes every padding byte as 0.
+ */
+#ifndef FP4_H
+#define FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum     */
+    FP4_ERR_UNSUPPORTED = 2,   /* shape or format combination not provided  */
+    FP4_ERR_ALIGNMENT = 3,     /* pointer or stride not aligned as required */
+    FP4_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed      */
+    FP4_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait           */
+} fp4_status;
+
+typedef enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1 } fp4_fmt;
+
+/* E2M1 tie rule at exact midpoints: even code (IEEE style, default) or the
+ * larger magnitude (reproduces the gpt-oss article's worked example). */
+typedef enum { FP4_ROUND_EVEN = 0, FP4_ROUND_AWAY = 1 } fp4_round;
+
+/* MXFP4 shared exponent: CEIL = smallest e with amax <= 6*2^e (no element
+ * clips; default); FLOOR = floor(log2 amax) - 2 (the OCP MX rule; values
+ * between 6 and 8 times the scale saturate to 6). */
+typedef enum { FP4_MX_SCALE_CEIL = 0, FP4_MX_SCALE_FLOOR = 1 } fp4_mx_scale_rule;
+
+typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_dtype;
+
+typedef struct {
+    int round;          /* fp4_round                                          */
+    int mx_scale_rule;  /* fp4_mx_scale_rule                                  */
+    int gscale_given;   /* NVFP4: 1 = *gscale holds s_g on entry (offline
+                           scale); 0 = s_g is computed from the tensor.       */
+} fp4_opts;
+
+/* Human-readable name of a status code (static string). */
+const char *fp4_status_string(fp4_status st);
+
+/* Sizes of the packed-element and scale buffers for a rows x cols tensor.
+ * q_bytes = rows*cols/2; s_bytes = pad128(rows) * pad4(cols/block).
+ * Host-only; block must be 32 for MXFP4 and 16 for NVFP4. */
+fp4_status fp4_quantize_sizes(int64_t rows, int64_t cols, int fmt, int block,
+                              size_t *q_bytes, size_t *s_bytes);
+
+/*
+ * fp4_quantize — microscaling quantization, TransFP4 Eq.(1), optionally after
+ * the block-diagonal Hadamard rotation H_k (MR-GPTQ §3.2.3) of every
+ * contiguous k-element chunk along K.
+ *
+ *   x       bf16 input, rows x cols, row stride ld_x elements.  16-byte
+ *           aligned; ld_x a multiple of 8.
+ *   fmt     FP4_MXFP4 (block 32) or FP4_NVFP4 (block 16).
+ *   hadamard_k  0 (no rotation) or 16, 32, 64, 128; cols % k == 0.  The
+ *           rotation is the normalised Sylvester Walsh-Hadamard transform
+ *           (stages h = 1, 2, ..., k/2, then x RN(1/sqrt(k))) in fp32.
+ *   opts    may be NULL (= round even, CEIL, s_g computed).
+ *   q       output, packed elements (layout above), 16-byte aligned.
+ *   s       output, scales in the tile layout above (padding written 0).
+ *   gscale  NVFP4 only (ignored for MXFP4, may be NULL): one device fp32.
+ *           gscale_given: read as s_g.  Otherwise written with
+ *           s_g = amax(|H_k x|) / (6*448), or 1 for an all-zero tensor.
+ * cols must be a multiple of 32 (also for NVFP4).  rows == 0 is a no-op.
+ */
+fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                        int fmt, int block, int hadamard_k, const fp4_opts *opts,
+                        uint8_t *q, uint8_t *s, float *gscale, void *stream);
+
+/*
+ * fp4_dequantize — x^ = s_g * s_b * q ("4.5 FP8 and NVFP4/MXFP4" §4.1; for
+ * MXFP4 s_g = 1 and s_b = 2^(byte-127)), NVFP4 computed as
+ * RN(RN(s_g*s_b) * q).  hadamard_k > 0 applies H_k again (it is its own
+ * inverse) to return to the unrotated domain; 0 leaves values rotated.
+ *   q, s, gscale   as produced by fp4_quantize (gscale ignored for MXFP4).
+ *   out_dtype      FP4_OUT_F32 or FP4_OUT_BF16 (round to nearest even).
+ *   out            rows x cols, row stride cols, 16-byte aligned.
+ */
+fp4_status fp4_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale,
+                          int64_t rows, int64_t cols, int fmt, int block,
+                          int hadamard_k, int out_dtype, void *out, void *stream);
+
+/* Bytes of scratch fp4_gemm needs for this shape (0 when none). Host-only. */
+fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt,
+                                   size_t *bytes);
+
+/*
+ * fp4_gemm — W4A4 linear C = alpha * A W^T with FP32 accumulation
+ * ("4.5 FP8 and NVFP4/MXFP4" §5: both operands in FP4 on the Blackwell
+ * tensor cores), A: M x K, W: N x K, both quantized along K in the same
+ * format by fp4_quantize (Aq/As, Wq/Ws).  alpha = s_gA * s_gW for NVFP4
+ * (gA, gW device fp32), 1 for MXFP4 (gA, gW ignored).
+ *   K          multiple of 256.
+ *   out_dtype  FP4_OUT_F32 or FP4_OUT_BF16.  C row-major, row stride ldc
+ *              elements (ldc >= N).
+ *   workspace  device scratch of at least fp4_gemm_workspace_size() bytes
+ *              (may be NULL when that size is 0).
+ * Rotated operands: quantize both A and W with the same hadamard_k;
+ * (X H)(W H)^T = X W^T, so C needs no correction.
+ * M <= 16 runs the decode (weight-streaming, split-K) kernel; larger M the
+ * tiled tensor-core kernel.
+ */
+fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA,
+                    const uint8_t *Wq, const uint8_t *Ws, const float *gW,
+                    int64_t M, int64_t N, int64_t K, int fmt, int out_dtype,
+                    void *C, int64_t ldc, void *workspace, size_t ws_bytes,
+                    void *stream);
+
+/* Number of kernels this library has launched in this process so far
+ * (host-side counter; diagnostics and launch accounting). */
+uint64_t fp4_kernel_launches(void);
+
+/* Reads and clears the device-side error word that kernels set when a
+ * bounded wait gives up.  Synchronizes `stream`.  Returns FP4_ERR_TIMEOUT if
+ * it was set, else FP4_OK (or FP4_ERR_CUDA). */
+fp4_status fp4_check_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

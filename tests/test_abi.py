@@ -1,0 +1,104 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared symbol,
+and rejects invalid calls on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp4_microscaling_quantization_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(fp4_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert "fp4_quantize" in names and "fp4_gemm" in names
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert set(_lib.SIGNATURES) <= names
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert L.fp4_status_string(code).startswith(b"FP4_")
+
+
+def test_quantize_sizes(L):
+    q, s = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.fp4_quantize_sizes(200, 320, 0, 32, ctypes.byref(q), ctypes.byref(s)) == 0
+    assert q.value == 200 * 160 and s.value == 256 * 12
+    assert L.fp4_quantize_sizes(200, 320, 1, 16, ctypes.byref(q), ctypes.byref(s)) == 0
+    assert s.value == 256 * 20
+    assert L.fp4_quantize_sizes(4, 64, 0, 16, ctypes.byref(q), ctypes.byref(s)) == 2  # MX needs 32
+    assert L.fp4_quantize_sizes(-1, 64, 0, 32, ctypes.byref(q), ctypes.byref(s)) == 1
+
+
+FAKE = 0x10000  # an aligned pointer value never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(rows=-1), 1),
+    (dict(fmt=0, block=16), 2),
+    (dict(fmt=1, block=32), 2),
+    (dict(hadamard_k=8), 2),
+    (dict(cols=48), 2),
+    (dict(cols=64, hadamard_k=128), 2),
+    (dict(ld=16), 1),
+    (dict(x=FAKE + 8), 3),
+    (dict(ld=68), 3),
+    (dict(q=FAKE + 4), 3),
+    (dict(fmt=1, block=16, g=None), 1),
+    (dict(x=None), 1),
+])
+def test_quantize_rejects_on_host(L, args, code):
+    a = dict(x=FAKE, rows=4, cols=64, ld=64, fmt=0, block=32, hadamard_k=0, q=FAKE, s=FAKE, g=FAKE)
+    a.update(args)
+    rc = L.fp4_quantize(a["x"], a["rows"], a["cols"], a["ld"], a["fmt"], a["block"], a["hadamard_k"],
+                        None, a["q"], a["s"], a["g"], None)
+    assert rc == code
+
+
+def test_bad_opts_rejected(L):
+    o = _lib.Fp4Opts(7, 0, 0)
+    assert L.fp4_quantize(FAKE, 4, 64, 64, 0, 32, 0, ctypes.byref(o), FAKE, FAKE, FAKE, None) == 1
+    o = _lib.Fp4Opts(0, 3, 0)
+    assert L.fp4_quantize(FAKE, 4, 64, 64, 0, 32, 0, ctypes.byref(o), FAKE, FAKE, FAKE, None) == 1
+
+
+def test_dequantize_rejects_on_host(L):
+    assert L.fp4_dequantize(FAKE, FAKE, FAKE, 4, 64, 0, 32, 0, 9, FAKE, None) == 1
+    assert L.fp4_dequantize(FAKE, FAKE, None, 4, 64, 1, 16, 0, 0, FAKE, None) == 1
+    assert L.fp4_dequantize(FAKE + 1, FAKE, FAKE, 4, 64, 0, 32, 0, 0, FAKE, None) == 3
+    assert L.fp4_dequantize(FAKE, FAKE, FAKE, 4, 48, 0, 32, 0, 0, FAKE, None) == 2
+
+
+def test_gemm_rejects_on_host(L):
+    g = L.fp4_gemm
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 100, 0, 1, FAKE, 8, None, 0, None) == 2  # K % 256
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 4, None, 0, None) == 1  # ldc < N
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 5, 1, FAKE, 8, None, 0, None) == 2
+    assert g(None, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 8, None, 0, None) == 1
+    assert g(FAKE, FAKE, None, FAKE, FAKE, FAKE, 4, 8, 256, 1, 1, FAKE, 8, None, 0, None) == 1
+    assert g(FAKE + 2, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 8, None, 0, None) == 3
+
+
+def test_empty_mx_is_noop(L):
+    assert L.fp4_quantize(None, 0, 64, 64, 0, 32, 0, None, None, None, None, None) == 0
+    assert L.fp4_dequantize(None, None, None, 0, 64, 0, 32, 0, 0, None, None) == 0

@@ -1,0 +1,184 @@
+"""GPU parity of fp4_quantize / fp4_dequantize against the CPU oracle.
+
+Packed nibbles, scale bytes (tile layout, padding included) and the NVFP4
+tensor scale must be bit-exact; dequantized fp32 values too (both sides do the
+same IEEE fp32 operations), and bf16 output is the RNE rounding of them.
+"""
+import numpy as np
+import pytest
+
+from fp4_microscaling_quantization_b200 import inputs
+
+from helpers import bf16_tensor_bits, to_dev_bf16, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp4():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fp4_microscaling_quantization_b200 import build
+    build.build()
+    import fp4_microscaling_quantization_b200 as m
+    return m
+
+
+def check_quantize(fp4, orc, x, fmt, hk=0, tie=0, rule=0, gscale=None, x_dev=None):
+    import torch
+    rows, cols = x.shape
+    xd = to_dev_bf16(x) if x_dev is None else x_dev
+    gs = None if gscale is None else torch.tensor([gscale], dtype=torch.float32, device="cuda")
+    q, s, g = fp4.quantize(xd, fmt, hadamard_k=hk, round=tie, mx_scale_rule=rule, gscale=gs)
+    torch.cuda.synchronize()
+    oq, os_, og = orc.quantize(x, fmt, hadamard_k=hk, tie=tie, mx_rule=rule, gscale=gscale)
+    q_np, s_np = to_np(q), to_np(s)
+    bad = np.argwhere(q_np != oq)
+    assert bad.size == 0, f"nibbles differ at {bad[:4].tolist()}: gpu {q_np[tuple(bad[0])]:#x} oracle {oq[tuple(bad[0])]:#x}"
+    os_atoms = orc.scales_to_atoms(os_)
+    assert s_np.shape == os_atoms.shape
+    sbad = np.flatnonzero(s_np != os_atoms)
+    assert sbad.size == 0, f"scales differ at {sbad[:4].tolist()}"
+    if fmt == fp4.FP4_NVFP4:
+        assert np.float32(to_np(g)[0]) == np.float32(og), (to_np(g)[0], og)
+    return q, s, g, (oq, os_, og)
+
+
+SHAPES = [(1, 32), (3, 96), (130, 512), (257, 1024), (64, 4096)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_parity_shapes(fp4, orc, shape, fmt):
+    rows, cols = shape
+    rng = np.random.default_rng(rows * 7 + cols)
+    v = rng.laplace(0, 1, shape).astype(np.float32)
+    v[rng.random(shape) < 0.01] *= 20
+    check_quantize(fp4, orc, inputs.f32_to_bf16_bits(v), fmt)
+
+
+@pytest.mark.parametrize("hk", [16, 32, 64, 128])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_parity_rotated(fp4, orc, hk, fmt):
+    x = inputs.rotate_acts(rows=136, cols=1024, seed=hk)
+    check_quantize(fp4, orc, x, fmt, hk=hk)
+
+
+@pytest.mark.parametrize("fmt,tie,rule", [(0, 1, 0), (0, 0, 1), (0, 1, 1), (1, 1, 0)])
+def test_quantize_parity_modes(fp4, orc, fmt, tie, rule):
+    x = inputs.quant_sweep(rows=40, cols=2048, seed=9)
+    check_quantize(fp4, orc, x, fmt, hk=32, tie=tie, rule=rule)
+    check_quantize(fp4, orc, x, fmt, hk=0, tie=tie, rule=rule)
+
+
+def edge_tensor():
+    """Rows of special values: zeros, -0, bf16 subnormals, exact E2M1 ties
+    under a power-of-two scale, saturation, lone outliers, huge values."""
+    rows = []
+    rows.append(np.zeros(64, np.float32))
+    rows.append(-np.zeros(64, np.float32))
+    sub = np.array([(i + 1) * 2.0 ** -133 for i in range(64)], np.float32)  # bf16 subnormals
+    rows.append(sub * np.where(np.arange(64) % 2, -1, 1))
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0] * 8, np.float32)
+    rows.append(ties * np.where(np.arange(64) % 3 == 0, -1, 1))   # block max 6 -> scale 1
+    rows.append(ties * 2.0 ** 20)
+    r = np.full(64, 1e-3, np.float32)
+    r[5] = 1e4
+    r[40] = -3e5
+    rows.append(r)
+    rows.append(np.linspace(-3e38, 3e38, 64).astype(np.float32))
+    rows.append(np.full(64, -1.0, np.float32))
+    x = np.stack(rows)
+    return inputs.f32_to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("fmt,tie", [(0, 0), (0, 1), (1, 0), (1, 1)])
+def test_quantize_edge_cases(fp4, orc, fmt, tie):
+    x = edge_tensor()
+    check_quantize(fp4, orc, x, fmt, tie=tie)
+    check_quantize(fp4, orc, x[:6], fmt, tie=tie, hk=64)
+
+
+@pytest.mark.parametrize("gscale", [1.0, 1e-3, 1e-30, 7.5e2, 3e30])
+def test_nvfp4_given_global_scale(fp4, orc, gscale):
+    """Offline s_g: saturation (tiny s_g), underflow to zero scales (huge s_g)."""
+    x = inputs.quant_sweep(rows=16, cols=512, seed=3)
+    check_quantize(fp4, orc, x, 1, gscale=gscale)
+
+
+def test_all_zero_tensor_nvfp4(fp4, orc):
+    x = np.zeros((5, 64), np.uint16)
+    q, s, g, _ = check_quantize(fp4, orc, x, 1)
+    assert to_np(g)[0] == 1.0
+
+
+def test_strided_input(fp4, orc):
+    import torch
+    x = inputs.quant_sweep(rows=33, cols=512, seed=4)
+    big = np.zeros((33, 640), np.uint16)
+    big[:, :512] = x
+    xd = to_dev_bf16(big)[:, :512]
+    assert xd.stride(0) == 640
+    for fmt in (0, 1):
+        check_quantize(fp4, orc, x, fmt, x_dev=xd)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("hk", [0, 32, 128])
+@pytest.mark.parametrize("bf16", [0, 1])
+def test_dequantize_parity(fp4, orc, fmt, hk, bf16):
+    import torch
+    x = inputs.rotate_acts(rows=130, cols=512, seed=5)
+    q, s, g, (oq, os_, og) = check_quantize(fp4, orc, x, fmt, hk=hk)
+    out = fp4.dequantize(q, s, g, fmt, hadamard_k=hk, out_dtype=bf16)
+    torch.cuda.synchronize()
+    ref = orc.dequantize(oq, os_, og, fmt, hadamard_k=hk)
+    if bf16:
+        got = bf16_tensor_bits(out)
+        want = inputs.f32_to_bf16_bits(ref)
+        assert np.array_equal(got, want)
+    else:
+        got = to_np(out)
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # leaving the values rotated: dequantize without the inverse rotation
+    if hk:
+        out2 = fp4.dequantize(q, s, g, fmt, hadamard_k=0)
+        ref2 = orc.dequantize(oq, os_, og, fmt, hadamard_k=0)
+        assert np.array_equal(to_np(out2).view(np.uint32), ref2.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_full_size_quant_sweep(fp4, orc, fmt):
+    """1024 x 131072 heavy-tailed tensor: whole-tensor parity at the
+    benchmark's size and launch configuration."""
+    import torch
+    x = inputs.quant_sweep()
+    check_quantize(fp4, orc, x, fmt)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("hk", [0, 16, 128])
+def test_full_size_rotate(fp4, orc, fmt, hk):
+    """8192 x 4096 activations with outlier channels, rotated then quantized."""
+    x = inputs.rotate_acts()
+    check_quantize(fp4, orc, x, fmt, hk=hk)
+
+
+def test_reuses_output_buffers(fp4, orc):
+    import torch
+    x = inputs.quant_sweep(rows=8, cols=256, seed=1)
+    xd = to_dev_bf16(x)
+    q, s, g = fp4.quantize(xd, 1)
+    q2, s2, g2 = fp4.quantize(xd, 1, out=(torch.empty_like(q), torch.empty_like(s), torch.empty_like(g)))
+    assert torch.equal(q, q2) and torch.equal(s, s2) and torch.equal(g, g2)
+
+
+@pytest.mark.parametrize("row", range(8))
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_edge_rows_alone(fp4, orc, row, fmt):
+    """Each special-value row as its own tensor, so the NVFP4 tensor scale is
+    computed from it (all-zero, -0, subnormal-only, tie-only, ... tensors)."""
+    x = edge_tensor()[row:row + 1]
+    check_quantize(fp4, orc, x, fmt)
