@@ -52,6 +52,64 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def fp4_tensor_peak():
+    """Dense FP4 tensor peak: the measured bf16 GEMM burst figure x 4, the
+    nominal fp4 / bf16 ratio (9 / 2.25 PFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return 4.0 * float(json.load(open(p))["bf16_tflops"]), "measured bf16 burst x 4"
+    return 4.0 * 1590.0, "fallback bf16 x 4"
+
+
+def time_graph(torch, fn, warmup: int, reps: int):
+    """Average device time of `fn` (ms) over `reps` launches captured in one
+    CUDA graph, after `warmup` captured launches."""
+    fn()
+    torch.cuda.synchronize()
+    gw = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw):
+        for _ in range(warmup):
+            fn()
+    gt = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gt):
+        for _ in range(reps):
+            fn()
+    gw.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    gt.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def bench_prefill(torch, fp4, inputs, dev, reps: int):
+    """W4A4 prefill GEMM, 70B-MLP shape: A 8192x8192, W 28672x8192, BF16 out."""
+    M, N, K = 8192, 28672, 8192
+    a, w = inputs.prefill_linear()
+    ad = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
+    del a, w
+    peak, kind = fp4_tensor_peak()
+    out = {"workload": f"prefill W4A4 linear M={M} N={N} K={K}, BF16 out", "peak_tflops": peak, "peak_kind": kind}
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    for fmt, name in ((fp4.FP4_NVFP4, "nvfp4"), (fp4.FP4_MXFP4, "mxfp4")):
+        A = fp4.quantize(ad, fmt)
+        W = fp4.quantize(wd, fmt)
+        ms = time_graph(torch, lambda: fp4.gemm(A, W, M, N, K, fmt, out=C), 3, reps)
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[name] = {"ms": ms, "tflops": tf, "frac": tf / peak}
+        q_ms = time_graph(torch, lambda: fp4.quantize(ad, fmt, out=A), 3, reps)
+        out[name]["act_quantize_ms"] = q_ms
+        out[name]["tflops_incl_act_quantize"] = 2.0 * M * N * K / ((ms + q_ms) * 1e-3) / 1e12
+        del A, W
+    del ad, wd, C
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------- clocks -----
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -129,11 +187,10 @@ def barrier(ws: int):
 
 
 # ---------------------------------------------------------------- oracle leg --
-def oracle_sample(rows: int, seed: int = 2):
-    """Times the CPU oracle on a `rows`-row slab of the same workload."""
+def oracle_step(x):
+    """Times the CPU oracle (as it stands, OpenMP over rows) on one step."""
     import oracle
-    from fp4_microscaling_quantization_b200 import inputs
-    x = inputs.quant_sweep(rows=rows, cols=COLS, seed=seed)
+    rows = x.shape[0]
     t0 = time.perf_counter()
     qm, sm, _ = oracle.quantize(x, oracle.MXFP4)
     qn, sn, gn = oracle.quantize(x, oracle.NVFP4)
@@ -149,11 +206,13 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
+    from fp4_microscaling_quantization_b200 import inputs
     oracle.build()
-    rows = 16
+    rows = 256
+    x = inputs.quant_sweep(rows=rows, seed=2)
     times = []
     for i in range(args.warmup + args.steps):
-        gbs, dt, cores = oracle_sample(rows)
+        gbs, dt, cores = oracle_step(x)
         if i >= args.warmup:
             times.append(dt)
     dt = statistics.mean(times)
@@ -205,7 +264,7 @@ def run_ours(args):
     def step(evs=None):
         def mark(i):
             if evs is not None:
-                evs[i].record(stream)
+                evs[i].record()
         mark(0)
         fp4.quantize(x, fp4.FP4_MXFP4, out=(qm, sm, gm))
         mark(1)
@@ -216,25 +275,38 @@ def run_ours(args):
         fp4.dequantize(qn, sn, gn, fp4.FP4_NVFP4, out_dtype=fp4.FP4_OUT_BF16, out=dn)
         mark(4)
 
-    for _ in range(args.warmup):
-        step()
+    # The W warm-up steps and the K timed steps are each captured once into a
+    # CUDA graph (no host work between kernels); the timed graph carries
+    # event-record nodes between the calls for the per-kernel breakdown.
+    step()
+    torch.cuda.synchronize()
+    launches0 = _lib.lib().fp4_kernel_launches()
+    g_warm = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm):
+        for _ in range(args.warmup):
+            step()
+    evsets = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(args.steps)]
+    launches1 = _lib.lib().fp4_kernel_launches()
+    g_timed = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_timed):
+        for i in range(args.steps):
+            step(evsets[i])
+    launches = _lib.lib().fp4_kernel_launches() - launches1
     torch.cuda.synchronize()
 
+    g_warm.replay()
+    torch.cuda.synchronize()
     per = {n: 0.0 for n in names}
-    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    launches0 = _lib.lib().fp4_kernel_launches()
     with ClockSampler(dev.index) as clk:
         barrier(ws)
         torch.cuda.synchronize()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        for i in range(args.steps):
-            step(evsets[i])
+        g_timed.replay()
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(ws)
-    launches = _lib.lib().fp4_kernel_launches() - launches0
     total_ms = t0.elapsed_time(t1)
     for ev in evsets:
         for j, n in enumerate(names):
@@ -294,14 +366,17 @@ def run_ours(args):
 
     nmse_vals = {"mxfp4": nmse(dm), "nvfp4": nmse(dn), "rows_sampled": 8}
 
+    gemm = None
+    if not args.no_gemm:
+        gemm = {"prefill": bench_prefill(torch, fp4, inputs, dev, reps=10)}
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        crow = 16
-        gbs, dt, cores = oracle_sample(crow)
+        gbs, dt, cores = oracle_step(x_np)
         cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": f"{crow} of {ROWS} rows of the same step, {dt:.1f} s"}
+               "sample": f"one full step ({rows} x {cols}) on the host, {dt:.1f} s"}
 
     if ws > 1:
         import torch.distributed as dist
@@ -321,6 +396,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": int(launches),
+        "gemm": gemm,
         "nmse": nmse_vals,
         "clocks": clk.summary(),
     }
@@ -336,6 +412,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--rows", type=int, default=ROWS, help="rows of the tensor (profiling runs use fewer)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-gemm", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

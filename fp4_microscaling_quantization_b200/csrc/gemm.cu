@@ -1,19 +1,300 @@
-// gemm.cu — block-scaled W4A4 GEMM kernels (placeholder until the tcgen05
-// kernels land: every call reports the shape as unsupported).
-#include "common.cuh"
+// gemm.cu — block-scaled W4A4 GEMM on the 5th-generation tensor cores:
+// C[M x N] = alpha * sum_k deq(A[m,k]) * deq(W[n,k]), FP32 accumulation in
+// tensor memory ("4.5 FP8 and NVFP4/MXFP4" §5: both operands FP4 on the
+// Blackwell tensor cores; "FP4 quantization analysis: MXFP4 vs NVFP4" §3.3:
+// FP4-specific operand re-layout feeding the GEMM).
+//
+// Operands come straight from fp4_quantize: packed E2M1 rows (K-major) and
+// scales already in the 128x4 atom layout the MMA reads, so no re-layout
+// pass exists.  alpha = s_gA * s_gW for NVFP4, 1 for MXFP4.
+//
+// Tiled kernel (one 128 x 256 output tile per CTA, 4 warps):
+//   warp 0 lane 0  TMA producer: A (128 x 256 fp4) and W (256 x 256 fp4)
+//                  tiles with 128-byte swizzle, plus the scale atoms, into a
+//                  4-stage shared-memory ring (mbarrier transaction counts);
+//   warp 1 lane 0  MMA issuer: tcgen05.cp of the scale atoms to TMEM, then
+//                  four K=64 block-scaled MMAs per stage into a 128 x 256 fp32
+//                  TMEM accumulator; tcgen05.commit frees the stage;
+//   warps 0-3      epilogue: tcgen05.ld of their 32-lane quarter, x alpha,
+//                  convert, store.
+// Every wait is bounded (%globaltimer); a wait that gives up sets the device
+// error word, the CTA drains its in-flight copies and MMAs, frees its TMEM and
+// returns without storing.
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
 
 namespace fp4 {
 
 static __device__ unsigned int g_gemm_error;
 
+namespace tiled {
+
+constexpr int BM = 128, BN = 256, BK = 256;  // BK in fp4 elements (128 bytes)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK / 2;         // 16 KB
+constexpr int B_BYTES = BN * BK / 2;         // 32 KB
+constexpr int SFA_BYTES = 4 * 512;           // up to 4 atoms (NVFP4)
+constexpr int SFB_BYTES = 2 * 4 * 512;       // 2 row blocks x 4 atoms
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296, multiple of 1024
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COL = 0;
+constexpr int SF_COL0 = 256;                 // per stage: SFA 16 cols, SFB 32 cols
+constexpr int SF_STAGE_COLS = 48;
+
+struct Params {
+    const uint8_t *As;
+    const uint8_t *Ws;
+    const float *gA;
+    const float *gW;
+    void *C;
+    int64_t ldc;
+    int M, N, K;
+    int nkb4;       // scale-atom columns per 128-row block (K / block / 4)
+    int nrb_w;      // 128-row scale blocks of W (pad128(N) / 128)
+};
+
+template <int FMT, int BF16OUT>
+__global__ void __launch_bounds__(128, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p)
+{
+    constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;  // scale atoms per stage per 128-row block
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    // bars[0..S): full, bars[S..2S): empty, bars[2S]: accumulator ready
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int mt = blockIdx.x, nt = blockIdx.y;
+    const int nk = p.K / BK;
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES), accb = smem_u32(bars + 2 * STAGES);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; s++) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(accb, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            const int nrb = (2 * nt + 1 < p.nrb_w) ? 2 : 1;
+            const uint32_t tx = A_BYTES + B_BYTES + KA * 512 * (1 + nrb);
+            int issued = 0;
+            for (int ks = 0; ks < nk; ks++) {
+                const int s = ks % STAGES;
+                const uint32_t ph = (ks / STAGES) & 1;
+                if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error)) break;
+                uint8_t *st = smem + s * STAGE_BYTES;
+                const uint32_t fb = full0 + 8 * s;
+                mbar_arrive_expect_tx(fb, tx);
+                tma_load_2d(smem_u32(st), &tmA, ks * (BK / 2), mt * BM, fb);
+                tma_load_2d(smem_u32(st + A_BYTES), &tmB, ks * (BK / 2), nt * BN, fb);
+                bulk_load(smem_u32(st + A_BYTES + B_BYTES), p.As + ((int64_t)mt * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+                for (int rb = 0; rb < nrb; rb++)
+                    bulk_load(smem_u32(st + A_BYTES + B_BYTES + SFA_BYTES + rb * KA * 512),
+                              p.Ws + ((int64_t)(2 * nt + rb) * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+                issued = ks + 1;
+            }
+            // drain: every issued copy must land before the CTA may exit
+            for (int ks = (issued > STAGES ? issued - STAGES : 0); ks < issued; ks++) {
+                volatile uint32_t no_abort = 0;
+                mbar_wait_bounded(full0 + 8 * (ks % STAGES), (ks / STAGES) & 1, &no_abort, &g_gemm_error);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            const uint32_t acc = tmem + ACC_COL;
+            for (int ks = 0; ks < nk; ks++) {
+                const int s = ks % STAGES;
+                const uint32_t ph = (ks / STAGES) & 1;
+                if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error)) break;
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+                const uint32_t sb = sa + A_BYTES;
+                const uint32_t ssfa = sb + B_BYTES;
+                const uint32_t ssfb = ssfa + SFA_BYTES;
+                const uint32_t tsfa = tmem + SF_COL0 + s * SF_STAGE_COLS;
+                const uint32_t tsfb = tsfa + 16;
+                for (int a = 0; a < KA; a++) {
+                    tc_cp_scale_atom(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
+                    tc_cp_scale_atom(tsfb + 8 * a, smem_desc(ssfb + 512 * a, 0, 128, 0));
+                    tc_cp_scale_atom(tsfb + 8 * a + 4, smem_desc(ssfb + KA * 512 + 512 * a, 0, 128, 0));
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; kk++) {
+                    // K step of 64 fp4 = 32 bytes inside the 128-byte swizzled row
+                    const uint64_t ad = smem_desc(sa + 32 * kk, 16, 1024, 2);
+                    const uint64_t bd = smem_desc(sb + 32 * kk, 16, 1024, 2);
+                    const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
+                    const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
+                    const uint32_t idesc = idesc_blockscaled(BM, BN, FMT == FP4_MXFP4, sfid, sfid);
+                    tc_mma_blockscaled<FMT>(acc, ad, bd, idesc, (tsfa + 4 * atom) | (sfid << 30),
+                                            (tsfb + 8 * atom) | (sfid << 30), (ks | kk) ? 1u : 0u);
+                }
+                tc_commit(empty0 + 8 * s);
+            }
+            // arrives once every MMA issued above has completed (also on abort)
+            tc_commit(accb);
+        }
+        __syncwarp();
+    }
+
+    // ---------------- epilogue (all four warps) ----------------
+    {
+        volatile uint32_t no_abort = 0;
+        bool ok = mbar_wait_bounded(accb, 0, &no_abort, &g_gemm_error) && !*abort_flag;
+        ok = __all_sync(0xFFFFFFFFu, ok);  // tcgen05.ld below is warp-collective
+        tc_fence_after();
+        if (ok) {
+            const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
+            const int m = mt * BM + warp * 32 + lane;
+            const uint32_t lane_base = tmem + ACC_COL + ((uint32_t)(warp * 32) << 16);
+            const bool vec_ok = BF16OUT ? (p.ldc % 8 == 0) : (p.ldc % 4 == 0);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; c++) {
+                uint32_t r[32];
+                __syncwarp();
+                tmem_ld32(lane_base + c * 32, r);
+                tmem_ld_wait();
+                const int n0 = nt * BN + c * 32;
+                if (m >= p.M || n0 >= p.N) continue;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; i++) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+                const bool full = vec_ok && (n0 + 32 <= p.N);
+                if (BF16OUT) {
+                    __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(p.C) + (int64_t)m * p.ldc + n0;
+                    if (full) {
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int i = 0; i < 4; i++) {
+                                __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * i], v[8 * q + 2 * i + 1]);
+                                w[i] = *reinterpret_cast<uint32_t *>(&h);
+                            }
+                            reinterpret_cast<uint4 *>(row)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    } else {
+                        for (int i = 0; i < 32 && n0 + i < p.N; i++) row[i] = __float2bfloat16_rn(v[i]);
+                    }
+                } else {
+                    float *row = reinterpret_cast<float *>(p.C) + (int64_t)m * p.ldc + n0;
+                    if (full) {
+#pragma unroll
+                        for (int q = 0; q < 8; q++)
+                            reinterpret_cast<float4 *>(row)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    } else {
+                        for (int i = 0; i < 32 && n0 + i < p.N; i++) row[i] = v[i];
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace tiled
+
+// ---------------------------------------------------------------------------
+// Host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// Row-major packed fp4 matrix (rows x K/2 bytes) as a 2-D byte tensor, boxes
+// of 128 bytes x box_rows rows with 128-byte swizzle; out-of-range rows read 0.
+static bool make_fp4_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int FMT, int BF>
+static cudaError_t launch_tiled(const CUtensorMap &ta, const CUtensorMap &tb, const tiled::Params &p, cudaStream_t st)
+{
+    auto kern = tiled::gemm_kernel<FMT, BF>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tiled::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid((p.M + tiled::BM - 1) / tiled::BM, (p.N + tiled::BN - 1) / tiled::BN);
+    count_launches(1);
+    kern<<<grid, 128, tiled::SMEM_BYTES, st>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
 size_t gemm_workspace_bytes(int64_t, int64_t, int64_t, int, int) { return 0; }
 
-cudaError_t launch_gemm(const uint8_t *, const uint8_t *, const float *, const uint8_t *,
-                        const uint8_t *, const float *, int64_t, int64_t, int64_t, int, int,
-                        void *, int64_t, void *, size_t, int, cudaStream_t, int *bad)
+cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
+                        const float *gW, int64_t M, int64_t N, int64_t K, int fmt, int bf16out, void *C, int64_t ldc,
+                        void *, size_t, int, cudaStream_t st, int *bad)
 {
-    *bad = 1;
-    return cudaSuccess;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) {
+        *bad = 1;
+        return cudaSuccess;
+    }
+    CUtensorMap ta, tb;
+    if (!make_fp4_map(&ta, Aq, M, K, tiled::BM) || !make_fp4_map(&tb, Wq, N, K, tiled::BN)) return cudaErrorInvalidValue;
+    tiled::Params p;
+    p.As = As;
+    p.Ws = Ws;
+    p.gA = gA;
+    p.gW = gW;
+    p.C = C;
+    p.ldc = ldc;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+    p.nrb_w = (int)((N + 127) / 128);
+    if (fmt == FP4_MXFP4)
+        return bf16out ? launch_tiled<FP4_MXFP4, 1>(ta, tb, p, st) : launch_tiled<FP4_MXFP4, 0>(ta, tb, p, st);
+    return bf16out ? launch_tiled<FP4_NVFP4, 1>(ta, tb, p, st) : launch_tiled<FP4_NVFP4, 0>(ta, tb, p, st);
 }
 
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err)

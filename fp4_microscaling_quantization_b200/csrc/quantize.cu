@@ -35,15 +35,27 @@ struct QuantArgs {
     int gscale_computed;    // NVFP4: *gscale holds amax bits (set by the amax pass)
 };
 
-// Load one 32-element unit as fp32.
-FP4_DEV void load_unit(const uint16_t *x, int64_t ld, int64_t upr, int64_t u, float *v)
+// Units processed per thread and loop trip: their loads are all issued
+// before any is consumed, so each thread keeps UNITS x 64 bytes in flight.
+constexpr int QUNITS = 2;  // quantize / amax
+constexpr int DUNITS = 4;  // dequantize (16 bytes of nibbles per unit)
+
+// Raw bytes of one 32-element unit (4 x 16-byte loads, read-only path).
+FP4_DEV void fetch_unit(const uint16_t *x, int64_t ld, int64_t upr, int64_t u, uint4 *w)
 {
-    int64_t row = u / upr;
-    int64_t j = u - row * upr;
+    const int64_t row = u / upr;
+    const int64_t j = u - row * upr;
     const uint4 *p = reinterpret_cast<const uint4 *>(x + row * ld + j * 32);
 #pragma unroll
+    for (int c = 0; c < 4; c++) w[c] = __ldg(p + c);
+}
+
+// bf16 pairs -> 32 fp32 values.
+FP4_DEV void unpack_unit(const uint4 *raw, float *v)
+{
+#pragma unroll
     for (int c = 0; c < 4; c++) {
-        uint4 w = __ldg(p + c);
+        const uint4 w = raw[c];
         v[8 * c + 0] = bf16lo(w.x);
         v[8 * c + 1] = bf16hi(w.x);
         v[8 * c + 2] = bf16lo(w.y);
@@ -106,18 +118,26 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     float m = 0.0f;
-    for (int64_t base = warp * 32; base < a.total_units; base += nwarps * 32) {
-        const int64_t u = base + lane;
-        float v[32];
-        if (u < a.total_units) {
-            load_unit(a.x, a.ld, a.units_per_row, u, v);
-        } else {
+    for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
+        uint4 raw[QUNITS][4];
 #pragma unroll
-            for (int j = 0; j < 32; j++) v[j] = 0.0f;
+        for (int i = 0; i < QUNITS; i++) {
+            const int64_t u = base + i * 32 + lane;
+            if (u < a.total_units) {
+                fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
+            }
         }
-        if (HK) fwht_unit<HK>(v, a.ck, lane);
 #pragma unroll
-        for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+        for (int i = 0; i < QUNITS; i++) {
+            float v[32];
+            unpack_unit(raw[i], v);
+            if (HK) fwht_unit<HK>(v, a.ck, lane);
+#pragma unroll
+            for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+        }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -152,60 +172,69 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
         six_sg = __fmul_rn(6.0f, sg);
     }
 
-    for (int64_t base = warp * 32; base < a.total_units; base += nwarps * 32) {
-        const int64_t u = base + lane;
-        const bool live = u < a.total_units;
-        float v[32];
-        if (live) {
-            load_unit(a.x, a.ld, a.units_per_row, u, v);
-        } else {
+    for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
+        uint4 raw[QUNITS][4];
 #pragma unroll
-            for (int j = 0; j < 32; j++) v[j] = 0.0f;
+        for (int i = 0; i < QUNITS; i++) {
+            const int64_t u = base + i * 32 + lane;
+            if (u < a.total_units) {
+                fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
+            }
         }
-        if (HK) fwht_unit<HK>(v, a.ck, lane);
-        if (!live) continue;
+#pragma unroll
+        for (int i = 0; i < QUNITS; i++) {
+            const int64_t u = base + i * 32 + lane;
+            const bool live = u < a.total_units;
+            float v[32];
+            unpack_unit(raw[i], v);
+            if (HK) fwht_unit<HK>(v, a.ck, lane);
+            if (!live) continue;
 
-        const int64_t row = u / a.units_per_row;
-        const int64_t j = u - row * a.units_per_row;
-        if (FMT == FP4_MXFP4) {
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
-            const int e = mx_exponent(amax, a.mx_floor);
-            const float inv = exp2i(-e);
-#pragma unroll
-            for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
-            a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)(e + 127);
-        } else {
-            uint32_t sb2 = 0;
-#pragma unroll
-            for (int b = 0; b < 2; b++) {
+            const int64_t row = u / a.units_per_row;
+            const int64_t j = u - row * a.units_per_row;
+            if (FMT == FP4_MXFP4) {
                 float amax = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[16 * b + i]));
-                const float t = __fdiv_rn(amax, six_sg);
-                const uint32_t sb = e4m3_rn(t);
-                const float d = __fmul_rn(sg, e4m3_to_f32(sb));
-                const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
+                for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+                const int e = mx_exponent(amax, a.mx_floor);
+                const float inv = exp2i(-e);
 #pragma unroll
-                for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
-                sb2 |= sb << (8 * b);
+                for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
+                a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)(e + 127);
+            } else {
+                uint32_t sb2 = 0;
+#pragma unroll
+                for (int b = 0; b < 2; b++) {
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[16 * b + i]));
+                    const float t = __fdiv_rn(amax, six_sg);
+                    const uint32_t sb = e4m3_rn(t);
+                    const float d = __fmul_rn(sg, e4m3_to_f32(sb));
+                    const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
+#pragma unroll
+                    for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
+                    sb2 |= sb << (8 * b);
+                }
+                *reinterpret_cast<uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4)) = (uint16_t)sb2;
             }
-            *reinterpret_cast<uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4)) = (uint16_t)sb2;
+            uint4 out;
+            if (!a.round_away) {
+                out.x = e2m1x8_rn(v + 0);
+                out.y = e2m1x8_rn(v + 8);
+                out.z = e2m1x8_rn(v + 16);
+                out.w = e2m1x8_rn(v + 24);
+            } else {
+                out.x = e2m1x8_away(v + 0);
+                out.y = e2m1x8_away(v + 8);
+                out.z = e2m1x8_away(v + 16);
+                out.w = e2m1x8_away(v + 24);
+            }
+            *reinterpret_cast<uint4 *>(a.q + row * a.q_row_bytes + j * 16) = out;
         }
-        uint4 out;
-        if (!a.round_away) {
-            out.x = e2m1x8_rn(v + 0);
-            out.y = e2m1x8_rn(v + 8);
-            out.z = e2m1x8_rn(v + 16);
-            out.w = e2m1x8_rn(v + 24);
-        } else {
-            out.x = e2m1x8_away(v + 0);
-            out.y = e2m1x8_away(v + 8);
-            out.z = e2m1x8_away(v + 16);
-            out.w = e2m1x8_away(v + 24);
-        }
-        *reinterpret_cast<uint4 *>(a.q + row * a.q_row_bytes + j * 16) = out;
     }
 }
 
@@ -254,67 +283,86 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const float sg = (FMT == FP4_NVFP4) ? *a.gscale : 1.0f;
 
-    for (int64_t base = warp * 32; base < a.total_units; base += nwarps * 32) {
-        const int64_t u = base + lane;
-        const bool live = u < a.total_units;
-        float v[32];
-        int64_t row = 0, j = 0;
-        if (live) {
-            row = u / a.units_per_row;
-            j = u - row * a.units_per_row;
-            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.q + row * a.q_row_bytes + j * 16));
-            const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-            float d0, d1;
-            if (FMT == FP4_MXFP4) {
-                const uint32_t sb = a.s[scale_offset(row, j, a.nkb4)];
-                d0 = d1 = (sb == 0xFF) ? __uint_as_float(0x7FC00000u) : exp2i((int)sb - 127);
-            } else {
-                const uint16_t sb2 = *reinterpret_cast<const uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4));
-                d0 = __fmul_rn(sg, e4m3_to_f32(sb2 & 0xFF));
-                d1 = __fmul_rn(sg, e4m3_to_f32(sb2 >> 8));
+    for (int64_t base = warp * 32 * DUNITS; base < a.total_units; base += nwarps * 32 * DUNITS) {
+        uint4 raw[DUNITS];
+        uint32_t sraw[DUNITS];
+#pragma unroll
+        for (int i = 0; i < DUNITS; i++) {
+            const int64_t u = base + i * 32 + lane;
+            raw[i] = make_uint4(0, 0, 0, 0);
+            sraw[i] = 0;
+            if (u < a.total_units) {
+                const int64_t row = u / a.units_per_row;
+                const int64_t j = u - row * a.units_per_row;
+                raw[i] = __ldg(reinterpret_cast<const uint4 *>(a.q + row * a.q_row_bytes + j * 16));
+                sraw[i] = (FMT == FP4_MXFP4)
+                              ? (uint32_t)__ldg(a.s + scale_offset(row, j, a.nkb4))
+                              : (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(a.s + scale_offset(row, 2 * j, a.nkb4)));
             }
-#pragma unroll
-            for (int c = 0; c < 4; c++) {
-#pragma unroll
-                for (int b = 0; b < 4; b++) {
-                    float lo, hi;
-                    e2m1x2_to_f32((words[c] >> (8 * b)) & 0xFF, lo, hi);
-                    const float d = (c < 2) ? d0 : d1;
-                    v[8 * c + 2 * b] = __fmul_rn(d, lo);
-                    v[8 * c + 2 * b + 1] = __fmul_rn(d, hi);
-                }
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; i++) v[i] = 0.0f;
         }
-        if (HK) fwht_unit<HK>(v, a.ck, lane);
-        if (!live) continue;
-        if (BF16OUT) {
-            uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(a.out) + row * a.cols + j * 32);
 #pragma unroll
-            for (int c = 0; c < 4; c++) {
-                uint32_t w[4];
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * c + 2 * i], v[8 * c + 2 * i + 1]);
-                    w[i] = *reinterpret_cast<uint32_t *>(&p);
+        for (int i = 0; i < DUNITS; i++) {
+            const int64_t u = base + i * 32 + lane;
+            const bool live = u < a.total_units;
+            float v[32];
+            int64_t row = 0, j = 0;
+            if (live) {
+                row = u / a.units_per_row;
+                j = u - row * a.units_per_row;
+                const uint4 w = raw[i];
+                const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+                float d0, d1;
+                if (FMT == FP4_MXFP4) {
+                    const uint32_t sb = sraw[i];
+                    d0 = d1 = (sb == 0xFF) ? __uint_as_float(0x7FC00000u) : exp2i((int)sb - 127);
+                } else {
+                    const uint32_t sb2 = sraw[i];
+                    d0 = __fmul_rn(sg, e4m3_to_f32(sb2 & 0xFF));
+                    d1 = __fmul_rn(sg, e4m3_to_f32(sb2 >> 8));
                 }
-                o[c] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-        } else {
-            float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + row * a.cols + j * 32);
 #pragma unroll
-            for (int c = 0; c < 8; c++) o[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                for (int c = 0; c < 4; c++) {
+#pragma unroll
+                    for (int b = 0; b < 4; b++) {
+                        float lo, hi;
+                        e2m1x2_to_f32((words[c] >> (8 * b)) & 0xFF, lo, hi);
+                        const float d = (c < 2) ? d0 : d1;
+                        v[8 * c + 2 * b] = __fmul_rn(d, lo);
+                        v[8 * c + 2 * b + 1] = __fmul_rn(d, hi);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; i++) v[i] = 0.0f;
+            }
+            if (HK) fwht_unit<HK>(v, a.ck, lane);
+            if (!live) continue;
+            if (BF16OUT) {
+                uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(a.out) + row * a.cols + j * 32);
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * c + 2 * i], v[8 * c + 2 * i + 1]);
+                        w[i] = *reinterpret_cast<uint32_t *>(&p);
+                    }
+                    o[c] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            } else {
+                float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + row * a.cols + j * 32);
+#pragma unroll
+                for (int c = 0; c < 8; c++) o[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
         }
     }
 }
 
 // ---------------------------------------------------------------------------
 // Host launchers (called from capi.cu after validation).
-static int grid_for(int64_t total_units, int sms)
+static int grid_for(int64_t total_units, int sms, int units_per_thread)
 {
-    const int64_t warps = (total_units + 31) / 32;
+    const int64_t warps = (total_units + 32 * units_per_thread - 1) / (32 * units_per_thread);
     const int64_t blocks = (warps + 7) / 8;  // 8 warps per 256-thread block
     const int64_t cap = (int64_t)sms * 8;
     return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
@@ -368,7 +416,7 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     a.round_away = round_away;
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
-    const int grid = grid_for(a.total_units, sms);
+    const int grid = grid_for(a.total_units, sms, QUNITS);
     cudaError_t err = cudaSuccess;
     if (a.gscale_computed) {
         if ((err = cudaMemsetAsync(gscale, 0, sizeof(float), st)) != cudaSuccess) return err;
@@ -428,7 +476,7 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
     a.out = out;
     a.ck = ck;
     if (a.total_units == 0) return cudaSuccess;
-    const int grid = grid_for(a.total_units, sms);
+    const int grid = grid_for(a.total_units, sms, DUNITS);
     if (fmt == FP4_MXFP4)
         return bf16out ? launch_deq_fmt<FP4_MXFP4, 1>(a, hk, grid, st) : launch_deq_fmt<FP4_MXFP4, 0>(a, hk, grid, st);
     return bf16out ? launch_deq_fmt<FP4_NVFP4, 1>(a, hk, grid, st) : launch_deq_fmt<FP4_NVFP4, 0>(a, hk, grid, st);

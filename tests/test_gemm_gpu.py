@@ -1,0 +1,215 @@
+"""GPU parity of fp4_gemm against the oracle's fp64 product of the
+dequantized operands.
+
+Acceptance per element: |C - C_ref| <= 1e-5 * sum_k |a_k||w_k| for FP32
+output; BF16 output adds half a bf16 ulp, 2^-8 |C_ref|.  With unit scales
+every product is a multiple of 1/4 and every partial sum is exact in FP32, so
+C must then be bit-exact.
+"""
+import numpy as np
+import pytest
+
+from fp4_microscaling_quantization_b200 import inputs
+
+from helpers import to_dev_bf16, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp4():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fp4_microscaling_quantization_b200 import build
+    build.build()
+    import fp4_microscaling_quantization_b200 as m
+    return m
+
+
+def upload(orc, q, s_logical, g):
+    import torch
+    qd = torch.from_numpy(np.ascontiguousarray(q)).cuda()
+    sd = torch.from_numpy(orc.scales_to_atoms(s_logical)).cuda()
+    gd = torch.tensor([g], dtype=torch.float32, device="cuda")
+    return qd, sd, gd
+
+
+def run_gemm(fp4, orc, qa, sa, ga, qw, sw, gw, fmt, out_dtype, ldc=None):
+    import torch
+    M, K = qa.shape[0], qa.shape[1] * 2
+    N = qw.shape[0]
+    a = upload(orc, qa, sa, ga)
+    w = upload(orc, qw, sw, gw)
+    dt = torch.float32 if out_dtype == 0 else torch.bfloat16
+    if ldc is None:
+        out = None
+    else:
+        out = torch.full((M, ldc), float("nan"), dtype=dt, device="cuda")[:, :N]
+    c = fp4.gemm(a, w, M, N, K, fmt, out_dtype=out_dtype, out=out)
+    torch.cuda.synchronize()
+    fp4.check_device_status()
+    if ldc is not None:
+        full = out.base if out.base is not None else out
+        pad = full.reshape(M, ldc)[:, N:]
+        assert torch.isnan(pad.float()).all(), "GEMM wrote outside the N columns"
+    return to_np(c.float())
+
+
+def reference(orc, qa, sa, ga, qw, sw, gw, fmt):
+    ah = orc.dequantize(qa, sa, ga, fmt)
+    wh = orc.dequantize(qw, sw, gw, fmt)
+    return orc.gemm_ref(ah, wh)
+
+
+def assert_close(c, ref, bound, out_dtype):
+    tol = 1e-5 * bound + (2.0 ** -8 * np.abs(ref) if out_dtype == 1 else 0.0)
+    err = np.abs(c.astype(np.float64) - ref)
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, (f"{bad.shape[0]} elements out of tolerance, first {bad[:3].tolist()}: "
+                           f"got {c[tuple(bad[0])]} want {ref[tuple(bad[0])]} tol {tol[tuple(bad[0])]}")
+
+
+def rand_q(rng, rows, K):
+    return rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+
+
+def unit_scales(fmt, rows, K):
+    block = 32 if fmt == 0 else 16
+    return np.full((rows, K // block), 127 if fmt == 0 else 0x38, np.uint8)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("shape", [(128, 256, 256), (128, 256, 1024), (256, 512, 512), (130, 300, 512)])
+def test_unit_scale_exact(fp4, orc, fmt, shape):
+    M, N, K = shape
+    rng = np.random.default_rng(M + N + K + fmt)
+    qa, qw = rand_q(rng, M, K), rand_q(rng, N, K)
+    sa, sw = unit_scales(fmt, M, K), unit_scales(fmt, N, K)
+    c = run_gemm(fp4, orc, qa, sa, 1.0, qw, sw, 1.0, fmt, 0)
+    ref, _ = reference(orc, qa, sa, 1.0, qw, sw, 1.0, fmt)
+    assert np.array_equal(c.astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_impulses_pin_operand_and_scale_layout(fp4, orc, fmt):
+    """One nonzero element in A and W and one distinct scale per block: C
+    lights exactly one entry, with the product of the two scales."""
+    M, N, K = 256, 512, 512
+    block = 32 if fmt == 0 else 16
+    rng = np.random.default_rng(fmt)
+    for trial in range(6):
+        m, n, k = int(rng.integers(M)), int(rng.integers(N)), int(rng.integers(K))
+        qa = np.zeros((M, K // 2), np.uint8)
+        qw = np.zeros((N, K // 2), np.uint8)
+        qa[m, k // 2] = (3 if k % 2 == 0 else 3 << 4)          # 1.5
+        qw[n, k // 2] = (0xD if k % 2 == 0 else 0xD << 4)      # -3
+        if fmt == 0:
+            sa = rng.integers(120, 135, (M, K // block)).astype(np.uint8)
+            sw = rng.integers(120, 135, (N, K // block)).astype(np.uint8)
+        else:
+            sa = rng.integers(0x20, 0x60, (M, K // block)).astype(np.uint8)
+            sw = rng.integers(0x20, 0x60, (N, K // block)).astype(np.uint8)
+        c = run_gemm(fp4, orc, qa, sa, 1.0, qw, sw, 1.0, fmt, 0)
+        ref, _ = reference(orc, qa, sa, 1.0, qw, sw, 1.0, fmt)
+        nz = np.argwhere(c != 0)
+        assert nz.tolist() == [[m, n]], (trial, nz[:4].tolist(), (m, n, k))
+        assert c[m, n] == ref[m, n]
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("out_dtype", [0, 1])
+@pytest.mark.parametrize("shape", [(128, 256, 512), (200, 520, 1024), (1, 8, 256), (16, 4096, 512), (300, 256, 2048)])
+def test_random_scales_within_tolerance(fp4, orc, fmt, out_dtype, shape):
+    M, N, K = shape
+    rng = np.random.default_rng(M * 3 + N + K)
+    va = rng.laplace(0, 1, (M, K)).astype(np.float32)
+    va[rng.random((M, K)) < 0.01] *= 20
+    vw = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
+    qa, sa, ga = orc.quantize(inputs.f32_to_bf16_bits(va), fmt)
+    qw, sw, gw = orc.quantize(inputs.f32_to_bf16_bits(vw), fmt)
+    c = run_gemm(fp4, orc, qa, sa, ga, qw, sw, gw, fmt, out_dtype)
+    ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, fmt)
+    assert_close(c, ref, bound, out_dtype)
+
+
+def test_tiny_linear_workload(fp4, orc):
+    """MXFP4 W4A4 linear, tiny: A 128x512, W 256x512, full brute force."""
+    a, w = inputs.tiny_linear()
+    qa, sa, ga = orc.quantize(a, 0)
+    qw, sw, gw = orc.quantize(w, 0)
+    for out_dtype in (0, 1):
+        c = run_gemm(fp4, orc, qa, sa, ga, qw, sw, gw, 0, out_dtype)
+        ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, 0)
+        assert_close(c, ref, bound, out_dtype)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_strided_output(fp4, orc, fmt):
+    M, N, K = 130, 264, 512
+    rng = np.random.default_rng(5)
+    qa, sa, ga = orc.quantize(inputs.f32_to_bf16_bits(rng.laplace(0, 1, (M, K)).astype(np.float32)), fmt)
+    qw, sw, gw = orc.quantize(inputs.f32_to_bf16_bits(rng.laplace(0, 1, (N, K)).astype(np.float32)), fmt)
+    ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, fmt)
+    for out_dtype, ldc in ((0, 300), (1, 304), (1, 270)):
+        c = run_gemm(fp4, orc, qa, sa, ga, qw, sw, gw, fmt, out_dtype, ldc=ldc)
+        assert_close(c, ref, bound, out_dtype)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_rotated_operands_preserve_product(fp4, orc, fmt):
+    """(X H)(W H)^T = X W^T: quantizing both operands with the same H_k gives
+    the product of the unrotated tensors up to quantization error."""
+    import torch
+    M, N, K = 128, 256, 1024
+    a = inputs.rotate_acts(rows=M, cols=K, seed=8)
+    rng = np.random.default_rng(9)
+    w = inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (N, K)).astype(np.float32))
+    exact = inputs.bf16_bits_to_f32(a).astype(np.float64) @ inputs.bf16_bits_to_f32(w).astype(np.float64).T
+    errs = {}
+    for hk in (0, 128):
+        A = fp4.quantize(to_dev_bf16(a), fmt, hadamard_k=hk)
+        W = fp4.quantize(to_dev_bf16(w), fmt, hadamard_k=hk)
+        c = to_np(fp4.gemm(A, W, M, N, K, fmt, out_dtype=0)).astype(np.float64)
+        torch.cuda.synchronize()
+        # the GEMM over the rotated operands equals the oracle product of their dequantized values
+        qa, sa, ga = orc.quantize(a, fmt, hadamard_k=hk)
+        qw, sw, gw = orc.quantize(w, fmt, hadamard_k=hk)
+        ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, fmt)
+        assert_close(c, ref, bound, 0)
+        errs[hk] = np.linalg.norm(c - exact) / np.linalg.norm(exact)
+    assert errs[128] < 0.25 and errs[0] < 0.5
+    assert errs[128] < errs[0]  # the rotation spreads the outlier channels
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_full_size_prefill_sampled(fp4, orc, fmt):
+    """8192 x 8192 activations times a 28672 x 8192 weight (70B MLP shape), in
+    the benchmark's launch configuration; 64 x 64 sampled outputs against the
+    oracle's fp64 product of the same quantized bytes."""
+    import torch
+    M, N, K = 8192, 28672, 8192
+    a, w = inputs.prefill_linear()
+    A = fp4.quantize(to_dev_bf16(a), fmt)
+    W = fp4.quantize(to_dev_bf16(w), fmt)
+    del a
+    c = fp4.gemm(A, W, M, N, K, fmt, out_dtype=1)
+    torch.cuda.synchronize()
+    fp4.check_device_status()
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(M, 64, replace=False))
+    cols = np.sort(rng.choice(N, 64, replace=False))
+    block = 32 if fmt == 0 else 16
+    nkb = K // block
+
+    def deq(T, idx, nrows):
+        q = to_np(T[0])[idx]
+        s_log = orc.scales_from_atoms(to_np(T[1]), nrows, nkb)[idx]
+        return orc.dequantize(q, s_log, float(to_np(T[2])[0]), fmt)
+
+    ah, wh = deq(A, rows, M), deq(W, cols, N)
+    ref, bound = orc.gemm_ref(ah, wh)
+    got = to_np(c.float())[np.ix_(rows, cols)]
+    assert_close(got, ref, bound, 1)
+    del c, A, W
+    torch.cuda.empty_cache()
