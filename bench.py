@@ -85,10 +85,48 @@ def time_graph(torch, fn, warmup: int, reps: int):
     return e0.elapsed_time(e1) / reps
 
 
-def bench_prefill(torch, fp4, inputs, dev, reps: int):
+def bench_decode(torch, fp4, inputs, dev, reps: int):
+    """Decode shapes: M in {1,4,16} bf16 activations quantized online inside
+    the timed call (fp4_linear), W 14336x4096 and 4096x14336 pre-quantized,
+    BF16 out.  W copies are rotated so the weight stream comes from HBM."""
+    hbm, kind = peaks()
+    res = {"peak_gbs": hbm, "peak_kind": kind, "copies": 0, "cases": {}}
+    for (N, K) in ((14336, 4096), (4096, 14336)):
+        _, w = inputs.decode_linear(1, N, K)
+        wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
+        del w
+        for fmt, name in ((fp4.FP4_NVFP4, "nvfp4"), (fp4.FP4_MXFP4, "mxfp4")):
+            W0 = fp4.quantize(wd, fmt)
+            wbytes = W0[0].numel() + W0[1].numel()
+            copies = max(2, int(2 * 126e6 // wbytes) + 1)
+            Ws = [tuple(t.clone() for t in W0) for _ in range(copies)]
+            res["copies"] = copies
+            for M in (1, 4, 16):
+                a, _ = inputs.decode_linear(M, 8, K)
+                x = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+                C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                ws = torch.empty((fp4.linear_workspace_size(M, N, K, fmt),), dtype=torch.uint8, device=dev)
+                it = [0]
+
+                def call():
+                    W = Ws[it[0] % copies]
+                    it[0] += 1
+                    fp4.linear(x, W, fmt, out=C, workspace=ws)
+
+                ms = time_graph(torch, call, 3, reps * copies)
+                b = wbytes + M * K * 2 + M * N * 2
+                res["cases"][f"{name}_M{M}_N{N}_K{K}"] = {"us": ms * 1e3, "gbs": b / (ms * 1e-3) / 1e9,
+                                                          "frac": b / (ms * 1e-3) / 1e9 / hbm}
+            del Ws, W0
+        del wd
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_prefill(torch, fp4, inputs, dev, reps: int, M: int = 8192, fmts=None):
     """W4A4 prefill GEMM, 70B-MLP shape: A 8192x8192, W 28672x8192, BF16 out."""
-    M, N, K = 8192, 28672, 8192
-    a, w = inputs.prefill_linear()
+    N, K = 28672, 8192
+    a, w = inputs.prefill_linear(m=M)
     ad = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
     wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
     del a, w
@@ -96,6 +134,8 @@ def bench_prefill(torch, fp4, inputs, dev, reps: int):
     out = {"workload": f"prefill W4A4 linear M={M} N={N} K={K}, BF16 out", "peak_tflops": peak, "peak_kind": kind}
     C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     for fmt, name in ((fp4.FP4_NVFP4, "nvfp4"), (fp4.FP4_MXFP4, "mxfp4")):
+        if fmts is not None and name not in fmts:
+            continue
         A = fp4.quantize(ad, fmt)
         W = fp4.quantize(wd, fmt)
         ms = time_graph(torch, lambda: fp4.gemm(A, W, M, N, K, fmt, out=C), 3, reps)
@@ -247,6 +287,15 @@ def run_ours(args):
     import fp4_microscaling_quantization_b200 as fp4
     from fp4_microscaling_quantization_b200 import _lib, inputs
 
+    if args.only:
+        # profiling helper: one leg alone, no JSON contract
+        if args.only == "prefill":
+            r = bench_prefill(torch, fp4, inputs, dev, reps=args.steps, M=args.prefill_m, fmts=args.fmts)
+        else:
+            r = bench_decode(torch, fp4, inputs, dev, reps=args.steps)
+        print(json.dumps({"only": args.only, "result": r}), flush=True)
+        return 0
+
     x_np = inputs.quant_sweep(rows=args.rows, seed=2 + rank)
     x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     x = x_host.to(dev)
@@ -368,7 +417,8 @@ def run_ours(args):
 
     gemm = None
     if not args.no_gemm:
-        gemm = {"prefill": bench_prefill(torch, fp4, inputs, dev, reps=10)}
+        gemm = {"prefill": bench_prefill(torch, fp4, inputs, dev, reps=10),
+                "decode": bench_decode(torch, fp4, inputs, dev, reps=10)}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -413,6 +463,10 @@ def main():
     ap.add_argument("--rows", type=int, default=ROWS, help="rows of the tensor (profiling runs use fewer)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gemm", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="profiling helper: run one GEMM leg alone")
+    ap.add_argument("--prefill-m", type=int, default=8192)
+    ap.add_argument("--fmts", nargs="*", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

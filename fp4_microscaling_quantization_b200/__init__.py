@@ -14,7 +14,7 @@ from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_NVFP4, 
                    FP4_OUT_F32, FP4_ROUND_AWAY, FP4_ROUND_EVEN, Fp4Error)
 
 __all__ = [
-    "quantize", "dequantize", "gemm", "quantize_sizes", "gemm_workspace_size", "check_device_status",
+    "quantize", "dequantize", "gemm", "linear", "linear_workspace_size", "quantize_sizes", "gemm_workspace_size", "check_device_status",
     "FP4_MXFP4", "FP4_NVFP4", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
     "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "Fp4Error", "block_of",
 ]
@@ -120,6 +120,39 @@ def gemm(a, w, M: int, N: int, K: int, fmt, out_dtype: int = FP4_OUT_BF16, out=N
         Aq.data_ptr(), As.data_ptr(), gA.data_ptr(), Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(),
         M, N, K, fmt, int(out_dtype), out.data_ptr(), out.stride(0), wp, wb,
         _stream_handle(torch, Aq.device)))
+    return out
+
+
+def linear_workspace_size(M: int, N: int, K: int, fmt) -> int:
+    b = ctypes.c_size_t()
+    _lib.check("fp4_linear_workspace_size",
+               _lib.lib().fp4_linear_workspace_size(M, N, K, _fmt(fmt), ctypes.byref(b)))
+    return b.value
+
+
+def linear(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale=None,
+           round: int = FP4_ROUND_EVEN, mx_scale_rule: int = FP4_MX_SCALE_CEIL, out=None, workspace=None):
+    """W4A4 linear from bf16 activations x (M x K) and a pre-quantized weight
+    w = (Wq, Ws, gW) (N x K): quantizes x online, returns C = x W^T."""
+    import torch
+
+    fmt = _fmt(fmt)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor, contiguous along K")
+    Wq, Ws, gW = w
+    M, K = x.shape
+    N = Wq.shape[0]
+    dt = torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, N), dtype=dt, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((linear_workspace_size(M, N, K, fmt),), dtype=torch.uint8, device=x.device)
+    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), 0)
+    _lib.check("fp4_linear", _lib.lib().fp4_linear(
+        x.data_ptr(), M, K, x.stride(0), fmt, int(hadamard_k), ctypes.byref(opts),
+        gscale.data_ptr() if gscale is not None else None, Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(), N,
+        int(out_dtype), out.data_ptr(), out.stride(0), workspace.data_ptr(), workspace.numel(),
+        _stream_handle(torch, x.device)))
     return out
 
 

@@ -153,6 +153,76 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+struct LinearLayout {
+    size_t aq, as, ga, gemm, total;
+};
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int fmt, int sms)
+{
+    LinearLayout L;
+    const int64_t nkb = K / (fmt == FP4_MXFP4 ? 32 : 16);
+    L.aq = 0;
+    L.as = round256((size_t)(M * (K / 2)));
+    L.ga = L.as + round256((size_t)(((M + 127) / 128 * 128) * ((nkb + 3) / 4 * 4)));
+    L.gemm = L.ga + 256;
+    L.total = L.gemm + round256(fp4::gemm_workspace_bytes(M, N, K, fmt, sms));
+    return L;
+}
+}  // namespace
+
+extern "C" {
+
+fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes)
+{
+    if (M < 0 || N < 0 || K < 0 || !bytes) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    *bytes = linear_layout(M, N, K, fmt, sm_count()).total;
+    return FP4_OK;
+}
+
+fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt, int hadamard_k,
+                      const fp4_opts *opts, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
+                      const float *gW, int64_t N, int out_dtype, void *C, int64_t ldc,
+                      void *workspace, size_t ws_bytes, void *stream)
+{
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0};
+    if (opts) o = *opts;
+    if (M < 0 || N < 0 || K < 0 || ld_x < K || ldc < N) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+    if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
+    if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
+    if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (K % 256 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return FP4_OK;
+    if (!x || !Wq || !Ws || !C || !workspace) return FP4_ERR_INVALID_ARG;
+    if (fmt == FP4_NVFP4 && !gW) return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || (ld_x % 8) || !aligned(Wq, 16) || !aligned(Ws, 16) || !aligned(C, 16) ||
+        !aligned(workspace, 256))
+        return FP4_ERR_ALIGNMENT;
+    const int sms = sm_count();
+    const LinearLayout L = linear_layout(M, N, K, fmt, sms);
+    if (ws_bytes < L.total) return FP4_ERR_INVALID_ARG;
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    uint8_t *aq = base + L.aq, *as = base + L.as;
+    float *ga = (fmt == FP4_NVFP4 && gA) ? const_cast<float *>(gA) : reinterpret_cast<float *>(base + L.ga);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = fp4::launch_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
+                                         hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
+                                         o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, sms, st);
+    if (e != cudaSuccess) return FP4_ERR_CUDA;
+    int bad = 0;
+    e = fp4::launch_gemm(aq, as, ga, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc, base + L.gemm,
+                         L.total - L.gemm, sms, st, &bad);
+    if (bad) return FP4_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
 uint64_t fp4_kernel_launches(void) { return fp4::g_launches.load(std::memory_order_relaxed); }
 
 fp4_status fp4_check_device_status(void *stream)

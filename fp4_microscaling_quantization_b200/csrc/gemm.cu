@@ -221,6 +221,256 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
 }  // namespace tiled
 
+
+// ---------------------------------------------------------------------------
+// Decode kernel (M <= 16): the weight stream dominates, so the roles swap: a
+// 128-row W tile is the MMA's M operand and the (up to 16) activation rows
+// are N = 16.  The (W tile, 256-wide K step) units are split evenly over the
+// SMs in tile-major order (stream-K); each CTA accumulates every tile segment
+// it owns in TMEM (two buffers, alternating) and writes the 128 x 16 fp32
+// partial to a workspace slot.  reduce_kernel then sums each output's partials
+// in a fixed CTA order (deterministic) and applies alpha.
+namespace decode {
+
+constexpr int BMW = 128, BNA = 16, BK = 256;
+constexpr int STAGES = 8;
+constexpr int W_BYTES = BMW * BK / 2;        // 16 KB
+constexpr int A_BYTES = BNA * BK / 2;        // 2 KB
+constexpr int SFW_BYTES = 4 * 512;
+constexpr int SFA_BYTES = 4 * 512;
+constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;  // 22528 = 22 KB
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int TMEM_COLS = 512;
+constexpr int SF_COL0 = 32;                  // accumulators at columns [0,16) and [16,32)
+constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation scales 16 cols
+
+struct Params {
+    const uint8_t *Ws;   // W scales (N rows)
+    const uint8_t *As;   // activation scales (M rows, padded to 128)
+    float *ws;           // partials: [G][maxseg][128][16]
+    int N, M, K;
+    int nk;              // K / BK
+    int ntiles;          // ceil(N / 128)
+    int G;               // CTAs
+    int maxseg;
+    int nkb4;
+};
+
+__host__ __device__ inline int64_t unit_begin(int c, int64_t U, int G) { return (int64_t)c * U / G; }
+
+template <int FMT>
+__global__ void __launch_bounds__(192, 1)
+decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, Params p)
+{
+    constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    // bars: full[S], empty[S], accfull[2], accempty[2], drain
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    const int64_t U = (int64_t)p.ntiles * p.nk;
+    const int64_t u0 = unit_begin(c, U, p.G), u1 = unit_begin(c + 1, U, p.G);
+    const int t_first = (int)(u0 / p.nk);
+    const int nseg = (int)((u1 - 1) / p.nk) - t_first + 1;
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+    const uint32_t accf0 = smem_u32(bars + 2 * STAGES), acce0 = smem_u32(bars + 2 * STAGES + 2);
+    const uint32_t drainb = smem_u32(bars + 2 * STAGES + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; s++) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(accf0 + 8 * b, 1);
+            mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
+        }
+        mbar_init(drainb, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmA);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
+            int64_t issued = 0;
+            for (int64_t u = u0; u < u1; u++) {
+                const int64_t i = u - u0;
+                const int s = (int)(i % STAGES);
+                const uint32_t ph = (uint32_t)((i / STAGES) & 1);
+                if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error)) break;
+                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
+                uint8_t *st = smem + s * STAGE_BYTES;
+                const uint32_t fb = full0 + 8 * s;
+                mbar_arrive_expect_tx(fb, tx);
+                tma_load_2d(smem_u32(st), &tmW, ks * (BK / 2), t * BMW, fb);
+                tma_load_2d(smem_u32(st + W_BYTES), &tmA, ks * (BK / 2), 0, fb);
+                bulk_load(smem_u32(st + W_BYTES + A_BYTES), p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+                bulk_load(smem_u32(st + W_BYTES + A_BYTES + SFW_BYTES), p.As + (int64_t)ks * KA * 512, KA * 512, fb);
+                issued = i + 1;
+            }
+            for (int64_t i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++) {
+                volatile uint32_t no_abort = 0;
+                mbar_wait_bounded(full0 + 8 * (int)(i % STAGES), (uint32_t)((i / STAGES) & 1), &no_abort, &g_gemm_error);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int seg = -1;
+            for (int64_t u = u0; u < u1; u++) {
+                const int64_t i = u - u0;
+                const int s = (int)(i % STAGES);
+                const uint32_t ph = (uint32_t)((i / STAGES) & 1);
+                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
+                const bool first = (u == u0) || ks == 0;
+                const bool last = (u == u1 - 1) || ks == p.nk - 1;
+                if (first) {
+                    seg++;
+                    if (seg >= 2 &&
+                        !mbar_wait_bounded(acce0 + 8 * (seg & 1), (uint32_t)(((seg >> 1) - 1) & 1), abort_flag, &g_gemm_error))
+                        break;
+                }
+                if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error)) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)(seg & 1) * BNA;
+                const uint32_t sw = smem_u32(smem + s * STAGE_BYTES);
+                const uint32_t sa = sw + W_BYTES;
+                const uint32_t ssfw = sa + A_BYTES;
+                const uint32_t ssfa = ssfw + SFW_BYTES;
+                const uint32_t tsfw = tmem + SF_COL0 + s * SF_STAGE_COLS;
+                const uint32_t tsfa = tsfw + 16;
+                for (int a = 0; a < KA; a++) {
+                    tc_cp_scale_atom(tsfw + 4 * a, smem_desc(ssfw + 512 * a, 0, 128, 0));
+                    tc_cp_scale_atom(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; kk++) {
+                    const uint64_t wd = smem_desc(sw + 32 * kk, 16, 1024, 2);
+                    const uint64_t ad = smem_desc(sa + 32 * kk, 16, 1024, 2);
+                    const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
+                    const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
+                    const uint32_t idesc = idesc_blockscaled(BMW, BNA, FMT == FP4_MXFP4, sfid, sfid);
+                    tc_mma_blockscaled<FMT>(acc, wd, ad, idesc, (tsfw + 4 * atom) | (sfid << 30),
+                                            (tsfa + 4 * atom) | (sfid << 30), (first && kk == 0) ? 0u : 1u);
+                }
+                tc_commit(empty0 + 8 * s);
+                if (last) tc_commit(accf0 + 8 * (seg & 1));
+            }
+            // arrives once every MMA issued above has completed
+            tc_commit(drainb);
+        }
+        __syncwarp();
+    } else {
+    // ---------------- epilogue warps 2-5: one partial per tile segment ----------------
+    // warp w may only read TMEM lanes 32*(w%4) .. 32*(w%4)+31
+    const int quarter = warp & 3;
+    for (int seg = 0; seg < nseg; seg++) {
+        const int b = seg & 1;
+        bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r[16];
+        tmem_ld16(tmem + (uint32_t)b * BNA + ((uint32_t)(quarter * 32) << 16), r);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");
+        float4 *dst = reinterpret_cast<float4 *>(p.ws + (((int64_t)c * p.maxseg + seg) * 128 + quarter * 32 + lane) * 16);
+#pragma unroll
+        for (int q = 0; q < 4; q++)
+            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                                 __uint_as_float(r[4 * q + 3]));
+    }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        // every MMA has completed before TMEM is released (also on the abort path)
+        volatile uint32_t no_abort = 0;
+        mbar_wait_bounded(drainb, 0, &no_abort, &g_gemm_error);
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// C[m][n] = alpha * sum over the CTAs that own a part of n's tile, in CTA order.
+template <int BF16OUT, int FMT>
+__global__ void __launch_bounds__(128) reduce_kernel(Params p, const float *gA, const float *gW, void *C, int64_t ldc)
+{
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= p.N) return;
+    const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*gA, *gW) : 1.0f;
+    const int t = n / BMW, r = n % BMW;
+    const int64_t U = (int64_t)p.ntiles * p.nk;
+    auto owner = [&](int64_t u) { return (int)(((u + 1) * p.G + U - 1) / U) - 1; };
+    const int c_lo = owner((int64_t)t * p.nk), c_hi = owner((int64_t)(t + 1) * p.nk - 1);
+    float acc[BNA];
+#pragma unroll
+    for (int m = 0; m < BNA; m++) acc[m] = 0.0f;
+    for (int c = c_lo; c <= c_hi; c++) {
+        const int seg = t - (int)(unit_begin(c, U, p.G) / p.nk);
+        const float4 *src = reinterpret_cast<const float4 *>(p.ws + (((int64_t)c * p.maxseg + seg) * 128 + r) * 16);
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const float4 v = src[q];
+            acc[4 * q] = __fadd_rn(acc[4 * q], v.x);
+            acc[4 * q + 1] = __fadd_rn(acc[4 * q + 1], v.y);
+            acc[4 * q + 2] = __fadd_rn(acc[4 * q + 2], v.z);
+            acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < BNA; m++) {
+        if (m >= p.M) break;
+        const float v = __fmul_rn(acc[m], alpha);
+        if (BF16OUT)
+            reinterpret_cast<__nv_bfloat16 *>(C)[(int64_t)m * ldc + n] = __float2bfloat16_rn(v);
+        else
+            reinterpret_cast<float *>(C)[(int64_t)m * ldc + n] = v;
+    }
+}
+
+struct Plan {
+    int G, maxseg, nk, ntiles;
+    size_t ws_bytes;
+};
+
+inline Plan plan(int64_t M, int64_t N, int64_t K, int sms)
+{
+    Plan pl;
+    pl.nk = (int)(K / BK);
+    pl.ntiles = (int)((N + BMW - 1) / BMW);
+    const int64_t U = (int64_t)pl.ntiles * pl.nk;
+    pl.G = (int)(U < sms ? U : sms);
+    pl.maxseg = 1;
+    for (int c = 0; c < pl.G; c++) {
+        const int64_t a = unit_begin(c, U, pl.G), b = unit_begin(c + 1, U, pl.G);
+        const int segs = (int)((b - 1) / pl.nk - a / pl.nk + 1);
+        if (segs > pl.maxseg) pl.maxseg = segs;
+    }
+    pl.ws_bytes = (size_t)pl.G * pl.maxseg * 128 * BNA * sizeof(float);
+    (void)M;
+    return pl;
+}
+
+}  // namespace decode
+
 // ---------------------------------------------------------------------------
 // Host side
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -268,15 +518,67 @@ static cudaError_t launch_tiled(const CUtensorMap &ta, const CUtensorMap &tb, co
     return cudaGetLastError();
 }
 
-size_t gemm_workspace_bytes(int64_t, int64_t, int64_t, int, int) { return 0; }
+constexpr int64_t kDecodeMaxM = 16;
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
+{
+    if (M < 1 || M > kDecodeMaxM || N < 1 || K < decode::BK) return 0;
+    return decode::plan(M, N, K, sms).ws_bytes;
+}
+
+template <int FMT, int BF>
+static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const decode::Params &p, const float *gA,
+                                 const float *gW, void *C, int64_t ldc, cudaStream_t st)
+{
+    auto kern = decode::decode_kernel<FMT>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, decode::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    count_launches(2);
+    kern<<<p.G, 192, decode::SMEM_BYTES, st>>>(tw, ta, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    decode::reduce_kernel<BF, FMT><<<(p.N + 127) / 128, 128, 0, st>>>(p, gA, gW, C, ldc);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
                         const float *gW, int64_t M, int64_t N, int64_t K, int fmt, int bf16out, void *C, int64_t ldc,
-                        void *, size_t, int, cudaStream_t st, int *bad)
+                        void *ws, size_t ws_bytes, int sms, cudaStream_t st, int *bad)
 {
     if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) {
         *bad = 1;
         return cudaSuccess;
+    }
+    if (M <= kDecodeMaxM) {
+        const decode::Plan pl = decode::plan(M, N, K, sms);
+        if (!ws || ws_bytes < pl.ws_bytes) {
+            *bad = 1;
+            return cudaSuccess;
+        }
+        CUtensorMap tw, ta;
+        if (!make_fp4_map(&tw, Wq, N, K, decode::BMW) || !make_fp4_map(&ta, Aq, M, K, decode::BNA))
+            return cudaErrorInvalidValue;
+        decode::Params dp;
+        dp.Ws = Ws;
+        dp.As = As;
+        dp.ws = static_cast<float *>(ws);
+        dp.N = (int)N;
+        dp.M = (int)M;
+        dp.K = (int)K;
+        dp.nk = pl.nk;
+        dp.ntiles = pl.ntiles;
+        dp.G = pl.G;
+        dp.maxseg = pl.maxseg;
+        dp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+        if (fmt == FP4_MXFP4)
+            return bf16out ? launch_decode<FP4_MXFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st)
+                           : launch_decode<FP4_MXFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st);
+        return bf16out ? launch_decode<FP4_NVFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st)
+                       : launch_decode<FP4_NVFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st);
     }
     CUtensorMap ta, tb;
     if (!make_fp4_map(&ta, Aq, M, K, tiled::BM) || !make_fp4_map(&tb, Wq, N, K, tiled::BN)) return cudaErrorInvalidValue;

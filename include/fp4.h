@@ -148,6 +148,30 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA,
                     void *C, int64_t ldc, void *workspace, size_t ws_bytes,
                     void *stream);
 
+/* Bytes of device scratch fp4_linear needs (quantized activations, their
+ * scales and tensor scale, and the GEMM workspace).  Host-only. */
+fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes);
+
+/*
+ * fp4_linear — the W4A4 linear layer from bf16 activations: x (M x K bf16,
+ * row stride ld_x) is quantized online ("4.5 FP8 and NVFP4/MXFP4" §4.2:
+ * online quantization from BF16 needs no calibration data) in the weight's
+ * format, optionally rotated by H_k ("FP4 quantization analysis" §3.2.3:
+ * activations rotated online, weights rotated offline — W must have been
+ * quantized with the same hadamard_k), then C = alpha * x_q W_q^T as in
+ * fp4_gemm.  M <= 16 is the decode case the weight stream dominates.
+ *   gA      NVFP4 activation tensor scale: NULL = computed from x (dynamic),
+ *           else a device fp32 holding a static s_g.  Ignored for MXFP4.
+ *   opts    rounding options for the activation quantization (may be NULL;
+ *           gscale_given is ignored, gA decides).
+ *   workspace  at least fp4_linear_workspace_size() bytes, 256-byte aligned;
+ *           its contents on entry do not matter.
+ */
+fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt, int hadamard_k,
+                      const fp4_opts *opts, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
+                      const float *gW, int64_t N, int out_dtype, void *C, int64_t ldc,
+                      void *workspace, size_t ws_bytes, void *stream);
+
 /* Number of kernels this library has launched in this process so far
  * (host-side counter; diagnostics and launch accounting). */
 uint64_t fp4_kernel_launches(void);

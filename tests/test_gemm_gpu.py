@@ -43,16 +43,15 @@ def run_gemm(fp4, orc, qa, sa, ga, qw, sw, gw, fmt, out_dtype, ldc=None):
     w = upload(orc, qw, sw, gw)
     dt = torch.float32 if out_dtype == 0 else torch.bfloat16
     if ldc is None:
-        out = None
+        out = full = None
     else:
-        out = torch.full((M, ldc), float("nan"), dtype=dt, device="cuda")[:, :N]
+        full = torch.full((M, ldc), float("nan"), dtype=dt, device="cuda")
+        out = full[:, :N]
     c = fp4.gemm(a, w, M, N, K, fmt, out_dtype=out_dtype, out=out)
     torch.cuda.synchronize()
     fp4.check_device_status()
-    if ldc is not None:
-        full = out.base if out.base is not None else out
-        pad = full.reshape(M, ldc)[:, N:]
-        assert torch.isnan(pad.float()).all(), "GEMM wrote outside the N columns"
+    if full is not None:
+        assert torch.isnan(full[:, N:].float()).all(), "GEMM wrote outside the N columns"
     return to_np(c.float())
 
 
@@ -179,7 +178,11 @@ def test_rotated_operands_preserve_product(fp4, orc, fmt):
         assert_close(c, ref, bound, 0)
         errs[hk] = np.linalg.norm(c - exact) / np.linalg.norm(exact)
     assert errs[128] < 0.25 and errs[0] < 0.5
-    assert errs[128] < errs[0]  # the rotation spreads the outlier channels
+    if fmt == 0:
+        # MXFP4: the rotation spreads the outlier channels and lowers the error.
+        # (For NVFP4 the pages report rotation can raise the error a little,
+        # which is what this workload shows too, so no ordering is asserted.)
+        assert errs[128] < errs[0]
 
 
 @pytest.mark.parametrize("fmt", [0, 1])
@@ -213,3 +216,101 @@ def test_full_size_prefill_sampled(fp4, orc, fmt):
     assert_close(got, ref, bound, 1)
     del c, A, W
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ decode ----
+DECODE_SHAPES = [(1, 4096, 512), (4, 1000, 768), (16, 4096, 1024), (3, 40000, 256), (16, 300, 4096), (7, 8, 256)]
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("out_dtype", [0, 1])
+@pytest.mark.parametrize("shape", DECODE_SHAPES)
+def test_decode_within_tolerance(fp4, orc, fmt, out_dtype, shape):
+    """M <= 16 takes the weight-streaming split-K kernel; (3, 40000, 256) gives
+    each CTA three tile segments, (16, 300, 4096) a ragged last tile."""
+    M, N, K = shape
+    rng = np.random.default_rng(M + N + K)
+    qa, sa, ga = orc.quantize(inputs.f32_to_bf16_bits(rng.laplace(0, 1, (M, K)).astype(np.float32)), fmt)
+    qw, sw, gw = orc.quantize(inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (N, K)).astype(np.float32)), fmt)
+    assert fp4.gemm_workspace_size(M, N, K, fmt) > 0
+    c = run_gemm(fp4, orc, qa, sa, ga, qw, sw, gw, fmt, out_dtype)
+    ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, fmt)
+    assert_close(c, ref, bound, out_dtype)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_decode_unit_scale_exact_and_deterministic(fp4, orc, fmt):
+    import torch
+    M, N, K = 16, 2048, 2048
+    rng = np.random.default_rng(3)
+    qa, qw = rand_q(rng, M, K), rand_q(rng, N, K)
+    sa, sw = unit_scales(fmt, M, K), unit_scales(fmt, N, K)
+    c1 = run_gemm(fp4, orc, qa, sa, 1.0, qw, sw, 1.0, fmt, 0)
+    c2 = run_gemm(fp4, orc, qa, sa, 1.0, qw, sw, 1.0, fmt, 0)
+    ref, _ = reference(orc, qa, sa, 1.0, qw, sw, 1.0, fmt)
+    assert np.array_equal(c1.astype(np.float64), ref)
+    assert np.array_equal(c1.view(np.uint32), c2.view(np.uint32))
+
+
+def test_decode_workspace_checked(fp4, orc):
+    import torch
+    M, N, K = 4, 1024, 512
+    need = fp4.gemm_workspace_size(M, N, K, 0)
+    qa = torch.zeros((M, K // 2), dtype=torch.uint8, device="cuda")
+    sa = torch.zeros((128 * K // 32,), dtype=torch.uint8, device="cuda")
+    qw = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    sw = torch.zeros((N * K // 32,), dtype=torch.uint8, device="cuda")
+    g = torch.ones((1,), dtype=torch.float32, device="cuda")
+    small = torch.empty((need - 16,), dtype=torch.uint8, device="cuda")
+    with pytest.raises(fp4.Fp4Error):
+        fp4.gemm((qa, sa, g), (qw, sw, g), M, N, K, 0, workspace=small)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("NK", [(14336, 4096), (4096, 14336)])
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_full_size_decode(fp4, orc, fmt, NK, M):
+    """Decode shapes of the 8B MLP: every output against the oracle."""
+    N, K = NK
+    a, w = inputs.decode_linear(M, N, K)
+    qa, sa, ga = orc.quantize(a, fmt)
+    qw, sw, gw = orc.quantize(w, fmt)
+    c = run_gemm(fp4, orc, qa, sa, ga, qw, sw, gw, fmt, 1)
+    ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, fmt)
+    assert_close(c, ref, bound, 1)
+
+
+# ------------------------------------------------------------------ linear ----
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("M,hk", [(1, 0), (16, 64), (5, 128), (200, 32)])
+def test_linear_online_activation_quantization(fp4, orc, fmt, M, hk):
+    """fp4_linear = online quantization of bf16 activations + the GEMM; the
+    reference quantizes the same activations with the oracle."""
+    import torch
+    N, K = 1024, 1024
+    rng = np.random.default_rng(M + hk)
+    x = inputs.f32_to_bf16_bits(rng.laplace(0, 1, (M, K)).astype(np.float32))
+    w = inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (N, K)).astype(np.float32))
+    qw, sw, gw = orc.quantize(w, fmt, hadamard_k=hk)
+    W = upload(orc, qw, sw, gw)
+    c = fp4.linear(to_dev_bf16(x), W, fmt, hadamard_k=hk, out_dtype=0)
+    torch.cuda.synchronize()
+    qa, sa, ga = orc.quantize(x, fmt, hadamard_k=hk)
+    ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, fmt)
+    assert_close(to_np(c), ref, bound, 0)
+
+
+def test_linear_static_activation_scale(fp4, orc):
+    import torch
+    M, N, K = 8, 512, 512
+    rng = np.random.default_rng(0)
+    x = inputs.f32_to_bf16_bits(rng.laplace(0, 1, (M, K)).astype(np.float32))
+    w = inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (N, K)).astype(np.float32))
+    qw, sw, gw = orc.quantize(w, 1)
+    W = upload(orc, qw, sw, gw)
+    gA = 0.004
+    c = fp4.linear(to_dev_bf16(x), W, 1, out_dtype=0, gscale=torch.tensor([gA], device="cuda"))
+    torch.cuda.synchronize()
+    qa, sa, ga = orc.quantize(x, 1, gscale=gA)
+    ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, 1)
+    assert_close(to_np(c), ref, bound, 0)
