@@ -38,7 +38,7 @@ struct QuantArgs {
 // Units processed per thread and loop trip: their loads are all issued
 // before any is consumed, so each thread keeps UNITS x 64 bytes in flight.
 constexpr int QUNITS = 2;  // quantize / amax
-constexpr int DUNITS = 4;  // dequantize (16 bytes of nibbles per unit)
+constexpr int DUNITS = 2;  // dequantize (16 bytes of nibbles per unit)
 
 // Raw bytes of one 32-element unit (4 x 16-byte loads, read-only path).
 FP4_DEV void fetch_unit(const uint16_t *x, int64_t ld, int64_t upr, int64_t u, uint4 *w)
@@ -278,6 +278,8 @@ struct DequantArgs {
 template <int FMT, int HK, int BF16OUT>
 __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
 {
+    constexpr int NC = BF16OUT ? 4 : 8;  // 16-byte output chunks per 32-element unit
+    __shared__ uint4 stage_all[8 * 32 * NC];
     const int lane = threadIdx.x & 31;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -305,10 +307,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
             const int64_t u = base + i * 32 + lane;
             const bool live = u < a.total_units;
             float v[32];
-            int64_t row = 0, j = 0;
             if (live) {
-                row = u / a.units_per_row;
-                j = u - row * a.units_per_row;
                 const uint4 w = raw[i];
                 const uint32_t words[4] = {w.x, w.y, w.z, w.w};
                 float d0, d1;
@@ -336,24 +335,41 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
                 for (int i = 0; i < 32; i++) v[i] = 0.0f;
             }
             if (HK) fwht_unit<HK>(v, a.ck, lane);
-            if (!live) continue;
+
+            // Stage the unit's output in shared memory (16-byte chunks, XOR
+            // swizzled so both the row-wise writes and the chunk-wise reads are
+            // free of bank conflicts), then store it as whole 512-byte warp
+            // segments: the warp's 32 units are contiguous in the output.
+            uint4 *stage = stage_all + (threadIdx.x >> 5) * (32 * NC);
             if (BF16OUT) {
-                uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(a.out) + row * a.cols + j * 32);
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
                     uint32_t w[4];
 #pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * c + 2 * i], v[8 * c + 2 * i + 1]);
-                        w[i] = *reinterpret_cast<uint32_t *>(&p);
+                    for (int e = 0; e < 4; e++) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * c + 2 * e], v[8 * c + 2 * e + 1]);
+                        w[e] = *reinterpret_cast<uint32_t *>(&h);
                     }
-                    o[c] = make_uint4(w[0], w[1], w[2], w[3]);
+                    stage[lane * NC + (c ^ ((lane >> 1) & 3))] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             } else {
-                float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + row * a.cols + j * 32);
 #pragma unroll
-                for (int c = 0; c < 8; c++) o[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                for (int c = 0; c < 8; c++)
+                    stage[lane * NC + (c ^ (lane & 7))] =
+                        make_uint4(__float_as_uint(v[4 * c]), __float_as_uint(v[4 * c + 1]),
+                                   __float_as_uint(v[4 * c + 2]), __float_as_uint(v[4 * c + 3]));
             }
+            __syncwarp();
+            const int64_t ubase = base + i * 32;
+            uint4 *out16 = reinterpret_cast<uint4 *>(a.out) + ubase * NC;
+#pragma unroll
+            for (int k = 0; k < NC; k++) {
+                const int ch = k * 32 + lane;   // chunk within the warp's segment
+                const int un = ch / NC, c = ch % NC;
+                const int cp = BF16OUT ? (c ^ ((un >> 1) & 3)) : (c ^ (un & 7));
+                if (ubase + un < a.total_units) out16[ch] = stage[un * NC + cp];
+            }
+            __syncwarp();
         }
     }
 }
