@@ -22,6 +22,8 @@
 // returns without storing.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "sm100.cuh"
 
 namespace fp4 {
@@ -220,6 +222,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 }
 
 }  // namespace tiled
+
 
 
 // ---------------------------------------------------------------------------
@@ -502,6 +505,7 @@ static bool make_fp4_map(CUtensorMap *m, const void *base, int64_t rows, int64_t
     return r == CUDA_SUCCESS;
 }
 
+
 template <int FMT, int BF>
 static cudaError_t launch_tiled(const CUtensorMap &ta, const CUtensorMap &tb, const tiled::Params &p, cudaStream_t st)
 {
@@ -612,3 +616,74 @@ cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err)
 }
 
 }  // namespace fp4
+
+namespace fp4 {
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode GEMM.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// decode product: code executing inside a CUDA stream capture that must not
+// add allocation nodes, plugins handed fixed buffers by a host framework, or
+// processes whose memory budget is fixed up front.  For them the decode
+// kernel's split-K partials live in a fixed, statically sized device array
+// owned by this library instead of a caller workspace.  The array is a
+// file-scope __device__ variable, so every GPU that loads the library keeps
+// it (kNoAllocScratchBytes) until the process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr int kMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device.  Host code only
+// sees a host-side stand-in under the array's name, so the address is looked
+// up once per device (with that device current) and cached.
+static cudaError_t noalloc_scratch(int dev, void **out)
+{
+    static std::mutex mu;
+    static void *ptrs[kMaxDevices] = {};
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return cudaSuccess;
+}
+
+}  // namespace fp4
+
+extern "C" fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *As, const float *gA,
+                                              const uint8_t *Wq, const uint8_t *Ws, const float *gW,
+                                              int64_t M, int64_t N, int64_t K, int fmt, int out_dtype,
+                                              void *C, int64_t ldc, void *stream)
+{
+    if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+    if (K % 256 || M > fp4::kDecodeMaxM) return FP4_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return FP4_OK;
+    if (!Aq || !As || !Wq || !Ws || !C) return FP4_ERR_INVALID_ARG;
+    if (fmt == FP4_NVFP4 && (!gA || !gW)) return FP4_ERR_INVALID_ARG;
+    auto aligned16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    if (!aligned16(Aq) || !aligned16(Wq) || !aligned16(As) || !aligned16(Ws) || !aligned16(C))
+        return FP4_ERR_ALIGNMENT;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return FP4_ERR_CUDA;
+    if (fp4::gemm_workspace_bytes(M, N, K, fmt, sms) > fp4::kNoAllocScratchBytes) return FP4_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if (fp4::noalloc_scratch(dev, &scratch) != cudaSuccess) return FP4_ERR_CUDA;
+    int bad = 0;
+    const cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc,
+                                           scratch, fp4::kNoAllocScratchBytes, sms,
+                                           static_cast<cudaStream_t>(stream), &bad);
+    if (bad) return FP4_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}

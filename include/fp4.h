@@ -172,6 +172,30 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
                       const float *gW, int64_t N, int out_dtype, void *C, int64_t ldc,
                       void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * fp4_gemm_decode_noalloc — the decode product of fp4_gemm (M <= 16) for
+ * callers that cannot allocate device memory at call time (inside a stream
+ * capture that must not add allocations, a plugin given fixed buffers, a
+ * process with a fixed memory budget).  It has no counterpart on the source
+ * pages: it is the same computation as fp4_gemm, with the split-K partials
+ * kept in a 4 MiB array inside this library instead of a caller workspace.
+ *   Arguments as fp4_gemm, without workspace.  M must be <= 16 and
+ *   fp4_gemm_workspace_size(M, N, K, fmt) must be <= 4 MiB, else
+ *   FP4_ERR_UNSUPPORTED (nothing launched).
+ *   The array is a device variable: every GPU that loads the library holds
+ *   4 MiB for it until the process exits.  The first call on a device looks
+ *   up the array's device address (with that device current); make that first
+ *   call before any stream capture.  All calls share the array: calls whose
+ *   kernels overlap on the GPU (different streams without ordering) race and
+ *   give wrong results.  Nothing in it needs to start at zero; it keeps the
+ *   last call's partial sums.
+ * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *As, const float *gA,
+                                   const uint8_t *Wq, const uint8_t *Ws, const float *gW,
+                                   int64_t M, int64_t N, int64_t K, int fmt, int out_dtype,
+                                   void *C, int64_t ldc, void *stream);
+
 /* Number of kernels this library has launched in this process so far
  * (host-side counter; diagnostics and launch accounting). */
 uint64_t fp4_kernel_launches(void);
