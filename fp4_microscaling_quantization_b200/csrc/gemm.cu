@@ -8,18 +8,13 @@
 // scales already in the 128x4 atom layout the MMA reads, so no re-layout
 // pass exists.  alpha = s_gA * s_gW for NVFP4, 1 for MXFP4.
 //
-// Tiled kernel (one 128 x 256 output tile per CTA, 4 warps):
-//   warp 0 lane 0  TMA producer: A (128 x 256 fp4) and W (256 x 256 fp4)
-//                  tiles with 128-byte swizzle, plus the scale atoms, into a
-//                  4-stage shared-memory ring (mbarrier transaction counts);
-//   warp 1 lane 0  MMA issuer: tcgen05.cp of the scale atoms to TMEM, then
-//                  four K=64 block-scaled MMAs per stage into a 128 x 256 fp32
-//                  TMEM accumulator; tcgen05.commit frees the stage;
-//   warps 0-3      epilogue: tcgen05.ld of their 32-lane quarter, x alpha,
-//                  convert, store.
+// Prefill (M > 16): a persistent kernel over 128*CG x 256 output tiles, CG = 2
+// (CTA pairs sharing one 2-SM MMA) once A spans more than 128 rows; see
+// pgemm_kernel.  Decode (M <= 16): a weight-streaming split-K kernel with a
+// deterministic reduction; see decode_kernel.
 // Every wait is bounded (%globaltimer); a wait that gives up sets the device
-// error word, the CTA drains its in-flight copies and MMAs, frees its TMEM and
-// returns without storing.
+// error word, the kernel stops issuing work, frees its TMEM and returns
+// without storing.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -30,200 +25,263 @@ namespace fp4 {
 
 static __device__ unsigned int g_gemm_error;
 
-namespace tiled {
 
-constexpr int BM = 128, BN = 256, BK = 256;  // BK in fp4 elements (128 bytes)
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK / 2;         // 16 KB
-constexpr int B_BYTES = BN * BK / 2;         // 32 KB
-constexpr int SFA_BYTES = 4 * 512;           // up to 4 atoms (NVFP4)
-constexpr int SFB_BYTES = 2 * 4 * 512;       // 2 row blocks x 4 atoms
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296, multiple of 1024
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
-constexpr int TMEM_COLS = 512;
-constexpr int ACC_COL = 0;
-constexpr int SF_COL0 = 256;                 // per stage: SFA 16 cols, SFB 32 cols
-constexpr int SF_STAGE_COLS = 48;
 
-struct Params {
-    const uint8_t *As;
-    const uint8_t *Ws;
+
+
+// ---------------------------------------------------------------------------
+// Persistent tiled kernel.  Each CTA (CG == 1) or CTA pair (CG == 2, one
+// 2-SM MMA covering 256 rows of A) walks output tiles of 128*CG x 256 in
+// M-fastest order, strided by the number of CTA groups, so the tiles resident
+// at one time share the same W columns in L2.  Roles:
+//   warp 0       TMA producer, runs ahead across tile boundaries: A rows of
+//                this CTA, its share of the 256 W rows (all of them for
+//                CG == 1, half for CG == 2) and the scale atoms (A: this CTA's
+//                128 rows; W: all 256 rows, both CTAs), counted on the full
+//                barrier of the group's leader CTA;
+//   warp 1       TMEM allocation; in the leader CTA also the MMA issuer:
+//                tcgen05.cp of the scale atoms, four K=64 block-scaled MMAs
+//                per stage, tcgen05.commit to free the stage (in both CTAs);
+//   warps 2-9    epilogue: two warps per 32-lane quarter, each draining 128
+//                accumulator columns into registers, then releasing the
+//                accumulator (so the next tile's MMAs start) before scaling,
+//                converting and storing.
+template <int CG>
+struct PCfg {
+    static constexpr int BM = 128;                       // rows of A per CTA
+    static constexpr int BN = 256;                       // output columns per tile
+    static constexpr int BK = 256;                       // fp4 elements per stage
+    static constexpr int B_ROWS = BN / CG;               // W rows loaded per CTA
+    static constexpr int A_BYTES = BM * BK / 2;
+    static constexpr int B_BYTES = B_ROWS * BK / 2;
+    static constexpr int SFA_BYTES = 4 * 512;
+    static constexpr int SFB_BYTES = 2 * 4 * 512;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGES = CG == 1 ? 4 : 5;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+    static constexpr int THREADS = 320;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int SF_COL0 = 256;
+    static constexpr int SF_STAGE_COLS = 48;
+    static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for the 128-byte swizzle");
+    static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "TMEM budget");
+};
+
+struct PParams {
     const float *gA;
     const float *gW;
     void *C;
     int64_t ldc;
     int M, N, K;
-    int nkb4;       // scale-atom columns per 128-row block (K / block / 4)
-    int nrb_w;      // 128-row scale blocks of W (pad128(N) / 128)
+    int nkb4;
+    int num_m_tiles, num_n_tiles;
 };
 
-template <int FMT, int BF16OUT>
-__global__ void __launch_bounds__(128, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p)
+template <int FMT, int BF16OUT, int CG>
+__global__ void __launch_bounds__(320, 1)
+pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+             const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, PParams p)
 {
-    constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;  // scale atoms per stage per 128-row block
+    using Cfg = PCfg<CG>;
+    constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
+    constexpr int STAGES = Cfg::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    // bars[0..S): full, bars[S..2S): empty, bars[2S]: accumulator ready
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * Cfg::STAGE_BYTES);
+    // bars: full[S] empty[S] accfull accempty
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 2);
     volatile uint32_t *abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mt = blockIdx.x, nt = blockIdx.y;
-    const int nk = p.K / BK;
-    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES), accb = smem_u32(bars + 2 * STAGES);
+    const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int group = blockIdx.x / CG, ngroups = gridDim.x / CG;
+    const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+    const int nk = p.K / Cfg::BK;
+
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+    const uint32_t accf = smem_u32(bars + 2 * STAGES), acce = smem_u32(bars + 2 * STAGES + 1);
+    // the leader's copies of the barriers every CTA of the group signals
+    const uint32_t full0_lead = (CG == 2) ? mapa_shared(full0, 0) : full0;
+    const uint32_t acce_lead = (CG == 2) ? mapa_shared(acce, 0) : acce;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
-            mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, 1);
+            mbar_init(full0 + 8 * s, CG);   // one arrive.expect_tx per CTA of the group
+            mbar_init(empty0 + 8 * s, 1);   // one tcgen05.commit
         }
-        mbar_init(accb, 1);
+        mbar_init(accf, 1);
+        mbar_init(acce, 8 * CG);            // every epilogue warp of the group
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmSA);
+        tma_prefetch_desc(&tmSB);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_cg<CG>(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish_cg<CG>();
     }
     tc_fence_before();
-    __syncthreads();
+    if (CG == 2) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
-            const int nrb = (2 * nt + 1 < p.nrb_w) ? 2 : 1;
-            const uint32_t tx = A_BYTES + B_BYTES + KA * 512 * (1 + nrb);
-            int issued = 0;
-            for (int ks = 0; ks < nk; ks++) {
-                const int s = ks % STAGES;
-                const uint32_t ph = (ks / STAGES) & 1;
-                if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error)) break;
-                uint8_t *st = smem + s * STAGE_BYTES;
-                const uint32_t fb = full0 + 8 * s;
-                mbar_arrive_expect_tx(fb, tx);
-                tma_load_2d(smem_u32(st), &tmA, ks * (BK / 2), mt * BM, fb);
-                tma_load_2d(smem_u32(st + A_BYTES), &tmB, ks * (BK / 2), nt * BN, fb);
-                bulk_load(smem_u32(st + A_BYTES + B_BYTES), p.As + ((int64_t)mt * p.nkb4 + ks * KA) * 512, KA * 512, fb);
-                for (int rb = 0; rb < nrb; rb++)
-                    bulk_load(smem_u32(st + A_BYTES + B_BYTES + SFA_BYTES + rb * KA * 512),
-                              p.Ws + ((int64_t)(2 * nt + rb) * p.nkb4 + ks * KA) * 512, KA * 512, fb);
-                issued = ks + 1;
-            }
-            // drain: every issued copy must land before the CTA may exit
-            for (int ks = (issued > STAGES ? issued - STAGES : 0); ks < issued; ks++) {
-                volatile uint32_t no_abort = 0;
-                mbar_wait_bounded(full0 + 8 * (ks % STAGES), (ks / STAGES) & 1, &no_abort, &g_gemm_error);
+            const uint32_t tx = Cfg::A_BYTES + Cfg::B_BYTES + 3 * KA * 512;
+            int it = 0;
+            for (int t = group; t < num_tiles; t += ngroups) {
+                const int mt = t % p.num_m_tiles, nt = t / p.num_m_tiles;
+                const int arow = (mt * CG + (int)rank) * Cfg::BM;
+                const int brow = nt * Cfg::BN + (int)rank * Cfg::B_ROWS;
+                const int sfa_atom = (mt * CG + (int)rank) * p.nkb4;
+                const int sfb_atom0 = (2 * nt) * p.nkb4, sfb_atom1 = (2 * nt + 1) * p.nkb4;
+                bool stop = false;
+                for (int ks = 0; ks < nk; ks++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error)) { stop = true; break; }
+                    uint8_t *st = smem + s * Cfg::STAGE_BYTES;
+                    const uint32_t fb = full0_lead + 8 * s;
+                    if (CG == 1) mbar_arrive_expect_tx(fb, tx); else mbar_arrive_expect_tx_cluster(fb, tx);
+                    tma_load_2d_cg<CG>(smem_u32(st), &tmA, ks * (Cfg::BK / 2), arow, fb);
+                    tma_load_2d_cg<CG>(smem_u32(st + Cfg::A_BYTES), &tmB, ks * (Cfg::BK / 2), brow, fb);
+                    const uint32_t ssf = smem_u32(st + Cfg::A_BYTES + Cfg::B_BYTES);
+                    tma_load_2d_cg<CG>(ssf, &tmSA, 0, sfa_atom + ks * KA, fb);
+                    tma_load_2d_cg<CG>(ssf + Cfg::SFA_BYTES, &tmSB, 0, sfb_atom0 + ks * KA, fb);
+                    tma_load_2d_cg<CG>(ssf + Cfg::SFA_BYTES + KA * 512, &tmSB, 0, sfb_atom1 + ks * KA, fb);
+                }
+                if (stop) break;
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer ----------------
-            const uint32_t acc = tmem + ACC_COL;
-            for (int ks = 0; ks < nk; ks++) {
-                const int s = ks % STAGES;
-                const uint32_t ph = (ks / STAGES) & 1;
-                if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error)) break;
+        if (lane == 0 && leader) {
+            // ---------------- MMA issuer (leader CTA) ----------------
+            int it = 0, tile_i = 0;
+            const uint16_t both = (uint16_t)((1u << CG) - 1u);
+            for (int t = group; t < num_tiles; t += ngroups, tile_i++) {
+                if (tile_i > 0 &&
+                    !mbar_wait_bounded(acce, (uint32_t)((tile_i - 1) & 1), abort_flag, &g_gemm_error))
+                    break;
                 tc_fence_after();
-                const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-                const uint32_t sb = sa + A_BYTES;
-                const uint32_t ssfa = sb + B_BYTES;
-                const uint32_t ssfb = ssfa + SFA_BYTES;
-                const uint32_t tsfa = tmem + SF_COL0 + s * SF_STAGE_COLS;
-                const uint32_t tsfb = tsfa + 16;
-                for (int a = 0; a < KA; a++) {
-                    tc_cp_scale_atom(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
-                    tc_cp_scale_atom(tsfb + 8 * a, smem_desc(ssfb + 512 * a, 0, 128, 0));
-                    tc_cp_scale_atom(tsfb + 8 * a + 4, smem_desc(ssfb + KA * 512 + 512 * a, 0, 128, 0));
-                }
+                bool stop = false;
+                for (int ks = 0; ks < nk; ks++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
+                    const uint32_t sb = sa + Cfg::A_BYTES;
+                    const uint32_t ssfa = sb + Cfg::B_BYTES;
+                    const uint32_t ssfb = ssfa + Cfg::SFA_BYTES;
+                    const uint32_t tsfa = tmem + Cfg::SF_COL0 + s * Cfg::SF_STAGE_COLS;
+                    const uint32_t tsfb = tsfa + 16;
+                    for (int a = 0; a < KA; a++) {
+                        tc_cp_scale_atom_cg<CG>(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
+                        tc_cp_scale_atom_cg<CG>(tsfb + 8 * a, smem_desc(ssfb + 512 * a, 0, 128, 0));
+                        tc_cp_scale_atom_cg<CG>(tsfb + 8 * a + 4, smem_desc(ssfb + KA * 512 + 512 * a, 0, 128, 0));
+                    }
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    // K step of 64 fp4 = 32 bytes inside the 128-byte swizzled row
-                    const uint64_t ad = smem_desc(sa + 32 * kk, 16, 1024, 2);
-                    const uint64_t bd = smem_desc(sb + 32 * kk, 16, 1024, 2);
-                    const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
-                    const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
-                    const uint32_t idesc = idesc_blockscaled(BM, BN, FMT == FP4_MXFP4, sfid, sfid);
-                    tc_mma_blockscaled<FMT>(acc, ad, bd, idesc, (tsfa + 4 * atom) | (sfid << 30),
-                                            (tsfb + 8 * atom) | (sfid << 30), (ks | kk) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; kk++) {
+                        const uint64_t ad = smem_desc(sa + 32 * kk, 16, 1024, 2);
+                        const uint64_t bd = smem_desc(sb + 32 * kk, 16, 1024, 2);
+                        const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
+                        const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
+                        const uint32_t idesc = idesc_blockscaled(Cfg::BM * CG, Cfg::BN, FMT == FP4_MXFP4, sfid, sfid);
+                        tc_mma_blockscaled_cg<FMT, CG>(tmem, ad, bd, idesc, (tsfa + 4 * atom) | (sfid << 30),
+                                                       (tsfb + 8 * atom) | (sfid << 30), (ks | kk) ? 1u : 0u);
+                    }
+                    tc_commit_cg<CG>(empty0 + 8 * s, both);
                 }
-                tc_commit(empty0 + 8 * s);
+                // the accumulator is ready (or, after an abort, no MMA is left in flight)
+                tc_commit_cg<CG>(accf, both);
+                if (stop) break;
             }
-            // arrives once every MMA issued above has completed (also on abort)
-            tc_commit(accb);
         }
         __syncwarp();
-    }
-
-    // ---------------- epilogue (all four warps) ----------------
-    {
-        volatile uint32_t no_abort = 0;
-        bool ok = mbar_wait_bounded(accb, 0, &no_abort, &g_gemm_error) && !*abort_flag;
-        ok = __all_sync(0xFFFFFFFFu, ok);  // tcgen05.ld below is warp-collective
-        tc_fence_after();
-        if (ok) {
+    } else {
+        // ---------------- epilogue: warps 2..9 ----------------
+        const int quarter = warp & 3;          // TMEM lanes this warp may read
+        const int half = (warp - 2) >> 2;      // accumulator columns [128*half, 128*half + 128)
+        const bool vec32 = BF16OUT ? (p.ldc % 16 == 0) : (p.ldc % 8 == 0);
+        const bool aligned_c = (reinterpret_cast<uintptr_t>(p.C) & 31) == 0;
+        int tile_i = 0;
+        for (int t = group; t < num_tiles; t += ngroups, tile_i++) {
+            bool ok = !*abort_flag && mbar_wait_bounded(accf, (uint32_t)(tile_i & 1), abort_flag, &g_gemm_error);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok || *abort_flag) break;
+            tc_fence_after();
+            const int mt = t % p.num_m_tiles, nt = t / p.num_m_tiles;
+            uint32_t r[128];
+            const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 128);
+            tmem_ld32(base + 0, r + 0);
+            tmem_ld32(base + 32, r + 32);
+            tmem_ld32(base + 64, r + 64);
+            tmem_ld32(base + 96, r + 96);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (CG == 1) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce) : "memory");
+                else mbar_arrive_cluster(acce_lead);
+            }
             const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
-            const int m = mt * BM + warp * 32 + lane;
-            const uint32_t lane_base = tmem + ACC_COL + ((uint32_t)(warp * 32) << 16);
-            const bool vec_ok = BF16OUT ? (p.ldc % 8 == 0) : (p.ldc % 4 == 0);
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; c++) {
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld32(lane_base + c * 32, r);
-                tmem_ld_wait();
-                const int n0 = nt * BN + c * 32;
-                if (m >= p.M || n0 >= p.N) continue;
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; i++) v[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
-                const bool full = vec_ok && (n0 + 32 <= p.N);
+            const int m = (mt * CG + (int)rank) * Cfg::BM + quarter * 32 + lane;
+            const int n0 = nt * Cfg::BN + half * 128;
+            if (m < p.M && n0 < p.N) {
                 if (BF16OUT) {
                     __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(p.C) + (int64_t)m * p.ldc + n0;
-                    if (full) {
+                    const bool fast = vec32 && aligned_c && n0 + 128 <= p.N;
 #pragma unroll
-                        for (int q = 0; q < 4; q++) {
-                            uint32_t w[4];
+                    for (int c = 0; c < 8; c++) {
+                        uint32_t w[8];
 #pragma unroll
-                            for (int i = 0; i < 4; i++) {
-                                __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * i], v[8 * q + 2 * i + 1]);
-                                w[i] = *reinterpret_cast<uint32_t *>(&h);
-                            }
-                            reinterpret_cast<uint4 *>(row)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+                        for (int e = 0; e < 8; e++) {
+                            __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[16 * c + 2 * e]), alpha),
+                                                                     __fmul_rn(__uint_as_float(r[16 * c + 2 * e + 1]), alpha));
+                            w[e] = *reinterpret_cast<uint32_t *>(&h);
                         }
-                    } else {
-                        for (int i = 0; i < 32 && n0 + i < p.N; i++) row[i] = __float2bfloat16_rn(v[i]);
+                        if (fast) {
+                            st_global_v8(row + 16 * c, w);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; e++)
+                                if (n0 + 16 * c + e < p.N)
+                                    reinterpret_cast<uint16_t *>(row)[16 * c + e] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+                        }
                     }
                 } else {
                     float *row = reinterpret_cast<float *>(p.C) + (int64_t)m * p.ldc + n0;
-                    if (full) {
+                    const bool fast = vec32 && aligned_c && n0 + 128 <= p.N;
 #pragma unroll
-                        for (int q = 0; q < 8; q++)
-                            reinterpret_cast<float4 *>(row)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    } else {
-                        for (int i = 0; i < 32 && n0 + i < p.N; i++) row[i] = v[i];
+                    for (int c = 0; c < 16; c++) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; e++) w[e] = __float_as_uint(__fmul_rn(__uint_as_float(r[8 * c + e]), alpha));
+                        if (fast) {
+                            st_global_v8(row + 8 * c, w);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; e++)
+                                if (n0 + 8 * c + e < p.N) row[8 * c + e] = __uint_as_float(w[e]);
+                        }
                     }
                 }
             }
         }
     }
+
     tc_fence_before();
-    __syncthreads();
+    if (CG == 2) cluster_sync(); else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_cg<CG>(tmem, Cfg::TMEM_COLS);
     }
 }
-
-}  // namespace tiled
-
-
 
 // ---------------------------------------------------------------------------
 // Decode kernel (M <= 16): the weight stream dominates, so the roles swap: a
@@ -506,21 +564,72 @@ static bool make_fp4_map(CUtensorMap *m, const void *base, int64_t rows, int64_t
 }
 
 
-template <int FMT, int BF>
-static cudaError_t launch_tiled(const CUtensorMap &ta, const CUtensorMap &tb, const tiled::Params &p, cudaStream_t st)
+// Scale-atom buffer (tile layout) as a 2-D tensor of 512-byte atoms: 256
+// uint16 per atom, one atom per row; boxes of `box_atoms` consecutive atoms.
+// Atoms past the end (row blocks beyond the padded rows) read as zeros.
+static bool make_sf_map(CUtensorMap *m, const void *base, int64_t n_atoms, int box_atoms)
 {
-    auto kern = tiled::gemm_kernel<FMT, BF>;
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {256u, (cuuint64_t)n_atoms};
+    cuuint64_t strides[1] = {512u};
+    cuuint32_t box[2] = {256u, (cuuint32_t)box_atoms};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int FMT, int BF, int CG>
+static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq, const uint8_t *Ws,
+                                const PParams &p, int sms, cudaStream_t st)
+{
+    using Cfg = PCfg<CG>;
+    constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
+    CUtensorMap ta, tb, tsa, tsb;
+    const int64_t nrb_a = (int64_t)((p.M + 127) / 128), nrb_w = (int64_t)((p.N + 127) / 128);
+    if (!make_fp4_map(&ta, Aq, p.M, p.K, Cfg::BM) || !make_fp4_map(&tb, Wq, p.N, p.K, Cfg::B_ROWS) ||
+        !make_sf_map(&tsa, As, nrb_a * p.nkb4, KA) || !make_sf_map(&tsb, Ws, nrb_w * p.nkb4, KA))
+        return cudaErrorInvalidValue;
+    auto kern = pgemm_kernel<FMT, BF, CG>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tiled::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid((p.M + tiled::BM - 1) / tiled::BM, (p.N + tiled::BN - 1) / tiled::BN);
+    const int tiles = p.num_m_tiles * p.num_n_tiles;
+    const int groups = tiles < sms / CG ? tiles : sms / CG;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(groups * CG, 1, 1);
+    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     count_launches(1);
-    kern<<<grid, 128, tiled::SMEM_BYTES, st>>>(ta, tb, p);
-    return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p);
 }
+
+template <int CG>
+static cudaError_t launch_pgemm_fmt(int fmt, int bf16out, const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq,
+                                    const uint8_t *Ws, const PParams &p, int sms, cudaStream_t st)
+{
+    if (fmt == FP4_MXFP4)
+        return bf16out ? launch_pgemm<FP4_MXFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st)
+                       : launch_pgemm<FP4_MXFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st);
+    return bf16out ? launch_pgemm<FP4_NVFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st)
+                   : launch_pgemm<FP4_NVFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st);
+}
+
+// CTA-pair (2-SM MMA) tiles are used once A spans more than one 128-row block.
+static int pgemm_cta_group(int64_t M) { return M > 128 ? 2 : 1; }
 
 constexpr int64_t kDecodeMaxM = 16;
 
@@ -584,23 +693,22 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         return bf16out ? launch_decode<FP4_NVFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st)
                        : launch_decode<FP4_NVFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st);
     }
-    CUtensorMap ta, tb;
-    if (!make_fp4_map(&ta, Aq, M, K, tiled::BM) || !make_fp4_map(&tb, Wq, N, K, tiled::BN)) return cudaErrorInvalidValue;
-    tiled::Params p;
-    p.As = As;
-    p.Ws = Ws;
-    p.gA = gA;
-    p.gW = gW;
-    p.C = C;
-    p.ldc = ldc;
-    p.M = (int)M;
-    p.N = (int)N;
-    p.K = (int)K;
-    p.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
-    p.nrb_w = (int)((N + 127) / 128);
-    if (fmt == FP4_MXFP4)
-        return bf16out ? launch_tiled<FP4_MXFP4, 1>(ta, tb, p, st) : launch_tiled<FP4_MXFP4, 0>(ta, tb, p, st);
-    return bf16out ? launch_tiled<FP4_NVFP4, 1>(ta, tb, p, st) : launch_tiled<FP4_NVFP4, 0>(ta, tb, p, st);
+    {
+        PParams pp;
+        pp.gA = gA;
+        pp.gW = gW;
+        pp.C = C;
+        pp.ldc = ldc;
+        pp.M = (int)M;
+        pp.N = (int)N;
+        pp.K = (int)K;
+        pp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+        const int cg = pgemm_cta_group(M);
+        pp.num_m_tiles = (int)((M + 128 * cg - 1) / (128 * cg));
+        pp.num_n_tiles = (int)((N + 255) / 256);
+        return cg == 2 ? launch_pgemm_fmt<2>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st)
+                       : launch_pgemm_fmt<1>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st);
+    }
 }
 
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err)
