@@ -11,14 +11,14 @@
 namespace fp4 {
 cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
                             int hk, float ck, int round_away, int mx_floor, int gscale_given,
-                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st);
+                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl);
 cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
                               int64_t cols, int fmt, int hk, float ck, int bf16out, void *out,
                               int sms, cudaStream_t st);
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
                         const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K,
                         int fmt, int bf16out, void *C, int64_t ldc, void *ws, size_t ws_bytes,
-                        int sms, cudaStream_t st, int *timeout_flag_out);
+                        int sms, cudaStream_t st, int *timeout_flag_out, bool pdl);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int sms);
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
 static std::atomic<uint64_t> g_launches{0};
@@ -99,7 +99,7 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                                          hadamard_k, hadamard_constant(hadamard_k),
                                          o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
                                          o.gscale_given, q, s, gscale, sm_count(),
-                                         static_cast<cudaStream_t>(stream));
+                                         static_cast<cudaStream_t>(stream), false);
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
@@ -148,7 +148,7 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const
     int bad = 0;
     cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16,
                                      C, ldc, workspace, ws_bytes, sms,
-                                     static_cast<cudaStream_t>(stream), &bad);
+                                     static_cast<cudaStream_t>(stream), &bad, false);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
@@ -214,11 +214,12 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = fp4::launch_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
                                          hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
-                                         o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, sms, st);
+                                         o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, sms, st,
+                                         true);
     if (e != cudaSuccess) return FP4_ERR_CUDA;
     int bad = 0;
     e = fp4::launch_gemm(aq, as, ga, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc, base + L.gemm,
-                         L.total - L.gemm, sms, st, &bad);
+                         L.total - L.gemm, sms, st, &bad, true);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

@@ -14,6 +14,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/fp4.h"
 
 #define FP4_DEV __device__ __forceinline__
@@ -23,7 +25,35 @@ namespace fp4 {
 // Host-side launch accounting (fp4_kernel_launches).
 void count_launches(int n);
 
+// Launches `kern` on `st`; with `pdl` the launch may overlap the tail of the
+// previous kernel in the stream (programmatic stream serialization).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                            Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    count_launches(1);
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 constexpr float kFltMax = 3.40282346638528859812e+38f;
+
+// ---- programmatic dependent launch -----------------------------------------
+// A kernel launched with programmatic stream serialization may start before
+// its predecessor in the stream has finished; it must call grid_dep_wait()
+// before reading anything the predecessor wrote (or writing anything it
+// reads).  Both are no-ops for ordinary launches.
+FP4_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+FP4_DEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- bf16 -----------------------------------------------------------------
 // Two bf16 values packed in a 32-bit word -> fp32 (exact).

@@ -127,6 +127,8 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     if (CG == 2) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    grid_dep_launch();
+    grid_dep_wait();  // operands may come from the preceding kernel
 
     if (warp == 0) {
         if (lane == 0) {
@@ -331,6 +333,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
     volatile uint32_t *abort_flag = tmem_slot + 1;
 
+    grid_dep_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
     const int64_t U = (int64_t)p.ntiles * p.nk;
@@ -368,20 +371,39 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     if (warp == 0) {
         if (lane == 0) {
             const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
-            int64_t issued = 0;
-            for (int64_t u = u0; u < u1; u++) {
+            auto load_w = [&](int64_t u, int s) {
+                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
+                uint8_t *st = smem + s * STAGE_BYTES;
+                const uint32_t fb = full0 + 8 * s;
+                tma_load_2d(smem_u32(st), &tmW, ks * (BK / 2), t * BMW, fb);
+                bulk_load(smem_u32(st + W_BYTES + A_BYTES), p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+            };
+            auto load_a = [&](int64_t u, int s) {
+                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
+                uint8_t *st = smem + s * STAGE_BYTES;
+                const uint32_t fb = full0 + 8 * s;
+                tma_load_2d(smem_u32(st + W_BYTES), &tmA, ks * (BK / 2), 0, fb);
+                bulk_load(smem_u32(st + W_BYTES + A_BYTES + SFW_BYTES), p.As + (int64_t)ks * KA * 512, KA * 512, fb);
+            };
+            // The weight stream does not depend on the preceding kernel (which
+            // may still be quantizing the activations): fill the first stages
+            // with W, then wait for the activations.
+            const int64_t npre = (u1 - u0) < STAGES ? (u1 - u0) : STAGES;
+            for (int64_t i = 0; i < npre; i++) {
+                mbar_arrive_expect_tx(full0 + 8 * (int)i, tx);
+                load_w(u0 + i, (int)i);
+            }
+            grid_dep_wait();
+            for (int64_t i = 0; i < npre; i++) load_a(u0 + i, (int)i);
+            int64_t issued = npre;
+            for (int64_t u = u0 + npre; u < u1; u++) {
                 const int64_t i = u - u0;
                 const int s = (int)(i % STAGES);
                 const uint32_t ph = (uint32_t)((i / STAGES) & 1);
                 if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error)) break;
-                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
-                uint8_t *st = smem + s * STAGE_BYTES;
-                const uint32_t fb = full0 + 8 * s;
-                mbar_arrive_expect_tx(fb, tx);
-                tma_load_2d(smem_u32(st), &tmW, ks * (BK / 2), t * BMW, fb);
-                tma_load_2d(smem_u32(st + W_BYTES), &tmA, ks * (BK / 2), 0, fb);
-                bulk_load(smem_u32(st + W_BYTES + A_BYTES), p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
-                bulk_load(smem_u32(st + W_BYTES + A_BYTES + SFW_BYTES), p.As + (int64_t)ks * KA * 512, KA * 512, fb);
+                mbar_arrive_expect_tx(full0 + 8 * s, tx);
+                load_w(u, s);
+                load_a(u, s);
                 issued = i + 1;
             }
             for (int64_t i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++) {
@@ -440,6 +462,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     // ---------------- epilogue warps 2-5: one partial per tile segment ----------------
     // warp w may only read TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
+    grid_dep_wait();
     for (int seg = 0; seg < nseg; seg++) {
         const int b = seg & 1;
         bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error);
@@ -474,6 +497,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
 template <int BF16OUT, int FMT>
 __global__ void __launch_bounds__(128) reduce_kernel(Params p, const float *gA, const float *gW, void *C, int64_t ldc)
 {
+    grid_dep_wait();
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     if (n >= p.N) return;
     const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*gA, *gW) : 1.0f;
@@ -583,7 +607,7 @@ static bool make_sf_map(CUtensorMap *m, const void *base, int64_t n_atoms, int b
 
 template <int FMT, int BF, int CG>
 static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq, const uint8_t *Ws,
-                                const PParams &p, int sms, cudaStream_t st)
+                                const PParams &p, int sms, cudaStream_t st, bool pdl)
 {
     using Cfg = PCfg<CG>;
     constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
@@ -606,26 +630,28 @@ static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint
     cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CG;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     count_launches(1);
     return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p);
 }
 
 template <int CG>
 static cudaError_t launch_pgemm_fmt(int fmt, int bf16out, const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq,
-                                    const uint8_t *Ws, const PParams &p, int sms, cudaStream_t st)
+                                    const uint8_t *Ws, const PParams &p, int sms, cudaStream_t st, bool pdl)
 {
     if (fmt == FP4_MXFP4)
-        return bf16out ? launch_pgemm<FP4_MXFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st)
-                       : launch_pgemm<FP4_MXFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st);
-    return bf16out ? launch_pgemm<FP4_NVFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st)
-                   : launch_pgemm<FP4_NVFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st);
+        return bf16out ? launch_pgemm<FP4_MXFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st, pdl)
+                       : launch_pgemm<FP4_MXFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
+    return bf16out ? launch_pgemm<FP4_NVFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st, pdl)
+                   : launch_pgemm<FP4_NVFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
 }
 
 // CTA-pair (2-SM MMA) tiles are used once A spans more than one 128-row block.
@@ -641,7 +667,7 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
 
 template <int FMT, int BF>
 static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const decode::Params &p, const float *gA,
-                                 const float *gW, void *C, int64_t ldc, cudaStream_t st)
+                                 const float *gW, void *C, int64_t ldc, cudaStream_t st, bool pdl)
 {
     auto kern = decode::decode_kernel<FMT>;
     static bool attr_set = false;
@@ -650,17 +676,16 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    count_launches(2);
-    kern<<<p.G, 192, decode::SMEM_BYTES, st>>>(tw, ta, p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_k(kern, dim3(p.G), dim3(192), decode::SMEM_BYTES, st, pdl, tw, ta, p);
     if (e != cudaSuccess) return e;
-    decode::reduce_kernel<BF, FMT><<<(p.N + 127) / 128, 128, 0, st>>>(p, gA, gW, C, ldc);
-    return cudaGetLastError();
+    // the reduction waits for the split-K kernel inside (grid_dep_wait)
+    return launch_k(decode::reduce_kernel<BF, FMT>, dim3((p.N + 127) / 128), dim3(128), 0, st, true, p, gA, gW, C,
+                    ldc);
 }
 
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
                         const float *gW, int64_t M, int64_t N, int64_t K, int fmt, int bf16out, void *C, int64_t ldc,
-                        void *ws, size_t ws_bytes, int sms, cudaStream_t st, int *bad)
+                        void *ws, size_t ws_bytes, int sms, cudaStream_t st, int *bad, bool pdl)
 {
     if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) {
         *bad = 1;
@@ -688,10 +713,10 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.maxseg = pl.maxseg;
         dp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
         if (fmt == FP4_MXFP4)
-            return bf16out ? launch_decode<FP4_MXFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st)
-                           : launch_decode<FP4_MXFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st);
-        return bf16out ? launch_decode<FP4_NVFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st)
-                       : launch_decode<FP4_NVFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st);
+            return bf16out ? launch_decode<FP4_MXFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st, pdl)
+                           : launch_decode<FP4_MXFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st, pdl);
+        return bf16out ? launch_decode<FP4_NVFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st, pdl)
+                       : launch_decode<FP4_NVFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st, pdl);
     }
     {
         PParams pp;
@@ -706,8 +731,8 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         const int cg = pgemm_cta_group(M);
         pp.num_m_tiles = (int)((M + 128 * cg - 1) / (128 * cg));
         pp.num_n_tiles = (int)((N + 255) / 256);
-        return cg == 2 ? launch_pgemm_fmt<2>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st)
-                       : launch_pgemm_fmt<1>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st);
+        return cg == 2 ? launch_pgemm_fmt<2>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st, pdl)
+                       : launch_pgemm_fmt<1>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st, pdl);
     }
 }
 
@@ -791,7 +816,7 @@ extern "C" fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *
     int bad = 0;
     const cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc,
                                            scratch, fp4::kNoAllocScratchBytes, sms,
-                                           static_cast<cudaStream_t>(stream), &bad);
+                                           static_cast<cudaStream_t>(stream), &bad, false);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

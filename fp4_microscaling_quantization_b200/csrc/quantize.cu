@@ -114,6 +114,8 @@ FP4_DEV float read_global_scale(const float *g, int computed)
 template <int HK>
 __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -155,6 +157,8 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
 // (1 for an all-zero tensor).  Runs after the quantize kernel has read it.
 __global__ void finalize_gscale_kernel(float *g)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     *g = nv_global_from_amax(*g);
 }
 
@@ -162,6 +166,8 @@ __global__ void finalize_gscale_kernel(float *g)
 template <int FMT, int HK>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -242,6 +248,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
 // [nkb, 4*nkb4) of real rows, and every byte of rows [rows, pad128(rows)).
 __global__ void scale_pad_kernel(uint8_t *s, int64_t rows, int64_t nkb, int64_t nkb4)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     const int64_t cpad = nkb4 * 4 - nkb;
     const int64_t rows_p = (rows + 127) / 128 * 128;
     const int64_t n1 = rows * cpad;
@@ -278,6 +286,8 @@ struct DequantArgs {
 template <int FMT, int HK, int BF16OUT>
 __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     constexpr int NC = BF16OUT ? 4 : 8;  // 16-byte output chunks per 32-element unit
     __shared__ uint4 stage_all[8 * 32 * NC];
     const int lane = threadIdx.x & 31;
@@ -385,37 +395,36 @@ static int grid_for(int64_t total_units, int sms, int units_per_thread)
 }
 
 template <int FMT>
-static cudaError_t launch_quant_fmt(const QuantArgs &a, int hk, int grid, cudaStream_t st)
+static void (*quant_kernel_for(int hk))(QuantArgs)
 {
-    count_launches(1);
     switch (hk) {
-    case 0: quantize_kernel<FMT, 0><<<grid, 256, 0, st>>>(a); break;
-    case 16: quantize_kernel<FMT, 16><<<grid, 256, 0, st>>>(a); break;
-    case 32: quantize_kernel<FMT, 32><<<grid, 256, 0, st>>>(a); break;
-    case 64: quantize_kernel<FMT, 64><<<grid, 256, 0, st>>>(a); break;
-    case 128: quantize_kernel<FMT, 128><<<grid, 256, 0, st>>>(a); break;
-    default: return cudaErrorInvalidValue;
+    case 0: return quantize_kernel<FMT, 0>;
+    case 16: return quantize_kernel<FMT, 16>;
+    case 32: return quantize_kernel<FMT, 32>;
+    case 64: return quantize_kernel<FMT, 64>;
+    case 128: return quantize_kernel<FMT, 128>;
     }
-    return cudaGetLastError();
+    return nullptr;
 }
 
-static cudaError_t launch_amax(const QuantArgs &a, int hk, int grid, cudaStream_t st)
+static void (*amax_kernel_for(int hk))(QuantArgs)
 {
-    count_launches(1);
     switch (hk) {
-    case 0: amax_kernel<0><<<grid, 256, 0, st>>>(a); break;
-    case 16: amax_kernel<16><<<grid, 256, 0, st>>>(a); break;
-    case 32: amax_kernel<32><<<grid, 256, 0, st>>>(a); break;
-    case 64: amax_kernel<64><<<grid, 256, 0, st>>>(a); break;
-    case 128: amax_kernel<128><<<grid, 256, 0, st>>>(a); break;
-    default: return cudaErrorInvalidValue;
+    case 0: return amax_kernel<0>;
+    case 16: return amax_kernel<16>;
+    case 32: return amax_kernel<32>;
+    case 64: return amax_kernel<64>;
+    case 128: return amax_kernel<128>;
     }
-    return cudaGetLastError();
+    return nullptr;
 }
 
+// Quantize launch sequence.  With `pdl` every launch after the first may
+// overlap its predecessor (each kernel waits for it before touching memory),
+// so a consumer launched the same way can start streaming early.
 cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
                             int hk, float ck, int round_away, int mx_floor, int gscale_given,
-                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st)
+                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl)
 {
     QuantArgs a;
     a.x = x;
@@ -433,46 +442,48 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
     const int grid = grid_for(a.total_units, sms, QUNITS);
+    void (*qk)(QuantArgs) = (fmt == FP4_MXFP4) ? quant_kernel_for<FP4_MXFP4>(hk) : quant_kernel_for<FP4_NVFP4>(hk);
+    void (*ak)(QuantArgs) = amax_kernel_for(hk);
+    if (!qk || !ak) return cudaErrorInvalidValue;
     cudaError_t err = cudaSuccess;
+    bool first = true;  // the first launch of the sequence is ordered normally after earlier work
     if (a.gscale_computed) {
         if ((err = cudaMemsetAsync(gscale, 0, sizeof(float), st)) != cudaSuccess) return err;
-        if ((err = launch_amax(a, hk, grid, st)) != cudaSuccess) return err;
+        if ((err = launch_k(ak, dim3(grid), dim3(256), 0, st, false, a)) != cudaSuccess) return err;
+        first = false;
     }
     if (a.total_units > 0) {
-        err = (fmt == FP4_MXFP4) ? launch_quant_fmt<FP4_MXFP4>(a, hk, grid, st)
-                                 : launch_quant_fmt<FP4_NVFP4>(a, hk, grid, st);
-        if (err != cudaSuccess) return err;
+        if ((err = launch_k(qk, dim3(grid), dim3(256), 0, st, pdl && !first, a)) != cudaSuccess) return err;
+        first = false;
     }
     if (a.gscale_computed) {
-        count_launches(1);
-        finalize_gscale_kernel<<<1, 1, 0, st>>>(gscale);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        if ((err = launch_k(finalize_gscale_kernel, dim3(1), dim3(1), 0, st, pdl && !first, gscale)) != cudaSuccess)
+            return err;
+        first = false;
     }
     const int64_t rows_p = (rows + 127) / 128 * 128;
     const int64_t npad = rows * (a.nkb4 * 4 - nkb) + (rows_p - rows) * a.nkb4 * 4;
     if (npad > 0) {
         int g = (int)((npad + 255) / 256);
         if (g > sms * 4) g = sms * 4;
-        count_launches(1);
-        scale_pad_kernel<<<g, 256, 0, st>>>(s, rows, nkb, a.nkb4);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        if ((err = launch_k(scale_pad_kernel, dim3(g), dim3(256), 0, st, pdl && !first, s, rows, nkb, a.nkb4)) !=
+            cudaSuccess)
+            return err;
     }
     return cudaSuccess;
 }
 
 template <int FMT, int BF>
-static cudaError_t launch_deq_fmt(const DequantArgs &a, int hk, int grid, cudaStream_t st)
+static void (*deq_kernel_for(int hk))(DequantArgs)
 {
-    count_launches(1);
     switch (hk) {
-    case 0: dequantize_kernel<FMT, 0, BF><<<grid, 256, 0, st>>>(a); break;
-    case 16: dequantize_kernel<FMT, 16, BF><<<grid, 256, 0, st>>>(a); break;
-    case 32: dequantize_kernel<FMT, 32, BF><<<grid, 256, 0, st>>>(a); break;
-    case 64: dequantize_kernel<FMT, 64, BF><<<grid, 256, 0, st>>>(a); break;
-    case 128: dequantize_kernel<FMT, 128, BF><<<grid, 256, 0, st>>>(a); break;
-    default: return cudaErrorInvalidValue;
+    case 0: return dequantize_kernel<FMT, 0, BF>;
+    case 16: return dequantize_kernel<FMT, 16, BF>;
+    case 32: return dequantize_kernel<FMT, 32, BF>;
+    case 64: return dequantize_kernel<FMT, 64, BF>;
+    case 128: return dequantize_kernel<FMT, 128, BF>;
     }
-    return cudaGetLastError();
+    return nullptr;
 }
 
 cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
@@ -493,9 +504,11 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
     a.ck = ck;
     if (a.total_units == 0) return cudaSuccess;
     const int grid = grid_for(a.total_units, sms, DUNITS);
-    if (fmt == FP4_MXFP4)
-        return bf16out ? launch_deq_fmt<FP4_MXFP4, 1>(a, hk, grid, st) : launch_deq_fmt<FP4_MXFP4, 0>(a, hk, grid, st);
-    return bf16out ? launch_deq_fmt<FP4_NVFP4, 1>(a, hk, grid, st) : launch_deq_fmt<FP4_NVFP4, 0>(a, hk, grid, st);
+    void (*k)(DequantArgs) = (fmt == FP4_MXFP4)
+                                 ? (bf16out ? deq_kernel_for<FP4_MXFP4, 1>(hk) : deq_kernel_for<FP4_MXFP4, 0>(hk))
+                                 : (bf16out ? deq_kernel_for<FP4_NVFP4, 1>(hk) : deq_kernel_for<FP4_NVFP4, 0>(hk));
+    if (!k) return cudaErrorInvalidValue;
+    return launch_k(k, dim3(grid), dim3(256), 0, st, false, a);
 }
 
 }  // namespace fp4
