@@ -29,6 +29,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 ROWS, COLS = 1024, 131072
+
+# DRAM bytes (read + write) per launch of the roofline kernel at 1024 x 131072,
+# from the ncu capture summarised in profiles/quantize_kernel_mx_512x131072_full.md
+# (512-row capture scaled by rows).  Set to None whenever that kernel changes,
+# until it is captured again.
+QUANT_MX_TRAFFIC_BYTES = 306.4e6
 WORKLOAD = "quantize sweep 1024x131072 bf16 Student-t(3)+1% outliers x20: MXFP4 + NVFP4 quantize and dequantize"
 METRIC = "FP4 quantize GB/s (% HBM peak)"
 
@@ -373,7 +379,7 @@ def run_ours(args):
     achieved = sb[dom] / (per[dom] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "quantize_kernel<MXFP4,k=0>", "achieved": achieved, "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": None,
+                "traffic": QUANT_MX_TRAFFIC_BYTES if rows == ROWS else None,
                 "per_call_ms": per,
                 "per_call_gbs": {n: sb[n] / (per[n] * 1e-3) / 1e9 for n in names}}
 
