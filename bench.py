@@ -91,6 +91,35 @@ def time_graph(torch, fn, warmup: int, reps: int):
     return e0.elapsed_time(e1) / reps
 
 
+def bench_rotate(torch, fp4, inputs, dev, reps: int):
+    """Fused rotate + quantize of 8192x4096 bf16 activations (Laplace(0,1), 1%
+    outlier channels x50), k in {0,16,32,64,128}, MXFP4 and NVFP4.  Four input
+    copies are rotated so every call reads x from HBM (one copy fits in L2).
+    Bytes per element: read 2 + nibbles 0.5 + scales 1/32 (MX) or 1/16 (NV);
+    the NVFP4 amax pass re-reads x from L2 and is not counted."""
+    hbm, kind = peaks()
+    x = inputs.rotate_acts()
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    copies = [xd.clone() for _ in range(4)]
+    n = xd.numel()
+    res = {"peak_gbs": hbm, "peak_kind": kind, "workload": "rotate+quantize 8192x4096 bf16", "cases": {}}
+    for fmt, name, bpe in ((fp4.FP4_MXFP4, "mxfp4", 2 + 0.5 + 1 / 32), (fp4.FP4_NVFP4, "nvfp4", 2 + 0.5 + 1 / 16)):
+        outs = fp4.quantize(xd, fmt)
+        for k in (0, 16, 32, 64, 128):
+            it = [0]
+
+            def call():
+                fp4.quantize(copies[it[0] % 4], fmt, hadamard_k=k, out=outs)
+                it[0] += 1
+
+            ms = time_graph(torch, call, 3, reps * 4)
+            gbs = n * bpe / (ms * 1e-3) / 1e9
+            res["cases"][f"{name}_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
+    del copies, xd
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_decode(torch, fp4, inputs, dev, reps: int):
     """Decode shapes: M in {1,4,16} bf16 activations quantized online inside
     the timed call (fp4_linear), W 14336x4096 and 4096x14336 pre-quantized,
@@ -297,6 +326,8 @@ def run_ours(args):
         # profiling helper: one leg alone, no JSON contract
         if args.only == "prefill":
             r = bench_prefill(torch, fp4, inputs, dev, reps=args.steps, M=args.prefill_m, fmts=args.fmts)
+        elif args.only == "rotate":
+            r = bench_rotate(torch, fp4, inputs, dev, reps=args.steps)
         else:
             r = bench_decode(torch, fp4, inputs, dev, reps=args.steps)
         print(json.dumps({"only": args.only, "result": r}), flush=True)
@@ -425,6 +456,7 @@ def run_ours(args):
     if not args.no_gemm:
         gemm = {"prefill": bench_prefill(torch, fp4, inputs, dev, reps=10),
                 "decode": bench_decode(torch, fp4, inputs, dev, reps=10)}
+    rotate = None if args.no_gemm else bench_rotate(torch, fp4, inputs, dev, reps=10)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -453,6 +485,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": int(launches),
         "gemm": gemm,
+        "rotate_quantize": rotate,
         "nmse": nmse_vals,
         "clocks": clk.summary(),
     }
@@ -469,7 +502,7 @@ def main():
     ap.add_argument("--rows", type=int, default=ROWS, help="rows of the tensor (profiling runs use fewer)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gemm", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "rotate"], default=None,
                     help="profiling helper: run one GEMM leg alone")
     ap.add_argument("--prefill-m", type=int, default=8192)
     ap.add_argument("--fmts", nargs="*", default=None)

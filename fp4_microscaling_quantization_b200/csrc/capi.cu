@@ -18,7 +18,10 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
                         const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K,
                         int fmt, int bf16out, void *C, int64_t ldc, void *ws, size_t ws_bytes,
-                        int sms, cudaStream_t st, int *timeout_flag_out, bool pdl);
+                        int sms, cudaStream_t st, int *timeout_flag_out, bool pdl, unsigned *counters);
+cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int hk, float ck,
+                                int round_away, int mx_floor, int gscale_given, uint8_t *q, uint8_t *s, float *gscale,
+                                unsigned *zero, int nzero, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int sms);
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
 static std::atomic<uint64_t> g_launches{0};
@@ -148,7 +151,7 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const
     int bad = 0;
     cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16,
                                      C, ldc, workspace, ws_bytes, sms,
-                                     static_cast<cudaStream_t>(stream), &bad, false);
+                                     static_cast<cudaStream_t>(stream), &bad, false, nullptr);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
@@ -157,7 +160,7 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const
 
 namespace {
 struct LinearLayout {
-    size_t aq, as, ga, gemm, total;
+    size_t aq, as, ga, gemm, counters, total;
 };
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
@@ -170,7 +173,9 @@ LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, int fmt, int sms)
     L.as = round256((size_t)(M * (K / 2)));
     L.ga = L.as + round256((size_t)(((M + 127) / 128 * 128) * ((nkb + 3) / 4 * 4)));
     L.gemm = L.ga + 256;
-    L.total = L.gemm + round256(fp4::gemm_workspace_bytes(M, N, K, fmt, sms));
+    L.counters = L.gemm + round256(fp4::gemm_workspace_bytes(M, N, K, fmt, sms));
+    // per-tile arrival counters of the decode kernel's fused reduction
+    L.total = L.counters + round256((size_t)((N + 127) / 128) * sizeof(unsigned));
     return L;
 }
 }  // namespace
@@ -212,14 +217,25 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     uint8_t *aq = base + L.aq, *as = base + L.as;
     float *ga = (fmt == FP4_NVFP4 && gA) ? const_cast<float *>(gA) : reinterpret_cast<float *>(base + L.ga);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = fp4::launch_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
-                                         hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
-                                         o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, sms, st,
-                                         true);
+    const bool decode = M <= 16;
+    unsigned *counters = decode ? reinterpret_cast<unsigned *>(base + L.counters) : nullptr;
+    cudaError_t e;
+    if (decode) {
+        // two launches: one cluster quantizes the activations (and zeroes the
+        // tile counters); the split-K kernel streams W meanwhile and reduces.
+        e = fp4::launch_act_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
+                                     hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
+                                     o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, counters,
+                                     (int)((N + 127) / 128), st);
+    } else {
+        e = fp4::launch_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
+                                 hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
+                                 o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, sms, st, true);
+    }
     if (e != cudaSuccess) return FP4_ERR_CUDA;
     int bad = 0;
     e = fp4::launch_gemm(aq, as, ga, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc, base + L.gemm,
-                         L.total - L.gemm, sms, st, &bad, true);
+                         L.counters - L.gemm, sms, st, &bad, true, counters);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

@@ -311,6 +311,13 @@ struct Params {
     const uint8_t *Ws;   // W scales (N rows)
     const uint8_t *As;   // activation scales (M rows, padded to 128)
     float *ws;           // partials: [G][maxseg][128][16]
+    // Fused reduction (counters != nullptr): per-tile arrival counters, zero
+    // on entry; the last CTA to finish a tile sums its partials and stores C.
+    unsigned *counters;
+    const float *gA, *gW;
+    void *C;
+    int64_t ldc;
+    int bf16out;
     int N, M, K;
     int nk;              // K / BK
     int ntiles;          // ceil(N / 128)
@@ -320,6 +327,22 @@ struct Params {
 };
 
 __host__ __device__ inline int64_t unit_begin(int c, int64_t U, int G) { return (int64_t)c * U / G; }
+// The CTA whose unit range contains unit u.
+__host__ __device__ inline int unit_owner(int64_t u, int64_t U, int G) { return (int)(((u + 1) * G + U - 1) / U) - 1; }
+
+// C[m][n] for the m < M activation rows of one output row n.
+FP4_DEV void store_row(const Params &p, int n, const float *acc, float alpha)
+{
+#pragma unroll
+    for (int m = 0; m < BNA; m++) {
+        if (m >= p.M) break;
+        const float v = __fmul_rn(acc[m], alpha);
+        if (p.bf16out)
+            reinterpret_cast<__nv_bfloat16 *>(p.C)[(int64_t)m * p.ldc + n] = __float2bfloat16_rn(v);
+        else
+            reinterpret_cast<float *>(p.C)[(int64_t)m * p.ldc + n] = v;
+    }
+}
 
 template <int FMT>
 __global__ void __launch_bounds__(192, 1)
@@ -331,6 +354,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     // bars: full[S], empty[S], accfull[2], accempty[2], drain
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    __shared__ volatile unsigned s_last;
     volatile uint32_t *abort_flag = tmem_slot + 1;
 
     grid_dep_launch();
@@ -475,11 +499,53 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         tc_fence_before();
         __syncwarp();
         if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");
-        float4 *dst = reinterpret_cast<float4 *>(p.ws + (((int64_t)c * p.maxseg + seg) * 128 + quarter * 32 + lane) * 16);
+        const int t = t_first + seg;
+        const int row = quarter * 32 + lane;  // row of the W tile = output column n
+        const int n = t * BMW + row;
+        const int c_lo = unit_owner((int64_t)t * p.nk, U, p.G), c_hi = unit_owner((int64_t)(t + 1) * p.nk - 1, U, p.G);
+        if (p.counters && c_lo == c_hi) {
+            // the whole K range of this tile is ours: store C directly
+            float acc[BNA];
+#pragma unroll
+            for (int m = 0; m < BNA; m++) acc[m] = __fadd_rn(0.0f, __uint_as_float(r[m]));
+            if (n < p.N) store_row(p, n, acc, (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
+            continue;
+        }
+        float4 *dst = reinterpret_cast<float4 *>(p.ws + (((int64_t)c * p.maxseg + seg) * 128 + row) * 16);
 #pragma unroll
         for (int q = 0; q < 4; q++)
             dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
                                  __uint_as_float(r[4 * q + 3]));
+        if (p.counters) {
+            // Fused reduction: the last of the tile's c_hi - c_lo + 1 CTAs to get
+            // here sums every partial in CTA order (the same order as
+            // reduce_kernel, so results do not depend on which CTA is last).
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (threadIdx.x == 64) s_last = (atomicAdd(&p.counters[t], 1u) == (unsigned)(c_hi - c_lo)) ? 1u : 0u;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (s_last) {
+                __threadfence();
+                float acc[BNA];
+#pragma unroll
+                for (int m = 0; m < BNA; m++) acc[m] = 0.0f;
+                for (int cc = c_lo; cc <= c_hi; cc++) {
+                    const int sg = t - (int)(unit_begin(cc, U, p.G) / p.nk);
+                    const float4 *src = reinterpret_cast<const float4 *>(p.ws + (((int64_t)cc * p.maxseg + sg) * 128 + row) * 16);
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        const float4 v = __ldcg(src + q);
+                        acc[4 * q] = __fadd_rn(acc[4 * q], v.x);
+                        acc[4 * q + 1] = __fadd_rn(acc[4 * q + 1], v.y);
+                        acc[4 * q + 2] = __fadd_rn(acc[4 * q + 2], v.z);
+                        acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
+                    }
+                }
+                if (n < p.N) store_row(p, n, acc, (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
+                if (threadIdx.x == 64) p.counters[t] = 0u;  // ready for the next call
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // s_last is reused by the next segment
+        }
     }
     }
     tc_fence_before();
@@ -494,17 +560,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
 }
 
 // C[m][n] = alpha * sum over the CTAs that own a part of n's tile, in CTA order.
-template <int BF16OUT, int FMT>
-__global__ void __launch_bounds__(128) reduce_kernel(Params p, const float *gA, const float *gW, void *C, int64_t ldc)
+template <int FMT>
+__global__ void __launch_bounds__(128) reduce_kernel(Params p)
 {
     grid_dep_wait();
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     if (n >= p.N) return;
-    const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*gA, *gW) : 1.0f;
+    const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
     const int t = n / BMW, r = n % BMW;
     const int64_t U = (int64_t)p.ntiles * p.nk;
-    auto owner = [&](int64_t u) { return (int)(((u + 1) * p.G + U - 1) / U) - 1; };
-    const int c_lo = owner((int64_t)t * p.nk), c_hi = owner((int64_t)(t + 1) * p.nk - 1);
+    const int c_lo = unit_owner((int64_t)t * p.nk, U, p.G), c_hi = unit_owner((int64_t)(t + 1) * p.nk - 1, U, p.G);
     float acc[BNA];
 #pragma unroll
     for (int m = 0; m < BNA; m++) acc[m] = 0.0f;
@@ -520,15 +585,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(Params p, const float *gA, 
             acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
         }
     }
-#pragma unroll
-    for (int m = 0; m < BNA; m++) {
-        if (m >= p.M) break;
-        const float v = __fmul_rn(acc[m], alpha);
-        if (BF16OUT)
-            reinterpret_cast<__nv_bfloat16 *>(C)[(int64_t)m * ldc + n] = __float2bfloat16_rn(v);
-        else
-            reinterpret_cast<float *>(C)[(int64_t)m * ldc + n] = v;
-    }
+    store_row(p, n, acc, alpha);
 }
 
 struct Plan {
@@ -665,9 +722,9 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
     return decode::plan(M, N, K, sms).ws_bytes;
 }
 
-template <int FMT, int BF>
-static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const decode::Params &p, const float *gA,
-                                 const float *gW, void *C, int64_t ldc, cudaStream_t st, bool pdl)
+template <int FMT>
+static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const decode::Params &p, cudaStream_t st,
+                                 bool pdl)
 {
     auto kern = decode::decode_kernel<FMT>;
     static bool attr_set = false;
@@ -677,15 +734,14 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
         attr_set = true;
     }
     cudaError_t e = launch_k(kern, dim3(p.G), dim3(192), decode::SMEM_BYTES, st, pdl, tw, ta, p);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || p.counters) return e;
     // the reduction waits for the split-K kernel inside (grid_dep_wait)
-    return launch_k(decode::reduce_kernel<BF, FMT>, dim3((p.N + 127) / 128), dim3(128), 0, st, true, p, gA, gW, C,
-                    ldc);
+    return launch_k(decode::reduce_kernel<FMT>, dim3((p.N + 127) / 128), dim3(128), 0, st, true, p);
 }
 
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
                         const float *gW, int64_t M, int64_t N, int64_t K, int fmt, int bf16out, void *C, int64_t ldc,
-                        void *ws, size_t ws_bytes, int sms, cudaStream_t st, int *bad, bool pdl)
+                        void *ws, size_t ws_bytes, int sms, cudaStream_t st, int *bad, bool pdl, unsigned *counters)
 {
     if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) {
         *bad = 1;
@@ -712,11 +768,13 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.G = pl.G;
         dp.maxseg = pl.maxseg;
         dp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
-        if (fmt == FP4_MXFP4)
-            return bf16out ? launch_decode<FP4_MXFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st, pdl)
-                           : launch_decode<FP4_MXFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st, pdl);
-        return bf16out ? launch_decode<FP4_NVFP4, 1>(tw, ta, dp, gA, gW, C, ldc, st, pdl)
-                       : launch_decode<FP4_NVFP4, 0>(tw, ta, dp, gA, gW, C, ldc, st, pdl);
+        dp.counters = counters;
+        dp.gA = gA;
+        dp.gW = gW;
+        dp.C = C;
+        dp.ldc = ldc;
+        dp.bf16out = bf16out;
+        return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4>(tw, ta, dp, st, pdl) : launch_decode<FP4_NVFP4>(tw, ta, dp, st, pdl);
     }
     {
         PParams pp;
@@ -816,7 +874,7 @@ extern "C" fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *
     int bad = 0;
     const cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc,
                                            scratch, fp4::kNoAllocScratchBytes, sms,
-                                           static_cast<cudaStream_t>(stream), &bad, false);
+                                           static_cast<cudaStream_t>(stream), &bad, false, nullptr);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

@@ -15,7 +15,7 @@
 // the last butterfly stages exchange values with shuffles.  Warps walk the
 // tensor in a grid-stride loop of 32 consecutive units, so neighbouring
 // lanes read and write neighbouring memory.
-#include "common.cuh"
+#include "sm100.cuh"
 
 namespace fp4 {
 
@@ -106,6 +106,55 @@ FP4_DEV float read_global_scale(const float *g, int computed)
 {
     float v = *g;
     return computed ? nv_global_from_amax(v) : v;
+}
+
+// Scale and element encoding of one rotated 32-element unit u, and the stores
+// of its nibbles and scale byte(s) (TransFP4 Eq.(1): MXFP4 power-of-two
+// scale; NVFP4 E4M3 block scale under the tensor scale sg).
+template <int FMT>
+FP4_DEV void encode_store_unit(float *v, int64_t u, const QuantArgs &a, float sg, float six_sg)
+{
+    const int64_t row = u / a.units_per_row;
+    const int64_t j = u - row * a.units_per_row;
+    if (FMT == FP4_MXFP4) {
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+        const int e = mx_exponent(amax, a.mx_floor);
+        const float inv = exp2i(-e);
+#pragma unroll
+        for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
+        a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)(e + 127);
+    } else {
+        uint32_t sb2 = 0;
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[16 * b + i]));
+            const float t = __fdiv_rn(amax, six_sg);
+            const uint32_t sb = e4m3_rn(t);
+            const float d = __fmul_rn(sg, e4m3_to_f32(sb));
+            const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
+#pragma unroll
+            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
+            sb2 |= sb << (8 * b);
+        }
+        *reinterpret_cast<uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4)) = (uint16_t)sb2;
+    }
+    uint4 out;
+    if (!a.round_away) {
+        out.x = e2m1x8_rn(v + 0);
+        out.y = e2m1x8_rn(v + 8);
+        out.z = e2m1x8_rn(v + 16);
+        out.w = e2m1x8_rn(v + 24);
+    } else {
+        out.x = e2m1x8_away(v + 0);
+        out.y = e2m1x8_away(v + 8);
+        out.z = e2m1x8_away(v + 16);
+        out.w = e2m1x8_away(v + 24);
+    }
+    *reinterpret_cast<uint4 *>(a.q + row * a.q_row_bytes + j * 16) = out;
 }
 
 // ---------------------------------------------------------------------------
@@ -199,47 +248,99 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
             if (HK) fwht_unit<HK>(v, a.ck, lane);
             if (!live) continue;
 
-            const int64_t row = u / a.units_per_row;
-            const int64_t j = u - row * a.units_per_row;
-            if (FMT == FP4_MXFP4) {
-                float amax = 0.0f;
+            encode_store_unit<FMT>(v, u, a, sg, six_sg);
+        }
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Activation quantization for the decode product (a few rows): one cluster of
+// ACT_CTAS CTAs quantizes the whole tensor in a single launch.  For NVFP4
+// with a computed tensor scale the CTAs exchange their partial maxima through
+// distributed shared memory, so no global scratch, memset or second kernel is
+// involved.  The kernel also zeroes `nzero` words at `zero` (the split-K
+// kernel's per-tile arrival counters) and writes no scale padding (the GEMM
+// never reads scales of rows past the tensor).
+constexpr int ACT_CTAS = 8, ACT_THREADS = 256;
+
+template <int FMT, int HK>
+__global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, unsigned *zero, int nzero)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    __shared__ float red[ACT_THREADS / 32];
+    __shared__ float cta_max;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (blockIdx.x * (int64_t)ACT_THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * ACT_THREADS) >> 5;
+    for (int i = blockIdx.x * ACT_THREADS + threadIdx.x; i < nzero; i += gridDim.x * ACT_THREADS) zero[i] = 0u;
+
+    float sg = 1.0f;
+    if (FMT == FP4_NVFP4) {
+        if (a.gscale_computed) {
+            float m = 0.0f;
+            for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
+                uint4 raw[QUNITS][4];
 #pragma unroll
-                for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
-                const int e = mx_exponent(amax, a.mx_floor);
-                const float inv = exp2i(-e);
+                for (int i = 0; i < QUNITS; i++) {
+                    const int64_t u = base + i * 32 + lane;
+                    if (u < a.total_units) {
+                        fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
+                    } else {
 #pragma unroll
-                for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
-                a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)(e + 127);
-            } else {
-                uint32_t sb2 = 0;
-#pragma unroll
-                for (int b = 0; b < 2; b++) {
-                    float amax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[16 * b + i]));
-                    const float t = __fdiv_rn(amax, six_sg);
-                    const uint32_t sb = e4m3_rn(t);
-                    const float d = __fmul_rn(sg, e4m3_to_f32(sb));
-                    const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
-#pragma unroll
-                    for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
-                    sb2 |= sb << (8 * b);
+                        for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
+                    }
                 }
-                *reinterpret_cast<uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4)) = (uint16_t)sb2;
+#pragma unroll
+                for (int i = 0; i < QUNITS; i++) {
+                    float v[32];
+                    unpack_unit(raw[i], v);
+                    if (HK) fwht_unit<HK>(v, a.ck, lane);
+#pragma unroll
+                    for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+                }
             }
-            uint4 out;
-            if (!a.round_away) {
-                out.x = e2m1x8_rn(v + 0);
-                out.y = e2m1x8_rn(v + 8);
-                out.z = e2m1x8_rn(v + 16);
-                out.w = e2m1x8_rn(v + 24);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+            if (lane == 0) red[threadIdx.x >> 5] = m;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float b = red[0];
+                for (int w = 1; w < ACT_THREADS / 32; w++) b = fmaxf(b, red[w]);
+                cta_max = b;
+            }
+            cluster_sync();  // every CTA's partial maximum is in place
+            float t = 0.0f;
+            for (unsigned r = 0; r < gridDim.x; r++) t = fmaxf(t, ld_shared_cluster_f32(mapa_shared(smem_u32(&cta_max), r)));
+            cluster_sync();  // no CTA leaves while another still reads its shared memory
+            sg = nv_global_from_amax(t);
+            if (blockIdx.x == 0 && threadIdx.x == 0) *a.gscale = sg;
+        } else {
+            sg = *a.gscale;
+        }
+    }
+    const float six_sg = __fmul_rn(6.0f, sg);
+
+    for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
+        uint4 raw[QUNITS][4];
+#pragma unroll
+        for (int i = 0; i < QUNITS; i++) {
+            const int64_t u = base + i * 32 + lane;
+            if (u < a.total_units) {
+                fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
             } else {
-                out.x = e2m1x8_away(v + 0);
-                out.y = e2m1x8_away(v + 8);
-                out.z = e2m1x8_away(v + 16);
-                out.w = e2m1x8_away(v + 24);
+#pragma unroll
+                for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
             }
-            *reinterpret_cast<uint4 *>(a.q + row * a.q_row_bytes + j * 16) = out;
+        }
+#pragma unroll
+        for (int i = 0; i < QUNITS; i++) {
+            const int64_t u = base + i * 32 + lane;
+            float v[32];
+            unpack_unit(raw[i], v);
+            if (HK) fwht_unit<HK>(v, a.ck, lane);
+            if (u < a.total_units) encode_store_unit<FMT>(v, u, a, sg, six_sg);
         }
     }
 }
@@ -471,6 +572,58 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
             return err;
     }
     return cudaSuccess;
+}
+
+
+template <int FMT>
+static void (*act_kernel_for(int hk))(QuantArgs, unsigned *, int)
+{
+    switch (hk) {
+    case 0: return act_quant_kernel<FMT, 0>;
+    case 16: return act_quant_kernel<FMT, 16>;
+    case 32: return act_quant_kernel<FMT, 32>;
+    case 64: return act_quant_kernel<FMT, 64>;
+    case 128: return act_quant_kernel<FMT, 128>;
+    }
+    return nullptr;
+}
+
+// Single-launch quantization of a small activation tensor (see
+// act_quant_kernel); scale padding is left unwritten.
+cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int hk, float ck,
+                                int round_away, int mx_floor, int gscale_given, uint8_t *q, uint8_t *s, float *gscale,
+                                unsigned *zero, int nzero, cudaStream_t st)
+{
+    QuantArgs a;
+    a.x = x;
+    a.ld = ld;
+    a.units_per_row = cols / 32;
+    a.total_units = rows * (cols / 32);
+    const int64_t nkb = cols / (fmt == FP4_MXFP4 ? 32 : 16);
+    a.nkb4 = (nkb + 3) / 4;
+    a.q_row_bytes = cols / 2;
+    a.q = q;
+    a.s = s;
+    a.gscale = gscale;
+    a.ck = ck;
+    a.round_away = round_away;
+    a.mx_floor = mx_floor;
+    a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
+    void (*k)(QuantArgs, unsigned *, int) = (fmt == FP4_MXFP4) ? act_kernel_for<FP4_MXFP4>(hk) : act_kernel_for<FP4_NVFP4>(hk);
+    if (!k) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ACT_CTAS);
+    cfg.blockDim = dim3(ACT_THREADS);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ACT_CTAS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    count_launches(1);
+    return cudaLaunchKernelEx(&cfg, k, a, zero, nzero);
 }
 
 template <int FMT, int BF>

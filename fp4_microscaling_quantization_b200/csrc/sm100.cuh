@@ -327,3 +327,13 @@ FP4_DEV void st_global_v8(void *p, const uint32_t *w)
 }
 
 }  // namespace fp4
+
+namespace fp4 {
+// Load a float from the shared memory of another CTA of the cluster.
+FP4_DEV float ld_shared_cluster_f32(uint32_t addr_cluster)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr_cluster) : "memory");
+    return v;
+}
+}  // namespace fp4

@@ -314,3 +314,30 @@ def test_linear_static_activation_scale(fp4, orc):
     qa, sa, ga = orc.quantize(x, 1, gscale=gA)
     ref, bound = reference(orc, qa, sa, ga, qw, sw, gw, 1)
     assert_close(to_np(c), ref, bound, 0)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("M,N,K,hk", [(16, 14336, 4096, 0), (4, 4096, 14336, 0), (3, 40000, 256, 0),
+                                      (1, 300, 4096, 32), (16, 2048, 2048, 128)])
+def test_linear_decode_fused_reduction_matches_gemm(fp4, orc, fmt, M, N, K, hk):
+    """fp4_linear's decode path (one-cluster activation quantizer + split-K with
+    the reduction fused into the last CTA of each tile) gives bit-identical
+    results to fp4_quantize + fp4_gemm (separate reduction kernel): the partial
+    sums are added in the same CTA order.  Tiles with one and with several
+    contributing CTAs are both exercised; repeated calls are identical."""
+    import torch
+    a, w = inputs.decode_linear(M, N, K, seed=N + K)
+    xd = to_dev_bf16(a)
+    W = fp4.quantize(to_dev_bf16(w), fmt, hadamard_k=hk)
+    A = fp4.quantize(xd, fmt, hadamard_k=hk)
+    ref = fp4.gemm(A, W, M, N, K, fmt, out_dtype=0)
+    c1 = fp4.linear(xd, W, fmt, hadamard_k=hk, out_dtype=0)
+    c2 = fp4.linear(xd, W, fmt, hadamard_k=hk, out_dtype=0)
+    torch.cuda.synchronize()
+    fp4.check_device_status()
+    assert torch.equal(c1.view(torch.int32), ref.view(torch.int32))
+    assert torch.equal(c1.view(torch.int32), c2.view(torch.int32))
+    # bf16 output of the fused path equals the rounding of the fp32 one
+    cb = fp4.linear(xd, W, fmt, hadamard_k=hk, out_dtype=1)
+    torch.cuda.synchronize()
+    assert torch.equal(cb, c1.to(torch.bfloat16))
