@@ -93,14 +93,14 @@ def time_graph(torch, fn, warmup: int, reps: int):
 
 def bench_rotate(torch, fp4, inputs, dev, reps: int):
     """Fused rotate + quantize of 8192x4096 bf16 activations (Laplace(0,1), 1%
-    outlier channels x50), k in {0,16,32,64,128}, MXFP4 and NVFP4.  Four input
-    copies are rotated so every call reads x from HBM (one copy fits in L2).
+    outlier channels x50), k in {0,16,32,64,128}, MXFP4 and NVFP4.  Eight input
+    copies (537 MB) are rotated so every call reads x from HBM (one fits in L2).
     Bytes per element: read 2 + nibbles 0.5 + scales 1/32 (MX) or 1/16 (NV);
     the NVFP4 amax pass re-reads x from L2 and is not counted."""
     hbm, kind = peaks()
     x = inputs.rotate_acts()
     xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
-    copies = [xd.clone() for _ in range(4)]
+    copies = [xd.clone() for _ in range(8)]
     n = xd.numel()
     res = {"peak_gbs": hbm, "peak_kind": kind, "workload": "rotate+quantize 8192x4096 bf16", "cases": {}}
     for fmt, name, bpe in ((fp4.FP4_MXFP4, "mxfp4", 2 + 0.5 + 1 / 32), (fp4.FP4_NVFP4, "nvfp4", 2 + 0.5 + 1 / 16)):
@@ -109,10 +109,10 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int):
             it = [0]
 
             def call():
-                fp4.quantize(copies[it[0] % 4], fmt, hadamard_k=k, out=outs)
+                fp4.quantize(copies[it[0] % 8], fmt, hadamard_k=k, out=outs)
                 it[0] += 1
 
-            ms = time_graph(torch, call, 3, reps * 4)
+            ms = time_graph(torch, call, 3, reps * 8)
             gbs = n * bpe / (ms * 1e-3) / 1e9
             res["cases"][f"{name}_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
     del copies, xd

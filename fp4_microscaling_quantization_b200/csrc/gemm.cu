@@ -593,13 +593,20 @@ struct Plan {
     size_t ws_bytes;
 };
 
+// Work split: each W tile is cut into S equal K ranges with S the largest
+// count that keeps ntiles * S CTAs within one per SM, so tiles are split only
+// when there are fewer of them than SMs (S = 1: no partial sums at all).
 inline Plan plan(int64_t M, int64_t N, int64_t K, int sms)
 {
     Plan pl;
     pl.nk = (int)(K / BK);
     pl.ntiles = (int)((N + BMW - 1) / BMW);
     const int64_t U = (int64_t)pl.ntiles * pl.nk;
-    pl.G = (int)(U < sms ? U : sms);
+    int64_t split = sms / pl.ntiles;
+    if (split < 1) split = 1;
+    if (split > pl.nk) split = pl.nk;
+    const int64_t G = (int64_t)pl.ntiles * split;
+    pl.G = (int)(G < sms ? G : (U < sms ? U : sms));
     pl.maxseg = 1;
     for (int c = 0; c < pl.G; c++) {
         const int64_t a = unit_begin(c, U, pl.G), b = unit_begin(c + 1, U, pl.G);

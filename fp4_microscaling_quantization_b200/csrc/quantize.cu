@@ -202,6 +202,15 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
     }
 }
 
+// Clears the amax accumulator (a kernel rather than a memset node, so the
+// whole sequence stays on the compute engine).
+__global__ void zero_word_kernel(float *g)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    *g = 0.0f;
+}
+
 // Converts the tensor max left by amax_kernel into s_g = amax / (6 * 448)
 // (1 for an all-zero tensor).  Runs after the quantize kernel has read it.
 __global__ void finalize_gscale_kernel(float *g)
@@ -549,8 +558,8 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     cudaError_t err = cudaSuccess;
     bool first = true;  // the first launch of the sequence is ordered normally after earlier work
     if (a.gscale_computed) {
-        if ((err = cudaMemsetAsync(gscale, 0, sizeof(float), st)) != cudaSuccess) return err;
-        if ((err = launch_k(ak, dim3(grid), dim3(256), 0, st, false, a)) != cudaSuccess) return err;
+        if ((err = launch_k(zero_word_kernel, dim3(1), dim3(1), 0, st, false, gscale)) != cudaSuccess) return err;
+        if ((err = launch_k(ak, dim3(grid), dim3(256), 0, st, pdl, a)) != cudaSuccess) return err;
         first = false;
     }
     if (a.total_units > 0) {
