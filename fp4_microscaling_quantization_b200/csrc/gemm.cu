@@ -17,6 +17,7 @@
 // without storing.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "sm100.cuh"
@@ -75,6 +76,8 @@ struct PParams {
     int M, N, K;
     int nkb4;
     int num_m_tiles, num_n_tiles;
+    uint64_t budget_ns;  // limit of every mbarrier wait
+    int stall;           // failure-detection test: the producer issues no loads
 };
 
 template <int FMT, int BF16OUT, int CG>
@@ -131,7 +134,7 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     grid_dep_wait();  // operands may come from the preceding kernel
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !p.stall) {
             // ---------------- TMA producer ----------------
             const uint32_t tx = Cfg::A_BYTES + Cfg::B_BYTES + 3 * KA * 512;
             int it = 0;
@@ -145,7 +148,7 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 for (int ks = 0; ks < nk; ks++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error)) { stop = true; break; }
+                    if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) { stop = true; break; }
                     uint8_t *st = smem + s * Cfg::STAGE_BYTES;
                     const uint32_t fb = full0_lead + 8 * s;
                     if (CG == 1) mbar_arrive_expect_tx(fb, tx); else mbar_arrive_expect_tx_cluster(fb, tx);
@@ -167,14 +170,14 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             const uint16_t both = (uint16_t)((1u << CG) - 1u);
             for (int t = group; t < num_tiles; t += ngroups, tile_i++) {
                 if (tile_i > 0 &&
-                    !mbar_wait_bounded(acce, (uint32_t)((tile_i - 1) & 1), abort_flag, &g_gemm_error))
+                    !mbar_wait_bounded(acce, (uint32_t)((tile_i - 1) & 1), abort_flag, &g_gemm_error, p.budget_ns))
                     break;
                 tc_fence_after();
                 bool stop = false;
                 for (int ks = 0; ks < nk; ks++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error)) { stop = true; break; }
+                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) { stop = true; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
                     const uint32_t sb = sa + Cfg::A_BYTES;
@@ -182,13 +185,16 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     const uint32_t ssfb = ssfa + Cfg::SFA_BYTES;
                     const uint32_t tsfa = tmem + Cfg::SF_COL0 + s * Cfg::SF_STAGE_COLS;
                     const uint32_t tsfb = tsfa + 16;
-                    for (int a = 0; a < KA; a++) {
-                        tc_cp_scale_atom_cg<CG>(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
-                        tc_cp_scale_atom_cg<CG>(tsfb + 8 * a, smem_desc(ssfb + 512 * a, 0, 128, 0));
-                        tc_cp_scale_atom_cg<CG>(tsfb + 8 * a + 4, smem_desc(ssfb + KA * 512 + 512 * a, 0, 128, 0));
-                    }
 #pragma unroll
                     for (int kk = 0; kk < 4; kk++) {
+                        // copy each scale atom just before its first MMA, so the
+                        // copies of one atom overlap the MMA of the previous one
+                        if (FMT == FP4_NVFP4 || (kk & 1) == 0) {
+                            const int a = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
+                            tc_cp_scale_atom_cg<CG>(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
+                            tc_cp_scale_atom_cg<CG>(tsfb + 8 * a, smem_desc(ssfb + 512 * a, 0, 128, 0));
+                            tc_cp_scale_atom_cg<CG>(tsfb + 8 * a + 4, smem_desc(ssfb + KA * 512 + 512 * a, 0, 128, 0));
+                        }
                         const uint64_t ad = smem_desc(sa + 32 * kk, 16, 1024, 2);
                         const uint64_t bd = smem_desc(sb + 32 * kk, 16, 1024, 2);
                         const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
@@ -198,6 +204,13 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                                                        (tsfb + 8 * atom) | (sfid << 30), (ks | kk) ? 1u : 0u);
                     }
                     tc_commit_cg<CG>(empty0 + 8 * s, both);
+                }
+                if (stop && CG == 2) {
+                    // the peer CTA's epilogue must not store after an abort
+                    asm volatile("st.shared::cluster.u32 [%0], %1;\n\tfence.acq_rel.cluster;" ::"r"(
+                                     mapa_shared(smem_u32((const void *)abort_flag), 1)),
+                                 "r"(1u)
+                                 : "memory");
                 }
                 // the accumulator is ready (or, after an abort, no MMA is left in flight)
                 tc_commit_cg<CG>(accf, both);
@@ -213,7 +226,7 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         const bool aligned_c = (reinterpret_cast<uintptr_t>(p.C) & 31) == 0;
         int tile_i = 0;
         for (int t = group; t < num_tiles; t += ngroups, tile_i++) {
-            bool ok = !*abort_flag && mbar_wait_bounded(accf, (uint32_t)(tile_i & 1), abort_flag, &g_gemm_error);
+            bool ok = !*abort_flag && mbar_wait_bounded(accf, (uint32_t)(tile_i & 1), abort_flag, &g_gemm_error, p.budget_ns);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (!ok || *abort_flag) break;
             tc_fence_after();
@@ -318,6 +331,8 @@ struct Params {
     void *C;
     int64_t ldc;
     int bf16out;
+    uint64_t budget_ns;  // limit of every mbarrier wait
+    int stall;           // failure-detection test: the producer issues no loads
     int N, M, K;
     int nk;              // K / BK
     int ntiles;          // ceil(N / 128)
@@ -393,7 +408,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !p.stall) {
             const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
             auto load_w = [&](int64_t u, int s) {
                 const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
@@ -424,7 +439,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 const int64_t i = u - u0;
                 const int s = (int)(i % STAGES);
                 const uint32_t ph = (uint32_t)((i / STAGES) & 1);
-                if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error)) break;
+                if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) break;
                 mbar_arrive_expect_tx(full0 + 8 * s, tx);
                 load_w(u, s);
                 load_a(u, s);
@@ -432,7 +447,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             }
             for (int64_t i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++) {
                 volatile uint32_t no_abort = 0;
-                mbar_wait_bounded(full0 + 8 * (int)(i % STAGES), (uint32_t)((i / STAGES) & 1), &no_abort, &g_gemm_error);
+                mbar_wait_bounded(full0 + 8 * (int)(i % STAGES), (uint32_t)((i / STAGES) & 1), &no_abort, &g_gemm_error, p.budget_ns);
             }
         }
         __syncwarp();
@@ -449,10 +464,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 if (first) {
                     seg++;
                     if (seg >= 2 &&
-                        !mbar_wait_bounded(acce0 + 8 * (seg & 1), (uint32_t)(((seg >> 1) - 1) & 1), abort_flag, &g_gemm_error))
+                        !mbar_wait_bounded(acce0 + 8 * (seg & 1), (uint32_t)(((seg >> 1) - 1) & 1), abort_flag, &g_gemm_error, p.budget_ns))
                         break;
                 }
-                if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error)) break;
+                if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) break;
                 tc_fence_after();
                 const uint32_t acc = tmem + (uint32_t)(seg & 1) * BNA;
                 const uint32_t sw = smem_u32(smem + s * STAGE_BYTES);
@@ -489,7 +504,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     grid_dep_wait();
     for (int seg = 0; seg < nseg; seg++) {
         const int b = seg & 1;
-        bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error);
+        bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error, p.budget_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -554,7 +569,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         tc_fence_after();
         // every MMA has completed before TMEM is released (also on the abort path)
         volatile uint32_t no_abort = 0;
-        mbar_wait_bounded(drainb, 0, &no_abort, &g_gemm_error);
+        mbar_wait_bounded(drainb, 0, &no_abort, &g_gemm_error, p.budget_ns);
         tmem_dealloc(tmem, TMEM_COLS);
     }
 }
@@ -723,6 +738,12 @@ static int pgemm_cta_group(int64_t M) { return M > 128 ? 2 : 1; }
 
 constexpr int64_t kDecodeMaxM = 16;
 
+// Failure-detection test hook (fp4_test_inject_stall): consumed by the next
+// GEMM launch.
+static std::atomic<int> g_inject_stall{0};
+static std::atomic<uint64_t> g_inject_budget{0};
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;
+
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
 {
     if (M < 1 || M > kDecodeMaxM || N < 1 || K < decode::BK) return 0;
@@ -754,6 +775,9 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         *bad = 1;
         return cudaSuccess;
     }
+    const int stall = g_inject_stall.exchange(0);
+    uint64_t budget = g_inject_budget.exchange(0);
+    if (budget == 0) budget = kWaitBudgetNs;
     if (M <= kDecodeMaxM) {
         const decode::Plan pl = decode::plan(M, N, K, sms);
         if (!ws || ws_bytes < pl.ws_bytes) {
@@ -776,6 +800,8 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.maxseg = pl.maxseg;
         dp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
         dp.counters = counters;
+        dp.budget_ns = budget;
+        dp.stall = stall;
         dp.gA = gA;
         dp.gW = gW;
         dp.C = C;
@@ -793,6 +819,8 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         pp.N = (int)N;
         pp.K = (int)K;
         pp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+        pp.budget_ns = budget;
+        pp.stall = stall;
         const int cg = pgemm_cta_group(M);
         pp.num_m_tiles = (int)((M + 128 * cg - 1) / (128 * cg));
         pp.num_n_tiles = (int)((N + 255) / 256);
@@ -855,6 +883,13 @@ static cudaError_t noalloc_scratch(int dev, void **out)
 }
 
 }  // namespace fp4
+
+extern "C" fp4_status fp4_test_inject_stall(int stall, uint64_t budget_ns)
+{
+    fp4::g_inject_budget.store(budget_ns);
+    fp4::g_inject_stall.store(stall ? 1 : 0);
+    return FP4_OK;
+}
 
 extern "C" fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *As, const float *gA,
                                               const uint8_t *Wq, const uint8_t *Ws, const float *gW,

@@ -200,6 +200,16 @@ fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *As, const f
  * (host-side counter; diagnostics and launch accounting). */
 uint64_t fp4_kernel_launches(void);
 
+/* Failure-detection test hook.  With stall != 0 the next GEMM launch
+ * (fp4_gemm, fp4_linear or fp4_gemm_decode_noalloc) issues no operand loads,
+ * so its MMA warp's bounded wait gives up after budget_ns nanoseconds
+ * (0 = the default of 2 s): the kernel sets the device error word, stores
+ * nothing, frees its tensor memory and returns, and fp4_check_device_status()
+ * then reports FP4_ERR_TIMEOUT.  The context stays usable.  A nonzero
+ * budget_ns with stall == 0 only shortens the waits of the next launch.
+ * Host-side, applies to one launch; not for production use. */
+fp4_status fp4_test_inject_stall(int stall, uint64_t budget_ns);
+
 /* Reads and clears the device-side error word that kernels set when a
  * bounded wait gives up.  Synchronizes `stream`.  Returns FP4_ERR_TIMEOUT if
  * it was set, else FP4_OK (or FP4_ERR_CUDA). */
