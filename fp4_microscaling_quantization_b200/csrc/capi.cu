@@ -46,6 +46,10 @@ bool valid_fmt(int fmt, int block)
 
 bool valid_k(int k) { return k == 0 || k == 16 || k == 32 || k == 64 || k == 128; }
 
+// The streaming kernels index 32-element units with 32-bit integers: 2^32
+// units are 2^37 elements, more than device memory holds as bf16.
+bool too_many_units(int64_t rows, int64_t cols) { return cols > 0 && rows > ((int64_t(1) << 32) - 1) / (cols / 32 > 0 ? cols / 32 : 1); }
+
 // RN_fp32(1/sqrt(k)): the double quotient is within 2^-52 relative of the
 // exact value, far inside half an fp32 ulp, so rounding it once to fp32 gives
 // the correctly rounded constant.
@@ -92,6 +96,7 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
         return FP4_ERR_INVALID_ARG;
     if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
     const bool empty = rows == 0 || cols == 0;
     if (fmt == FP4_NVFP4 && !gscale) return FP4_ERR_INVALID_ARG;
     if (!empty && (!x || !q || !s)) return FP4_ERR_INVALID_ARG;
@@ -114,6 +119,7 @@ fp4_status fp4_dequantize(const uint8_t *q, const uint8_t *s, const float *gscal
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
     if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
     if (rows == 0 || cols == 0) return FP4_OK;
     if (!q || !s || !out || (fmt == FP4_NVFP4 && !gscale)) return FP4_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(s, 16) || !aligned(out, 16)) return FP4_ERR_ALIGNMENT;
@@ -204,6 +210,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
     if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (K % 256 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (too_many_units(M, K)) return FP4_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return FP4_OK;
     if (!x || !Wq || !Ws || !C || !workspace) return FP4_ERR_INVALID_ARG;
     if (fmt == FP4_NVFP4 && !gW) return FP4_ERR_INVALID_ARG;

@@ -47,6 +47,38 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
 
 constexpr float kFltMax = 3.40282346638528859812e+38f;
 
+// ---- division by a launch-invariant divisor ---------------------------------
+// q = floor(n / d) for 32-bit unsigned n and d >= 1 by one high multiply, a
+// subtract and two shifts: the round-up multiplier with one extra bit of
+// Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication" (PLDI 1994), section 4:
+//   l = ceil(log2 d),  m = floor(2^32 (2^l - d) / d) + 1,
+//   t = mulhi(m, n),   q = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0).
+// Exact for every n < 2^32.  The kernels use it for the row of a 32-element
+// unit (unit index / units per row), which a 64-bit division made the largest
+// integer cost of the streaming kernels.
+struct FastDiv {
+    uint32_t d, m, s1, s2;
+};
+
+inline FastDiv make_fastdiv(uint32_t d)
+{
+    uint32_t l = 0;
+    while ((1ull << l) < (uint64_t)d) l++;
+    FastDiv f;
+    f.d = d;
+    f.m = (uint32_t)(((1ull << 32) * ((1ull << l) - (uint64_t)d)) / d + 1);
+    f.s1 = l > 0 ? 1u : 0u;
+    f.s2 = l > 0 ? l - 1 : 0u;
+    return f;
+}
+
+FP4_DEV uint32_t fastdiv(uint32_t n, const FastDiv &f)
+{
+    const uint32_t t = __umulhi(n, f.m);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
 // ---- programmatic dependent launch -----------------------------------------
 // A kernel launched with programmatic stream serialization may start before
 // its predecessor in the stream has finished; it must call grid_dep_wait()

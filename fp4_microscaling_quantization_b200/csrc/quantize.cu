@@ -23,7 +23,8 @@ struct QuantArgs {
     const uint16_t *x;
     int64_t ld;             // row stride of x, elements
     int64_t units_per_row;  // cols / 32
-    int64_t total_units;    // rows * units_per_row
+    int64_t total_units;    // rows * units_per_row (< 2^32, checked by the launcher)
+    FastDiv upr_div;        // division by units_per_row
     int64_t nkb4;           // ceil(blocks per row / 4)
     int64_t q_row_bytes;    // cols / 2
     uint8_t *q;
@@ -40,12 +41,17 @@ struct QuantArgs {
 constexpr int QUNITS = 2;  // quantize / amax
 constexpr int DUNITS = 2;  // dequantize (16 bytes of nibbles per unit)
 
-// Raw bytes of one 32-element unit (4 x 16-byte loads, read-only path).
-FP4_DEV void fetch_unit(const uint16_t *x, int64_t ld, int64_t upr, int64_t u, uint4 *w)
+// Row and position in the row of unit u.
+FP4_DEV void unit_rc(int64_t u, const FastDiv &upr, uint32_t &row, uint32_t &j)
 {
-    const int64_t row = u / upr;
-    const int64_t j = u - row * upr;
-    const uint4 *p = reinterpret_cast<const uint4 *>(x + row * ld + j * 32);
+    row = fastdiv((uint32_t)u, upr);
+    j = (uint32_t)u - row * upr.d;
+}
+
+// Raw bytes of unit j of row `row` (4 x 16-byte loads, read-only path).
+FP4_DEV void fetch_unit(const uint16_t *x, int64_t ld, uint32_t row, uint32_t j, uint4 *w)
+{
+    const uint4 *p = reinterpret_cast<const uint4 *>(x + (int64_t)row * ld + (int64_t)j * 32);
 #pragma unroll
     for (int c = 0; c < 4; c++) w[c] = __ldg(p + c);
 }
@@ -112,10 +118,8 @@ FP4_DEV float read_global_scale(const float *g, int computed)
 // of its nibbles and scale byte(s) (TransFP4 Eq.(1): MXFP4 power-of-two
 // scale; NVFP4 E4M3 block scale under the tensor scale sg).
 template <int FMT>
-FP4_DEV void encode_store_unit(float *v, int64_t u, const QuantArgs &a, float sg, float six_sg)
+FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, const QuantArgs &a, float sg, float six_sg)
 {
-    const int64_t row = u / a.units_per_row;
-    const int64_t j = u - row * a.units_per_row;
     if (FMT == FP4_MXFP4) {
         float amax = 0.0f;
 #pragma unroll
@@ -154,7 +158,7 @@ FP4_DEV void encode_store_unit(float *v, int64_t u, const QuantArgs &a, float sg
         out.z = e2m1x8_away(v + 16);
         out.w = e2m1x8_away(v + 24);
     }
-    *reinterpret_cast<uint4 *>(a.q + row * a.q_row_bytes + j * 16) = out;
+    *reinterpret_cast<uint4 *>(a.q + u * 16) = out;  // q rows are contiguous: row * cols/2 + j * 16 = u * 16
 }
 
 // ---------------------------------------------------------------------------
@@ -171,11 +175,13 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
     float m = 0.0f;
     for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
         uint4 raw[QUNITS][4];
+        uint32_t row[QUNITS] = {}, col[QUNITS] = {};
 #pragma unroll
         for (int i = 0; i < QUNITS; i++) {
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
-                fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
+                unit_rc(u, a.upr_div, row[i], col[i]);
+                fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -238,11 +244,13 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
 
     for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
         uint4 raw[QUNITS][4];
+        uint32_t row[QUNITS] = {}, col[QUNITS] = {};
 #pragma unroll
         for (int i = 0; i < QUNITS; i++) {
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
-                fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
+                unit_rc(u, a.upr_div, row[i], col[i]);
+                fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -257,7 +265,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
             if (HK) fwht_unit<HK>(v, a.ck, lane);
             if (!live) continue;
 
-            encode_store_unit<FMT>(v, u, a, sg, six_sg);
+            encode_store_unit<FMT>(v, u, row[i], col[i], a, sg, six_sg);
         }
     }
 }
@@ -276,8 +284,11 @@ constexpr int ACT_CTAS = 8, ACT_THREADS = 256;
 template <int FMT, int HK>
 __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, unsigned *zero, int nzero)
 {
-    grid_dep_launch();
+    // Launched programmatically after the previous work in the stream.  The
+    // dependent split-K kernel streams W before it waits, so it may only start
+    // once everything before this kernel has finished: trigger after the wait.
     grid_dep_wait();
+    grid_dep_launch();
     __shared__ float red[ACT_THREADS / 32];
     __shared__ float cta_max;
     const int lane = threadIdx.x & 31;
@@ -291,11 +302,13 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
             float m = 0.0f;
             for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
                 uint4 raw[QUNITS][4];
+        uint32_t row[QUNITS] = {}, col[QUNITS] = {};
 #pragma unroll
                 for (int i = 0; i < QUNITS; i++) {
                     const int64_t u = base + i * 32 + lane;
                     if (u < a.total_units) {
-                        fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
+                        unit_rc(u, a.upr_div, row[i], col[i]);
+                        fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
                     } else {
 #pragma unroll
                         for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -333,11 +346,13 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
 
     for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
         uint4 raw[QUNITS][4];
+        uint32_t row[QUNITS] = {}, col[QUNITS] = {};
 #pragma unroll
         for (int i = 0; i < QUNITS; i++) {
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
-                fetch_unit(a.x, a.ld, a.units_per_row, u, raw[i]);
+                unit_rc(u, a.upr_div, row[i], col[i]);
+                fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -349,7 +364,7 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
             float v[32];
             unpack_unit(raw[i], v);
             if (HK) fwht_unit<HK>(v, a.ck, lane);
-            if (u < a.total_units) encode_store_unit<FMT>(v, u, a, sg, six_sg);
+            if (u < a.total_units) encode_store_unit<FMT>(v, u, row[i], col[i], a, sg, six_sg);
         }
     }
 }
@@ -385,7 +400,8 @@ struct DequantArgs {
     const uint8_t *s;
     const float *gscale;
     int64_t units_per_row;
-    int64_t total_units;
+    int64_t total_units;    // < 2^32, checked by the launcher
+    FastDiv upr_div;        // division by units_per_row
     int64_t nkb4;
     int64_t q_row_bytes;
     int64_t cols;
@@ -414,9 +430,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
             raw[i] = make_uint4(0, 0, 0, 0);
             sraw[i] = 0;
             if (u < a.total_units) {
-                const int64_t row = u / a.units_per_row;
-                const int64_t j = u - row * a.units_per_row;
-                raw[i] = __ldg(reinterpret_cast<const uint4 *>(a.q + row * a.q_row_bytes + j * 16));
+                uint32_t row, j;
+                unit_rc(u, a.upr_div, row, j);
+                raw[i] = __ldg(reinterpret_cast<const uint4 *>(a.q + u * 16));
                 sraw[i] = (FMT == FP4_MXFP4)
                               ? (uint32_t)__ldg(a.s + scale_offset(row, j, a.nkb4))
                               : (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(a.s + scale_offset(row, 2 * j, a.nkb4)));
@@ -541,6 +557,8 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     a.ld = ld;
     a.units_per_row = cols / 32;
     a.total_units = rows * (cols / 32);
+    if (a.total_units >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
+    a.upr_div = make_fastdiv((uint32_t)(a.units_per_row > 0 ? a.units_per_row : 1));
     const int64_t nkb = cols / (fmt == FP4_MXFP4 ? 32 : 16);
     a.nkb4 = (nkb + 3) / 4;
     a.q_row_bytes = cols / 2;
@@ -608,6 +626,8 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     a.ld = ld;
     a.units_per_row = cols / 32;
     a.total_units = rows * (cols / 32);
+    if (a.total_units >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
+    a.upr_div = make_fastdiv((uint32_t)(a.units_per_row > 0 ? a.units_per_row : 1));
     const int64_t nkb = cols / (fmt == FP4_MXFP4 ? 32 : 16);
     a.nkb4 = (nkb + 3) / 4;
     a.q_row_bytes = cols / 2;
@@ -624,13 +644,17 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     cfg.gridDim = dim3(ACT_CTAS);
     cfg.blockDim = dim3(ACT_THREADS);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = ACT_CTAS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // May start while the previous kernel drains (its launch latency is then
+    // hidden); the kernel waits for it before touching memory.
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     count_launches(1);
     return cudaLaunchKernelEx(&cfg, k, a, zero, nzero);
 }
@@ -658,6 +682,8 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
     a.gscale = gscale;
     a.units_per_row = cols / 32;
     a.total_units = rows * (cols / 32);
+    if (a.total_units >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
+    a.upr_div = make_fastdiv((uint32_t)(a.units_per_row > 0 ? a.units_per_row : 1));
     const int64_t nkb = cols / (fmt == FP4_MXFP4 ? 32 : 16);
     a.nkb4 = (nkb + 3) / 4;
     a.q_row_bytes = cols / 2;

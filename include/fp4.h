@@ -104,6 +104,9 @@ fp4_status fp4_quantize_sizes(int64_t rows, int64_t cols, int fmt, int block,
  *           gscale_given: read as s_g.  Otherwise written with
  *           s_g = amax(|H_k x|) / (6*448), or 1 for an all-zero tensor.
  * cols must be a multiple of 32 (also for NVFP4).  rows == 0 is a no-op.
+ * rows * cols / 32 must stay below 2^32 (FP4_ERR_UNSUPPORTED otherwise; the
+ * bound is above what device memory holds as bf16); the same holds for
+ * fp4_dequantize and for M * K in fp4_linear.
  */
 fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                         int fmt, int block, int hadamard_k, const fp4_opts *opts,

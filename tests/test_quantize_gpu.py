@@ -45,7 +45,7 @@ def check_quantize(fp4, orc, x, fmt, hk=0, tie=0, rule=0, gscale=None, x_dev=Non
     return q, s, g, (oq, os_, og)
 
 
-SHAPES = [(1, 32), (3, 96), (130, 512), (257, 1024), (64, 4096)]
+SHAPES = [(1, 32), (3, 96), (130, 512), (257, 1024), (64, 4096), (37, 3104), (5, 32736)]
 
 
 @pytest.mark.parametrize("shape", SHAPES)
