@@ -301,11 +301,19 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 // ---------------------------------------------------------------------------
 // Decode kernel (M <= 16): the weight stream dominates, so the roles swap: a
 // 128-row W tile is the MMA's M operand and the (up to 16) activation rows
-// are N = 16.  The (W tile, 256-wide K step) units are split evenly over the
-// SMs in tile-major order (stream-K); each CTA accumulates every tile segment
-// it owns in TMEM (two buffers, alternating) and writes the 128 x 16 fp32
-// partial to a workspace slot.  reduce_kernel then sums each output's partials
-// in a fixed CTA order (deterministic) and applies alpha.
+// are N = 16.  Work is cut into (W tile, 256-wide K step) units, and each CTA
+// accumulates the units it owns in TMEM (two buffers, alternating per tile).
+// Three ways to spread the tiles over the SMs (plan()):
+//   * whole tiles (ntiles <= SMs, no spare SMs for a split): one CTA per
+//     tile, C stored straight from the accumulator;
+//   * cluster split: each tile's K range is cut into S = 2, 4 or 8 slices,
+//     one CTA each, and the S CTAs form a thread-block cluster.  Every CTA
+//     leaves its 128 x 16 fp32 partial in shared memory and the cluster's
+//     first CTA sums them in rank order over distributed shared memory;
+//   * global split (very few tiles, or more tiles than SMs: stream-K over
+//     the units): partials go to a workspace and are summed in CTA order,
+//     either by the last CTA of the tile (per-tile arrival counters) or by
+//     reduce_kernel.
 namespace decode {
 
 constexpr int BMW = 128, BNA = 16, BK = 256;
@@ -319,6 +327,7 @@ constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 constexpr int TMEM_COLS = 512;
 constexpr int SF_COL0 = 32;                  // accumulators at columns [0,16) and [16,32)
 constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation scales 16 cols
+constexpr int MAX_CLUSTER = 8;               // portable cluster size
 
 struct Params {
     const uint8_t *Ws;   // W scales (N rows)
@@ -339,6 +348,7 @@ struct Params {
     int G;               // CTAs
     int maxseg;
     int nkb4;
+    int csize;           // > 1: the CTAs of a tile form a cluster of csize and reduce through DSMEM
 };
 
 __host__ __device__ inline int64_t unit_begin(int c, int64_t U, int G) { return (int64_t)c * U / G; }
@@ -371,6 +381,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
     __shared__ volatile unsigned s_last;
     volatile uint32_t *abort_flag = tmem_slot + 1;
+    // cluster split: this CTA's 128 x 16 partial, [4][128][4] floats (16-byte
+    // groups of one row's columns 4q..4q+3), in stage 0's W buffer, which no
+    // load or MMA touches once the accumulator is complete
+    float4 *part = reinterpret_cast<float4 *>(smem);
 
     grid_dep_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -382,6 +396,23 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
     const uint32_t accf0 = smem_u32(bars + 2 * STAGES), acce0 = smem_u32(bars + 2 * STAGES + 2);
     const uint32_t drainb = smem_u32(bars + 2 * STAGES + 4);
+    const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
+    const int64_t npre = (u1 - u0) < STAGES ? (u1 - u0) : STAGES;
+
+    auto load_w = [&](int64_t u, int st_i) {
+        const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
+        uint8_t *st = smem + st_i * STAGE_BYTES;
+        const uint32_t fb = full0 + 8 * st_i;
+        tma_load_2d(smem_u32(st), &tmW, ks * (BK / 2), t * BMW, fb);
+        bulk_load(smem_u32(st + W_BYTES + A_BYTES), p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+    };
+    auto load_a = [&](int64_t u, int st_i) {
+        const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
+        uint8_t *st = smem + st_i * STAGE_BYTES;
+        const uint32_t fb = full0 + 8 * st_i;
+        tma_load_2d(smem_u32(st + W_BYTES), &tmA, ks * (BK / 2), 0, fb);
+        bulk_load(smem_u32(st + W_BYTES + A_BYTES + SFW_BYTES), p.As + (int64_t)ks * KA * 512, KA * 512, fb);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
@@ -397,6 +428,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         fence_barrier_init();
         tma_prefetch_desc(&tmW);
         tma_prefetch_desc(&tmA);
+        // The weight stream depends on no earlier kernel (the one before may
+        // still be quantizing the activations): start it at once, while warp
+        // 1 allocates tensor memory.
+        if (!p.stall) {
+            for (int64_t i = 0; i < npre; i++) {
+                mbar_arrive_expect_tx(full0 + 8 * (int)i, tx);
+                load_w(u0 + i, (int)i);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -409,29 +449,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
 
     if (warp == 0) {
         if (lane == 0 && !p.stall) {
-            const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
-            auto load_w = [&](int64_t u, int s) {
-                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
-                uint8_t *st = smem + s * STAGE_BYTES;
-                const uint32_t fb = full0 + 8 * s;
-                tma_load_2d(smem_u32(st), &tmW, ks * (BK / 2), t * BMW, fb);
-                bulk_load(smem_u32(st + W_BYTES + A_BYTES), p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
-            };
-            auto load_a = [&](int64_t u, int s) {
-                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
-                uint8_t *st = smem + s * STAGE_BYTES;
-                const uint32_t fb = full0 + 8 * s;
-                tma_load_2d(smem_u32(st + W_BYTES), &tmA, ks * (BK / 2), 0, fb);
-                bulk_load(smem_u32(st + W_BYTES + A_BYTES + SFW_BYTES), p.As + (int64_t)ks * KA * 512, KA * 512, fb);
-            };
-            // The weight stream does not depend on the preceding kernel (which
-            // may still be quantizing the activations): fill the first stages
-            // with W, then wait for the activations.
-            const int64_t npre = (u1 - u0) < STAGES ? (u1 - u0) : STAGES;
-            for (int64_t i = 0; i < npre; i++) {
-                mbar_arrive_expect_tx(full0 + 8 * (int)i, tx);
-                load_w(u0 + i, (int)i);
-            }
             grid_dep_wait();
             for (int64_t i = 0; i < npre; i++) load_a(u0 + i, (int)i);
             int64_t issued = npre;
@@ -498,10 +515,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         }
         __syncwarp();
     } else {
-    // ---------------- epilogue warps 2-5: one partial per tile segment ----------------
+    // ---------------- epilogue warps 2-5: one result per tile segment ----------------
     // warp w may only read TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
     grid_dep_wait();
+    const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
     for (int seg = 0; seg < nseg; seg++) {
         const int b = seg & 1;
         bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error, p.budget_ns);
@@ -517,13 +535,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         const int t = t_first + seg;
         const int row = quarter * 32 + lane;  // row of the W tile = output column n
         const int n = t * BMW + row;
+        if (p.csize > 1) {
+            // cluster split (one segment per CTA): leave the partial for the
+            // cluster's first CTA
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+                part[q * 128 + row] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                                  __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+            continue;
+        }
         const int c_lo = unit_owner((int64_t)t * p.nk, U, p.G), c_hi = unit_owner((int64_t)(t + 1) * p.nk - 1, U, p.G);
-        if (p.counters && c_lo == c_hi) {
+        if (c_lo == c_hi) {
             // the whole K range of this tile is ours: store C directly
             float acc[BNA];
 #pragma unroll
             for (int m = 0; m < BNA; m++) acc[m] = __fadd_rn(0.0f, __uint_as_float(r[m]));
-            if (n < p.N) store_row(p, n, acc, (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
+            if (n < p.N) store_row(p, n, acc, alpha);
             continue;
         }
         float4 *dst = reinterpret_cast<float4 *>(p.ws + (((int64_t)c * p.maxseg + seg) * 128 + row) * 16);
@@ -556,7 +583,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                         acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
                     }
                 }
-                if (n < p.N) store_row(p, n, acc, (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
+                if (n < p.N) store_row(p, n, acc, alpha);
                 if (threadIdx.x == 64) p.counters[t] = 0u;  // ready for the next call
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");  // s_last is reused by the next segment
@@ -565,6 +592,34 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     }
     tc_fence_before();
     __syncthreads();
+    if (p.csize > 1) {
+        // Every partial of the cluster is in place once all its CTAs pass
+        // this barrier; the first CTA sums them in rank order (the CTA order
+        // of the global reduction) and stores C.  The second barrier keeps
+        // the other CTAs' shared memory alive until it has read it.  Both are
+        // reached on every path, the abort paths included.
+        cluster_sync();
+        if (cluster_ctarank() == 0 && warp >= 2) {
+            const int row = (warp & 3) * 32 + lane;
+            const int t = c / p.csize;
+            const int n = t * BMW + row;
+            float acc[BNA];
+#pragma unroll
+            for (int m = 0; m < BNA; m++) acc[m] = 0.0f;
+            for (int rk = 0; rk < p.csize; rk++) {
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const float4 v = ld_shared_cluster_f32x4(mapa_shared(smem_u32(part + q * 128 + row), (uint32_t)rk));
+                    acc[4 * q] = __fadd_rn(acc[4 * q], v.x);
+                    acc[4 * q + 1] = __fadd_rn(acc[4 * q + 1], v.y);
+                    acc[4 * q + 2] = __fadd_rn(acc[4 * q + 2], v.z);
+                    acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
+                }
+            }
+            if (n < p.N && !*abort_flag) store_row(p, n, acc, (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
+        }
+        cluster_sync();
+    }
     if (warp == 1) {
         tc_fence_after();
         // every MMA has completed before TMEM is released (also on the abort path)
@@ -574,7 +629,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     }
 }
 
-// C[m][n] = alpha * sum over the CTAs that own a part of n's tile, in CTA order.
+// C[m][n] = alpha * sum over the CTAs that own a part of n's tile, in CTA
+// order, for the tiles cut between CTAs (whole tiles were stored directly).
 template <int FMT>
 __global__ void __launch_bounds__(128) reduce_kernel(Params p)
 {
@@ -585,6 +641,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(Params p)
     const int t = n / BMW, r = n % BMW;
     const int64_t U = (int64_t)p.ntiles * p.nk;
     const int c_lo = unit_owner((int64_t)t * p.nk, U, p.G), c_hi = unit_owner((int64_t)(t + 1) * p.nk - 1, U, p.G);
+    if (c_lo == c_hi) return;
     float acc[BNA];
 #pragma unroll
     for (int m = 0; m < BNA; m++) acc[m] = 0.0f;
@@ -605,30 +662,46 @@ __global__ void __launch_bounds__(128) reduce_kernel(Params p)
 
 struct Plan {
     int G, maxseg, nk, ntiles;
+    int csize;       // cluster split: CTAs per tile (1: not a cluster split)
+    bool any_cut;    // some tile is cut between CTAs outside a cluster (global reduction)
     size_t ws_bytes;
 };
 
-// Work split: each W tile is cut into S equal K ranges with S the largest
-// count that keeps ntiles * S CTAs within one per SM, so tiles are split only
-// when there are fewer of them than SMs (S = 1: no partial sums at all).
+// Work split (see the comment above the kernel):
+//   ntiles > SMs          stream-K: G = SMs CTAs over the units;
+//   ntiles <= SMs / 16    global split: S = min(SMs / ntiles, nk) slices per tile;
+//   otherwise             S = the largest power of two <= 8 with ntiles * S
+//                         <= SMs (and S <= nk); S > 1 is a cluster split.
 inline Plan plan(int64_t M, int64_t N, int64_t K, int sms)
 {
     Plan pl;
     pl.nk = (int)(K / BK);
     pl.ntiles = (int)((N + BMW - 1) / BMW);
+    pl.csize = 1;
     const int64_t U = (int64_t)pl.ntiles * pl.nk;
-    int64_t split = sms / pl.ntiles;
-    if (split < 1) split = 1;
-    if (split > pl.nk) split = pl.nk;
-    const int64_t G = (int64_t)pl.ntiles * split;
-    pl.G = (int)(G < sms ? G : (U < sms ? U : sms));
+    if (pl.ntiles > sms) {
+        pl.G = (int)(U < sms ? U : sms);
+    } else if ((int64_t)pl.ntiles * 2 * MAX_CLUSTER <= sms) {
+        int64_t split = sms / pl.ntiles;
+        if (split > pl.nk) split = pl.nk;
+        pl.G = (int)(pl.ntiles * split);
+    } else {
+        int split = 1;
+        while (split * 2 <= MAX_CLUSTER && (int64_t)pl.ntiles * split * 2 <= sms && split * 2 <= pl.nk) split *= 2;
+        pl.G = pl.ntiles * split;
+        pl.csize = split;
+    }
     pl.maxseg = 1;
     for (int c = 0; c < pl.G; c++) {
         const int64_t a = unit_begin(c, U, pl.G), b = unit_begin(c + 1, U, pl.G);
         const int segs = (int)((b - 1) / pl.nk - a / pl.nk + 1);
         if (segs > pl.maxseg) pl.maxseg = segs;
     }
-    pl.ws_bytes = (size_t)pl.G * pl.maxseg * 128 * BNA * sizeof(float);
+    pl.any_cut = false;
+    if (pl.csize == 1)
+        for (int t = 0; t < pl.ntiles && !pl.any_cut; t++)
+            pl.any_cut = unit_owner((int64_t)t * pl.nk, U, pl.G) != unit_owner((int64_t)(t + 1) * pl.nk - 1, U, pl.G);
+    pl.ws_bytes = pl.any_cut ? (size_t)pl.G * pl.maxseg * 128 * BNA * sizeof(float) : 0;
     (void)M;
     return pl;
 }
@@ -751,8 +824,8 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
 }
 
 template <int FMT>
-static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const decode::Params &p, cudaStream_t st,
-                                 bool pdl)
+static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const decode::Params &p, bool any_cut,
+                                 cudaStream_t st, bool pdl)
 {
     auto kern = decode::decode_kernel<FMT>;
     static bool attr_set = false;
@@ -761,8 +834,30 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    cudaError_t e = launch_k(kern, dim3(p.G), dim3(192), decode::SMEM_BYTES, st, pdl, tw, ta, p);
-    if (e != cudaSuccess || p.counters) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.G);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = decode::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (p.csize > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = p.csize;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        na++;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        na++;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    count_launches(1);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, ta, p);
+    if (e != cudaSuccess || p.counters || !any_cut) return e;
     // the reduction waits for the split-K kernel inside (grid_dep_wait)
     return launch_k(decode::reduce_kernel<FMT>, dim3((p.N + 127) / 128), dim3(128), 0, st, true, p);
 }
@@ -780,7 +875,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
     if (budget == 0) budget = kWaitBudgetNs;
     if (M <= kDecodeMaxM) {
         const decode::Plan pl = decode::plan(M, N, K, sms);
-        if (!ws || ws_bytes < pl.ws_bytes) {
+        if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes)) {
             *bad = 1;
             return cudaSuccess;
         }
@@ -798,6 +893,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.ntiles = pl.ntiles;
         dp.G = pl.G;
         dp.maxseg = pl.maxseg;
+        dp.csize = pl.csize;
         dp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
         dp.counters = counters;
         dp.budget_ns = budget;
@@ -807,7 +903,8 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.C = C;
         dp.ldc = ldc;
         dp.bf16out = bf16out;
-        return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4>(tw, ta, dp, st, pdl) : launch_decode<FP4_NVFP4>(tw, ta, dp, st, pdl);
+        return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4>(tw, ta, dp, pl.any_cut, st, pdl)
+                                : launch_decode<FP4_NVFP4>(tw, ta, dp, pl.any_cut, st, pdl);
     }
     {
         PParams pp;

@@ -33,7 +33,7 @@ struct QuantArgs {
     float ck;               // RN(1/sqrt(k)) of the rotation
     int round_away;         // E2M1 ties to the larger magnitude
     int mx_floor;           // MX scale: floor rule
-    int gscale_computed;    // NVFP4: *gscale holds amax bits (set by the amax pass)
+    int gscale_computed;    // NVFP4: *gscale was set by the amax pass (see amax_kernel)
 };
 
 // Units processed per thread and loop trip: their loads are all issued
@@ -108,10 +108,20 @@ FP4_DEV float nv_global_from_amax(float amax)
     return (amax > 0.0f && amax <= kFltMax) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
 }
 
-FP4_DEV float read_global_scale(const float *g, int computed)
+// s_g as left in *g by amax_kernel: max over CTAs of RN(amax_cta / 2688)
+// equals RN(amax / 2688) (division by a positive constant and rounding are
+// both monotonic), so only the all-zero and the non-finite cases remain,
+// both mapped to 1.  The quantize kernel writes that 1 back; other CTAs may
+// read 0 / inf or 1 meanwhile and decode either to the same s_g.
+FP4_DEV float computed_global_scale(float v) { return (v > 0.0f && v <= kFltMax) ? v : 1.0f; }
+
+FP4_DEV float read_global_scale(float *g, int computed)
 {
-    float v = *g;
-    return computed ? nv_global_from_amax(v) : v;
+    const float v = __ldcg(g);
+    if (!computed) return v;
+    const float sg = computed_global_scale(v);
+    if (!(sg == v) && blockIdx.x == 0 && threadIdx.x == 0) atomicExch(g, sg);
+    return sg;
 }
 
 // Scale and element encoding of one rotated 32-element unit u, and the stores
@@ -162,8 +172,10 @@ FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, co
 }
 
 // ---------------------------------------------------------------------------
-// NVFP4 tensor max |H_k x| -> *gscale (as the bits of a non-negative float;
-// integer order equals float order).  *gscale must be 0 on entry.
+// NVFP4 tensor scale: every CTA folds RN(max |H_k x| over its part / 2688)
+// into *gscale with an integer atomicMax (the bits of a non-negative float
+// order like the float; *gscale must be 0 on entry).  The result is s_g =
+// RN(amax / (6 * 448)) itself, or 0 for an all-zero tensor.
 template <int HK>
 __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
 {
@@ -204,7 +216,8 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
     if (threadIdx.x == 0) {
         float b = red[0];
         for (int w = 1; w < (int)(blockDim.x >> 5); w++) b = fmaxf(b, red[w]);
-        atomicMax(reinterpret_cast<unsigned int *>(a.gscale), __float_as_uint(b));
+        // integer order of non-negative float bits is float order
+        atomicMax(reinterpret_cast<unsigned int *>(a.gscale), __float_as_uint(__fdiv_rn(b, 2688.0f)));
     }
 }
 
@@ -215,15 +228,6 @@ __global__ void zero_word_kernel(float *g)
     grid_dep_launch();
     grid_dep_wait();
     *g = 0.0f;
-}
-
-// Converts the tensor max left by amax_kernel into s_g = amax / (6 * 448)
-// (1 for an all-zero tensor).  Runs after the quantize kernel has read it.
-__global__ void finalize_gscale_kernel(float *g)
-{
-    grid_dep_launch();
-    grid_dep_wait();
-    *g = nv_global_from_amax(*g);
 }
 
 // ---------------------------------------------------------------------------
@@ -580,13 +584,8 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
         if ((err = launch_k(ak, dim3(grid), dim3(256), 0, st, pdl, a)) != cudaSuccess) return err;
         first = false;
     }
-    if (a.total_units > 0) {
+    if (a.total_units > 0 || a.gscale_computed) {  // an empty NVFP4 tensor still gets s_g = 1
         if ((err = launch_k(qk, dim3(grid), dim3(256), 0, st, pdl && !first, a)) != cudaSuccess) return err;
-        first = false;
-    }
-    if (a.gscale_computed) {
-        if ((err = launch_k(finalize_gscale_kernel, dim3(1), dim3(1), 0, st, pdl && !first, gscale)) != cudaSuccess)
-            return err;
         first = false;
     }
     const int64_t rows_p = (rows + 127) / 128 * 128;

@@ -336,4 +336,14 @@ FP4_DEV float ld_shared_cluster_f32(uint32_t addr_cluster)
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr_cluster) : "memory");
     return v;
 }
+
+FP4_DEV float4 ld_shared_cluster_f32x4(uint32_t addr_cluster)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr_cluster)
+                 : "memory");
+    return v;
+}
 }  // namespace fp4

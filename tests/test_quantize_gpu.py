@@ -182,3 +182,23 @@ def test_edge_rows_alone(fp4, orc, row, fmt):
     computed from it (all-zero, -0, subnormal-only, tie-only, ... tensors)."""
     x = edge_tensor()[row:row + 1]
     check_quantize(fp4, orc, x, fmt)
+
+
+def test_nvfp4_scale_buffer_reused_across_tensors(fp4, orc):
+    """The computed s_g never keeps a value from an earlier call through the
+    same output word: a large-range tensor, then a small-range one, then an
+    all-zero one (s_g = 1), then an empty one (s_g = 1)."""
+    import torch
+    big = inputs.quant_sweep(rows=8, cols=256, seed=11)
+    small = inputs.f32_to_bf16_bits(inputs.bf16_bits_to_f32(big) * np.float32(2.0 ** -20))
+    q, s, g = fp4.quantize(to_dev_bf16(big), 1)
+    for x in (small, np.zeros_like(big)):
+        fp4.quantize(to_dev_bf16(x), 1, out=(q, s, g))
+        torch.cuda.synchronize()
+        _, _, og = orc.quantize(x, 1)
+        assert np.float32(to_np(g)[0]) == np.float32(og)
+    empty = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    g.fill_(123.0)
+    fp4.quantize(empty, 1, out=(q[:0], s, g))
+    torch.cuda.synchronize()
+    assert to_np(g)[0] == 1.0

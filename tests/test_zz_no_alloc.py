@@ -69,5 +69,22 @@ def test_noalloc_rejects_what_it_cannot_hold(fp4):
     # M above the decode range, and K not a multiple of 256: refused before any launch
     assert f(p, p, g.data_ptr(), p, p, g.data_ptr(), 17, 8, 256, 0, 0, p, 8, None) == 2
     assert f(p, p, g.data_ptr(), p, p, g.data_ptr(), 4, 8, 100, 0, 0, p, 8, None) == 2
-    # partials larger than the fixed array (many tiny-K tiles spread over every SM)
-    assert f(p, p, g.data_ptr(), p, p, g.data_ptr(), 16, 1 << 22, 256, 0, 0, p, 1 << 22, None) == 2
+    # Partials larger than the fixed array: many more tiles than SMs with two
+    # K steps each, so the stream-K split cuts tiles and every CTA holds
+    # several segments.  The size is settled on the host first, and every
+    # buffer is allocated at full size, so the call could run safely even if
+    # it were accepted.
+    M, K, fmt = 16, 512, 0
+    N = 128 * 600
+    while fp4.gemm_workspace_size(M, N, K, fmt) <= 4 << 20:
+        N *= 2
+        assert N <= 128 * 600 * 16, "no decode shape needs more than the fixed array"
+    qa = torch.zeros((M, K // 2), dtype=torch.uint8, device="cuda")
+    sa = torch.zeros((128 * K // 32,), dtype=torch.uint8, device="cuda")
+    qw = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    sw = torch.zeros(((N + 127) // 128 * 128 * K // 32,), dtype=torch.uint8, device="cuda")
+    c = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    rc = f(qa.data_ptr(), sa.data_ptr(), g.data_ptr(), qw.data_ptr(), sw.data_ptr(), g.data_ptr(), M, N, K, fmt,
+           0, c.data_ptr(), N, None)
+    torch.cuda.synchronize()
+    assert rc == 2
