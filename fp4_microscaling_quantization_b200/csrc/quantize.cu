@@ -15,6 +15,9 @@
 // the last butterfly stages exchange values with shuffles.  Warps walk the
 // tensor in a grid-stride loop of 32 consecutive units, so neighbouring
 // lanes read and write neighbouring memory.
+#include <map>
+#include <mutex>
+
 #include "sm100.cuh"
 
 namespace fp4 {
@@ -277,13 +280,34 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
 
 // ---------------------------------------------------------------------------
 // Activation quantization for the decode product (a few rows): one cluster of
-// ACT_CTAS CTAs quantizes the whole tensor in a single launch.  For NVFP4
-// with a computed tensor scale the CTAs exchange their partial maxima through
-// distributed shared memory, so no global scratch, memset or second kernel is
-// involved.  The kernel also zeroes `nzero` words at `zero` (the split-K
-// kernel's per-tile arrival counters) and writes no scale padding (the GEMM
-// never reads scales of rows past the tensor).
-constexpr int ACT_CTAS = 8, ACT_THREADS = 256;
+// up to ACT_CTAS CTAs quantizes the whole tensor in a single launch.  Each
+// thread owns the units u = (warp + i * warps) * 32 + lane, i < ACT_UPT, and
+// when they cover the tensor it keeps their raw bytes in registers, so the
+// NVFP4 tensor-max pass and the encode pass read x once.  The CTAs exchange
+// their partial maxima through distributed shared memory: no global scratch,
+// memset or second kernel.  The kernel also zeroes `nzero` words at `zero`
+// (the split-K kernel's per-tile arrival counters) and writes no scale
+// padding (the GEMM never reads scales of rows past the tensor).
+constexpr int ACT_CTAS = 16, ACT_CTAS_PORTABLE = 8, ACT_THREADS = 256, ACT_UPT = 2;
+
+// Loads units base + 32 i + lane (i < N) of the tensor, zeros past the end.
+template <int N>
+FP4_DEV void fetch_units(const QuantArgs &a, int64_t base, int64_t stride, int lane, uint4 (*raw)[4], uint32_t *row,
+                         uint32_t *col)
+{
+#pragma unroll
+    for (int i = 0; i < N; i++) {
+        const int64_t u = base + i * stride + lane;
+        row[i] = col[i] = 0;
+        if (u < a.total_units) {
+            unit_rc(u, a.upr_div, row[i], col[i]);
+            fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
 
 template <int FMT, int HK>
 __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, unsigned *zero, int nzero)
@@ -300,31 +324,38 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
     const int64_t nwarps = ((int64_t)gridDim.x * ACT_THREADS) >> 5;
     for (int i = blockIdx.x * ACT_THREADS + threadIdx.x; i < nzero; i += gridDim.x * ACT_THREADS) zero[i] = 0u;
 
+    const int64_t stride = nwarps * 32;  // units between a thread's consecutive units
+    const bool cached = a.total_units <= stride * ACT_UPT;
+    uint4 raw[ACT_UPT][4];
+    uint32_t row[ACT_UPT], col[ACT_UPT];
+    if (cached) fetch_units<ACT_UPT>(a, warp * 32, stride, lane, raw, row, col);
+
     float sg = 1.0f;
     if (FMT == FP4_NVFP4) {
         if (a.gscale_computed) {
             float m = 0.0f;
-            for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
-                uint4 raw[QUNITS][4];
-        uint32_t row[QUNITS] = {}, col[QUNITS] = {};
+            if (cached) {
 #pragma unroll
-                for (int i = 0; i < QUNITS; i++) {
-                    const int64_t u = base + i * 32 + lane;
-                    if (u < a.total_units) {
-                        unit_rc(u, a.upr_div, row[i], col[i]);
-                        fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < QUNITS; i++) {
+                for (int i = 0; i < ACT_UPT; i++) {
                     float v[32];
                     unpack_unit(raw[i], v);
                     if (HK) fwht_unit<HK>(v, a.ck, lane);
 #pragma unroll
                     for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+                }
+            } else {
+                for (int64_t base = warp * 32; base < a.total_units; base += stride * QUNITS) {
+                    uint4 r2[QUNITS][4];
+                    uint32_t rw[QUNITS], cl[QUNITS];
+                    fetch_units<QUNITS>(a, base, stride, lane, r2, rw, cl);
+#pragma unroll
+                    for (int i = 0; i < QUNITS; i++) {
+                        float v[32];
+                        unpack_unit(r2[i], v);
+                        if (HK) fwht_unit<HK>(v, a.ck, lane);
+#pragma unroll
+                        for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+                    }
                 }
             }
 #pragma unroll
@@ -348,27 +379,28 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
     }
     const float six_sg = __fmul_rn(6.0f, sg);
 
-    for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
-        uint4 raw[QUNITS][4];
-        uint32_t row[QUNITS] = {}, col[QUNITS] = {};
+    if (cached) {
 #pragma unroll
-        for (int i = 0; i < QUNITS; i++) {
-            const int64_t u = base + i * 32 + lane;
-            if (u < a.total_units) {
-                unit_rc(u, a.upr_div, row[i], col[i]);
-                fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < QUNITS; i++) {
-            const int64_t u = base + i * 32 + lane;
+        for (int i = 0; i < ACT_UPT; i++) {
+            const int64_t u = warp * 32 + i * stride + lane;
             float v[32];
             unpack_unit(raw[i], v);
             if (HK) fwht_unit<HK>(v, a.ck, lane);
             if (u < a.total_units) encode_store_unit<FMT>(v, u, row[i], col[i], a, sg, six_sg);
+        }
+        return;
+    }
+    for (int64_t base = warp * 32; base < a.total_units; base += stride * QUNITS) {
+        uint4 r2[QUNITS][4];
+        uint32_t rw[QUNITS], cl[QUNITS];
+        fetch_units<QUNITS>(a, base, stride, lane, r2, rw, cl);
+#pragma unroll
+        for (int i = 0; i < QUNITS; i++) {
+            const int64_t u = base + i * stride + lane;
+            float v[32];
+            unpack_unit(r2[i], v);
+            if (HK) fwht_unit<HK>(v, a.ck, lane);
+            if (u < a.total_units) encode_store_unit<FMT>(v, u, rw[i], cl[i], a, sg, six_sg);
         }
     }
 }
@@ -614,6 +646,42 @@ static void (*act_kernel_for(int hk))(QuantArgs, unsigned *, int)
     return nullptr;
 }
 
+// Cluster size of the activation quantizer: ACT_CTAS (a non-portable size)
+// where the device schedules such clusters, else the portable ACT_CTAS_PORTABLE.
+// Decided once per kernel instance.
+static int act_cluster_size(void (*k)(QuantArgs, unsigned *, int))
+{
+    static std::mutex mu;
+    static std::map<const void *, int> sizes;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = sizes.find(reinterpret_cast<const void *>(k));
+    if (it != sizes.end()) return it->second;
+    int n = ACT_CTAS_PORTABLE;
+    bool refused = false;  // a refused call leaves its error for cudaGetLastError: clear only ours
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        refused = true;
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(ACT_CTAS);
+        cfg.blockDim = dim3(ACT_THREADS);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = ACT_CTAS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, k, &cfg) != cudaSuccess)
+            refused = true;
+        else if (clusters > 0)
+            n = ACT_CTAS;
+    }
+    if (refused) cudaGetLastError();
+    sizes[reinterpret_cast<const void *>(k)] = n;
+    return n;
+}
+
 // Single-launch quantization of a small activation tensor (see
 // act_quant_kernel); scale padding is left unwritten.
 cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int hk, float ck,
@@ -639,13 +707,14 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
     void (*k)(QuantArgs, unsigned *, int) = (fmt == FP4_MXFP4) ? act_kernel_for<FP4_MXFP4>(hk) : act_kernel_for<FP4_NVFP4>(hk);
     if (!k) return cudaErrorInvalidValue;
+    const int ctas = act_cluster_size(k);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ACT_CTAS);
+    cfg.gridDim = dim3(ctas);
     cfg.blockDim = dim3(ACT_THREADS);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = ACT_CTAS;
+    attr[0].val.clusterDim.x = ctas;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     // May start while the previous kernel drains (its launch latency is then
