@@ -26,10 +26,6 @@ namespace fp4 {
 
 static __device__ unsigned int g_gemm_error;
 
-
-
-
-
 // ---------------------------------------------------------------------------
 // Persistent tiled kernel.  Each CTA (CG == 1) or CTA pair (CG == 2, one
 // 2-SM MMA covering 256 rows of A) walks output tiles of 128*CG x 256 in
@@ -41,8 +37,14 @@ static __device__ unsigned int g_gemm_error;
 //                128 rows; W: all 256 rows, both CTAs), counted on the full
 //                barrier of the group's leader CTA;
 //   warp 1       TMEM allocation; in the leader CTA also the MMA issuer:
-//                tcgen05.cp of the scale atoms, four K=64 block-scaled MMAs
-//                per stage, tcgen05.commit to free the stage (in both CTAs);
+//                four K=64 block-scaled MMAs per stage once the stage's
+//                scales are in TMEM, tcgen05.commit to free the stage (in
+//                both CTAs);
+//   warps 10-11  (leader CTA) scale copiers: tcgen05.cp of the stage's scale
+//                atoms into TMEM, half each, then a commit that releases the
+//                stage to the MMA issuer.  A tcgen05 instruction costs its
+//                issuing thread tens of cycles, so copies issued from other
+//                warps overlap the MMAs instead of queueing in front of them;
 //   warps 2-9    epilogue: two warps per 32-lane quarter, each draining 128
 //                accumulator columns into registers, then releasing the
 //                accumulator (so the next tile's MMAs start) before scaling,
@@ -60,7 +62,8 @@ struct PCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int STAGES = CG == 1 ? 4 : 5;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
-    static constexpr int THREADS = 320;
+    static constexpr int NCOPY = 2;                      // scale-copier warps (10 and 11)
+    static constexpr int THREADS = 384;
     static constexpr int TMEM_COLS = 512;
     static constexpr int SF_COL0 = 256;
     static constexpr int SF_STAGE_COLS = 48;
@@ -81,7 +84,7 @@ struct PParams {
 };
 
 template <int FMT, int BF16OUT, int CG>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
              const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, PParams p)
 {
@@ -91,8 +94,8 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * Cfg::STAGE_BYTES);
-    // bars: full[S] empty[S] accfull accempty
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 2);
+    // bars: full[S] empty[S] sfready[S] accfull accempty drain
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 3);
     volatile uint32_t *abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,8 +105,9 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     const int num_tiles = p.num_m_tiles * p.num_n_tiles;
     const int nk = p.K / Cfg::BK;
 
-    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
-    const uint32_t accf = smem_u32(bars + 2 * STAGES), acce = smem_u32(bars + 2 * STAGES + 1);
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES), sfr0 = smem_u32(bars + 2 * STAGES);
+    const uint32_t accf = smem_u32(bars + 3 * STAGES), acce = smem_u32(bars + 3 * STAGES + 1);
+    const uint32_t drainb = smem_u32(bars + 3 * STAGES + 2);
     // the leader's copies of the barriers every CTA of the group signals
     const uint32_t full0_lead = (CG == 2) ? mapa_shared(full0, 0) : full0;
     const uint32_t acce_lead = (CG == 2) ? mapa_shared(acce, 0) : acce;
@@ -112,8 +116,10 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         for (int s = 0; s < STAGES; s++) {
             mbar_init(full0 + 8 * s, CG);   // one arrive.expect_tx per CTA of the group
             mbar_init(empty0 + 8 * s, 1);   // one tcgen05.commit
+            mbar_init(sfr0 + 8 * s, Cfg::NCOPY);  // one commit per scale copier
         }
         mbar_init(accf, 1);
+        mbar_init(drainb, 1 + Cfg::NCOPY);  // MMA issuer and copiers, once each at the end
         mbar_init(acce, 8 * CG);            // every epilogue warp of the group
         *abort_flag = 0u;
         fence_barrier_init();
@@ -168,6 +174,11 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             // ---------------- MMA issuer (leader CTA) ----------------
             int it = 0, tile_i = 0;
             const uint16_t both = (uint16_t)((1u << CG) - 1u);
+            // stage-0 descriptors; stages and K steps add to the 16-byte-unit
+            // address field (offsets stay below 256 KB: no carry)
+            const uint32_t sa0 = smem_u32(smem);
+            const uint64_t adesc0 = smem_desc(sa0, 16, 1024, 2);
+            const uint64_t bdesc0 = smem_desc(sa0 + Cfg::A_BYTES, 16, 1024, 2);
             for (int t = group; t < num_tiles; t += ngroups, tile_i++) {
                 if (tile_i > 0 &&
                     !mbar_wait_bounded(acce, (uint32_t)((tile_i - 1) & 1), abort_flag, &g_gemm_error, p.budget_ns))
@@ -177,26 +188,16 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 for (int ks = 0; ks < nk; ks++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) { stop = true; break; }
+                    // operands landed and the scale copiers' tcgen05.cp done
+                    if (!mbar_wait_bounded(sfr0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) { stop = true; break; }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
-                    const uint32_t sb = sa + Cfg::A_BYTES;
-                    const uint32_t ssfa = sb + Cfg::B_BYTES;
-                    const uint32_t ssfb = ssfa + Cfg::SFA_BYTES;
+                    const uint64_t so = (uint64_t)((s * Cfg::STAGE_BYTES) >> 4);
                     const uint32_t tsfa = tmem + Cfg::SF_COL0 + s * Cfg::SF_STAGE_COLS;
                     const uint32_t tsfb = tsfa + 16;
 #pragma unroll
                     for (int kk = 0; kk < 4; kk++) {
-                        // copy each scale atom just before its first MMA, so the
-                        // copies of one atom overlap the MMA of the previous one
-                        if (FMT == FP4_NVFP4 || (kk & 1) == 0) {
-                            const int a = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
-                            tc_cp_scale_atom_cg<CG>(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
-                            tc_cp_scale_atom_cg<CG>(tsfb + 8 * a, smem_desc(ssfb + 512 * a, 0, 128, 0));
-                            tc_cp_scale_atom_cg<CG>(tsfb + 8 * a + 4, smem_desc(ssfb + KA * 512 + 512 * a, 0, 128, 0));
-                        }
-                        const uint64_t ad = smem_desc(sa + 32 * kk, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(sb + 32 * kk, 16, 1024, 2);
+                        const uint64_t ad = adesc0 + so + 2 * kk;
+                        const uint64_t bd = bdesc0 + so + 2 * kk;
                         const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
                         const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
                         const uint32_t idesc = idesc_blockscaled(Cfg::BM * CG, Cfg::BN, FMT == FP4_MXFP4, sfid, sfid);
@@ -216,6 +217,45 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 tc_commit_cg<CG>(accf, both);
                 if (stop) break;
             }
+            // TMEM is released only after every MMA and scale copy of the
+            // group has completed, also on the abort path
+            tc_commit_cg<CG>(drainb, 1);
+            volatile uint32_t no_abort = 0;
+            mbar_wait_bounded(drainb, 0, &no_abort, &g_gemm_error, p.budget_ns);
+        }
+        __syncwarp();
+    } else if (warp >= 10) {
+        // ---------------- scale copiers (leader CTA) ----------------
+        if (lane == 0 && leader) {
+            constexpr int APC = KA / Cfg::NCOPY;  // scale atoms per copier per stage
+            const int c = warp - 10;
+            const uint32_t sa0 = smem_u32(smem);
+            const uint64_t sfadesc0 = smem_desc(sa0 + Cfg::A_BYTES + Cfg::B_BYTES, 0, 128, 0);
+            const uint64_t sfbdesc0 = sfadesc0 + (Cfg::SFA_BYTES >> 4);
+            int it = 0;
+            bool stop = false;
+            for (int t = group; t < num_tiles && !stop; t += ngroups) {
+                for (int ks = 0; ks < nk; ks++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    // the stage's previous MMAs finished before it was reloaded
+                    // (empty -> producer -> full), so its scale columns are free
+                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint64_t so = (uint64_t)((s * Cfg::STAGE_BYTES) >> 4);
+                    const uint32_t tsfa = tmem + Cfg::SF_COL0 + s * Cfg::SF_STAGE_COLS;
+                    const uint32_t tsfb = tsfa + 16;
+#pragma unroll
+                    for (int q = 0; q < APC; q++) {
+                        const int a = c * APC + q;
+                        tc_cp_scale_atom_cg<CG>(tsfa + 4 * a, sfadesc0 + so + 32 * a);
+                        tc_cp_scale_atom_cg<CG>(tsfb + 8 * a, sfbdesc0 + so + 32 * a);
+                        tc_cp_scale_atom_cg<CG>(tsfb + 8 * a + 4, sfbdesc0 + so + 32 * (KA + a));
+                    }
+                    tc_commit_cg<CG>(sfr0 + 8 * s, 1);
+                }
+            }
+            tc_commit_cg<CG>(drainb, 1);
         }
         __syncwarp();
     } else {
@@ -325,7 +365,7 @@ constexpr int SFA_BYTES = 4 * 512;
 constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;  // 22528 = 22 KB
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 constexpr int TMEM_COLS = 512;
-constexpr int SF_COL0 = 32;                  // accumulators at columns [0,16) and [16,32)
+constexpr int SF_COL0 = 64;                  // accumulators: buffer b, issuer j at columns 32 b + 16 j
 constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation scales 16 cols
 constexpr int MAX_CLUSTER = 8;               // portable cluster size
 
@@ -369,8 +409,12 @@ FP4_DEV void store_row(const Params &p, int n, const float *acc, float alpha)
     }
 }
 
+// Threads: warp 0 loads, warps 1 and 6 issue MMAs, warps 2-5 drain the
+// accumulators (warp w may read TMEM lanes 32 (w % 4) .. + 31).
+constexpr int DECODE_THREADS = 224;
+
 template <int FMT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(DECODE_THREADS, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, Params p)
 {
     constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
@@ -391,27 +435,43 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const int c = blockIdx.x;
     const int64_t U = (int64_t)p.ntiles * p.nk;
     const int64_t u0 = unit_begin(c, U, p.G), u1 = unit_begin(c + 1, U, p.G);
+    // The loops below run on single threads, where integer latency is not
+    // hidden: positions advance incrementally instead of by division.
+    const int n_units = (int)(u1 - u0);
     const int t_first = (int)(u0 / p.nk);
+    const int ks_first = (int)(u0 - (int64_t)t_first * p.nk);
     const int nseg = (int)((u1 - 1) / p.nk) - t_first + 1;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
     const uint32_t accf0 = smem_u32(bars + 2 * STAGES), acce0 = smem_u32(bars + 2 * STAGES + 2);
     const uint32_t drainb = smem_u32(bars + 2 * STAGES + 4);
     const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
-    const int64_t npre = (u1 - u0) < STAGES ? (u1 - u0) : STAGES;
+    const int npre = n_units < STAGES ? n_units : STAGES;
+    const uint32_t smem0 = smem_u32(smem);
+    // Dual issue: a tcgen05 instruction costs its issuing thread tens of
+    // cycles, far longer than the tensor pipe needs for an N = 16 MMA, so two
+    // warps issue alternate K steps into two accumulators that the epilogue
+    // adds.  Used when the CTA owns one tile segment of at least two units
+    // (whole tiles and cluster splits); otherwise warp 1 issues alone.
+    const bool dual = nseg == 1 && n_units >= 2;
+    const uint32_t issuers = dual ? 2u : 1u;
 
-    auto load_w = [&](int64_t u, int st_i) {
-        const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
-        uint8_t *st = smem + st_i * STAGE_BYTES;
-        const uint32_t fb = full0 + 8 * st_i;
-        tma_load_2d(smem_u32(st), &tmW, ks * (BK / 2), t * BMW, fb);
-        bulk_load(smem_u32(st + W_BYTES + A_BYTES), p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+    auto advance = [&](int &t, int &ks) {
+        if (++ks == p.nk) {
+            ks = 0;
+            ++t;
+        }
     };
-    auto load_a = [&](int64_t u, int st_i) {
-        const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
-        uint8_t *st = smem + st_i * STAGE_BYTES;
+    auto load_w = [&](int t, int ks, int st_i) {
+        const uint32_t st = smem0 + st_i * STAGE_BYTES;
         const uint32_t fb = full0 + 8 * st_i;
-        tma_load_2d(smem_u32(st + W_BYTES), &tmA, ks * (BK / 2), 0, fb);
-        bulk_load(smem_u32(st + W_BYTES + A_BYTES + SFW_BYTES), p.As + (int64_t)ks * KA * 512, KA * 512, fb);
+        tma_load_2d(st, &tmW, ks * (BK / 2), t * BMW, fb);
+        bulk_load(st + W_BYTES + A_BYTES, p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+    };
+    auto load_a = [&](int ks, int st_i) {
+        const uint32_t st = smem0 + st_i * STAGE_BYTES;
+        const uint32_t fb = full0 + 8 * st_i;
+        tma_load_2d(st + W_BYTES, &tmA, ks * (BK / 2), 0, fb);
+        bulk_load(st + W_BYTES + A_BYTES + SFW_BYTES, p.As + (int64_t)ks * KA * 512, KA * 512, fb);
     };
 
     if (threadIdx.x == 0) {
@@ -420,10 +480,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             mbar_init(empty0 + 8 * s, 1);
         }
         for (int b = 0; b < 2; b++) {
-            mbar_init(accf0 + 8 * b, 1);
+            mbar_init(accf0 + 8 * b, issuers);
             mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
         }
-        mbar_init(drainb, 1);
+        mbar_init(drainb, issuers);
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch_desc(&tmW);
@@ -432,9 +492,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         // still be quantizing the activations): start it at once, while warp
         // 1 allocates tensor memory.
         if (!p.stall) {
-            for (int64_t i = 0; i < npre; i++) {
-                mbar_arrive_expect_tx(full0 + 8 * (int)i, tx);
-                load_w(u0 + i, (int)i);
+            int t = t_first, ks = ks_first;
+            for (int i = 0; i < npre; i++) {
+                mbar_arrive_expect_tx(full0 + 8 * i, tx);
+                load_w(t, ks, i);
+                advance(t, ks);
             }
         }
     }
@@ -450,34 +512,48 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     if (warp == 0) {
         if (lane == 0 && !p.stall) {
             grid_dep_wait();
-            for (int64_t i = 0; i < npre; i++) load_a(u0 + i, (int)i);
-            int64_t issued = npre;
-            for (int64_t u = u0 + npre; u < u1; u++) {
-                const int64_t i = u - u0;
-                const int s = (int)(i % STAGES);
+            int t = t_first, ks = ks_first;
+            for (int i = 0; i < npre; i++) {
+                load_a(ks, i);
+                advance(t, ks);
+            }
+            int issued = npre;
+            for (int i = npre; i < n_units; i++) {
+                const int s = i % STAGES;
                 const uint32_t ph = (uint32_t)((i / STAGES) & 1);
                 if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) break;
                 mbar_arrive_expect_tx(full0 + 8 * s, tx);
-                load_w(u, s);
-                load_a(u, s);
+                load_w(t, ks, s);
+                load_a(ks, s);
+                advance(t, ks);
                 issued = i + 1;
             }
-            for (int64_t i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++) {
+            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++) {
                 volatile uint32_t no_abort = 0;
-                mbar_wait_bounded(full0 + 8 * (int)(i % STAGES), (uint32_t)((i / STAGES) & 1), &no_abort, &g_gemm_error, p.budget_ns);
+                mbar_wait_bounded(full0 + 8 * (i % STAGES), (uint32_t)((i / STAGES) & 1), &no_abort, &g_gemm_error, p.budget_ns);
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        if (lane == 0) {
+    } else if (warp == 1 || warp == 6) {
+        const int j = warp == 1 ? 0 : 1;  // issuer index
+        if (lane == 0 && (j == 0 || dual)) {
+            // Descriptors of stage 0: a stage, atom or K step only moves the
+            // 16-byte-unit start address in the low 14 bits (shared memory
+            // offsets stay below 256 KB, so the add never carries out).
+            const uint64_t wdesc0 = smem_desc(smem0, 16, 1024, 2);
+            const uint64_t adesc0 = smem_desc(smem0 + W_BYTES, 16, 1024, 2);
+            const uint64_t sfwdesc0 = smem_desc(smem0 + W_BYTES + A_BYTES, 0, 128, 0);
+            const uint64_t sfadesc0 = smem_desc(smem0 + W_BYTES + A_BYTES + SFW_BYTES, 0, 128, 0);
+            const int step = dual ? 2 : 1;
             int seg = -1;
-            for (int64_t u = u0; u < u1; u++) {
-                const int64_t i = u - u0;
-                const int s = (int)(i % STAGES);
+            int t = t_first, ks = ks_first;
+            if (j == 1) advance(t, ks);
+            for (int i = j; i < n_units; i += step) {
+                const int s = i % STAGES;
                 const uint32_t ph = (uint32_t)((i / STAGES) & 1);
-                const int t = (int)(u / p.nk), ks = (int)(u - (int64_t)t * p.nk);
-                const bool first = (u == u0) || ks == 0;
-                const bool last = (u == u1 - 1) || ks == p.nk - 1;
+                // first / last unit of a tile segment among this warp's units
+                const bool first = dual ? (i == j) : ((i == 0) || ks == 0);
+                const bool last = dual ? (i + 2 >= n_units) : ((i == n_units - 1) || ks == p.nk - 1);
                 if (first) {
                     seg++;
                     if (seg >= 2 &&
@@ -486,21 +562,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 }
                 if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) break;
                 tc_fence_after();
-                const uint32_t acc = tmem + (uint32_t)(seg & 1) * BNA;
-                const uint32_t sw = smem_u32(smem + s * STAGE_BYTES);
-                const uint32_t sa = sw + W_BYTES;
-                const uint32_t ssfw = sa + A_BYTES;
-                const uint32_t ssfa = ssfw + SFW_BYTES;
+                const uint32_t acc = tmem + (uint32_t)(seg & 1) * 2 * BNA + (uint32_t)j * BNA;
+                const uint64_t so = (uint64_t)((s * STAGE_BYTES) >> 4);
                 const uint32_t tsfw = tmem + SF_COL0 + s * SF_STAGE_COLS;
                 const uint32_t tsfa = tsfw + 16;
+#pragma unroll
                 for (int a = 0; a < KA; a++) {
-                    tc_cp_scale_atom(tsfw + 4 * a, smem_desc(ssfw + 512 * a, 0, 128, 0));
-                    tc_cp_scale_atom(tsfa + 4 * a, smem_desc(ssfa + 512 * a, 0, 128, 0));
+                    tc_cp_scale_atom(tsfw + 4 * a, sfwdesc0 + so + 32 * a);
+                    tc_cp_scale_atom(tsfa + 4 * a, sfadesc0 + so + 32 * a);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 4; kk++) {
-                    const uint64_t wd = smem_desc(sw + 32 * kk, 16, 1024, 2);
-                    const uint64_t ad = smem_desc(sa + 32 * kk, 16, 1024, 2);
+                    const uint64_t wd = wdesc0 + so + 2 * kk;
+                    const uint64_t ad = adesc0 + so + 2 * kk;
                     const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
                     const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
                     const uint32_t idesc = idesc_blockscaled(BMW, BNA, FMT == FP4_MXFP4, sfid, sfid);
@@ -509,6 +583,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 }
                 tc_commit(empty0 + 8 * s);
                 if (last) tc_commit(accf0 + 8 * (seg & 1));
+                advance(t, ks);
+                if (dual) advance(t, ks);
             }
             // arrives once every MMA issued above has completed
             tc_commit(drainb);
@@ -527,8 +603,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         if (!ok) break;
         tc_fence_after();
         uint32_t r[16];
-        tmem_ld16(tmem + (uint32_t)b * BNA + ((uint32_t)(quarter * 32) << 16), r);
-        tmem_ld_wait();
+        const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+        tmem_ld16(tmem + (uint32_t)b * 2 * BNA + lanes, r);
+        if (dual) {
+            // the second issuer's accumulator, added in a fixed order
+            uint32_t r2[16];
+            tmem_ld16(tmem + (uint32_t)b * 2 * BNA + BNA + lanes, r2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int m = 0; m < BNA; m++) r[m] = __float_as_uint(__fadd_rn(__uint_as_float(r[m]), __uint_as_float(r2[m])));
+        } else {
+            tmem_ld_wait();
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");
@@ -599,7 +685,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         // the other CTAs' shared memory alive until it has read it.  Both are
         // reached on every path, the abort paths included.
         cluster_sync();
-        if (cluster_ctarank() == 0 && warp >= 2) {
+        if (cluster_ctarank() == 0 && warp >= 2 && warp <= 5) {
             const int row = (warp & 3) * 32 + lane;
             const int t = c / p.csize;
             const int n = t * BMW + row;
@@ -836,7 +922,7 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(decode::DECODE_THREADS);
     cfg.dynamicSmemBytes = decode::SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
