@@ -18,7 +18,8 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
                         const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K,
                         int fmt, int bf16out, void *C, int64_t ldc, void *ws, size_t ws_bytes,
-                        int sms, cudaStream_t st, int *timeout_flag_out, bool pdl, unsigned *counters);
+                        int sms, cudaStream_t st, int *timeout_flag_out, bool pdl, unsigned *counters,
+                        bool w_before_wait);
 cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int hk, float ck,
                                 int round_away, int mx_floor, int gscale_given, uint8_t *q, uint8_t *s, float *gscale,
                                 unsigned *zero, int nzero, cudaStream_t st);
@@ -157,7 +158,7 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const
     int bad = 0;
     cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16,
                                      C, ldc, workspace, ws_bytes, sms,
-                                     static_cast<cudaStream_t>(stream), &bad, false, nullptr);
+                                     static_cast<cudaStream_t>(stream), &bad, true, nullptr, false);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
@@ -242,7 +243,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     if (e != cudaSuccess) return FP4_ERR_CUDA;
     int bad = 0;
     e = fp4::launch_gemm(aq, as, ga, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc, base + L.gemm,
-                         L.counters - L.gemm, sms, st, &bad, true, counters);
+                         L.counters - L.gemm, sms, st, &bad, true, counters, decode);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

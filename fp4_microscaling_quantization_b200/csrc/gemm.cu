@@ -389,6 +389,11 @@ struct Params {
     int maxseg;
     int nkb4;
     int csize;           // > 1: the CTAs of a tile form a cluster of csize and reduce through DSMEM
+    // Stream W before waiting for the preceding kernel.  Only when that
+    // kernel triggers its dependents after its own wait (the decode
+    // activation quantizer), so every earlier kernel, whatever wrote W,
+    // has finished.
+    int w_before_wait;
 };
 
 __host__ __device__ inline int64_t unit_begin(int c, int64_t U, int G) { return (int64_t)c * U / G; }
@@ -492,6 +497,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         // still be quantizing the activations): start it at once, while warp
         // 1 allocates tensor memory.
         if (!p.stall) {
+            if (!p.w_before_wait) grid_dep_wait();
             int t = t_first, ks = ks_first;
             for (int i = 0; i < npre; i++) {
                 mbar_arrive_expect_tx(full0 + 8 * i, tx);
@@ -950,7 +956,8 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
 
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
                         const float *gW, int64_t M, int64_t N, int64_t K, int fmt, int bf16out, void *C, int64_t ldc,
-                        void *ws, size_t ws_bytes, int sms, cudaStream_t st, int *bad, bool pdl, unsigned *counters)
+                        void *ws, size_t ws_bytes, int sms, cudaStream_t st, int *bad, bool pdl, unsigned *counters,
+                        bool w_before_wait)
 {
     if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) {
         *bad = 1;
@@ -980,6 +987,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.G = pl.G;
         dp.maxseg = pl.maxseg;
         dp.csize = pl.csize;
+        dp.w_before_wait = (pdl && w_before_wait) ? 1 : 0;
         dp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
         dp.counters = counters;
         dp.budget_ns = budget;
@@ -1099,7 +1107,7 @@ extern "C" fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *
     int bad = 0;
     const cudaError_t e = fp4::launch_gemm(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc,
                                            scratch, fp4::kNoAllocScratchBytes, sms,
-                                           static_cast<cudaStream_t>(stream), &bad, false, nullptr);
+                                           static_cast<cudaStream_t>(stream), &bad, false, nullptr, false);
     if (bad) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

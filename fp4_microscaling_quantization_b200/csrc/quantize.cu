@@ -95,11 +95,14 @@ FP4_DEV void fwht_unit(float *v, float ck, int lane)
     }
 #pragma unroll
     for (int lm = 1; lm < HK / 32; lm <<= 1) {
-        const bool lower = (lane & lm) == 0;
+        // lower lane: a + b; upper lane: b - a, i.e. b + (-a): the same
+        // rounded sum either way, with the operand's sign flipped by bit
+        // (exact) instead of a second add and a select
+        const uint32_t flip = (lane & lm) ? 0x80000000u : 0u;
 #pragma unroll
         for (int j = 0; j < 32; j++) {
-            float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
-            v[j] = lower ? __fadd_rn(v[j], o) : __fsub_rn(o, v[j]);
+            const float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
+            v[j] = __fadd_rn(o, __uint_as_float(__float_as_uint(v[j]) ^ flip));
         }
     }
 #pragma unroll
