@@ -108,7 +108,7 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                                          hadamard_k, hadamard_constant(hadamard_k),
                                          o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
                                          o.gscale_given, q, s, gscale, sm_count(),
-                                         static_cast<cudaStream_t>(stream), false);
+                                         static_cast<cudaStream_t>(stream), true);
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 

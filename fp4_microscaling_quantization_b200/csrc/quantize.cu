@@ -59,6 +59,33 @@ FP4_DEV void fetch_unit(const uint16_t *x, int64_t ld, uint32_t row, uint32_t j,
     for (int c = 0; c < 4; c++) w[c] = __ldg(p + c);
 }
 
+// L2 eviction policies for the two passes of an NVFP4 quantization with a
+// computed tensor scale: the tensor-max pass marks x evict-last so that the
+// encode pass, which marks it evict-first, finds it in L2 when it fits.
+FP4_DEV uint64_t l2_policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+FP4_DEV uint64_t l2_policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+FP4_DEV void fetch_unit_hint(const uint16_t *x, int64_t ld, uint32_t row, uint32_t j, uint4 *w, uint64_t pol)
+{
+    const uint4 *p = reinterpret_cast<const uint4 *>(x + (int64_t)row * ld + (int64_t)j * 32);
+#pragma unroll
+    for (int c = 0; c < 4; c++)
+        asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                     : "=r"(w[c].x), "=r"(w[c].y), "=r"(w[c].z), "=r"(w[c].w)
+                     : "l"(p + c), "l"(pol));
+}
+
 // bf16 pairs -> 32 fp32 values.
 FP4_DEV void unpack_unit(const uint4 *raw, float *v)
 {
@@ -187,6 +214,7 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
 {
     grid_dep_launch();
     grid_dep_wait();
+    const uint64_t pol = l2_policy_evict_last();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -199,7 +227,7 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
                 unit_rc(u, a.upr_div, row[i], col[i]);
-                fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
+                fetch_unit_hint(a.x, a.ld, row[i], col[i], raw[i], pol);
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -251,6 +279,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
         sg = read_global_scale(a.gscale, a.gscale_computed);
         six_sg = __fmul_rn(6.0f, sg);
     }
+    const bool hinted = FMT == FP4_NVFP4 && a.gscale_computed;  // second read of x
+    const uint64_t pol = l2_policy_evict_first();
 
     for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
         uint4 raw[QUNITS][4];
@@ -260,7 +290,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
                 unit_rc(u, a.upr_div, row[i], col[i]);
-                fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
+                if (hinted) fetch_unit_hint(a.x, a.ld, row[i], col[i], raw[i], pol); else fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -584,9 +614,7 @@ static void (*amax_kernel_for(int hk))(QuantArgs)
     return nullptr;
 }
 
-// Quantize launch sequence.  With `pdl` every launch after the first may
-// overlap its predecessor (each kernel waits for it before touching memory),
-// so a consumer launched the same way can start streaming early.
+// Quantize launch sequence (see the note on `pdl` below).
 cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
                             int hk, float ck, int round_away, int mx_floor, int gscale_given,
                             uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl)
@@ -613,23 +641,22 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     void (*ak)(QuantArgs) = amax_kernel_for(hk);
     if (!qk || !ak) return cudaErrorInvalidValue;
     cudaError_t err = cudaSuccess;
-    bool first = true;  // the first launch of the sequence is ordered normally after earlier work
+    // With `pdl` every launch, the first included, may start while its
+    // predecessor drains: each kernel waits for it before touching memory,
+    // and none reads anything before that wait.
     if (a.gscale_computed) {
-        if ((err = launch_k(zero_word_kernel, dim3(1), dim3(1), 0, st, false, gscale)) != cudaSuccess) return err;
+        if ((err = launch_k(zero_word_kernel, dim3(1), dim3(1), 0, st, pdl, gscale)) != cudaSuccess) return err;
         if ((err = launch_k(ak, dim3(grid), dim3(256), 0, st, pdl, a)) != cudaSuccess) return err;
-        first = false;
     }
     if (a.total_units > 0 || a.gscale_computed) {  // an empty NVFP4 tensor still gets s_g = 1
-        if ((err = launch_k(qk, dim3(grid), dim3(256), 0, st, pdl && !first, a)) != cudaSuccess) return err;
-        first = false;
+        if ((err = launch_k(qk, dim3(grid), dim3(256), 0, st, pdl, a)) != cudaSuccess) return err;
     }
     const int64_t rows_p = (rows + 127) / 128 * 128;
     const int64_t npad = rows * (a.nkb4 * 4 - nkb) + (rows_p - rows) * a.nkb4 * 4;
     if (npad > 0) {
         int g = (int)((npad + 255) / 256);
         if (g > sms * 4) g = sms * 4;
-        if ((err = launch_k(scale_pad_kernel, dim3(g), dim3(256), 0, st, pdl && !first, s, rows, nkb, a.nkb4)) !=
-            cudaSuccess)
+        if ((err = launch_k(scale_pad_kernel, dim3(g), dim3(256), 0, st, pdl, s, rows, nkb, a.nkb4)) != cudaSuccess)
             return err;
     }
     return cudaSuccess;
@@ -767,7 +794,8 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
                                  ? (bf16out ? deq_kernel_for<FP4_MXFP4, 1>(hk) : deq_kernel_for<FP4_MXFP4, 0>(hk))
                                  : (bf16out ? deq_kernel_for<FP4_NVFP4, 1>(hk) : deq_kernel_for<FP4_NVFP4, 0>(hk));
     if (!k) return cudaErrorInvalidValue;
-    return launch_k(k, dim3(grid), dim3(256), 0, st, false, a);
+    // programmatic launch: the kernel waits for its predecessor before touching memory
+    return launch_k(k, dim3(grid), dim3(256), 0, st, true, a);
 }
 
 }  // namespace fp4
