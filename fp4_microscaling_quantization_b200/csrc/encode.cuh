@@ -1,0 +1,132 @@
+// encode.cuh — the per-unit arithmetic of FP4 quantization, shared by the
+// streaming quantize kernels and the decode GEMM's fused activation
+// quantizer so both produce the same bits.
+//
+// Method: "Portable FP4 quantization (TransFP4)" §1.1 Eq.(1) with absmax
+// block scales and nearest rounding; the NVFP4 two-level scale ("4.5 FP8 and
+// NVFP4/MXFP4" §4.1); the block-diagonal Hadamard rotation H_k ("FP4
+// quantization analysis: MXFP4 vs NVFP4" §3.2.3).  A unit is 32 consecutive
+// elements of a row: one MXFP4 block or two NVFP4 blocks.
+#pragma once
+
+#include "common.cuh"
+
+namespace fp4 {
+
+// bf16 pairs -> 32 fp32 values.
+FP4_DEV void unpack_unit(const uint4 *raw, float *v)
+{
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+        const uint4 w = raw[c];
+        v[8 * c + 0] = bf16lo(w.x);
+        v[8 * c + 1] = bf16hi(w.x);
+        v[8 * c + 2] = bf16lo(w.y);
+        v[8 * c + 3] = bf16hi(w.y);
+        v[8 * c + 4] = bf16lo(w.z);
+        v[8 * c + 5] = bf16hi(w.z);
+        v[8 * c + 6] = bf16lo(w.w);
+        v[8 * c + 7] = bf16hi(w.w);
+    }
+}
+
+// Normalised Sylvester Walsh-Hadamard transform of every k-chunk, stages
+// h = 1, 2, ..., k/2 in ascending order: (a, b) -> (a + b, a - b) with a the
+// element whose index has bit h clear; then every value times ck.  Stages
+// with h >= 32 pair this lane with lane ^ (h / 32).
+template <int HK>
+FP4_DEV void fwht_unit(float *v, float ck, int lane)
+{
+#pragma unroll
+    for (int h = 1; h < (HK < 32 ? HK : 32); h <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            if (j & h) continue;
+            float a = v[j], b = v[j + h];
+            v[j] = __fadd_rn(a, b);
+            v[j + h] = __fsub_rn(a, b);
+        }
+    }
+#pragma unroll
+    for (int lm = 1; lm < HK / 32; lm <<= 1) {
+        // lower lane: a + b; upper lane: b - a, i.e. b + (-a): the same
+        // rounded sum either way, with the operand's sign flipped by bit
+        // (exact) instead of a second add and a select
+        const uint32_t flip = (lane & lm) ? 0x80000000u : 0u;
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            const float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
+            v[j] = __fadd_rn(o, __uint_as_float(__float_as_uint(v[j]) ^ flip));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; j++) v[j] = __fmul_rn(v[j], ck);
+}
+
+FP4_DEV float nv_global_from_amax(float amax)
+{
+    return (amax > 0.0f && amax <= kFltMax) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// Largest |v_i| of N consecutive values, as a balanced tree of pairwise
+// maxima: the maximum is exact and independent of order, so this equals a
+// running maximum, with a dependency chain of log2 N steps instead of N.
+template <int N>
+FP4_DEV float absmax_tree(const float *v)
+{
+    float t[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; i++) t[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
+#pragma unroll
+    for (int w = N / 4; w >= 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w; i++) t[i] = fmaxf(t[i], t[i + w]);
+    }
+    return t[0];
+}
+
+// Scale and element encoding of one rotated 32-element unit (TransFP4
+// Eq.(1): MXFP4 power-of-two scale; NVFP4 E4M3 block scale under the tensor
+// scale sg).  v is scaled in place; the 32 E2M1 codes come back as 16 bytes
+// of nibbles (even element in the low nibble) and the return value holds the
+// scale byte (MXFP4) or the two block-scale bytes, first block low (NVFP4).
+template <int FMT>
+FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, int mx_floor, uint4 &out)
+{
+    uint32_t sbytes;
+    if (FMT == FP4_MXFP4) {
+        const float amax = absmax_tree<32>(v);
+        const int e = mx_exponent(amax, mx_floor);
+        const float inv = exp2i(-e);
+#pragma unroll
+        for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
+        sbytes = (uint32_t)(e + 127);
+    } else {
+        sbytes = 0;
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            const float amax = absmax_tree<16>(v + 16 * b);
+            const float t = __fdiv_rn(amax, six_sg);
+            const uint32_t sb = e4m3_rn(t);
+            const float d = __fmul_rn(sg, e4m3_to_f32(sb));
+            const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
+#pragma unroll
+            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
+            sbytes |= sb << (8 * b);
+        }
+    }
+    if (!round_away) {
+        out.x = e2m1x8_rn(v + 0);
+        out.y = e2m1x8_rn(v + 8);
+        out.z = e2m1x8_rn(v + 16);
+        out.w = e2m1x8_rn(v + 24);
+    } else {
+        out.x = e2m1x8_away(v + 0);
+        out.y = e2m1x8_away(v + 8);
+        out.z = e2m1x8_away(v + 16);
+        out.w = e2m1x8_away(v + 24);
+    }
+    return sbytes;
+}
+
+}  // namespace fp4

@@ -18,6 +18,7 @@
 #include <map>
 #include <mutex>
 
+#include "encode.cuh"
 #include "sm100.cuh"
 
 namespace fp4 {
@@ -86,61 +87,6 @@ FP4_DEV void fetch_unit_hint(const uint16_t *x, int64_t ld, uint32_t row, uint32
                      : "l"(p + c), "l"(pol));
 }
 
-// bf16 pairs -> 32 fp32 values.
-FP4_DEV void unpack_unit(const uint4 *raw, float *v)
-{
-#pragma unroll
-    for (int c = 0; c < 4; c++) {
-        const uint4 w = raw[c];
-        v[8 * c + 0] = bf16lo(w.x);
-        v[8 * c + 1] = bf16hi(w.x);
-        v[8 * c + 2] = bf16lo(w.y);
-        v[8 * c + 3] = bf16hi(w.y);
-        v[8 * c + 4] = bf16lo(w.z);
-        v[8 * c + 5] = bf16hi(w.z);
-        v[8 * c + 6] = bf16lo(w.w);
-        v[8 * c + 7] = bf16hi(w.w);
-    }
-}
-
-// Normalised Sylvester Walsh-Hadamard transform of every k-chunk, stages
-// h = 1, 2, ..., k/2 in ascending order: (a, b) -> (a + b, a - b) with a the
-// element whose index has bit h clear; then every value times ck.  Stages
-// with h >= 32 pair this lane with lane ^ (h / 32).
-template <int HK>
-FP4_DEV void fwht_unit(float *v, float ck, int lane)
-{
-#pragma unroll
-    for (int h = 1; h < (HK < 32 ? HK : 32); h <<= 1) {
-#pragma unroll
-        for (int j = 0; j < 32; j++) {
-            if (j & h) continue;
-            float a = v[j], b = v[j + h];
-            v[j] = __fadd_rn(a, b);
-            v[j + h] = __fsub_rn(a, b);
-        }
-    }
-#pragma unroll
-    for (int lm = 1; lm < HK / 32; lm <<= 1) {
-        // lower lane: a + b; upper lane: b - a, i.e. b + (-a): the same
-        // rounded sum either way, with the operand's sign flipped by bit
-        // (exact) instead of a second add and a select
-        const uint32_t flip = (lane & lm) ? 0x80000000u : 0u;
-#pragma unroll
-        for (int j = 0; j < 32; j++) {
-            const float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
-            v[j] = __fadd_rn(o, __uint_as_float(__float_as_uint(v[j]) ^ flip));
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < 32; j++) v[j] = __fmul_rn(v[j], ck);
-}
-
-FP4_DEV float nv_global_from_amax(float amax)
-{
-    return (amax > 0.0f && amax <= kFltMax) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
-}
-
 // s_g as left in *g by amax_kernel: max over CTAs of RN(amax_cta / 2688)
 // equals RN(amax / 2688) (division by a positive constant and rounding are
 // both monotonic), so only the all-zero and the non-finite cases remain,
@@ -157,50 +103,17 @@ FP4_DEV float read_global_scale(float *g, int computed)
     return sg;
 }
 
-// Scale and element encoding of one rotated 32-element unit u, and the stores
-// of its nibbles and scale byte(s) (TransFP4 Eq.(1): MXFP4 power-of-two
-// scale; NVFP4 E4M3 block scale under the tensor scale sg).
+// Encodes one rotated 32-element unit u (encode_unit) and stores its nibbles
+// and scale byte(s) in the tile layout.
 template <int FMT>
 FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, const QuantArgs &a, float sg, float six_sg)
 {
-    if (FMT == FP4_MXFP4) {
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
-        const int e = mx_exponent(amax, a.mx_floor);
-        const float inv = exp2i(-e);
-#pragma unroll
-        for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
-        a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)(e + 127);
-    } else {
-        uint32_t sb2 = 0;
-#pragma unroll
-        for (int b = 0; b < 2; b++) {
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[16 * b + i]));
-            const float t = __fdiv_rn(amax, six_sg);
-            const uint32_t sb = e4m3_rn(t);
-            const float d = __fmul_rn(sg, e4m3_to_f32(sb));
-            const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
-#pragma unroll
-            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
-            sb2 |= sb << (8 * b);
-        }
-        *reinterpret_cast<uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4)) = (uint16_t)sb2;
-    }
     uint4 out;
-    if (!a.round_away) {
-        out.x = e2m1x8_rn(v + 0);
-        out.y = e2m1x8_rn(v + 8);
-        out.z = e2m1x8_rn(v + 16);
-        out.w = e2m1x8_rn(v + 24);
-    } else {
-        out.x = e2m1x8_away(v + 0);
-        out.y = e2m1x8_away(v + 8);
-        out.z = e2m1x8_away(v + 16);
-        out.w = e2m1x8_away(v + 24);
-    }
+    const uint32_t sb = encode_unit<FMT>(v, sg, six_sg, a.round_away, a.mx_floor, out);
+    if (FMT == FP4_MXFP4)
+        a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)sb;
+    else
+        *reinterpret_cast<uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4)) = (uint16_t)sb;
     *reinterpret_cast<uint4 *>(a.q + u * 16) = out;  // q rows are contiguous: row * cols/2 + j * 16 = u * 16
 }
 
@@ -238,8 +151,7 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
             float v[32];
             unpack_unit(raw[i], v);
             if (HK) fwht_unit<HK>(v, a.ck, lane);
-#pragma unroll
-            for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+            m = fmaxf(m, absmax_tree<32>(v));
         }
     }
 #pragma unroll
@@ -373,8 +285,7 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
                     float v[32];
                     unpack_unit(raw[i], v);
                     if (HK) fwht_unit<HK>(v, a.ck, lane);
-#pragma unroll
-                    for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+                    m = fmaxf(m, absmax_tree<32>(v));
                 }
             } else {
                 for (int64_t base = warp * 32; base < a.total_units; base += stride * QUNITS) {
@@ -386,8 +297,7 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
                         float v[32];
                         unpack_unit(r2[i], v);
                         if (HK) fwht_unit<HK>(v, a.ck, lane);
-#pragma unroll
-                        for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(v[j]));
+                        m = fmaxf(m, absmax_tree<32>(v));
                     }
                 }
             }

@@ -314,9 +314,12 @@ def test_linear_online_activation_quantization(fp4, orc, fmt, M, hk):
     assert_close(to_np(c), ref, bound, 0)
 
 
-def test_linear_static_activation_scale(fp4, orc):
+@pytest.mark.parametrize("N,K", [(512, 512), (4096, 2048)])
+def test_linear_static_activation_scale(fp4, orc, N, K):
+    """A given activation tensor scale, with a global split (4 tiles) and a
+    cluster split (32 tiles) of the decode product."""
     import torch
-    M, N, K = 8, 512, 512
+    M = 8
     rng = np.random.default_rng(0)
     x = inputs.f32_to_bf16_bits(rng.laplace(0, 1, (M, K)).astype(np.float32))
     w = inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (N, K)).astype(np.float32))
@@ -332,14 +335,15 @@ def test_linear_static_activation_scale(fp4, orc):
 
 @pytest.mark.parametrize("fmt", [0, 1])
 @pytest.mark.parametrize("M,N,K,hk", [(16, 14336, 4096, 0), (4, 4096, 14336, 0), (3, 40000, 256, 0),
-                                      (2, 20000, 512, 0), (1, 300, 4096, 32), (16, 2048, 2048, 128)])
+                                      (2, 20000, 512, 0), (1, 300, 4096, 32), (16, 2048, 2048, 128),
+                                      (5, 14336, 1024, 64), (8, 4096, 2048, 32), (16, 14336, 512, 16)])
 def test_linear_decode_fused_reduction_matches_gemm(fp4, orc, fmt, M, N, K, hk):
     """fp4_linear's decode path (one-cluster activation quantizer + split-K,
     with partials of a globally split tile summed by the last CTA of the tile)
     gives bit-identical results to fp4_quantize + fp4_gemm (separate reduction
     kernel): the partial sums are added in the same CTA order.  Whole tiles,
-    cluster splits and global splits are all exercised; repeated calls are
-    identical."""
+    cluster splits and global splits, every rotation size and M from 1 to 16
+    are exercised; repeated calls are identical."""
     import torch
     a, w = inputs.decode_linear(M, N, K, seed=N + K)
     xd = to_dev_bf16(a)
