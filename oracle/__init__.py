@@ -80,6 +80,8 @@ def lib():
         L.fp4o_fwht.restype = None
         L.fp4o_quantize.argtypes = [vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp]
         L.fp4o_quantize.restype = i32
+        L.fp4o_quantize_f32.argtypes = [vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+        L.fp4o_quantize_f32.restype = i32
         L.fp4o_dequantize.argtypes = [vp, vp, f32, i64, i64, i32, i32, i32, vp]
         L.fp4o_dequantize.restype = i32
         L.fp4o_scales_to_atoms.argtypes = [vp, i64, i64, vp]
@@ -155,6 +157,22 @@ def quantize(x_bf16: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_E
     g = np.array([gscale if gscale is not None else 0.0], np.float32)
     rc = lib().fp4o_quantize(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie,
                              mx_rule, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
+    if rc != 0:
+        raise ValueError("oracle quantize: invalid arguments")
+    return q, s, (float(g[0]) if fmt == NVFP4 else 1.0)
+
+
+def quantize_f32(x: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_EVEN,
+                 mx_rule: int = MX_CEIL, gscale: float | None = None):
+    """quantize() for fp32 elements (rows, cols): same outputs."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    block = block_of(fmt)
+    q = np.zeros((rows, cols // 2), np.uint8)
+    s = np.zeros((rows, cols // block), np.uint8)
+    g = np.array([gscale if gscale is not None else 0.0], np.float32)
+    rc = lib().fp4o_quantize_f32(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie,
+                                 mx_rule, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
     if rc != 0:
         raise ValueError("oracle quantize: invalid arguments")
     return q, s, (float(g[0]) if fmt == NVFP4 else 1.0)

@@ -195,10 +195,14 @@ static int valid_shape(int fmt, int block, int hk, int64_t rows, int64_t cols)
 }
 
 /* Row r of x as fp32, rotated when hk > 0. */
-static void load_row(const uint16_t *x, int64_t ld, int64_t r, int64_t cols,
-                     int hk, float *y)
+/* One row of the input, as fp32: either bf16 elements (xb) or fp32 elements
+ * (xf, e.g. a product that is quantized again for the next layer); then the
+ * rotation, if any. */
+static void load_row(const uint16_t *xb, const float *xf, int64_t ld, int64_t r,
+                     int64_t cols, int hk, float *y)
 {
-    for (int64_t c = 0; c < cols; c++) y[c] = bf16_to_f32(x[r * ld + c]);
+    for (int64_t c = 0; c < cols; c++)
+        y[c] = xb ? bf16_to_f32(xb[r * ld + c]) : xf[r * ld + c];
     if (hk)
         for (int64_t c = 0; c < cols; c += hk) fp4o_fwht(y + c, hk);
 }
@@ -213,10 +217,10 @@ static float nv_global_scale(float amax_t)
     return 1.0f;
 }
 
-int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                  int fmt, int block, int hadamard_k, int tie, int mx_rule,
-                  int gscale_given, float *gscale,
-                  uint8_t *q, uint8_t *s_logical)
+static int quantize_rows(const uint16_t *xb, const float *xf, int64_t rows, int64_t cols,
+                         int64_t ld, int fmt, int block, int hadamard_k, int tie,
+                         int mx_rule, int gscale_given, float *gscale, uint8_t *q,
+                         uint8_t *s_logical)
 {
     if (!valid_shape(fmt, block, hadamard_k, rows, cols) || ld < cols) return -1;
     const int64_t nkb = cols / block;
@@ -233,7 +237,7 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                 float local = 0.0f;
 #pragma omp for schedule(static)
                 for (int64_t r = 0; r < rows; r++) {
-                    load_row(x, ld, r, cols, hadamard_k, y);
+                    load_row(xb, xf, ld, r, cols, hadamard_k, y);
                     for (int64_t c = 0; c < cols; c++) {
                         float a = fabsf(y[c]);
                         if (a > local) local = a;
@@ -253,7 +257,7 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
         float *y = (float *)malloc(sizeof(float) * (size_t)(cols ? cols : 1));
 #pragma omp for schedule(static)
         for (int64_t r = 0; r < rows; r++) {
-            load_row(x, ld, r, cols, hadamard_k, y);
+            load_row(xb, xf, ld, r, cols, hadamard_k, y);
             uint8_t *qrow = q + r * (cols / 2);
             memset(qrow, 0, (size_t)(cols / 2));
             for (int64_t kb = 0; kb < nkb; kb++) {
@@ -298,6 +302,24 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
         free(y);
     }
     return 0;
+}
+
+int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                  int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                  int gscale_given, float *gscale,
+                  uint8_t *q, uint8_t *s_logical)
+{
+    return quantize_rows(x, NULL, rows, cols, ld, fmt, block, hadamard_k, tie, mx_rule,
+                         gscale_given, gscale, q, s_logical);
+}
+
+int fp4o_quantize_f32(const float *x, int64_t rows, int64_t cols, int64_t ld,
+                      int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                      int gscale_given, float *gscale,
+                      uint8_t *q, uint8_t *s_logical)
+{
+    return quantize_rows(NULL, x, rows, cols, ld, fmt, block, hadamard_k, tie, mx_rule,
+                         gscale_given, gscale, q, s_logical);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -52,6 +52,13 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                   int gscale_given, float *gscale,
                   uint8_t *q, uint8_t *s_logical);
 
+/* The same with fp32 elements (row stride ld floats): a product quantized
+ * again, e.g. for the next layer. */
+int fp4o_quantize_f32(const float *x, int64_t rows, int64_t cols, int64_t ld,
+                      int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                      int gscale_given, float *gscale,
+                      uint8_t *q, uint8_t *s_logical);
+
 /* out: rows x cols fp32.  hadamard_k > 0 applies the (self-inverse)
  * rotation again to return to the original domain. */
 int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,

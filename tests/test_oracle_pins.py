@@ -431,3 +431,52 @@ def test_table5_nmse_directional(orc):
         assert got["nvfp4"] < got["rot_mxfp4"] < got["mxfp4"]
         for m, v in want.items():
             assert v / 2 < got[m] < v * 2, (key, m, got[m], v)
+
+
+# ---- quantization of fp32 elements (a product quantized for the next layer) ----
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("hk,tie", [(0, 0), (32, 0), (0, 1)])
+def test_quantize_f32_equals_bf16_path_on_bf16_values(orc, fmt, hk, tie):
+    """Widening bf16 to fp32 is exact, so the fp32 entry point must give the
+    bf16 one's bytes on every bf16 tensor."""
+    x = inputs.quant_sweep(rows=24, cols=1024, seed=17)
+    a = orc.quantize(x, fmt, hadamard_k=hk, tie=tie)
+    b = orc.quantize_f32(inputs.bf16_bits_to_f32(x), fmt, hadamard_k=hk, tie=tie)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and a[2] == b[2]
+
+
+@pytest.mark.parametrize("tie", [0, 1])
+def test_quantize_f32_brute_force_nearest(orc, tie):
+    """Blocks whose largest magnitude is exactly 6 get scale 1 (MXFP4 byte 127;
+    NVFP4 with s_g = 1: block scale 1.0 = 0x38), so every other element's code
+    must be the nearest E2M1 value found by brute force over the grid, ties by
+    the rule; the values are fp32 ones a bf16 tensor cannot hold."""
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    rng = np.random.default_rng(23)
+    v = rng.uniform(-6, 6, (8, 64)).astype(np.float32)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    v[:, 1:8] = mids                                  # exact midpoints
+    v[:, 8:15] = np.nextafter(mids, np.float32(10))   # just above them
+    v[:, 15:22] = np.nextafter(mids, np.float32(-10)) # just below them
+    v[:, 0] = 6.0
+    v[:, 32] = -6.0                                   # second MX block's max, both NV blocks of it too
+    v[:, 16] = 6.0                                    # the other NV blocks' max
+    v[:, 48] = 6.0
+
+    def nearest(a):
+        d = np.abs(grid - abs(float(a)))
+        best = np.flatnonzero(d == d.min())
+        if len(best) > 1:  # a midpoint
+            i = best[-1] if tie == 1 else (best[0] if best[0] % 2 == 0 else best[1])
+        else:
+            i = best[0]
+        return int(i) | (8 if np.signbit(a) else 0)
+
+    want = np.array([[nearest(a) for a in row] for row in v])
+    for fmt, gs in ((0, None), (1, 1.0)):
+        q, s, _ = orc.quantize_f32(v, fmt, tie=tie, gscale=gs)
+        codes = np.zeros_like(want)
+        codes[:, 0::2] = q & 0xF
+        codes[:, 1::2] = q >> 4
+        assert np.array_equal(codes, want), fmt
+        assert np.all(s == (127 if fmt == 0 else 0x38))
