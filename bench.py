@@ -179,7 +179,18 @@ def bench_prefill(torch, fp4, inputs, dev, reps: int, M: int = 8192, fmts=None):
         q_ms = time_graph(torch, lambda: fp4.quantize(ad, fmt, out=A), 3, reps)
         out[name]["act_quantize_ms"] = q_ms
         out[name]["tflops_incl_act_quantize"] = 2.0 * M * N * K / ((ms + q_ms) * 1e-3) / 1e12
-        del A, W
+        # C quantized for the next layer in the GEMM epilogue (NVFP4 with a
+        # given tensor scale), against BF16 C followed by a quantize pass.
+        gC = torch.full((1,), 0.05, dtype=torch.float32, device=dev)
+        Cq = fp4.gemm_quantized(A, W, M, N, K, fmt, fmt, gscale=gC if fmt == fp4.FP4_NVFP4 else None)
+        fq_ms = time_graph(torch, lambda: fp4.gemm_quantized(A, W, M, N, K, fmt, fmt, out=Cq), 3, reps)
+        gs = gC if fmt == fp4.FP4_NVFP4 else None
+        Cb = fp4.quantize(C, fmt, gscale=gs)
+        cq_ms = time_graph(torch, lambda: fp4.quantize(C, fmt, gscale=gs, out=Cb), 3, reps)
+        out[name]["quantized_out"] = {"ms": fq_ms, "tflops": 2.0 * M * N * K / (fq_ms * 1e-3) / 1e12,
+                                      "frac": 2.0 * M * N * K / (fq_ms * 1e-3) / 1e12 / peak,
+                                      "unfused_bf16_then_quantize_ms": ms + cq_ms}
+        del A, W, Cq, Cb
     del ad, wd, C
     torch.cuda.empty_cache()
     return out

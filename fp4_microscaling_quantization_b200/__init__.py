@@ -14,7 +14,8 @@ from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_NVFP4, 
                    FP4_OUT_F32, FP4_ROUND_AWAY, FP4_ROUND_EVEN, Fp4Error)
 
 __all__ = [
-    "quantize", "dequantize", "gemm", "linear", "linear_workspace_size", "quantize_sizes", "gemm_workspace_size", "check_device_status",
+    "quantize", "dequantize", "gemm", "gemm_quantized", "linear", "linear_workspace_size", "quantize_sizes",
+    "gemm_workspace_size", "check_device_status",
     "FP4_MXFP4", "FP4_NVFP4", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
     "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "Fp4Error", "block_of",
 ]
@@ -121,6 +122,37 @@ def gemm(a, w, M: int, N: int, K: int, fmt, out_dtype: int = FP4_OUT_BF16, out=N
         M, N, K, fmt, int(out_dtype), out.data_ptr(), out.stride(0), wp, wb,
         _stream_handle(torch, Aq.device)))
     return out
+
+
+def gemm_quantized(a, w, M: int, N: int, K: int, fmt, out_fmt, gscale=None, round: int = FP4_ROUND_EVEN,
+                   mx_scale_rule: int = FP4_MX_SCALE_CEIL, out=None):
+    """C = A W^T quantized along N for the next layer, in the GEMM's epilogue.
+
+    a = (Aq, As, gA), w = (Wq, Ws, gW) as for :func:`gemm`.  Returns
+    (Cq, Cs, gC) like :func:`quantize`: Cq (M, N/2) packed nibbles, Cs the
+    tile-layout scales, gC the NVFP4 tensor scale of C, which must be given
+    (``gscale``) for an NVFP4 output.
+    """
+    import torch
+
+    fmt, out_fmt = _fmt(fmt), _fmt(out_fmt)
+    Aq, As, gA = a
+    Wq, Ws, gW = w
+    qb, sb = quantize_sizes(M, N, out_fmt)
+    if out is None:
+        Cq = torch.empty((M, N // 2), dtype=torch.uint8, device=Aq.device)
+        Cs = torch.empty((sb,), dtype=torch.uint8, device=Aq.device)
+        gC = torch.ones((1,), dtype=torch.float32, device=Aq.device)
+    else:
+        Cq, Cs, gC = out
+    if gscale is not None:
+        gC.copy_(gscale.reshape(1).to(torch.float32))
+    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(gscale is not None))
+    _lib.check("fp4_gemm_quantized", _lib.lib().fp4_gemm_quantized(
+        Aq.data_ptr(), As.data_ptr(), gA.data_ptr(), Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(),
+        M, N, K, fmt, out_fmt, ctypes.byref(opts), gC.data_ptr() if out_fmt == FP4_NVFP4 else None,
+        Cq.data_ptr(), Cs.data_ptr(), _stream_handle(torch, Aq.device)))
+    return Cq, Cs, gC
 
 
 def linear_workspace_size(M: int, N: int, K: int, fmt) -> int:

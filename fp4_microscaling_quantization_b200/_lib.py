@@ -37,6 +37,8 @@ SIGNATURES = {
     "fp4_gemm_workspace_size": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_sz)]),
     "fp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _i64,
                         _vp, _sz, _vp]),
+    "fp4_gemm_quantized": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp,
+                                  _vp, _vp]),
     "fp4_check_device_status": (_int, [_vp]),
     "fp4_linear_workspace_size": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_sz)]),
     "fp4_linear": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _int, _vp, _i64,

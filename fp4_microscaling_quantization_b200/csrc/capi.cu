@@ -24,6 +24,10 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
                                 int round_away, int mx_floor, int gscale_given, uint8_t *q, uint8_t *s, float *gscale,
                                 unsigned *zero, int nzero, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int sms);
+cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
+                                  const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K, int fmt,
+                                  int out_fmt, int round_away, int mx_floor, const float *gC, uint8_t *Cq, uint8_t *Cs,
+                                  int sms, cudaStream_t st);
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -245,6 +249,33 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     e = fp4::launch_gemm(aq, as, ga, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc, base + L.gemm,
                          L.counters - L.gemm, sms, st, &bad, true, counters, decode);
     if (bad) return FP4_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
+                              const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K, int fmt,
+                              int out_fmt, const fp4_opts *opts, const float *gC, uint8_t *Cq, uint8_t *Cs,
+                              void *stream)
+{
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0};
+    if (opts) o = *opts;
+    if (M < 0 || N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (out_fmt != FP4_MXFP4 && out_fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
+    if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
+    if (M <= 16 || K % 256 || N % 128) return FP4_ERR_UNSUPPORTED;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP4_ERR_UNSUPPORTED;
+    if (!Aq || !As || !Wq || !Ws || !Cq || !Cs) return FP4_ERR_INVALID_ARG;
+    if (fmt == FP4_NVFP4 && (!gA || !gW)) return FP4_ERR_INVALID_ARG;
+    if (out_fmt == FP4_NVFP4 && !gC) return FP4_ERR_INVALID_ARG;
+    if (!aligned(Aq, 16) || !aligned(Wq, 16) || !aligned(As, 16) || !aligned(Ws, 16) || !aligned(Cq, 16) ||
+        !aligned(Cs, 16))
+        return FP4_ERR_ALIGNMENT;
+    if (gC && !aligned(gC, 4)) return FP4_ERR_ALIGNMENT;
+    cudaError_t e = fp4::launch_gemm_quantized(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_fmt,
+                                               o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
+                                               gC, Cq, Cs, sm_count(), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 

@@ -20,6 +20,7 @@
 #include <atomic>
 #include <mutex>
 
+#include "encode.cuh"
 #include "sm100.cuh"
 
 namespace fp4 {
@@ -71,11 +72,19 @@ struct PCfg {
     static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "TMEM budget");
 };
 
+// Output modes of the prefill kernel.
+enum { OUT_F32 = 0, OUT_BF16 = 1, OUT_MXFP4 = 2, OUT_NVFP4 = 3 };
+
 struct PParams {
     const float *gA;
     const float *gW;
-    void *C;
+    void *C;             // fp32 / bf16 C, or the packed FP4 elements of C (M x N/2 bytes)
     int64_t ldc;
+    // FP4 output (the product quantized again along N for the next layer):
+    uint8_t *Cs;         // scales in the tile layout
+    const float *gC;     // NVFP4: the given tensor scale of C
+    int nkb4c;           // ceil(N / block / 4)
+    int round_away, mx_floor;
     int M, N, K;
     int nkb4;
     int num_m_tiles, num_n_tiles;
@@ -83,7 +92,7 @@ struct PParams {
     int stall;           // failure-detection test: the producer issues no loads
 };
 
-template <int FMT, int BF16OUT, int CG>
+template <int FMT, int OUT, int CG>
 __global__ void __launch_bounds__(384, 1)
 pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
              const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, PParams p)
@@ -260,6 +269,7 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         __syncwarp();
     } else {
         // ---------------- epilogue: warps 2..9 ----------------
+        constexpr bool BF16OUT = OUT == OUT_BF16;
         const int quarter = warp & 3;          // TMEM lanes this warp may read
         const int half = (warp - 2) >> 2;      // accumulator columns [128*half, 128*half + 128)
         const bool vec32 = BF16OUT ? (p.ldc % 16 == 0) : (p.ldc % 8 == 0);
@@ -287,7 +297,35 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
             const int m = (mt * CG + (int)rank) * Cfg::BM + quarter * 32 + lane;
             const int n0 = nt * Cfg::BN + half * 128;
-            if (m < p.M && n0 < p.N) {
+            if (OUT >= OUT_MXFP4) {
+                // C quantized along N for the next layer: this thread's 128
+                // columns are 4 units of 32 (encode.cuh, as in the quantize
+                // kernels); rows past M (up to the tile layout's padding to
+                // 128 rows) get zero scales and no elements.
+                constexpr int QF = OUT == OUT_MXFP4 ? FP4_MXFP4 : FP4_NVFP4;
+                const float sgc = (QF == FP4_NVFP4) ? *p.gC : 1.0f;
+                const float six_sgc = __fmul_rn(6.0f, sgc);
+                uint8_t *cq = static_cast<uint8_t *>(p.C);
+                const bool in_layout = m < (p.M + 127) / 128 * 128;  // the scale tile layout's rows
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const int n = n0 + 32 * u;
+                    if (n >= p.N || !in_layout) break;
+                    float v[32];
+#pragma unroll
+                    for (int e = 0; e < 32; e++) v[e] = __fmul_rn(__uint_as_float(r[32 * u + e]), alpha);
+                    uint4 nib;
+                    uint32_t sb = encode_unit<QF>(v, sgc, six_sgc, p.round_away, p.mx_floor, nib);
+                    if (m < p.M)
+                        *reinterpret_cast<uint4 *>(cq + (int64_t)m * (p.N / 2) + n / 2) = nib;
+                    else
+                        sb = 0;
+                    if (QF == FP4_MXFP4)
+                        p.Cs[scale_offset(m, n / 32, p.nkb4c)] = (uint8_t)sb;
+                    else
+                        *reinterpret_cast<uint16_t *>(p.Cs + scale_offset(m, n / 16, p.nkb4c)) = (uint16_t)sb;
+                }
+            } else if (m < p.M && n0 < p.N) {
                 if (BF16OUT) {
                     __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(p.C) + (int64_t)m * p.ldc + n0;
                     const bool fast = vec32 && aligned_c && n0 + 128 <= p.N;
@@ -849,7 +887,7 @@ static bool make_sf_map(CUtensorMap *m, const void *base, int64_t n_atoms, int b
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int BF, int CG>
+template <int FMT, int OUT, int CG>
 static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq, const uint8_t *Ws,
                                 const PParams &p, int sms, cudaStream_t st, bool pdl)
 {
@@ -860,7 +898,7 @@ static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint
     if (!make_fp4_map(&ta, Aq, p.M, p.K, Cfg::BM) || !make_fp4_map(&tb, Wq, p.N, p.K, Cfg::B_ROWS) ||
         !make_sf_map(&tsa, As, nrb_a * p.nkb4, KA) || !make_sf_map(&tsb, Ws, nrb_w * p.nkb4, KA))
         return cudaErrorInvalidValue;
-    auto kern = pgemm_kernel<FMT, BF, CG>;
+    auto kern = pgemm_kernel<FMT, OUT, CG>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
@@ -887,15 +925,25 @@ static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint
     return cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p);
 }
 
+template <int FMT, int CG>
+static cudaError_t launch_pgemm_out(int out, const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq, const uint8_t *Ws,
+                                    const PParams &p, int sms, cudaStream_t st, bool pdl)
+{
+    switch (out) {
+    case OUT_F32: return launch_pgemm<FMT, OUT_F32, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
+    case OUT_BF16: return launch_pgemm<FMT, OUT_BF16, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
+    case OUT_MXFP4: return launch_pgemm<FMT, OUT_MXFP4, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
+    case OUT_NVFP4: return launch_pgemm<FMT, OUT_NVFP4, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
+    }
+    return cudaErrorInvalidValue;
+}
+
 template <int CG>
-static cudaError_t launch_pgemm_fmt(int fmt, int bf16out, const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq,
+static cudaError_t launch_pgemm_fmt(int fmt, int out, const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq,
                                     const uint8_t *Ws, const PParams &p, int sms, cudaStream_t st, bool pdl)
 {
-    if (fmt == FP4_MXFP4)
-        return bf16out ? launch_pgemm<FP4_MXFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st, pdl)
-                       : launch_pgemm<FP4_MXFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
-    return bf16out ? launch_pgemm<FP4_NVFP4, 1, CG>(Aq, As, Wq, Ws, p, sms, st, pdl)
-                   : launch_pgemm<FP4_NVFP4, 0, CG>(Aq, As, Wq, Ws, p, sms, st, pdl);
+    return fmt == FP4_MXFP4 ? launch_pgemm_out<FP4_MXFP4, CG>(out, Aq, As, Wq, Ws, p, sms, st, pdl)
+                            : launch_pgemm_out<FP4_NVFP4, CG>(out, Aq, As, Wq, Ws, p, sms, st, pdl);
 }
 
 // CTA-pair (2-SM MMA) tiles are used once A spans more than one 128-row block.
@@ -1006,6 +1054,10 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         pp.gW = gW;
         pp.C = C;
         pp.ldc = ldc;
+        pp.Cs = nullptr;
+        pp.gC = nullptr;
+        pp.nkb4c = 0;
+        pp.round_away = pp.mx_floor = 0;
         pp.M = (int)M;
         pp.N = (int)N;
         pp.K = (int)K;
@@ -1015,9 +1067,42 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         const int cg = pgemm_cta_group(M);
         pp.num_m_tiles = (int)((M + 128 * cg - 1) / (128 * cg));
         pp.num_n_tiles = (int)((N + 255) / 256);
-        return cg == 2 ? launch_pgemm_fmt<2>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st, pdl)
-                       : launch_pgemm_fmt<1>(fmt, bf16out, Aq, As, Wq, Ws, pp, sms, st, pdl);
+        const int out = bf16out ? OUT_BF16 : OUT_F32;
+        return cg == 2 ? launch_pgemm_fmt<2>(fmt, out, Aq, As, Wq, Ws, pp, sms, st, pdl)
+                       : launch_pgemm_fmt<1>(fmt, out, Aq, As, Wq, Ws, pp, sms, st, pdl);
     }
+}
+
+// C = A W^T quantized along N by the prefill kernel's epilogue (M > 16,
+// K % 256 == 0, N % 128 == 0; checked by the caller).
+cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
+                                  const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K, int fmt,
+                                  int out_fmt, int round_away, int mx_floor, const float *gC, uint8_t *Cq, uint8_t *Cs,
+                                  int sms, cudaStream_t st)
+{
+    PParams pp;
+    pp.gA = gA;
+    pp.gW = gW;
+    pp.C = Cq;
+    pp.ldc = N / 2;
+    pp.Cs = Cs;
+    pp.gC = gC;
+    pp.nkb4c = (int)((N / (out_fmt == FP4_MXFP4 ? 32 : 16) + 3) / 4);
+    pp.round_away = round_away;
+    pp.mx_floor = mx_floor;
+    pp.M = (int)M;
+    pp.N = (int)N;
+    pp.K = (int)K;
+    pp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+    uint64_t budget = g_inject_budget.exchange(0);
+    pp.budget_ns = budget ? budget : kWaitBudgetNs;
+    pp.stall = g_inject_stall.exchange(0);
+    const int cg = pgemm_cta_group(M);
+    pp.num_m_tiles = (int)((M + 128 * cg - 1) / (128 * cg));
+    pp.num_n_tiles = (int)((N + 255) / 256);
+    const int out = out_fmt == FP4_MXFP4 ? OUT_MXFP4 : OUT_NVFP4;
+    return cg == 2 ? launch_pgemm_fmt<2>(fmt, out, Aq, As, Wq, Ws, pp, sms, st, true)
+                   : launch_pgemm_fmt<1>(fmt, out, Aq, As, Wq, Ws, pp, sms, st, true);
 }
 
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err)

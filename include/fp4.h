@@ -151,6 +151,36 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA,
                     void *C, int64_t ldc, void *workspace, size_t ws_bytes,
                     void *stream);
 
+/*
+ * fp4_gemm_quantized — the product of fp4_gemm, C = alpha * A W^T with FP32
+ * accumulation, quantized again along N in the tensor-core kernel's epilogue
+ * for the next layer, which then takes C as its activations: the "custom
+ * epilogue fusing quantization and scale computation" that "FP4
+ * quantization analysis: MXFP4 vs NVFP4" §3.3 describes for QuTLASS, with
+ * the per-unit encoding of fp4_quantize (TransFP4 §1.1 Eq.(1)) applied to
+ * the FP32 values alpha * acc.
+ *   Aq/As/gA, Wq/Ws/gW, fmt   as for fp4_gemm.
+ *   out_fmt   FP4_MXFP4 or FP4_NVFP4 (may differ from fmt).
+ *   opts      round and mx_scale_rule as for fp4_quantize; may be NULL.
+ *   gC        NVFP4 output: the tensor scale s_g of C, one device fp32, given
+ *             (a whole-tensor maximum is not known until every tile is done,
+ *             so it is not computed here).  Ignored for MXFP4.
+ *   Cq        output, M x N/2 bytes of packed elements, 16-byte aligned.
+ *   Cs        output, the scales in the tile layout of fp4_quantize
+ *             (fp4_quantize_sizes(M, N, out_fmt, ...) bytes; the padding rows
+ *             are written 0), 16-byte aligned.
+ * Shapes: M > 16 (the tiled kernel), K multiple of 256, N multiple of 128;
+ * otherwise FP4_ERR_UNSUPPORTED with nothing launched.  Each 32-element unit
+ * is encoded as fp4_quantize encodes one, from the FP32 values fp4_gemm
+ * returns with FP4_OUT_F32 for the same operands.
+ */
+fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float *gA,
+                              const uint8_t *Wq, const uint8_t *Ws, const float *gW,
+                              int64_t M, int64_t N, int64_t K, int fmt, int out_fmt,
+                              const fp4_opts *opts, const float *gC, uint8_t *Cq,
+                              uint8_t *Cs, void *stream);
+
+
 /* Bytes of device scratch fp4_linear needs (quantized activations, their
  * scales and tensor scale, and the GEMM workspace).  Host-only. */
 fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes);

@@ -99,6 +99,21 @@ def test_gemm_rejects_on_host(L):
     assert g(FAKE + 2, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 8, None, 0, None) == 3
 
 
+def test_gemm_quantized_rejects_on_host(L):
+    g = L.fp4_gemm_quantized
+    F = FAKE
+    assert g(F, F, F, F, F, F, 16, 256, 256, 0, 0, None, None, F, F, None) == 2      # M <= 16: decode shapes
+    assert g(F, F, F, F, F, F, 256, 192, 256, 0, 0, None, None, F, F, None) == 2     # N % 128
+    assert g(F, F, F, F, F, F, 256, 256, 128, 0, 0, None, None, F, F, None) == 2     # K % 256
+    assert g(F, F, F, F, F, F, 256, 256, 256, 0, 3, None, None, F, F, None) == 2     # output format
+    assert g(F, F, F, F, F, F, 256, 256, 256, 0, 1, None, None, F, F, None) == 1     # NVFP4 out needs gC
+    assert g(F, F, None, F, F, F, 256, 256, 256, 1, 0, None, None, F, F, None) == 1  # NVFP4 in needs gA
+    assert g(F, F, F, F, F, F, 256, 256, 256, 0, 0, None, None, None, F, None) == 1  # Cq
+    assert g(F, F, F, F, F, F, 256, 256, 256, 0, 0, None, None, F + 4, F, None) == 3
+    o = _lib.Fp4Opts(7, 0, 0)
+    assert g(F, F, F, F, F, F, 256, 256, 256, 0, 0, ctypes.byref(o), None, F, F, None) == 1
+
+
 def test_empty_mx_is_noop(L):
     assert L.fp4_quantize(None, 0, 64, 64, 0, 32, 0, None, None, None, None, None) == 0
     assert L.fp4_dequantize(None, None, None, 0, 64, 0, 32, 0, 0, None, None) == 0
