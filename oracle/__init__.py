@@ -18,6 +18,9 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   quantize / dequantize   pinned: worked examples, power-of-two invariants,
                           Eq.(2) norm identity
   gemm reference          pinned: numpy fp64 matmul
+  MSE block-scale search  pinned: hand-derived blocks, exhaustive numpy search
+                          over every representable scale, nearest-element
+                          property (tests/test_oracle_mse_pins.py)
   NMSE vs the page's table   directional only (the page's generator is unknown)
 """
 from __future__ import annotations
@@ -35,6 +38,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 MXFP4, NVFP4 = 0, 1
 TIE_EVEN, TIE_AWAY = 0, 1
 MX_CEIL, MX_FLOOR = 0, 1
+SCALE_ABSMAX, SCALE_MSE = 0, 1
 
 
 def build(force: bool = False) -> str:
@@ -78,9 +82,9 @@ def lib():
         L.fp4o_hadamard_ck.restype = f32
         L.fp4o_fwht.argtypes = [vp, i32]
         L.fp4o_fwht.restype = None
-        L.fp4o_quantize.argtypes = [vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+        L.fp4o_quantize.argtypes = [vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp]
         L.fp4o_quantize.restype = i32
-        L.fp4o_quantize_f32.argtypes = [vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+        L.fp4o_quantize_f32.argtypes = [vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp]
         L.fp4o_quantize_f32.restype = i32
         L.fp4o_dequantize.argtypes = [vp, vp, f32, i64, i64, i32, i32, i32, vp]
         L.fp4o_dequantize.restype = i32
@@ -143,8 +147,9 @@ def fwht(y: np.ndarray, k: int) -> np.ndarray:
 
 # ---- tensors ----------------------------------------------------------------
 def quantize(x_bf16: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_EVEN,
-             mx_rule: int = MX_CEIL, gscale: float | None = None):
-    """x_bf16: (rows, cols) uint16 bf16 bit patterns.
+             mx_rule: int = MX_CEIL, gscale: float | None = None, search: int = SCALE_ABSMAX):
+    """x_bf16: (rows, cols) uint16 bf16 bit patterns.  search: SCALE_ABSMAX
+    or SCALE_MSE (block scales by the MSE search; mx_rule is then unused).
 
     Returns (q, s_logical, s_g): q (rows, cols/2) uint8 packed nibbles,
     s_logical (rows, cols/block) uint8, s_g the NVFP4 tensor scale (1.0 for MX).
@@ -156,14 +161,14 @@ def quantize(x_bf16: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_E
     s = np.zeros((rows, cols // block), np.uint8)
     g = np.array([gscale if gscale is not None else 0.0], np.float32)
     rc = lib().fp4o_quantize(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie,
-                             mx_rule, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
+                             mx_rule, search, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
     if rc != 0:
         raise ValueError("oracle quantize: invalid arguments")
     return q, s, (float(g[0]) if fmt == NVFP4 else 1.0)
 
 
 def quantize_f32(x: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_EVEN,
-                 mx_rule: int = MX_CEIL, gscale: float | None = None):
+                 mx_rule: int = MX_CEIL, gscale: float | None = None, search: int = SCALE_ABSMAX):
     """quantize() for fp32 elements (rows, cols): same outputs."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     rows, cols = x.shape
@@ -172,7 +177,7 @@ def quantize_f32(x: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_EV
     s = np.zeros((rows, cols // block), np.uint8)
     g = np.array([gscale if gscale is not None else 0.0], np.float32)
     rc = lib().fp4o_quantize_f32(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie,
-                                 mx_rule, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
+                                 mx_rule, search, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
     if rc != 0:
         raise ValueError("oracle quantize: invalid arguments")
     return q, s, (float(g[0]) if fmt == NVFP4 else 1.0)

@@ -18,7 +18,9 @@
  *   [Explainer] "MXFP4 quantization explainer" (AI Daily 2026-08-05), §3:
  *               32-element blocks, scale maps the block max to the FP4 max.
  *   [MR-GPTQ]   "FP4 quantization analysis: MXFP4 vs NVFP4" (jsqmd.com),
- *               §3.2.3: block-diagonal Hadamard H_k, k in {16,32,64,128}.
+ *               §3.2.3: block-diagonal Hadamard H_k, k in {16,32,64,128};
+ *               §3.2.1: block scales chosen to minimise the squared error
+ *               sum ||Y^_i - X_i||^2; §3.3: "MSE" and "Abs-Max" methods.
  *   [gpt-oss]   "gpt-oss MXFP4" article (juejin.cn), MXFP4 section: the
  *               worked example 0.0625, 0.375, 0.078125, 0.25.
  *
@@ -27,7 +29,9 @@
  * MXFP4 scale exponent = the smallest power of two that keeps the block
  * max <= 6 (default) or the OCP floor rule; E8M0 bias 127; NVFP4 global
  * scale s_g = amax/(6*448); one reciprocal per NVFP4 block, then a multiply;
- * the rotation is the normalised Sylvester FWHT along K, stages h ascending.
+ * the rotation is the normalised Sylvester FWHT along K, stages h ascending;
+ * the MSE method searches a fixed window of scales around the absmax one
+ * and compares fp32 block errors summed in a fixed pairwise order.
  */
 #include "fp4_oracle.h"
 
@@ -217,12 +221,105 @@ static float nv_global_scale(float amax_t)
     return 1.0f;
 }
 
+/* The absmax scale byte of one block ([TransFP4] §3.1): MX the E8M0 byte of
+ * fp4o_mx_scale_exponent(amax, rule); NV the E4M3 code of t = amax / (6 s_g). */
+static int absmax_scale_byte(const float *blk, int block, int fmt, int mx_rule, float sg)
+{
+    float amax_b = 0.0f;
+    for (int i = 0; i < block; i++)
+        if (fabsf(blk[i]) > amax_b) amax_b = fabsf(blk[i]);
+    if (fmt == FP4O_MXFP4) return fp4o_mx_scale_exponent(amax_b, mx_rule) + 127;
+    float six_sg = 6.0f * sg;
+    return fp4o_e4m3_encode(amax_b / six_sg);
+}
+
+/* Elements of one block under a given scale byte ([TransFP4] Eq.(1),
+ * q_i = Q_f(x_i / d)).  MX: d = 2^e, and x / 2^e is the exact product
+ * x * 2^-e.  NV: d = s_g * s_b, the values are multiplied by r = 1/d
+ * (clamped to the largest float); d = 0 gives signed zeros. */
+static void encode_block(const float *blk, int block, int fmt, int sbyte, float sg, int tie,
+                         int *codes)
+{
+    if (fmt == FP4O_MXFP4) {
+        float inv = ldexpf(1.0f, -(sbyte - 127));
+        for (int i = 0; i < block; i++) codes[i] = fp4o_e2m1_encode(blk[i] * inv, tie);
+        return;
+    }
+    float d = sg * (float)fp4o_e4m3_decode(sbyte);
+    if (d == 0.0f) {
+        for (int i = 0; i < block; i++) codes[i] = signbit(blk[i]) ? 8 : 0;
+        return;
+    }
+    float rcp = 1.0f / d;
+    if (rcp > FLT_MAX) rcp = FLT_MAX;
+    for (int i = 0; i < block; i++) codes[i] = fp4o_e2m1_encode(blk[i] * rcp, tie);
+}
+
+/* Squared reconstruction error of one encoded block ([MR-GPTQ] §3.2.1,
+ * sum_i (Y^_i - X_i)^2 with Y^_i = d * q_i), one fp32 operation per step:
+ * y_i = RN(q_i * d), e_i = RN(x_i - y_i), e_i^2 rounded; then a fixed
+ * pairwise sum: adjacent pairs first, then the first half of the partial
+ * sums plus the second half, until one value remains. */
+static float block_sse(const float *blk, int block, int fmt, int sbyte, float sg, const int *codes)
+{
+    float d = (fmt == FP4O_MXFP4) ? ldexpf(1.0f, sbyte - 127) : sg * (float)fp4o_e4m3_decode(sbyte);
+    float t[32];
+    for (int i = 0; i < block; i++) {
+        float y = (float)fp4o_e2m1_decode(codes[i]) * d;
+        float e = blk[i] - y;
+        t[i] = e * e;
+    }
+    for (int i = 0; i < block / 2; i++) t[i] = t[2 * i] + t[2 * i + 1];
+    for (int w = block / 4; w >= 1; w /= 2)
+        for (int i = 0; i < w; i++) t[i] = t[i] + t[i + w];
+    return t[0];
+}
+
+/* The "MSE" method ([MR-GPTQ] §3.2.1, §3.3): of a short list of candidate
+ * scales around the absmax one, the block takes the one whose encoding has
+ * the smallest block_sse; of equal ones the first.  Candidates, in order:
+ *   MX: e_c, then e_c - 1 (above -127 only), e_c the CEIL exponent; the
+ *       FLOOR rule's exponent is one of the two.  Larger exponents only
+ *       coarsen the grid; smaller ones clip the block max to half or less.
+ *   NV: t0, then t0 - 2, t0 - 1, t0 + 1, ..., t0 + 6, t0 the absmax E4M3
+ *       code; only codes 1 .. 0x7E (0x7F is NaN, 0 zeroes the block).  The
+ *       window maps the block max to between about 3.6 and 7.3 on the E2M1
+ *       grid: below 6 the top of the grid (spacing 2 between 4 and 6) may
+ *       serve the largest values of a block better.
+ * Writes the chosen block's codes and returns its scale byte. */
+static int mse_scale_byte(const float *blk, int block, int fmt, float sg, int tie, int *codes)
+{
+    int cand[9], nc = 0;
+    int s0 = absmax_scale_byte(blk, block, fmt, FP4O_MX_CEIL, sg);
+    cand[nc++] = s0;
+    if (fmt == FP4O_MXFP4) {
+        if (s0 > 0) cand[nc++] = s0 - 1;
+    } else {
+        for (int j = -2; j <= 6; j++)
+            if (j != 0 && s0 + j >= 1 && s0 + j <= 0x7E) cand[nc++] = s0 + j;
+    }
+    int best = -1;
+    float best_sse = 0.0f;
+    int trial[32];
+    for (int c = 0; c < nc; c++) {
+        encode_block(blk, block, fmt, cand[c], sg, tie, trial);
+        float e = block_sse(blk, block, fmt, cand[c], sg, trial);
+        if (best < 0 || e < best_sse) {
+            best = cand[c];
+            best_sse = e;
+            memcpy(codes, trial, sizeof(int) * (size_t)block);
+        }
+    }
+    return best;
+}
+
 static int quantize_rows(const uint16_t *xb, const float *xf, int64_t rows, int64_t cols,
                          int64_t ld, int fmt, int block, int hadamard_k, int tie,
-                         int mx_rule, int gscale_given, float *gscale, uint8_t *q,
+                         int mx_rule, int search, int gscale_given, float *gscale, uint8_t *q,
                          uint8_t *s_logical)
 {
     if (!valid_shape(fmt, block, hadamard_k, rows, cols) || ld < cols) return -1;
+    if (search != FP4O_SCALE_ABSMAX && search != FP4O_SCALE_MSE) return -1;
     const int64_t nkb = cols / block;
 
     float sg = 1.0f;
@@ -262,37 +359,15 @@ static int quantize_rows(const uint16_t *xb, const float *xf, int64_t rows, int6
             memset(qrow, 0, (size_t)(cols / 2));
             for (int64_t kb = 0; kb < nkb; kb++) {
                 const float *blk = y + kb * block;
-                float amax_b = 0.0f;
-                for (int i = 0; i < block; i++)
-                    if (fabsf(blk[i]) > amax_b) amax_b = fabsf(blk[i]);
-
                 int codes[32];
-                uint8_t sbyte;
-                if (fmt == FP4O_MXFP4) {
-                    /* Power-of-two scale: x / 2^e is a plain exponent shift. */
-                    int e = fp4o_mx_scale_exponent(amax_b, mx_rule);
-                    sbyte = (uint8_t)(e + 127);
-                    float inv = ldexpf(1.0f, -e);
-                    for (int i = 0; i < block; i++)
-                        codes[i] = fp4o_e2m1_encode(blk[i] * inv, tie);
+                int sbyte;
+                if (search == FP4O_SCALE_MSE) {
+                    sbyte = mse_scale_byte(blk, block, fmt, sg, tie, codes);
                 } else {
-                    /* Two-level scale: t = amax_b / (6 s_g) is stored as E4M3,
-                     * d = s_g * s_b, values are multiplied by r = 1/d. */
-                    float six_sg = 6.0f * sg;
-                    float t = amax_b / six_sg;
-                    int sb = fp4o_e4m3_encode(t);
-                    sbyte = (uint8_t)sb;
-                    float d = sg * (float)fp4o_e4m3_decode(sb);
-                    if (d == 0.0f) {
-                        for (int i = 0; i < block; i++) codes[i] = signbit(blk[i]) ? 8 : 0;
-                    } else {
-                        float rcp = 1.0f / d;
-                        if (rcp > FLT_MAX) rcp = FLT_MAX;
-                        for (int i = 0; i < block; i++)
-                            codes[i] = fp4o_e2m1_encode(blk[i] * rcp, tie);
-                    }
+                    sbyte = absmax_scale_byte(blk, block, fmt, mx_rule, sg);
+                    encode_block(blk, block, fmt, sbyte, sg, tie, codes);
                 }
-                s_logical[r * nkb + kb] = sbyte;
+                s_logical[r * nkb + kb] = (uint8_t)sbyte;
                 for (int i = 0; i < block; i++) {
                     int64_t c = kb * block + i;
                     qrow[c / 2] |= (uint8_t)((codes[i] & 0xF) << ((c & 1) ? 4 : 0));
@@ -305,21 +380,21 @@ static int quantize_rows(const uint16_t *xb, const float *xf, int64_t rows, int6
 }
 
 int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                  int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                  int fmt, int block, int hadamard_k, int tie, int mx_rule, int search,
                   int gscale_given, float *gscale,
                   uint8_t *q, uint8_t *s_logical)
 {
     return quantize_rows(x, NULL, rows, cols, ld, fmt, block, hadamard_k, tie, mx_rule,
-                         gscale_given, gscale, q, s_logical);
+                         search, gscale_given, gscale, q, s_logical);
 }
 
 int fp4o_quantize_f32(const float *x, int64_t rows, int64_t cols, int64_t ld,
-                      int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                      int fmt, int block, int hadamard_k, int tie, int mx_rule, int search,
                       int gscale_given, float *gscale,
                       uint8_t *q, uint8_t *s_logical)
 {
     return quantize_rows(NULL, x, rows, cols, ld, fmt, block, hadamard_k, tie, mx_rule,
-                         gscale_given, gscale, q, s_logical);
+                         search, gscale_given, gscale, q, s_logical);
 }
 
 /* ------------------------------------------------------------------------ */

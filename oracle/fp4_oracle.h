@@ -30,6 +30,7 @@ extern "C" {
 enum { FP4O_MXFP4 = 0, FP4O_NVFP4 = 1 };
 enum { FP4O_TIE_EVEN = 0, FP4O_TIE_AWAY = 1 };
 enum { FP4O_MX_CEIL = 0, FP4O_MX_FLOOR = 1 };
+enum { FP4O_SCALE_ABSMAX = 0, FP4O_SCALE_MSE = 1 };
 
 /* ---- element and scale codecs ------------------------------------------- */
 int    fp4o_e2m1_encode(float v, int tie);      /* 4-bit code, sign in bit 3 */
@@ -45,17 +46,19 @@ void   fp4o_fwht(float *y, int k);              /* in place, incl. c_k       */
 
 /* ---- quantize / dequantize --------------------------------------------- */
 /* gscale: NVFP4 only.  If gscale_given, *gscale is read as s_g; otherwise
- * s_g is computed from the tensor and written to *gscale.  Returns 0 on
- * success, -1 on an invalid argument. */
+ * s_g is computed from the tensor and written to *gscale.  search: block
+ * scale by absmax (mx_rule applies) or by the MSE search over the absmax
+ * scale's neighbours (mx_rule ignored).  Returns 0 on success, -1 on an
+ * invalid argument. */
 int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                  int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                  int fmt, int block, int hadamard_k, int tie, int mx_rule, int search,
                   int gscale_given, float *gscale,
                   uint8_t *q, uint8_t *s_logical);
 
 /* The same with fp32 elements (row stride ld floats): a product quantized
  * again, e.g. for the next layer. */
 int fp4o_quantize_f32(const float *x, int64_t rows, int64_t cols, int64_t ld,
-                      int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                      int fmt, int block, int hadamard_k, int tie, int mx_rule, int search,
                       int gscale_given, float *gscale,
                       uint8_t *q, uint8_t *s_logical);
 

@@ -1,0 +1,254 @@
+"""Pins of the oracle's MSE block-scale search ("FP4 quantization analysis:
+MXFP4 vs NVFP4" §3.2.1: group scales chosen to minimise sum ||Y^_i - X_i||^2;
+§3.3: kernels with the "MSE" and the "Abs-Max" method).
+
+What fixes it, independently of the oracle's own arithmetic:
+  - hand-derived blocks whose best scale differs from the absmax one, with
+    the reconstruction error worked out in the docstrings;
+  - special cases: all-zero blocks, blocks exact on the grid (the inference
+    guide's §3.3 example), which must keep the absmax scale;
+  - per block, the chosen scale's fp64 error is the minimum over the
+    candidate window and never above the absmax scale's; against EVERY
+    representable scale (an exhaustive numpy search) the window reaches the
+    optimum in nearly all blocks of the workloads' distributions;
+  - per element, the chosen scale's reconstruction is a nearest grid point.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from fp4_microscaling_quantization_b200 import inputs
+
+GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def codes_of(q, n):
+    q = np.asarray(q)
+    c = np.stack([q & 15, q >> 4], -1).reshape(q.shape[0], -1)
+    return c[:, :n]
+
+
+def nearest_grid_value(s):
+    """Nearest E2M1 magnitude of |s| (saturating at 6), sign of s; ties are
+    irrelevant to the error, which is all this is used for."""
+    a = np.minimum(np.abs(s), 6.0)
+    return np.sign(s) * GRID[np.abs(a[..., None] - GRID).argmin(-1)]
+
+
+def block_sse64(x, d):
+    """fp64 squared error of the best grid reconstruction of block(s) x
+    under decode scale(s) d (broadcast)."""
+    x = np.asarray(x, np.float64)
+    d = np.asarray(d, np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = np.where(d > 0, d * nearest_grid_value(np.where(d > 0, x / np.where(d > 0, d, 1), 0)), 0.0)
+    return ((x - y) ** 2).sum(-1)
+
+
+def decode_scales(orc, fmt, s, gscale):
+    if fmt == orc.MXFP4:
+        return np.array([[orc.e8m0_decode(int(b)) for b in row] for row in s])
+    return np.array([[gscale * orc.e4m3_decode(int(b)) for b in row] for row in s])
+
+
+def one_block(vals, n):
+    x = np.zeros((1, n), np.float32)
+    x[0, :len(vals)] = vals
+    return x
+
+
+# ------------------------------------------------------- worked examples ----
+def test_mx_outlier_block_takes_the_smaller_exponent(orc):
+    """Block (6.5, 0.703125 x 31).  Absmax (CEIL): amax 6.5 > 6 gives e = 1,
+    scale 2: 6.5/2 = 3.25 -> 3 (y = 6, error 0.5); 0.703125/2 = 0.3515625 ->
+    0.5 (y = 1, error 0.296875).  SSE = 0.25 + 31 * 0.088134765625 =
+    2.982177734375.  e = 0: 6.5 -> 6 (clipped, error 0.5); 0.703125 -> 0.5
+    (error 0.203125).  SSE = 0.25 + 31 * 0.041259765625 = 1.529052734375,
+    smaller: the MSE search stores e = 0 (byte 127)."""
+    x = one_block([6.5] + [0.703125] * 31, 32)
+    qa, sa, _ = orc.quantize_f32(x, orc.MXFP4)
+    qm, sm, _ = orc.quantize_f32(x, orc.MXFP4, search=orc.SCALE_MSE)
+    assert int(sa[0, 0]) == 128 and int(sm[0, 0]) == 127
+    assert codes_of(qm, 32)[0].tolist() == [7] + [1] * 31
+    for q, s, want in ((qa, sa, 2.982177734375), (qm, sm, 1.529052734375)):
+        xh = orc.dequantize(q, s, 1.0, orc.MXFP4)
+        assert np.sum((xh.astype(np.float64) - x) ** 2) == want
+
+
+def test_nv_block_takes_a_slightly_smaller_scale(orc):
+    """s_g = 1, block (6.125, 3.75 x 15).  Absmax: t = 6.125/6 -> E4M3 1.0
+    (0x38): 6.125 -> 6 (error 0.125), 3.75 -> 4 (error 0.25), SSE =
+    0.015625 + 15 * 0.0625 = 0.953125.  Scale 0.9375 (0x37): 6.125/0.9375 =
+    6.53 -> 6 (y = 5.625, error 0.5); 3.75/0.9375 = 4 exactly (error 0):
+    SSE = 0.25, the smallest of the window (1.125: 2.5; 0.875: 1.703)."""
+    x = one_block([6.125] + [3.75] * 15, 16)
+    qa, sa, _ = orc.quantize_f32(x, orc.NVFP4, gscale=1.0)
+    qm, sm, _ = orc.quantize_f32(x, orc.NVFP4, gscale=1.0, search=orc.SCALE_MSE)
+    assert int(sa[0, 0]) == 0x38 and int(sm[0, 0]) == 0x37
+    assert codes_of(qm, 16)[0].tolist() == [7] + [6] * 15
+    for q, s, want in ((qa, sa, 0.953125), (qm, sm, 0.25)):
+        xh = orc.dequantize(q, s, 1.0, orc.NVFP4)
+        assert np.sum((xh.astype(np.float64) - x) ** 2) == want
+
+
+def test_nv_block_max_mapped_near_four(orc):
+    """s_g = 1, block (6, 5 x 15): every 5 sits on the midpoint of the grid's
+    widest gap (4..6) under the absmax scale 1.0: SSE = 15.  Scale 1.625
+    (0x3D, five codes up): 6/1.625 = 3.69 -> 4 (y = 6.5, error 0.5) and
+    5/1.625 = 3.08 -> 3 (y = 4.875, error 0.125): SSE = 0.25 + 15/64 =
+    0.484375.  The rest of the window: 0x36 1.5, 0x37 6.0, 0x39 4.3125,
+    0x3A 1.0, 0x3B 4.0, 0x3C 3.75, 0x3E 1.5."""
+    x = one_block([6.0] + [5.0] * 15, 16)
+    _, sa, _ = orc.quantize_f32(x, orc.NVFP4, gscale=1.0)
+    qm, sm, _ = orc.quantize_f32(x, orc.NVFP4, gscale=1.0, search=orc.SCALE_MSE)
+    assert int(sa[0, 0]) == 0x38 and int(sm[0, 0]) == 0x3D
+    assert orc.e4m3_decode(0x3D) == 1.625
+    assert codes_of(qm, 16)[0].tolist() == [6] + [5] * 15
+    xh = orc.dequantize(qm, sm, 1.0, orc.NVFP4)
+    assert np.sum((xh.astype(np.float64) - x) ** 2) == 0.484375
+
+
+# ---------------------------------------------------------- special cases ----
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_all_zero_blocks(orc, fmt):
+    x = np.zeros((2, 64), np.float32)
+    q, s, g = orc.quantize_f32(x, fmt, search=orc.SCALE_MSE)
+    assert not q.any() and not s.any() and g == 1.0
+
+
+def test_blocks_exact_on_the_grid_keep_the_absmax_scale(orc):
+    """Inference guide §3.3: (5, 10, 20, 60) is exact under the NVFP4 scale
+    10, and (0.5, 1, 2, 6) under scale 1; zero error, so no other candidate
+    can be strictly better."""
+    g = {}
+    with open(os.path.join(GOLD, "guide_scale_example.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, *v = line.split()
+                g[k] = [float(t) for t in v]
+    for key, scale in (("block_a", g["scale_a"][0]), ("block_b", g["scale_b"][0])):
+        x = one_block(g[key], 16)
+        q, s, _ = orc.quantize_f32(x, orc.NVFP4, gscale=1.0, search=orc.SCALE_MSE)
+        assert orc.e4m3_decode(int(s[0, 0])) == scale
+        assert np.array_equal(orc.dequantize(q, s, 1.0, orc.NVFP4), x)
+    x = one_block([v * 8 for v in g["block_a"]], 32)
+    q, s, _ = orc.quantize_f32(x, orc.MXFP4, search=orc.SCALE_MSE)
+    assert int(s[0, 0]) == 127 + 3
+    assert np.array_equal(orc.dequantize(q, s, 1.0, orc.MXFP4), x)
+
+
+# ------------------------------------------------------------- properties ----
+def _workload(kind, rows, cols, seed):
+    rng = np.random.default_rng(seed)
+    if kind == "laplace_outliers":
+        return inputs.draw(rng, rows, cols, "laplace", 1.0, outlier_p=0.01, outlier_mult=20.0)
+    if kind == "student_t":
+        return inputs.draw(rng, rows, cols, "student_t", 1.0, nu=5.0)
+    return inputs.f32_to_bf16_bits(inputs.table5_weight(rows * cols, seed=seed).reshape(rows, cols))
+
+
+KINDS = ["laplace_outliers", "student_t", "table5_weight"]
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("tie", [0, 1])
+def test_mse_minimises_over_its_window_and_reaches_the_exhaustive_optimum(orc, kind, fmt, tie):
+    """Every block's chosen scale has the smallest fp64 error of its
+    candidate window (MX: e_c, e_c - 1; NV: t0 - 2 .. t0 + 6), within fp32
+    rounding of the error, and never more than the absmax scale's.  Against
+    ALL representable scales (254 E8M0 / 126 E4M3, exhaustive numpy search)
+    the window finds the optimum in at least 99.5 % of blocks and the
+    tensor's error is within 0.05 % of the exhaustive one."""
+    x = _workload(kind, 8, 1024, 7 + fmt + 2 * tie)
+    xf = inputs.bf16_bits_to_f32(x).astype(np.float64)
+    B = 32 if fmt == 0 else 16
+    qa, sa, ga = orc.quantize(x, fmt, tie=tie)
+    qm, sm, gm = orc.quantize(x, fmt, tie=tie, search=orc.SCALE_MSE)
+    assert gm == ga
+    blocks = xf.reshape(-1, B)
+    if fmt == 0:
+        all_d = np.array([orc.e8m0_decode(c) for c in range(255)])
+        _, s_ceil, _ = orc.quantize(x, fmt, tie=tie, mx_rule=orc.MX_CEIL)
+        t0, offs, lo, hi = s_ceil.reshape(-1).astype(int), range(-1, 1), 0, 254
+    else:
+        all_d = np.array([ga * orc.e4m3_decode(c) for c in range(127)])
+        t0, offs, lo, hi = sa.reshape(-1).astype(int), range(-2, 7), 1, 126
+    every = block_sse64(blocks[:, None, :], all_d[None, :, None])       # (blocks, scales)
+    idx = np.arange(len(blocks))
+    window = np.full(len(blocks), np.inf)
+    for j in offs:
+        c = t0 + j
+        ok = (c >= lo) & (c <= hi) | (j == 0)
+        window = np.where(ok, np.minimum(window, every[idx, np.clip(c, 0, len(all_d) - 1)]), window)
+    chosen = block_sse64(blocks, decode_scales(orc, fmt, sm, gm).reshape(-1, 1))
+    absmax = block_sse64(blocks, decode_scales(orc, fmt, sa, ga).reshape(-1, 1))
+    assert np.all(chosen <= window * (1 + 1e-6) + 1e-30), np.max(chosen / np.maximum(window, 1e-300))
+    assert np.all(chosen <= absmax * (1 + 1e-6) + 1e-30)
+    assert chosen.sum() < absmax.sum()
+    best = every.min(1)
+    assert np.mean(chosen <= best * (1 + 1e-6) + 1e-30) >= 0.995
+    assert chosen.sum() <= best.sum() * 1.0005
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("tie", [0, 1])
+def test_elements_are_nearest_under_the_chosen_scale(orc, fmt, tie):
+    """Whatever scale the search picks, every element's reconstruction is a
+    nearest point of that scale's grid (checked by brute force over the 15
+    signed grid values)."""
+    x = _workload("laplace_outliers", 8, 512, 21 + fmt + tie)
+    xf = inputs.bf16_bits_to_f32(x).astype(np.float64)
+    B = 32 if fmt == 0 else 16
+    q, s, g = orc.quantize(x, fmt, tie=tie, search=orc.SCALE_MSE)
+    xh = orc.dequantize(q, s, g, fmt).astype(np.float64)
+    d = np.repeat(decode_scales(orc, fmt, s, g), B, axis=1)
+    signed = np.concatenate([-GRID[:0:-1], GRID])
+    dist = np.abs(xf[..., None] - d[..., None] * signed).min(-1)
+    # the decode scale is an fp32 product RN(s_g * s_b): allow its rounding
+    assert np.all(np.abs(xf - xh) <= dist + 1e-6 * 6 * d + 1e-30)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_mx_choice_matches_one_of_the_two_rules(orc, fmt):
+    """MXFP4: the chosen exponent is the CEIL or the FLOOR one, and the
+    block's codes equal that rule's quantization of the block.  NVFP4: the
+    chosen code lies in the window t0 - 2 .. t0 + 6, and blocks that keep t0
+    have the absmax codes."""
+    x = _workload("student_t", 16, 1024, 33)
+    B = 32 if fmt == 0 else 16
+    qm, sm, gm = orc.quantize(x, fmt, search=orc.SCALE_MSE)
+    qc, sc, _ = orc.quantize(x, fmt)
+    cm, cc = codes_of(qm, 1024), codes_of(qc, 1024)
+    same_c = np.repeat(sm == sc, B, axis=1)
+    assert np.array_equal(cm[same_c], cc[same_c])
+    if fmt == 0:
+        qf, sf, _ = orc.quantize(x, fmt, mx_rule=orc.MX_FLOOR)
+        assert np.all((sm == sc) | (sm == sf))
+        same_f = np.repeat(sm == sf, B, axis=1)
+        assert np.array_equal(cm[same_f], codes_of(qf, 1024)[same_f])
+        assert (sm != sc).any()
+    else:
+        off = sm.astype(int) - sc.astype(int)
+        assert off.min() >= -2 and off.max() <= 6 and (off != 0).any()
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("hk", [32, 128])
+def test_with_rotation_lowers_the_tensor_error(orc, fmt, hk):
+    """With H_k the search works on the rotated blocks; H_k is orthogonal, so
+    the tensor's error after the inverse rotation still drops."""
+    x = _workload("laplace_outliers", 16, 1024, 41 + fmt)
+    xf = inputs.bf16_bits_to_f32(x)
+    qa, sa, ga = orc.quantize(x, fmt, hadamard_k=hk)
+    qm, sm, gm = orc.quantize(x, fmt, hadamard_k=hk, search=orc.SCALE_MSE)
+    na = orc.nmse(xf, orc.dequantize(qa, sa, ga, fmt, hadamard_k=hk))
+    nm = orc.nmse(xf, orc.dequantize(qm, sm, gm, fmt, hadamard_k=hk))
+    assert nm < na
+
+
+def test_invalid_search_rejected(orc):
+    with pytest.raises(ValueError):
+        orc.quantize(np.zeros((1, 32), np.uint16), 0, search=2)
