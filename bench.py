@@ -115,6 +115,17 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int):
             ms = time_graph(torch, call, 3, reps * 8)
             gbs = n * bpe / (ms * 1e-3) / 1e9
             res["cases"][f"{name}_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
+        # the MSE block-scale search (same bytes, more arithmetic per block)
+        for k in (0, 128):
+            it = [0]
+
+            def call_mse():
+                fp4.quantize(copies[it[0] % 8], fmt, hadamard_k=k, out=outs, scale_search=fp4.FP4_SCALE_MSE)
+                it[0] += 1
+
+            ms = time_graph(torch, call_mse, 3, reps * 8)
+            gbs = n * bpe / (ms * 1e-3) / 1e9
+            res["cases"][f"{name}_mse_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
     del copies, xd
     torch.cuda.empty_cache()
     return res

@@ -11,13 +11,14 @@ import ctypes
 
 from . import _lib
 from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_NVFP4, FP4_OUT_BF16,
-                   FP4_OUT_F32, FP4_ROUND_AWAY, FP4_ROUND_EVEN, Fp4Error)
+                   FP4_OUT_F32, FP4_ROUND_AWAY, FP4_ROUND_EVEN, FP4_SCALE_ABSMAX, FP4_SCALE_MSE, Fp4Error)
 
 __all__ = [
     "quantize", "dequantize", "gemm", "gemm_quantized", "linear", "linear_workspace_size", "quantize_sizes",
     "gemm_workspace_size", "check_device_status",
     "FP4_MXFP4", "FP4_NVFP4", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
-    "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "Fp4Error", "block_of",
+    "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "FP4_SCALE_ABSMAX", "FP4_SCALE_MSE",
+    "Fp4Error", "block_of",
 ]
 
 
@@ -44,13 +45,15 @@ def quantize_sizes(rows: int, cols: int, fmt) -> tuple[int, int]:
 
 
 def quantize(x, fmt, hadamard_k: int = 0, round: int = FP4_ROUND_EVEN,
-             mx_scale_rule: int = FP4_MX_SCALE_CEIL, gscale=None, out=None):
+             mx_scale_rule: int = FP4_MX_SCALE_CEIL, gscale=None, out=None,
+             scale_search: int = FP4_SCALE_ABSMAX):
     """Quantize a 2-D bf16 CUDA tensor along its last axis.
 
     Returns (q, s, g): q uint8 (rows, cols/2) packed nibbles, s uint8 scales in
     the tensor-core tile layout, g a 1-element fp32 tensor holding s_g (NVFP4;
     for MXFP4 a tensor holding 1).  If ``gscale`` is given (NVFP4) it is used
     as s_g instead of computing it.  ``out`` = (q, s, g) reuses buffers.
+    ``scale_search`` = FP4_SCALE_MSE picks each block scale by the MSE search.
     """
     import torch
 
@@ -70,7 +73,7 @@ def quantize(x, fmt, hadamard_k: int = 0, round: int = FP4_ROUND_EVEN,
     given = gscale is not None
     if given:
         g.copy_(gscale.reshape(1).to(torch.float32))
-    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(given))
+    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(given), int(scale_search))
     gp = g.data_ptr() if fmt == FP4_NVFP4 else None
     _lib.check("fp4_quantize", _lib.lib().fp4_quantize(
         x.data_ptr(), rows, cols, x.stride(0), fmt, block_of(fmt), int(hadamard_k), ctypes.byref(opts),

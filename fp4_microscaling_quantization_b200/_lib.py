@@ -17,6 +17,7 @@ FP4_MXFP4, FP4_NVFP4 = 0, 1
 FP4_ROUND_EVEN, FP4_ROUND_AWAY = 0, 1
 FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR = 0, 1
 FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
+FP4_SCALE_ABSMAX, FP4_SCALE_MSE = 0, 1
 
 STATUS = {
     0: "FP4_OK",
@@ -49,7 +50,8 @@ SIGNATURES = {
 
 
 class Fp4Opts(ctypes.Structure):
-    _fields_ = [("round", ctypes.c_int), ("mx_scale_rule", ctypes.c_int), ("gscale_given", ctypes.c_int)]
+    _fields_ = [("round", ctypes.c_int), ("mx_scale_rule", ctypes.c_int), ("gscale_given", ctypes.c_int),
+                ("scale_search", ctypes.c_int)]
 
 
 class Fp4Error(RuntimeError):

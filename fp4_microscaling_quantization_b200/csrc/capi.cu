@@ -10,7 +10,7 @@
 
 namespace fp4 {
 cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
-                            int hk, float ck, int round_away, int mx_floor, int gscale_given,
+                            int hk, float ck, int round_away, int mx_floor, int mse, int gscale_given,
                             uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl);
 cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
                               int64_t cols, int fmt, int hk, float ck, int bf16out, void *out,
@@ -93,12 +93,13 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                         int hadamard_k, const fp4_opts *opts, uint8_t *q, uint8_t *s, float *gscale,
                         void *stream)
 {
-    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0};
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX};
     if (opts) o = *opts;
     if (rows < 0 || cols < 0 || ld_x < cols) return FP4_ERR_INVALID_ARG;
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR)
         return FP4_ERR_INVALID_ARG;
+    if (o.scale_search != FP4_SCALE_ABSMAX && o.scale_search != FP4_SCALE_MSE) return FP4_ERR_INVALID_ARG;
     if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
@@ -111,7 +112,7 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
     cudaError_t e = fp4::launch_quantize(static_cast<const uint16_t *>(x), rows, cols, ld_x, fmt,
                                          hadamard_k, hadamard_constant(hadamard_k),
                                          o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
-                                         o.gscale_given, q, s, gscale, sm_count(),
+                                         o.scale_search == FP4_SCALE_MSE, o.gscale_given, q, s, gscale, sm_count(),
                                          static_cast<cudaStream_t>(stream), true);
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
@@ -206,13 +207,14 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
                       const float *gW, int64_t N, int out_dtype, void *C, int64_t ldc,
                       void *workspace, size_t ws_bytes, void *stream)
 {
-    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0};
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX};
     if (opts) o = *opts;
     if (M < 0 || N < 0 || K < 0 || ld_x < K || ldc < N) return FP4_ERR_INVALID_ARG;
     if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
+    if (o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;  // absmax scales only
     if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (K % 256 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(M, K)) return FP4_ERR_UNSUPPORTED;
@@ -242,7 +244,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     } else {
         e = fp4::launch_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
                                  hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
-                                 o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, sms, st, true);
+                                 o.mx_scale_rule == FP4_MX_SCALE_FLOOR, 0, gA != nullptr, aq, as, ga, sms, st, true);
     }
     if (e != cudaSuccess) return FP4_ERR_CUDA;
     int bad = 0;
@@ -257,13 +259,14 @@ fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float 
                               int out_fmt, const fp4_opts *opts, const float *gC, uint8_t *Cq, uint8_t *Cs,
                               void *stream)
 {
-    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0};
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX};
     if (opts) o = *opts;
     if (M < 0 || N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
     if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
     if (out_fmt != FP4_MXFP4 && out_fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
+    if (o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;  // absmax scales only
     if (M <= 16 || K % 256 || N % 128) return FP4_ERR_UNSUPPORTED;
     if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP4_ERR_UNSUPPORTED;
     if (!Aq || !As || !Wq || !Ws || !Cq || !Cs) return FP4_ERR_INVALID_ARG;

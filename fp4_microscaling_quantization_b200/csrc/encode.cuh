@@ -85,6 +85,23 @@ FP4_DEV float absmax_tree(const float *v)
     return t[0];
 }
 
+// E2M1 codes of 32 values already divided by their block scale, packed as
+// 16 bytes of nibbles (even element in the low nibble).
+FP4_DEV void e2m1_pack_unit(const float *v, int round_away, uint4 &out)
+{
+    if (!round_away) {
+        out.x = e2m1x8_rn(v + 0);
+        out.y = e2m1x8_rn(v + 8);
+        out.z = e2m1x8_rn(v + 16);
+        out.w = e2m1x8_rn(v + 24);
+    } else {
+        out.x = e2m1x8_away(v + 0);
+        out.y = e2m1x8_away(v + 8);
+        out.z = e2m1x8_away(v + 16);
+        out.w = e2m1x8_away(v + 24);
+    }
+}
+
 // Scale and element encoding of one rotated 32-element unit (TransFP4
 // Eq.(1): MXFP4 power-of-two scale; NVFP4 E4M3 block scale under the tensor
 // scale sg).  v is scaled in place; the 32 E2M1 codes come back as 16 bytes
@@ -115,17 +132,115 @@ FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, i
             sbytes |= sb << (8 * b);
         }
     }
-    if (!round_away) {
-        out.x = e2m1x8_rn(v + 0);
-        out.y = e2m1x8_rn(v + 8);
-        out.z = e2m1x8_rn(v + 16);
-        out.w = e2m1x8_rn(v + 24);
-    } else {
-        out.x = e2m1x8_away(v + 0);
-        out.y = e2m1x8_away(v + 8);
-        out.z = e2m1x8_away(v + 16);
-        out.w = e2m1x8_away(v + 24);
+    e2m1_pack_unit(v, round_away, out);
+    return sbytes;
+}
+
+// ---- the "MSE" scale method ------------------------------------------------
+// "FP4 quantization analysis: MXFP4 vs NVFP4" §3.2.1 (block scales chosen to
+// minimise sum ||Y^_i - X_i||^2) and §3.3 (quantization kernels with the MSE
+// and the Abs-Max method).  Each block tries a fixed window of scales around
+// its absmax scale and keeps the one whose reconstruction has the smallest
+// squared error; of equal ones the first tried.
+
+// The E2M1 grid value nearest to s (magnitude saturating at 6, sign of s),
+// ties as the encoder breaks them: the value the hardware conversion's code
+// decodes to, computed in fp32 without a conversion.  Below 2 the grid step
+// is 1/2, up to 4 it is 1, up to 6 it is 2, so |s| times 2, 1 or 1/2 (exact)
+// is rounded to an integer and scaled back.  Adding and subtracting
+// 1.5 * 2^23 rounds a non-negative value below 2^22 to an integer, ties to
+// even (larger values saturate at 6 anyway); the even-tie grid value and the
+// even code coincide in every step.  Ties away: a value exactly half above
+// its even rounding goes up.
+FP4_DEV float e2m1_grid_value(float s, int round_away)
+{
+    const float a = fabsf(s);
+    const float k = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
+    const float ik = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+    const float t = __fmul_rn(a, k);
+    float r = __fsub_rn(__fadd_rn(t, 12582912.0f), 12582912.0f);
+    if (round_away && __fsub_rn(t, r) == 0.5f) r = __fadd_rn(r, 1.0f);
+    return copysignf(fminf(__fmul_rn(r, ik), 6.0f), s);
+}
+
+// Squared reconstruction error of N values x under the block scale with
+// decode factor d and encode factor r (x_i * r is what the encoder rounds):
+// y_i = RN(q_i * d), e_i = RN(x_i - y_i), each e_i^2 rounded, then summed
+// as a fixed pairwise tree: adjacent pairs first, then the first half of
+// the partial sums plus the second half until one value remains.
+template <int N>
+FP4_DEV float block_sq_error(const float *x, float r, float d, int round_away)
+{
+    float t[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; i++) {
+        const float y0 = __fmul_rn(e2m1_grid_value(__fmul_rn(x[2 * i], r), round_away), d);
+        const float y1 = __fmul_rn(e2m1_grid_value(__fmul_rn(x[2 * i + 1], r), round_away), d);
+        const float e0 = __fsub_rn(x[2 * i], y0);
+        const float e1 = __fsub_rn(x[2 * i + 1], y1);
+        t[i] = __fadd_rn(__fmul_rn(e0, e0), __fmul_rn(e1, e1));
     }
+#pragma unroll
+    for (int w = N / 4; w >= 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w; i++) t[i] = __fadd_rn(t[i], t[i + w]);
+    }
+    return t[0];
+}
+
+// NVFP4 encode factor of a block scale with decode factor d: RN(1/d),
+// clamped to the largest float; 0 for d = 0 (the block encodes as zeros).
+FP4_DEV float nv_encode_factor(float d) { return (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax); }
+
+// encode_unit with the MSE method.  Candidates, in the order tried:
+//   MXFP4: e_c (the CEIL exponent), then e_c - 1 unless e_c = -127; the
+//          FLOOR rule's exponent is always one of the two.
+//   NVFP4: t0 (the absmax E4M3 code), then t0 - 2, t0 - 1, t0 + 1 .. t0 + 6,
+//          each only within 1 .. 0x7E: scales that put the block max between
+//          about 3.6 and 7.3 on the grid.
+template <int FMT>
+FP4_DEV uint32_t encode_unit_mse(float *v, float sg, float six_sg, int round_away, uint4 &out)
+{
+    uint32_t sbytes;
+    if (FMT == FP4_MXFP4) {
+        int e = mx_exponent(absmax_tree<32>(v), 0);
+        if (e > -127) {
+            const float e0 = block_sq_error<32>(v, exp2i(-e), exp2i(e), round_away);
+            const float e1 = block_sq_error<32>(v, exp2i(1 - e), exp2i(e - 1), round_away);
+            if (e1 < e0) e -= 1;
+        }
+        const float inv = exp2i(-e);
+#pragma unroll
+        for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
+        sbytes = (uint32_t)(e + 127);
+    } else {
+        sbytes = 0;
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            float *x = v + 16 * b;
+            const int t0 = (int)e4m3_rn(__fdiv_rn(absmax_tree<16>(x), six_sg));
+            int best = t0;
+            float best_r = nv_encode_factor(__fmul_rn(sg, e4m3_to_f32((uint32_t)t0)));
+            float best_err = block_sq_error<16>(x, best_r, __fmul_rn(sg, e4m3_to_f32((uint32_t)t0)), round_away);
+#pragma unroll 1
+            for (int j = -2; j <= 6; j++) {
+                const int c = t0 + j;
+                if (j == 0 || c < 1 || c > 0x7E) continue;
+                const float d = __fmul_rn(sg, e4m3_to_f32((uint32_t)c));
+                const float r = nv_encode_factor(d);
+                const float err = block_sq_error<16>(x, r, d, round_away);
+                if (err < best_err) {
+                    best = c;
+                    best_r = r;
+                    best_err = err;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; i++) x[i] = __fmul_rn(x[i], best_r);
+            sbytes |= (uint32_t)best << (8 * b);
+        }
+    }
+    e2m1_pack_unit(v, round_away, out);
     return sbytes;
 }
 

@@ -103,13 +103,15 @@ FP4_DEV float read_global_scale(float *g, int computed)
     return sg;
 }
 
-// Encodes one rotated 32-element unit u (encode_unit) and stores its nibbles
-// and scale byte(s) in the tile layout.
-template <int FMT>
+// Encodes one rotated 32-element unit u (encode_unit, or encode_unit_mse for
+// the MSE scale method) and stores its nibbles and scale byte(s) in the tile
+// layout.
+template <int FMT, bool MSE = false>
 FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, const QuantArgs &a, float sg, float six_sg)
 {
     uint4 out;
-    const uint32_t sb = encode_unit<FMT>(v, sg, six_sg, a.round_away, a.mx_floor, out);
+    const uint32_t sb = MSE ? encode_unit_mse<FMT>(v, sg, six_sg, a.round_away, out)
+                            : encode_unit<FMT>(v, sg, six_sg, a.round_away, a.mx_floor, out);
     if (FMT == FP4_MXFP4)
         a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)sb;
     else
@@ -177,7 +179,7 @@ __global__ void zero_word_kernel(float *g)
 }
 
 // ---------------------------------------------------------------------------
-template <int FMT, int HK>
+template <int FMT, int HK, bool MSE>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
 {
     grid_dep_launch();
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
             if (HK) fwht_unit<HK>(v, a.ck, lane);
             if (!live) continue;
 
-            encode_store_unit<FMT>(v, u, row[i], col[i], a, sg, six_sg);
+            encode_store_unit<FMT, MSE>(v, u, row[i], col[i], a, sg, six_sg);
         }
     }
 }
@@ -499,15 +501,15 @@ static int grid_for(int64_t total_units, int sms, int units_per_thread)
     return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
 }
 
-template <int FMT>
+template <int FMT, bool MSE>
 static void (*quant_kernel_for(int hk))(QuantArgs)
 {
     switch (hk) {
-    case 0: return quantize_kernel<FMT, 0>;
-    case 16: return quantize_kernel<FMT, 16>;
-    case 32: return quantize_kernel<FMT, 32>;
-    case 64: return quantize_kernel<FMT, 64>;
-    case 128: return quantize_kernel<FMT, 128>;
+    case 0: return quantize_kernel<FMT, 0, MSE>;
+    case 16: return quantize_kernel<FMT, 16, MSE>;
+    case 32: return quantize_kernel<FMT, 32, MSE>;
+    case 64: return quantize_kernel<FMT, 64, MSE>;
+    case 128: return quantize_kernel<FMT, 128, MSE>;
     }
     return nullptr;
 }
@@ -526,7 +528,7 @@ static void (*amax_kernel_for(int hk))(QuantArgs)
 
 // Quantize launch sequence (see the note on `pdl` below).
 cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
-                            int hk, float ck, int round_away, int mx_floor, int gscale_given,
+                            int hk, float ck, int round_away, int mx_floor, int mse, int gscale_given,
                             uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl)
 {
     QuantArgs a;
@@ -547,7 +549,10 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
     const int grid = grid_for(a.total_units, sms, QUNITS);
-    void (*qk)(QuantArgs) = (fmt == FP4_MXFP4) ? quant_kernel_for<FP4_MXFP4>(hk) : quant_kernel_for<FP4_NVFP4>(hk);
+    void (*qk)(QuantArgs) = (fmt == FP4_MXFP4) ? (mse ? quant_kernel_for<FP4_MXFP4, true>(hk)
+                                                      : quant_kernel_for<FP4_MXFP4, false>(hk))
+                                               : (mse ? quant_kernel_for<FP4_NVFP4, true>(hk)
+                                                      : quant_kernel_for<FP4_NVFP4, false>(hk));
     void (*ak)(QuantArgs) = amax_kernel_for(hk);
     if (!qk || !ak) return cudaErrorInvalidValue;
     cudaError_t err = cudaSuccess;

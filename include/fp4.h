@@ -68,6 +68,21 @@ typedef enum { FP4_ROUND_EVEN = 0, FP4_ROUND_AWAY = 1 } fp4_round;
  * between 6 and 8 times the scale saturate to 6). */
 typedef enum { FP4_MX_SCALE_CEIL = 0, FP4_MX_SCALE_FLOOR = 1 } fp4_mx_scale_rule;
 
+/* Block-scale method ("FP4 quantization analysis: MXFP4 vs NVFP4" §3.3:
+ * kernels with the "MSE" and the "Abs-Max" method).  ABSMAX (default): the
+ * scale from the block max (mx_scale_rule for MXFP4).  MSE (§3.2.1, scales
+ * that minimise sum ||Y^_i - X_i||^2): each block tries a fixed window of
+ * scales around the absmax one and keeps the one with the smallest fp32
+ * squared reconstruction error, summed in a fixed pairwise order; of equal
+ * ones the first tried.  Windows, in the order tried:
+ *   MXFP4: e_c (the CEIL exponent), e_c - 1 (unless e_c = -127);
+ *          mx_scale_rule is not used;
+ *   NVFP4: t0 (the absmax E4M3 code), t0-2, t0-1, t0+1, ..., t0+6, within
+ *          1 .. 0x7E.  The tensor scale s_g stays the absmax one.
+ * fp4_quantize only; fp4_linear and fp4_gemm_quantized return
+ * FP4_ERR_UNSUPPORTED for MSE. */
+typedef enum { FP4_SCALE_ABSMAX = 0, FP4_SCALE_MSE = 1 } fp4_scale_search;
+
 typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_dtype;
 
 typedef struct {
@@ -75,6 +90,7 @@ typedef struct {
     int mx_scale_rule;  /* fp4_mx_scale_rule                                  */
     int gscale_given;   /* NVFP4: 1 = *gscale holds s_g on entry (offline
                            scale); 0 = s_g is computed from the tensor.       */
+    int scale_search;   /* fp4_scale_search                                   */
 } fp4_opts;
 
 /* Human-readable name of a status code (static string). */

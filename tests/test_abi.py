@@ -80,6 +80,15 @@ def test_bad_opts_rejected(L):
     assert L.fp4_quantize(FAKE, 4, 64, 64, 0, 32, 0, ctypes.byref(o), FAKE, FAKE, FAKE, None) == 1
     o = _lib.Fp4Opts(0, 3, 0)
     assert L.fp4_quantize(FAKE, 4, 64, 64, 0, 32, 0, ctypes.byref(o), FAKE, FAKE, FAKE, None) == 1
+    o = _lib.Fp4Opts(0, 0, 0, 2)  # no such scale method
+    assert L.fp4_quantize(FAKE, 4, 64, 64, 0, 32, 0, ctypes.byref(o), FAKE, FAKE, FAKE, None) == 1
+
+
+def test_mse_scales_only_in_quantize(L):
+    o = _lib.Fp4Opts(0, 0, 0, _lib.FP4_SCALE_MSE)
+    F = FAKE
+    assert L.fp4_linear(F, 4, 256, 256, 0, 0, ctypes.byref(o), None, F, F, F, 8, 1, F, 8, F, 1 << 20, None) == 2
+    assert L.fp4_gemm_quantized(F, F, F, F, F, F, 256, 256, 256, 0, 0, ctypes.byref(o), None, F, F, None) == 2
 
 
 def test_dequantize_rejects_on_host(L):

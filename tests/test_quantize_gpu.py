@@ -25,14 +25,14 @@ def fp4():
     return m
 
 
-def check_quantize(fp4, orc, x, fmt, hk=0, tie=0, rule=0, gscale=None, x_dev=None):
+def check_quantize(fp4, orc, x, fmt, hk=0, tie=0, rule=0, gscale=None, x_dev=None, search=0):
     import torch
     rows, cols = x.shape
     xd = to_dev_bf16(x) if x_dev is None else x_dev
     gs = None if gscale is None else torch.tensor([gscale], dtype=torch.float32, device="cuda")
-    q, s, g = fp4.quantize(xd, fmt, hadamard_k=hk, round=tie, mx_scale_rule=rule, gscale=gs)
+    q, s, g = fp4.quantize(xd, fmt, hadamard_k=hk, round=tie, mx_scale_rule=rule, gscale=gs, scale_search=search)
     torch.cuda.synchronize()
-    oq, os_, og = orc.quantize(x, fmt, hadamard_k=hk, tie=tie, mx_rule=rule, gscale=gscale)
+    oq, os_, og = orc.quantize(x, fmt, hadamard_k=hk, tie=tie, mx_rule=rule, gscale=gscale, search=search)
     q_np, s_np = to_np(q), to_np(s)
     bad = np.argwhere(q_np != oq)
     assert bad.size == 0, f"nibbles differ at {bad[:4].tolist()}: gpu {q_np[tuple(bad[0])]:#x} oracle {oq[tuple(bad[0])]:#x}"
@@ -202,3 +202,59 @@ def test_nvfp4_scale_buffer_reused_across_tensors(fp4, orc):
     fp4.quantize(empty, 1, out=(q[:0], s, g))
     torch.cuda.synchronize()
     assert to_np(g)[0] == 1.0
+
+
+# ------------------------------------------------------------- MSE scales ----
+# The "MSE" block-scale method ("FP4 quantization analysis: MXFP4 vs NVFP4"
+# §3.2.1, §3.3): the same bit-exact bar as the absmax path.
+@pytest.mark.parametrize("shape", [(1, 32), (130, 512), (37, 3104), (5, 32736)])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_mse_parity_shapes(fp4, orc, shape, fmt):
+    rows, cols = shape
+    rng = np.random.default_rng(rows * 5 + cols)
+    v = rng.laplace(0, 1, shape).astype(np.float32)
+    v[rng.random(shape) < 0.01] *= 20
+    check_quantize(fp4, orc, inputs.f32_to_bf16_bits(v), fmt, search=1)
+
+
+@pytest.mark.parametrize("hk", [16, 32, 64, 128])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_mse_parity_rotated(fp4, orc, hk, fmt):
+    x = inputs.rotate_acts(rows=136, cols=1024, seed=hk + 1)
+    check_quantize(fp4, orc, x, fmt, hk=hk, search=1)
+
+
+@pytest.mark.parametrize("fmt,tie", [(0, 0), (0, 1), (1, 0), (1, 1)])
+def test_mse_edge_cases(fp4, orc, fmt, tie):
+    """Zeros, -0, subnormals, exact ties, saturation, lone outliers and
+    values near the fp32 maximum (whose squared errors overflow to inf on
+    both sides, leaving the absmax scale)."""
+    x = edge_tensor()
+    check_quantize(fp4, orc, x, fmt, tie=tie, search=1)
+    check_quantize(fp4, orc, x[:6], fmt, tie=tie, hk=64, search=1)
+    for row in range(x.shape[0]):
+        check_quantize(fp4, orc, x[row:row + 1], fmt, tie=tie, search=1)
+
+
+@pytest.mark.parametrize("gscale", [1.0, 1e-3, 1e-30, 3e30])
+def test_mse_nvfp4_given_global_scale(fp4, orc, gscale):
+    x = inputs.quant_sweep(rows=16, cols=512, seed=13)
+    check_quantize(fp4, orc, x, 1, gscale=gscale, search=1)
+    check_quantize(fp4, orc, x, 1, gscale=gscale, search=1, tie=1)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_mse_full_size_quant_sweep(fp4, orc, fmt):
+    """1024 x 131072 heavy-tailed tensor, whole-tensor parity, and the
+    tensor's error below the absmax method's."""
+    import torch
+    x = inputs.quant_sweep()
+    q, s, g, (oq, os_, og) = check_quantize(fp4, orc, x, fmt, search=1)
+    del q, s, g
+    torch.cuda.empty_cache()
+    xs = x[:64]
+    aq, as_, ag = orc.quantize(xs, fmt, gscale=og if fmt else None)
+    xf = inputs.bf16_bits_to_f32(xs)
+    n_abs = orc.nmse(xf, orc.dequantize(aq, as_, ag, fmt))
+    n_mse = orc.nmse(xf, orc.dequantize(oq[:64], os_[:64], og, fmt))
+    assert n_mse < n_abs
