@@ -145,22 +145,24 @@ FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, i
 
 // The E2M1 grid value nearest to s (magnitude saturating at 6, sign of s),
 // ties as the encoder breaks them: the value the hardware conversion's code
-// decodes to, computed in fp32 without a conversion.  Below 2 the grid step
-// is 1/2, up to 4 it is 1, up to 6 it is 2, so |s| times 2, 1 or 1/2 (exact)
-// is rounded to an integer and scaled back.  Adding and subtracting
-// 1.5 * 2^23 rounds a non-negative value below 2^22 to an integer, ties to
-// even (larger values saturate at 6 anyway); the even-tie grid value and the
-// even code coincide in every step.  Ties away: a value exactly half above
-// its even rounding goes up.
+// decodes to, computed in fp32 without a conversion.  The grid step is 1/2
+// below 2, 1 up to 4 and 2 from 4 to 6.  Adding and then subtracting
+// M = 1.5 * 2^22, 2^23 or 2^24 rounds |s| to a multiple of that step, ties to
+// even (a + M lies in the binade whose ulp is the step; the subtraction is
+// exact); the even multiple is the even code in every step.  Magnitudes past
+// 6 saturate.  Ties away: a value exactly half a step above its even
+// rounding goes up one step.
 FP4_DEV float e2m1_grid_value(float s, int round_away)
 {
     const float a = fabsf(s);
-    const float k = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-    const float ik = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-    const float t = __fmul_rn(a, k);
-    float r = __fsub_rn(__fadd_rn(t, 12582912.0f), 12582912.0f);
-    if (round_away && __fsub_rn(t, r) == 0.5f) r = __fadd_rn(r, 1.0f);
-    return copysignf(fminf(__fmul_rn(r, ik), 6.0f), s);
+    const bool lo = a < 2.0f, mid = a < 4.0f;
+    const float m = lo ? 6291456.0f : (mid ? 12582912.0f : 25165824.0f);
+    float r = __fsub_rn(__fadd_rn(a, m), m);
+    if (round_away) {
+        const float h = lo ? 0.25f : (mid ? 0.5f : 1.0f);
+        if (__fsub_rn(a, r) == h) r = __fadd_rn(r, __fadd_rn(h, h));
+    }
+    return copysignf(fminf(r, 6.0f), s);
 }
 
 // Squared reconstruction error of N values x under the block scale with
@@ -192,14 +194,32 @@ FP4_DEV float block_sq_error(const float *x, float r, float d, int round_away)
 // clamped to the largest float; 0 for d = 0 (the block encodes as zeros).
 FP4_DEV float nv_encode_factor(float d) { return (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax); }
 
+// Per-CTA tables for the NVFP4 MSE search: the decode factor d = RN(s_g *
+// s_b) and the encode factor RN(1/d) of every E4M3 code 0 .. 0x7E.
+struct NvScaleTables {
+    float d[128];
+    float r[128];
+};
+
+// Fills the tables (any number of threads; the caller synchronises).
+FP4_DEV void nv_tables_fill(NvScaleTables &t, float sg, int tid, int nthreads)
+{
+    for (int c = tid; c < 128; c += nthreads) {
+        const float d = (c < 0x7F) ? __fmul_rn(sg, e4m3_to_f32((uint32_t)c)) : 0.0f;
+        t.d[c] = d;
+        t.r[c] = nv_encode_factor(d);
+    }
+}
+
 // encode_unit with the MSE method.  Candidates, in the order tried:
 //   MXFP4: e_c (the CEIL exponent), then e_c - 1 unless e_c = -127; the
 //          FLOOR rule's exponent is always one of the two.
 //   NVFP4: t0 (the absmax E4M3 code), then t0 - 2, t0 - 1, t0 + 1 .. t0 + 6,
 //          each only within 1 .. 0x7E: scales that put the block max between
-//          about 3.6 and 7.3 on the grid.
+//          about 3.6 and 7.3 on the grid.  Decode and encode factors come
+//          from `tab`.
 template <int FMT>
-FP4_DEV uint32_t encode_unit_mse(float *v, float sg, float six_sg, int round_away, uint4 &out)
+FP4_DEV uint32_t encode_unit_mse(float *v, float six_sg, int round_away, const NvScaleTables *tab, uint4 &out)
 {
     uint32_t sbytes;
     if (FMT == FP4_MXFP4) {
@@ -220,23 +240,20 @@ FP4_DEV uint32_t encode_unit_mse(float *v, float sg, float six_sg, int round_awa
             float *x = v + 16 * b;
             const int t0 = (int)e4m3_rn(__fdiv_rn(absmax_tree<16>(x), six_sg));
             int best = t0;
-            float best_r = nv_encode_factor(__fmul_rn(sg, e4m3_to_f32((uint32_t)t0)));
-            float best_err = block_sq_error<16>(x, best_r, __fmul_rn(sg, e4m3_to_f32((uint32_t)t0)), round_away);
+            float best_err = block_sq_error<16>(x, tab->r[t0], tab->d[t0], round_away);
 #pragma unroll 1
             for (int j = -2; j <= 6; j++) {
                 const int c = t0 + j;
                 if (j == 0 || c < 1 || c > 0x7E) continue;
-                const float d = __fmul_rn(sg, e4m3_to_f32((uint32_t)c));
-                const float r = nv_encode_factor(d);
-                const float err = block_sq_error<16>(x, r, d, round_away);
+                const float err = block_sq_error<16>(x, tab->r[c], tab->d[c], round_away);
                 if (err < best_err) {
                     best = c;
-                    best_r = r;
                     best_err = err;
                 }
             }
+            const float r = tab->r[best];
 #pragma unroll
-            for (int i = 0; i < 16; i++) x[i] = __fmul_rn(x[i], best_r);
+            for (int i = 0; i < 16; i++) x[i] = __fmul_rn(x[i], r);
             sbytes |= (uint32_t)best << (8 * b);
         }
     }

@@ -107,10 +107,11 @@ FP4_DEV float read_global_scale(float *g, int computed)
 // the MSE scale method) and stores its nibbles and scale byte(s) in the tile
 // layout.
 template <int FMT, bool MSE = false>
-FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, const QuantArgs &a, float sg, float six_sg)
+FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, const QuantArgs &a, float sg, float six_sg,
+                               const NvScaleTables *tab = nullptr)
 {
     uint4 out;
-    const uint32_t sb = MSE ? encode_unit_mse<FMT>(v, sg, six_sg, a.round_away, out)
+    const uint32_t sb = MSE ? encode_unit_mse<FMT>(v, six_sg, a.round_away, tab, out)
                             : encode_unit<FMT>(v, sg, six_sg, a.round_away, a.mx_floor, out);
     if (FMT == FP4_MXFP4)
         a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)sb;
@@ -180,7 +181,7 @@ __global__ void zero_word_kernel(float *g)
 
 // ---------------------------------------------------------------------------
 template <int FMT, int HK, bool MSE>
-__global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
+FP4_DEV void quantize_body(const QuantArgs &a)
 {
     grid_dep_launch();
     grid_dep_wait();
@@ -195,12 +196,20 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
     }
     const bool hinted = FMT == FP4_NVFP4 && a.gscale_computed;  // second read of x
     const uint64_t pol = l2_policy_evict_first();
+    __shared__ NvScaleTables tab;  // NVFP4 MSE search only
+    if (MSE && FMT == FP4_NVFP4) {
+        nv_tables_fill(tab, sg, threadIdx.x, blockDim.x);
+        __syncthreads();
+    }
 
-    for (int64_t base = warp * 32 * QUNITS; base < a.total_units; base += nwarps * 32 * QUNITS) {
-        uint4 raw[QUNITS][4];
-        uint32_t row[QUNITS] = {}, col[QUNITS] = {};
+    // The MSE search is arithmetic-bound: one unit per trip keeps its
+    // registers within three CTAs per SM.
+    constexpr int NU = MSE ? 1 : QUNITS;
+    for (int64_t base = warp * 32 * NU; base < a.total_units; base += nwarps * 32 * NU) {
+        uint4 raw[NU][4];
+        uint32_t row[NU] = {}, col[NU] = {};
 #pragma unroll
-        for (int i = 0; i < QUNITS; i++) {
+        for (int i = 0; i < NU; i++) {
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
                 unit_rc(u, a.upr_div, row[i], col[i]);
@@ -211,7 +220,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
             }
         }
 #pragma unroll
-        for (int i = 0; i < QUNITS; i++) {
+        for (int i = 0; i < NU; i++) {
             const int64_t u = base + i * 32 + lane;
             const bool live = u < a.total_units;
             float v[32];
@@ -219,9 +228,22 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
             if (HK) fwht_unit<HK>(v, a.ck, lane);
             if (!live) continue;
 
-            encode_store_unit<FMT, MSE>(v, u, row[i], col[i], a, sg, six_sg);
+            encode_store_unit<FMT, MSE>(v, u, row[i], col[i], a, sg, six_sg, &tab);
         }
     }
+}
+
+template <int FMT, int HK>
+__global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
+{
+    quantize_body<FMT, HK, false>(a);
+}
+
+// The MSE scale search: arithmetic-bound, so sized for three CTAs per SM.
+template <int FMT, int HK>
+__global__ void __launch_bounds__(256, 3) quantize_mse_kernel(QuantArgs a)
+{
+    quantize_body<FMT, HK, true>(a);
 }
 
 
@@ -505,11 +527,11 @@ template <int FMT, bool MSE>
 static void (*quant_kernel_for(int hk))(QuantArgs)
 {
     switch (hk) {
-    case 0: return quantize_kernel<FMT, 0, MSE>;
-    case 16: return quantize_kernel<FMT, 16, MSE>;
-    case 32: return quantize_kernel<FMT, 32, MSE>;
-    case 64: return quantize_kernel<FMT, 64, MSE>;
-    case 128: return quantize_kernel<FMT, 128, MSE>;
+    case 0: return MSE ? quantize_mse_kernel<FMT, 0> : quantize_kernel<FMT, 0>;
+    case 16: return MSE ? quantize_mse_kernel<FMT, 16> : quantize_kernel<FMT, 16>;
+    case 32: return MSE ? quantize_mse_kernel<FMT, 32> : quantize_kernel<FMT, 32>;
+    case 64: return MSE ? quantize_mse_kernel<FMT, 64> : quantize_kernel<FMT, 64>;
+    case 128: return MSE ? quantize_mse_kernel<FMT, 128> : quantize_kernel<FMT, 128>;
     }
     return nullptr;
 }
