@@ -150,7 +150,7 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const
     if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
     if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
-    if (K % 256) return FP4_ERR_UNSUPPORTED;
+    if (K % 32) return FP4_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return FP4_OK;
     if (!Aq || !As || !Wq || !Ws || !C) return FP4_ERR_INVALID_ARG;
     if (fmt == FP4_NVFP4 && (!gA || !gW)) return FP4_ERR_INVALID_ARG;
@@ -216,7 +216,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
     if (o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;  // absmax scales only
     if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
-    if (K % 256 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (K % 32 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(M, K)) return FP4_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return FP4_OK;
     if (!x || !Wq || !Ws || !C || !workspace) return FP4_ERR_INVALID_ARG;
@@ -267,7 +267,7 @@ fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float 
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
     if (o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;  // absmax scales only
-    if (M <= 16 || K % 256 || N % 128) return FP4_ERR_UNSUPPORTED;
+    if (M <= 16 || K % 32 || N % 128) return FP4_ERR_UNSUPPORTED;
     if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP4_ERR_UNSUPPORTED;
     if (!Aq || !As || !Wq || !Ws || !Cq || !Cs) return FP4_ERR_INVALID_ARG;
     if (fmt == FP4_NVFP4 && (!gA || !gW)) return FP4_ERR_INVALID_ARG;

@@ -112,7 +112,7 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     const bool leader = rank == 0;
     const int group = blockIdx.x / CG, ngroups = gridDim.x / CG;
     const int num_tiles = p.num_m_tiles * p.num_n_tiles;
-    const int nk = p.K / Cfg::BK;
+    const int nk = (p.K + Cfg::BK - 1) / Cfg::BK;  // a K tail reads zeros past K (TMA fill)
 
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES), sfr0 = smem_u32(bars + 2 * STAGES);
     const uint32_t accf = smem_u32(bars + 3 * STAGES), acce = smem_u32(bars + 3 * STAGES + 1);
@@ -157,8 +157,8 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 const int mt = t % p.num_m_tiles, nt = t / p.num_m_tiles;
                 const int arow = (mt * CG + (int)rank) * Cfg::BM;
                 const int brow = nt * Cfg::BN + (int)rank * Cfg::B_ROWS;
-                const int sfa_atom = (mt * CG + (int)rank) * p.nkb4;
-                const int sfb_atom0 = (2 * nt) * p.nkb4, sfb_atom1 = (2 * nt + 1) * p.nkb4;
+                const int sfa_rb = mt * CG + (int)rank;  // 128-row blocks of the scale layouts
+                const int sfb_rb0 = 2 * nt, sfb_rb1 = 2 * nt + 1;
                 bool stop = false;
                 for (int ks = 0; ks < nk; ks++, it++) {
                     const int s = it % STAGES;
@@ -170,9 +170,9 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     tma_load_2d_cg<CG>(smem_u32(st), &tmA, ks * (Cfg::BK / 2), arow, fb);
                     tma_load_2d_cg<CG>(smem_u32(st + Cfg::A_BYTES), &tmB, ks * (Cfg::BK / 2), brow, fb);
                     const uint32_t ssf = smem_u32(st + Cfg::A_BYTES + Cfg::B_BYTES);
-                    tma_load_2d_cg<CG>(ssf, &tmSA, 0, sfa_atom + ks * KA, fb);
-                    tma_load_2d_cg<CG>(ssf + Cfg::SFA_BYTES, &tmSB, 0, sfb_atom0 + ks * KA, fb);
-                    tma_load_2d_cg<CG>(ssf + Cfg::SFA_BYTES + KA * 512, &tmSB, 0, sfb_atom1 + ks * KA, fb);
+                    tma_load_3d_cg<CG>(ssf, &tmSA, 0, ks * KA, sfa_rb, fb);
+                    tma_load_3d_cg<CG>(ssf + Cfg::SFA_BYTES, &tmSB, 0, ks * KA, sfb_rb0, fb);
+                    tma_load_3d_cg<CG>(ssf + Cfg::SFA_BYTES + KA * 512, &tmSB, 0, ks * KA, sfb_rb1, fb);
                 }
                 if (stop) break;
             }
@@ -421,7 +421,7 @@ struct Params {
     uint64_t budget_ns;  // limit of every mbarrier wait
     int stall;           // failure-detection test: the producer issues no loads
     int N, M, K;
-    int nk;              // K / BK
+    int nk;              // ceil(K / BK); the last K step of a tail reads zeros past K
     int ntiles;          // ceil(N / 128)
     int G;               // CTAs
     int maxseg;
@@ -458,7 +458,8 @@ constexpr int DECODE_THREADS = 224;
 
 template <int FMT>
 __global__ void __launch_bounds__(DECODE_THREADS, 1)
-decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, Params p)
+decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
+              const __grid_constant__ CUtensorMap tmSW, const __grid_constant__ CUtensorMap tmSA, Params p)
 {
     constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -508,13 +509,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         const uint32_t st = smem0 + st_i * STAGE_BYTES;
         const uint32_t fb = full0 + 8 * st_i;
         tma_load_2d(st, &tmW, ks * (BK / 2), t * BMW, fb);
-        bulk_load(st + W_BYTES + A_BYTES, p.Ws + ((int64_t)t * p.nkb4 + ks * KA) * 512, KA * 512, fb);
+        tma_load_3d(st + W_BYTES + A_BYTES, &tmSW, 0, ks * KA, t, fb);
     };
     auto load_a = [&](int ks, int st_i) {
         const uint32_t st = smem0 + st_i * STAGE_BYTES;
         const uint32_t fb = full0 + 8 * st_i;
         tma_load_2d(st + W_BYTES, &tmA, ks * (BK / 2), 0, fb);
-        bulk_load(st + W_BYTES + A_BYTES + SFW_BYTES, p.As + (int64_t)ks * KA * 512, KA * 512, fb);
+        tma_load_3d(st + W_BYTES + A_BYTES + SFW_BYTES, &tmSA, 0, ks * KA, 0, fb);
     };
 
     if (threadIdx.x == 0) {
@@ -531,6 +532,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         fence_barrier_init();
         tma_prefetch_desc(&tmW);
         tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmSW);
+        tma_prefetch_desc(&tmSA);
         // The weight stream depends on no earlier kernel (the one before may
         // still be quantizing the activations): start it at once, while warp
         // 1 allocates tensor memory.
@@ -805,7 +808,7 @@ struct Plan {
 inline Plan plan(int64_t M, int64_t N, int64_t K, int sms)
 {
     Plan pl;
-    pl.nk = (int)(K / BK);
+    pl.nk = (int)((K + BK - 1) / BK);
     pl.ntiles = (int)((N + BMW - 1) / BMW);
     pl.csize = 1;
     const int64_t U = (int64_t)pl.ntiles * pl.nk;
@@ -870,18 +873,19 @@ static bool make_fp4_map(CUtensorMap *m, const void *base, int64_t rows, int64_t
 }
 
 
-// Scale-atom buffer (tile layout) as a 2-D tensor of 512-byte atoms: 256
-// uint16 per atom, one atom per row; boxes of `box_atoms` consecutive atoms.
-// Atoms past the end (row blocks beyond the padded rows) read as zeros.
-static bool make_sf_map(CUtensorMap *m, const void *base, int64_t n_atoms, int box_atoms)
+// Scale-atom buffer (tile layout) as a 3-D tensor: 512-byte atoms (256
+// uint16), nkb4 atoms per 128-row block, nrb row blocks; boxes of
+// `box_atoms` consecutive atoms of one row block.  Atoms past a row block's
+// nkb4 (a K tail) or past the last row block read as zeros.
+static bool make_sf_map(CUtensorMap *m, const void *base, int64_t nkb4, int64_t nrb, int box_atoms)
 {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {256u, (cuuint64_t)n_atoms};
-    cuuint64_t strides[1] = {512u};
-    cuuint32_t box[2] = {256u, (cuuint32_t)box_atoms};
-    cuuint32_t estr[2] = {1u, 1u};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+    cuuint64_t dims[3] = {256u, (cuuint64_t)nkb4, (cuuint64_t)nrb};
+    cuuint64_t strides[2] = {512u, (cuuint64_t)(nkb4 * 512)};
+    cuuint32_t box[3] = {256u, (cuuint32_t)box_atoms, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -896,7 +900,7 @@ static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint
     CUtensorMap ta, tb, tsa, tsb;
     const int64_t nrb_a = (int64_t)((p.M + 127) / 128), nrb_w = (int64_t)((p.N + 127) / 128);
     if (!make_fp4_map(&ta, Aq, p.M, p.K, Cfg::BM) || !make_fp4_map(&tb, Wq, p.N, p.K, Cfg::B_ROWS) ||
-        !make_sf_map(&tsa, As, nrb_a * p.nkb4, KA) || !make_sf_map(&tsb, Ws, nrb_w * p.nkb4, KA))
+        !make_sf_map(&tsa, As, p.nkb4, nrb_a, KA) || !make_sf_map(&tsb, Ws, p.nkb4, nrb_w, KA))
         return cudaErrorInvalidValue;
     auto kern = pgemm_kernel<FMT, OUT, CG>;
     static bool attr_set = false;
@@ -959,13 +963,13 @@ constexpr uint64_t kWaitBudgetNs = 2000000000ull;
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
 {
-    if (M < 1 || M > kDecodeMaxM || N < 1 || K < decode::BK) return 0;
+    if (M < 1 || M > kDecodeMaxM || N < 1 || K < 32) return 0;
     return decode::plan(M, N, K, sms).ws_bytes;
 }
 
 template <int FMT>
-static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const decode::Params &p, bool any_cut,
-                                 cudaStream_t st, bool pdl)
+static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const CUtensorMap &tsw,
+                                 const CUtensorMap &tsa, const decode::Params &p, bool any_cut, cudaStream_t st, bool pdl)
 {
     auto kern = decode::decode_kernel<FMT>;
     static bool attr_set = false;
@@ -996,7 +1000,7 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
     cfg.attrs = attr;
     cfg.numAttrs = na;
     count_launches(1);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, ta, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, ta, tsw, tsa, p);
     if (e != cudaSuccess || p.counters || !any_cut) return e;
     // the reduction waits for the split-K kernel inside (grid_dep_wait)
     return launch_k(decode::reduce_kernel<FMT>, dim3((p.N + 127) / 128), dim3(128), 0, st, true, p);
@@ -1020,8 +1024,11 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
             *bad = 1;
             return cudaSuccess;
         }
-        CUtensorMap tw, ta;
-        if (!make_fp4_map(&tw, Wq, N, K, decode::BMW) || !make_fp4_map(&ta, Aq, M, K, decode::BNA))
+        const int64_t nkb4 = (K / (fmt == FP4_MXFP4 ? 32 : 16) + 3) / 4;
+        const int KA = fmt == FP4_MXFP4 ? 2 : 4;
+        CUtensorMap tw, ta, tsw, tsa;
+        if (!make_fp4_map(&tw, Wq, N, K, decode::BMW) || !make_fp4_map(&ta, Aq, M, K, decode::BNA) ||
+            !make_sf_map(&tsw, Ws, nkb4, (N + 127) / 128, KA) || !make_sf_map(&tsa, As, nkb4, 1, KA))
             return cudaErrorInvalidValue;
         decode::Params dp;
         dp.Ws = Ws;
@@ -1036,7 +1043,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.maxseg = pl.maxseg;
         dp.csize = pl.csize;
         dp.w_before_wait = (pdl && w_before_wait) ? 1 : 0;
-        dp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+        dp.nkb4 = (int)nkb4;
         dp.counters = counters;
         dp.budget_ns = budget;
         dp.stall = stall;
@@ -1045,8 +1052,8 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.C = C;
         dp.ldc = ldc;
         dp.bf16out = bf16out;
-        return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4>(tw, ta, dp, pl.any_cut, st, pdl)
-                                : launch_decode<FP4_NVFP4>(tw, ta, dp, pl.any_cut, st, pdl);
+        return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl)
+                                : launch_decode<FP4_NVFP4>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl);
     }
     {
         PParams pp;
@@ -1061,7 +1068,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         pp.M = (int)M;
         pp.N = (int)N;
         pp.K = (int)K;
-        pp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+        pp.nkb4 = (int)((K / (fmt == FP4_MXFP4 ? 32 : 16) + 3) / 4);
         pp.budget_ns = budget;
         pp.stall = stall;
         const int cg = pgemm_cta_group(M);
@@ -1074,7 +1081,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
 }
 
 // C = A W^T quantized along N by the prefill kernel's epilogue (M > 16,
-// K % 256 == 0, N % 128 == 0; checked by the caller).
+// K % 32 == 0, N % 128 == 0; checked by the caller).
 cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
                                   const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K, int fmt,
                                   int out_fmt, int round_away, int mx_floor, const float *gC, uint8_t *Cq, uint8_t *Cs,
@@ -1093,7 +1100,7 @@ cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const fl
     pp.M = (int)M;
     pp.N = (int)N;
     pp.K = (int)K;
-    pp.nkb4 = (int)(K / (fmt == FP4_MXFP4 ? 32 : 16) / 4);
+    pp.nkb4 = (int)((K / (fmt == FP4_MXFP4 ? 32 : 16) + 3) / 4);
     uint64_t budget = g_inject_budget.exchange(0);
     pp.budget_ns = budget ? budget : kWaitBudgetNs;
     pp.stall = g_inject_stall.exchange(0);
@@ -1175,7 +1182,7 @@ extern "C" fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *
     if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
     if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
-    if (K % 256 || M > fp4::kDecodeMaxM) return FP4_ERR_UNSUPPORTED;
+    if (K % 32 || M > fp4::kDecodeMaxM) return FP4_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return FP4_OK;
     if (!Aq || !As || !Wq || !Ws || !C) return FP4_ERR_INVALID_ARG;
     if (fmt == FP4_NVFP4 && (!gA || !gW)) return FP4_ERR_INVALID_ARG;

@@ -255,8 +255,11 @@ __global__ void __launch_bounds__(256, 3) quantize_mse_kernel(QuantArgs a)
 // NVFP4 tensor-max pass and the encode pass read x once.  The CTAs exchange
 // their partial maxima through distributed shared memory: no global scratch,
 // memset or second kernel.  The kernel also zeroes `nzero` words at `zero`
-// (the split-K kernel's per-tile arrival counters) and writes no scale
-// padding (the GEMM never reads scales of rows past the tensor).
+// (the split-K kernel's per-tile arrival counters) and the padding scale
+// columns of the tensor's rows (with K not a multiple of 128 (MX) or 64
+// (NV) the GEMM's last K step multiplies the zeros past K by them, so they
+// must be finite), but not the padding rows, whose products the GEMM never
+// stores.
 constexpr int ACT_CTAS = 16, ACT_CTAS_PORTABLE = 8, ACT_THREADS = 256, ACT_UPT = 2;
 
 // Loads units base + 32 i + lane (i < N) of the tensor, zeros past the end.
@@ -292,6 +295,13 @@ __global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, uns
     const int64_t warp = (blockIdx.x * (int64_t)ACT_THREADS + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * ACT_THREADS) >> 5;
     for (int i = blockIdx.x * ACT_THREADS + threadIdx.x; i < nzero; i += gridDim.x * ACT_THREADS) zero[i] = 0u;
+    {
+        const int64_t nkb = a.units_per_row * (FMT == FP4_MXFP4 ? 1 : 2);
+        const int pad = (int)(a.nkb4 * 4 - nkb);  // 0 .. 3
+        const int64_t rows = a.units_per_row > 0 ? a.total_units / a.units_per_row : 0;
+        for (int64_t i = blockIdx.x * ACT_THREADS + threadIdx.x; i < rows * pad; i += gridDim.x * ACT_THREADS)
+            a.s[scale_offset(i / pad, nkb + i % pad, a.nkb4)] = 0;
+    }
 
     const int64_t stride = nwarps * 32;  // units between a thread's consecutive units
     const bool cached = a.total_units <= stride * ACT_UPT;

@@ -78,6 +78,15 @@ FP4_DEV void tma_load_2d(uint32_t dst, const CUtensorMap *m, int x, int y, uint3
         : "memory");
 }
 
+// 3-D tiled load (no multicast) into shared memory, completing on `bar`.
+FP4_DEV void tma_load_3d(uint32_t dst, const CUtensorMap *m, int x, int y, int z, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
 // Contiguous bulk copy global -> shared (16-byte aligned, size % 16 == 0).
 FP4_DEV void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {
@@ -242,6 +251,20 @@ FP4_DEV void tma_load_2d_cg(uint32_t dst, const CUtensorMap *m, int x, int y, ui
         asm volatile(
             "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
             "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar)
+            : "memory");
+    }
+}
+
+// 3-D counterpart of tma_load_2d_cg.
+template <int CG>
+FP4_DEV void tma_load_3d_cg(uint32_t dst, const CUtensorMap *m, int x, int y, int z, uint32_t bar)
+{
+    if (CG == 1) {
+        tma_load_3d(dst, m, x, y, z, bar);
+    } else {
+        asm volatile(
+            "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+            "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
             : "memory");
     }
 }

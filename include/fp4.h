@@ -151,7 +151,10 @@ fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt,
  * tensor cores), A: M x K, W: N x K, both quantized along K in the same
  * format by fp4_quantize (Aq/As, Wq/Ws).  alpha = s_gA * s_gW for NVFP4
  * (gA, gW device fp32), 1 for MXFP4 (gA, gW ignored).
- *   K          multiple of 256.
+ *   K          multiple of 32 ("Portable FP4 quantization (TransFP4)" Table 3:
+ *              the GEMM's K alignment is 32).  The tensor cores step K by
+ *              256 per stage; the last step of a tail multiplies zeros read
+ *              past K with the zero padding scales fp4_quantize writes.
  *   out_dtype  FP4_OUT_F32 or FP4_OUT_BF16.  C row-major, row stride ldc
  *              elements (ldc >= N).
  *   workspace  device scratch of at least fp4_gemm_workspace_size() bytes
@@ -185,7 +188,7 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA,
  *   Cs        output, the scales in the tile layout of fp4_quantize
  *             (fp4_quantize_sizes(M, N, out_fmt, ...) bytes; the padding rows
  *             are written 0), 16-byte aligned.
- * Shapes: M > 16 (the tiled kernel), K multiple of 256, N multiple of 128;
+ * Shapes: M > 16 (the tiled kernel), K multiple of 32, N multiple of 128;
  * otherwise FP4_ERR_UNSUPPORTED with nothing launched.  Each 32-element unit
  * is encoded as fp4_quantize encodes one, from the FP32 values fp4_gemm
  * returns with FP4_OUT_F32 for the same operands.

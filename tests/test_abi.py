@@ -100,7 +100,7 @@ def test_dequantize_rejects_on_host(L):
 
 def test_gemm_rejects_on_host(L):
     g = L.fp4_gemm
-    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 100, 0, 1, FAKE, 8, None, 0, None) == 2  # K % 256
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 100, 0, 1, FAKE, 8, None, 0, None) == 2  # K % 32
     assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 4, None, 0, None) == 1  # ldc < N
     assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 5, 1, FAKE, 8, None, 0, None) == 2
     assert g(None, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 8, None, 0, None) == 1
@@ -113,7 +113,7 @@ def test_gemm_quantized_rejects_on_host(L):
     F = FAKE
     assert g(F, F, F, F, F, F, 16, 256, 256, 0, 0, None, None, F, F, None) == 2      # M <= 16: decode shapes
     assert g(F, F, F, F, F, F, 256, 192, 256, 0, 0, None, None, F, F, None) == 2     # N % 128
-    assert g(F, F, F, F, F, F, 256, 256, 128, 0, 0, None, None, F, F, None) == 2     # K % 256
+    assert g(F, F, F, F, F, F, 256, 256, 112, 0, 0, None, None, F, F, None) == 2     # K % 32
     assert g(F, F, F, F, F, F, 256, 256, 256, 0, 3, None, None, F, F, None) == 2     # output format
     assert g(F, F, F, F, F, F, 256, 256, 256, 0, 1, None, None, F, F, None) == 1     # NVFP4 out needs gC
     assert g(F, F, None, F, F, F, 256, 256, 256, 1, 0, None, None, F, F, None) == 1  # NVFP4 in needs gA

@@ -66,7 +66,7 @@ def test_noalloc_rejects_what_it_cannot_hold(fp4):
     z = torch.zeros(16, dtype=torch.uint8, device="cuda")
     g = torch.ones(1, device="cuda")
     p = z.data_ptr()
-    # M above the decode range, and K not a multiple of 256: refused before any launch
+    # M above the decode range, and K not a multiple of 32: refused before any launch
     assert f(p, p, g.data_ptr(), p, p, g.data_ptr(), 17, 8, 256, 0, 0, p, 8, None) == 2
     assert f(p, p, g.data_ptr(), p, p, g.data_ptr(), 4, 8, 100, 0, 0, p, 8, None) == 2
     # Partials larger than the fixed array: many more tiles than SMs with two
