@@ -166,9 +166,12 @@ def linear_workspace_size(M: int, N: int, K: int, fmt) -> int:
 
 
 def linear(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale=None,
-           round: int = FP4_ROUND_EVEN, mx_scale_rule: int = FP4_MX_SCALE_CEIL, out=None, workspace=None):
+           round: int = FP4_ROUND_EVEN, mx_scale_rule: int = FP4_MX_SCALE_CEIL, out=None, workspace=None,
+           weights_static: bool = False):
     """W4A4 linear from bf16 activations x (M x K) and a pre-quantized weight
-    w = (Wq, Ws, gW) (N x K): quantizes x online, returns C = x W^T."""
+    w = (Wq, Ws, gW) (N x K): quantizes x online, returns C = x W^T.
+    ``weights_static``: w is written by no kernel still in flight (inference
+    weights), so the decode kernel may stream it early."""
     import torch
 
     fmt = _fmt(fmt)
@@ -182,7 +185,7 @@ def linear(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale
         out = torch.empty((M, N), dtype=dt, device=x.device)
     if workspace is None:
         workspace = torch.empty((linear_workspace_size(M, N, K, fmt),), dtype=torch.uint8, device=x.device)
-    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), 0)
+    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), 0, 0, int(bool(weights_static)))
     _lib.check("fp4_linear", _lib.lib().fp4_linear(
         x.data_ptr(), M, K, x.stride(0), fmt, int(hadamard_k), ctypes.byref(opts),
         gscale.data_ptr() if gscale is not None else None, Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(), N,

@@ -51,7 +51,7 @@ SIGNATURES = {
 
 class Fp4Opts(ctypes.Structure):
     _fields_ = [("round", ctypes.c_int), ("mx_scale_rule", ctypes.c_int), ("gscale_given", ctypes.c_int),
-                ("scale_search", ctypes.c_int)]
+                ("scale_search", ctypes.c_int), ("weights_static", ctypes.c_int)]
 
 
 class Fp4Error(RuntimeError):

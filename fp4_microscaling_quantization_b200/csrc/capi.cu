@@ -22,7 +22,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
                         bool w_before_wait);
 cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int hk, float ck,
                                 int round_away, int mx_floor, int gscale_given, uint8_t *q, uint8_t *s, float *gscale,
-                                unsigned *zero, int nzero, cudaStream_t st);
+                                unsigned *zero, int nzero, int early, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int sms);
 cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
                                   const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K, int fmt,
@@ -93,7 +93,7 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                         int hadamard_k, const fp4_opts *opts, uint8_t *q, uint8_t *s, float *gscale,
                         void *stream)
 {
-    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX};
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
     if (opts) o = *opts;
     if (rows < 0 || cols < 0 || ld_x < cols) return FP4_ERR_INVALID_ARG;
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
@@ -207,7 +207,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
                       const float *gW, int64_t N, int out_dtype, void *C, int64_t ldc,
                       void *workspace, size_t ws_bytes, void *stream)
 {
-    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX};
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
     if (opts) o = *opts;
     if (M < 0 || N < 0 || K < 0 || ld_x < K || ldc < N) return FP4_ERR_INVALID_ARG;
     if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
@@ -215,6 +215,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
     if (o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;  // absmax scales only
+    if (o.weights_static != 0 && o.weights_static != 1) return FP4_ERR_INVALID_ARG;
     if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (K % 32 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(M, K)) return FP4_ERR_UNSUPPORTED;
@@ -240,7 +241,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
         e = fp4::launch_act_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
                                      hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
                                      o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, counters,
-                                     (int)((N + 127) / 128), st);
+                                     (int)((N + 127) / 128), o.weights_static != 0, st);
     } else {
         e = fp4::launch_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
                                  hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
@@ -259,7 +260,7 @@ fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float 
                               int out_fmt, const fp4_opts *opts, const float *gC, uint8_t *Cq, uint8_t *Cs,
                               void *stream)
 {
-    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX};
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
     if (opts) o = *opts;
     if (M < 0 || N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
     if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;

@@ -85,6 +85,29 @@ FP4_DEV float absmax_tree(const float *v)
     return t[0];
 }
 
+// NVFP4 encode factor of a block scale with decode factor d: RN(1/d),
+// clamped to the largest float; 0 for d = 0 (the block encodes as zeros).
+FP4_DEV float nv_encode_factor(float d) { return (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax); }
+
+// Per-CTA tables of the NVFP4 block scales under one tensor scale s_g: the
+// decode factor d = RN(s_g * s_b) and the encode factor RN(1/d) of every
+// E4M3 code 0 .. 0x7E, so that a block looks them up instead of converting
+// its code and dividing (the same values, computed once per CTA).
+struct NvScaleTables {
+    float d[128];
+    float r[128];
+};
+
+// Fills the tables (any number of threads; the caller synchronises).
+FP4_DEV void nv_tables_fill(NvScaleTables &t, float sg, int tid, int nthreads)
+{
+    for (int c = tid; c < 128; c += nthreads) {
+        const float d = (c < 0x7F) ? __fmul_rn(sg, e4m3_to_f32((uint32_t)c)) : 0.0f;
+        t.d[c] = d;
+        t.r[c] = nv_encode_factor(d);
+    }
+}
+
 // E2M1 codes of 32 values already divided by their block scale, packed as
 // 16 bytes of nibbles (even element in the low nibble).
 FP4_DEV void e2m1_pack_unit(const float *v, int round_away, uint4 &out)
@@ -108,7 +131,8 @@ FP4_DEV void e2m1_pack_unit(const float *v, int round_away, uint4 &out)
 // of nibbles (even element in the low nibble) and the return value holds the
 // scale byte (MXFP4) or the two block-scale bytes, first block low (NVFP4).
 template <int FMT>
-FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, int mx_floor, uint4 &out)
+FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, int mx_floor, uint4 &out,
+                             const NvScaleTables *tab = nullptr)
 {
     uint32_t sbytes;
     if (FMT == FP4_MXFP4) {
@@ -125,8 +149,7 @@ FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, i
             const float amax = absmax_tree<16>(v + 16 * b);
             const float t = __fdiv_rn(amax, six_sg);
             const uint32_t sb = e4m3_rn(t);
-            const float d = __fmul_rn(sg, e4m3_to_f32(sb));
-            const float r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax);
+            const float r = tab ? tab->r[sb] : nv_encode_factor(__fmul_rn(sg, e4m3_to_f32(sb)));
 #pragma unroll
             for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
             sbytes |= sb << (8 * b);
@@ -188,27 +211,6 @@ FP4_DEV float block_sq_error(const float *x, float r, float d, int round_away)
         for (int i = 0; i < w; i++) t[i] = __fadd_rn(t[i], t[i + w]);
     }
     return t[0];
-}
-
-// NVFP4 encode factor of a block scale with decode factor d: RN(1/d),
-// clamped to the largest float; 0 for d = 0 (the block encodes as zeros).
-FP4_DEV float nv_encode_factor(float d) { return (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax); }
-
-// Per-CTA tables for the NVFP4 MSE search: the decode factor d = RN(s_g *
-// s_b) and the encode factor RN(1/d) of every E4M3 code 0 .. 0x7E.
-struct NvScaleTables {
-    float d[128];
-    float r[128];
-};
-
-// Fills the tables (any number of threads; the caller synchronises).
-FP4_DEV void nv_tables_fill(NvScaleTables &t, float sg, int tid, int nthreads)
-{
-    for (int c = tid; c < 128; c += nthreads) {
-        const float d = (c < 0x7F) ? __fmul_rn(sg, e4m3_to_f32((uint32_t)c)) : 0.0f;
-        t.d[c] = d;
-        t.r[c] = nv_encode_factor(d);
-    }
 }
 
 // encode_unit with the MSE method.  Candidates, in the order tried:

@@ -403,7 +403,8 @@ constexpr int SFA_BYTES = 4 * 512;
 constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;  // 22528 = 22 KB
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 constexpr int TMEM_COLS = 512;
-constexpr int SF_COL0 = 64;                  // accumulators: buffer b, issuer j at columns 32 b + 16 j
+constexpr int NI = 4;                        // MMA issuer warps
+constexpr int SF_COL0 = 2 * NI * 16;         // accumulators: buffer b, issuer j at columns 16 (NI b + j)
 constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation scales 16 cols
 constexpr int MAX_CLUSTER = 8;               // portable cluster size
 
@@ -452,9 +453,11 @@ FP4_DEV void store_row(const Params &p, int n, const float *acc, float alpha)
     }
 }
 
-// Threads: warp 0 loads, warps 1 and 6 issue MMAs, warps 2-5 drain the
+// Threads: warp 0 loads, warps 1, 6, 7, 8 issue MMAs, warps 2-5 drain the
 // accumulators (warp w may read TMEM lanes 32 (w % 4) .. + 31).
-constexpr int DECODE_THREADS = 224;
+constexpr int DECODE_THREADS = 32 * (6 + NI - 1);
+static_assert(STAGES % NI == 0, "a stage is always issued by the same warp");
+static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "TMEM budget");
 
 template <int FMT>
 __global__ void __launch_bounds__(DECODE_THREADS, 1)
@@ -491,13 +494,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
     const int npre = n_units < STAGES ? n_units : STAGES;
     const uint32_t smem0 = smem_u32(smem);
-    // Dual issue: a tcgen05 instruction costs its issuing thread tens of
-    // cycles, far longer than the tensor pipe needs for an N = 16 MMA, so two
-    // warps issue alternate K steps into two accumulators that the epilogue
-    // adds.  Used when the CTA owns one tile segment of at least two units
-    // (whole tiles and cluster splits); otherwise warp 1 issues alone.
-    const bool dual = nseg == 1 && n_units >= 2;
-    const uint32_t issuers = dual ? 2u : 1u;
+    // NI issuers: a tcgen05 instruction costs its issuing thread tens of
+    // cycles, far longer than the tensor pipe needs for an N = 16 MMA, so NI
+    // warps take the units i = j (mod NI) and accumulate them in their own
+    // accumulators, which the epilogue adds in issuer order.  Every issuer
+    // commits once per tile segment (also one that owns no unit of it), so
+    // the segment barrier counts NI arrivals.
 
     auto advance = [&](int &t, int &ks) {
         if (++ks == p.nk) {
@@ -524,10 +526,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             mbar_init(empty0 + 8 * s, 1);
         }
         for (int b = 0; b < 2; b++) {
-            mbar_init(accf0 + 8 * b, issuers);
+            mbar_init(accf0 + 8 * b, NI);
             mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
         }
-        mbar_init(drainb, issuers);
+        mbar_init(drainb, NI);
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch_desc(&tmW);
@@ -581,9 +583,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             }
         }
         __syncwarp();
-    } else if (warp == 1 || warp == 6) {
-        const int j = warp == 1 ? 0 : 1;  // issuer index
-        if (lane == 0 && (j == 0 || dual)) {
+    } else if (warp == 1 || warp >= 6) {
+        const int j = warp == 1 ? 0 : warp - 5;  // issuer index
+        if (lane == 0) {
             // Descriptors of stage 0: a stage, atom or K step only moves the
             // 16-byte-unit start address in the low 14 bits (shared memory
             // offsets stay below 256 KB, so the add never carries out).
@@ -591,47 +593,52 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             const uint64_t adesc0 = smem_desc(smem0 + W_BYTES, 16, 1024, 2);
             const uint64_t sfwdesc0 = smem_desc(smem0 + W_BYTES + A_BYTES, 0, 128, 0);
             const uint64_t sfadesc0 = smem_desc(smem0 + W_BYTES + A_BYTES + SFW_BYTES, 0, 128, 0);
-            const int step = dual ? 2 : 1;
-            int seg = -1;
-            int t = t_first, ks = ks_first;
-            if (j == 1) advance(t, ks);
-            for (int i = j; i < n_units; i += step) {
-                const int s = i % STAGES;
-                const uint32_t ph = (uint32_t)((i / STAGES) & 1);
-                // first / last unit of a tile segment among this warp's units
-                const bool first = dual ? (i == j) : ((i == 0) || ks == 0);
-                const bool last = dual ? (i + 2 >= n_units) : ((i == n_units - 1) || ks == p.nk - 1);
-                if (first) {
-                    seg++;
-                    if (seg >= 2 &&
-                        !mbar_wait_bounded(acce0 + 8 * (seg & 1), (uint32_t)(((seg >> 1) - 1) & 1), abort_flag, &g_gemm_error, p.budget_ns))
+            int i0 = 0, ks0 = ks_first;  // first unit of the segment and its K step
+            bool stop = false;
+            for (int seg = 0; seg < nseg && !stop; seg++) {
+                const int len = (p.nk - ks0 < n_units - i0) ? p.nk - ks0 : n_units - i0;
+                const int b = seg & 1;
+                const int first = i0 + ((j - i0) % NI + NI) % NI;  // this issuer's first unit of the segment
+                // Buffer b is free once the epilogue has drained segment seg - 2.
+                // Every issuer waits, also one without units here: its commit
+                // below must not count toward the barrier's previous phase.
+                if (seg >= 2 &&
+                    !mbar_wait_bounded(acce0 + 8 * b, (uint32_t)(((seg >> 1) - 1) & 1), abort_flag, &g_gemm_error, p.budget_ns))
+                    break;
+                const uint32_t acc = tmem + (uint32_t)(b * NI + j) * BNA;
+                for (int i = first; i < i0 + len; i += NI) {
+                    const int s = i % STAGES;
+                    const uint32_t ph = (uint32_t)((i / STAGES) & 1);
+                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) {
+                        stop = true;
                         break;
-                }
-                if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) break;
-                tc_fence_after();
-                const uint32_t acc = tmem + (uint32_t)(seg & 1) * 2 * BNA + (uint32_t)j * BNA;
-                const uint64_t so = (uint64_t)((s * STAGE_BYTES) >> 4);
-                const uint32_t tsfw = tmem + SF_COL0 + s * SF_STAGE_COLS;
-                const uint32_t tsfa = tsfw + 16;
+                    }
+                    tc_fence_after();
+                    const uint64_t so = (uint64_t)((s * STAGE_BYTES) >> 4);
+                    const uint32_t tsfw = tmem + SF_COL0 + s * SF_STAGE_COLS;
+                    const uint32_t tsfa = tsfw + 16;
 #pragma unroll
-                for (int a = 0; a < KA; a++) {
-                    tc_cp_scale_atom(tsfw + 4 * a, sfwdesc0 + so + 32 * a);
-                    tc_cp_scale_atom(tsfa + 4 * a, sfadesc0 + so + 32 * a);
-                }
+                    for (int a = 0; a < KA; a++) {
+                        tc_cp_scale_atom(tsfw + 4 * a, sfwdesc0 + so + 32 * a);
+                        tc_cp_scale_atom(tsfa + 4 * a, sfadesc0 + so + 32 * a);
+                    }
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) {
-                    const uint64_t wd = wdesc0 + so + 2 * kk;
-                    const uint64_t ad = adesc0 + so + 2 * kk;
-                    const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
-                    const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
-                    const uint32_t idesc = idesc_blockscaled(BMW, BNA, FMT == FP4_MXFP4, sfid, sfid);
-                    tc_mma_blockscaled<FMT>(acc, wd, ad, idesc, (tsfw + 4 * atom) | (sfid << 30),
-                                            (tsfa + 4 * atom) | (sfid << 30), (first && kk == 0) ? 0u : 1u);
+                    for (int kk = 0; kk < 4; kk++) {
+                        const uint64_t wd = wdesc0 + so + 2 * kk;
+                        const uint64_t ad = adesc0 + so + 2 * kk;
+                        const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
+                        const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
+                        const uint32_t idesc = idesc_blockscaled(BMW, BNA, FMT == FP4_MXFP4, sfid, sfid);
+                        tc_mma_blockscaled<FMT>(acc, wd, ad, idesc, (tsfw + 4 * atom) | (sfid << 30),
+                                                (tsfa + 4 * atom) | (sfid << 30), (i == first && kk == 0) ? 0u : 1u);
+                    }
+                    tc_commit(empty0 + 8 * s);
                 }
-                tc_commit(empty0 + 8 * s);
-                if (last) tc_commit(accf0 + 8 * (seg & 1));
-                advance(t, ks);
-                if (dual) advance(t, ks);
+                if (stop) break;
+                // this issuer's part of the segment is complete (at once if it had none)
+                tc_commit(accf0 + 8 * b);
+                i0 += len;
+                ks0 = 0;
             }
             // arrives once every MMA issued above has completed
             tc_commit(drainb);
@@ -649,19 +656,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) break;
         tc_fence_after();
+        // the segment's units and the issuers that own some of them
+        const int i0 = seg == 0 ? 0 : (p.nk - ks_first) + (seg - 1) * p.nk;
+        const int len = (seg == 0) ? ((p.nk - ks_first < n_units) ? p.nk - ks_first : n_units)
+                                   : ((p.nk < n_units - i0) ? p.nk : n_units - i0);
         uint32_t r[16];
         const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
-        tmem_ld16(tmem + (uint32_t)b * 2 * BNA + lanes, r);
-        if (dual) {
-            // the second issuer's accumulator, added in a fixed order
-            uint32_t r2[16];
-            tmem_ld16(tmem + (uint32_t)b * 2 * BNA + BNA + lanes, r2);
+        float sum[BNA];
+#pragma unroll
+        for (int m = 0; m < BNA; m++) sum[m] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NI; j++) {
+            if (((j - i0) % NI + NI) % NI >= len) continue;  // issuer j owns no unit of this segment
+            tmem_ld16(tmem + (uint32_t)(b * NI + j) * BNA + lanes, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int m = 0; m < BNA; m++) r[m] = __float_as_uint(__fadd_rn(__uint_as_float(r[m]), __uint_as_float(r2[m])));
-        } else {
-            tmem_ld_wait();
+            for (int m = 0; m < BNA; m++) sum[m] = __fadd_rn(sum[m], __uint_as_float(r[m]));
         }
+#pragma unroll
+        for (int m = 0; m < BNA; m++) r[m] = __float_as_uint(sum[m]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");

@@ -112,7 +112,7 @@ FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, co
 {
     uint4 out;
     const uint32_t sb = MSE ? encode_unit_mse<FMT>(v, six_sg, a.round_away, tab, out)
-                            : encode_unit<FMT>(v, sg, six_sg, a.round_away, a.mx_floor, out);
+                            : encode_unit<FMT>(v, sg, six_sg, a.round_away, a.mx_floor, out, tab);
     if (FMT == FP4_MXFP4)
         a.s[scale_offset(row, j, a.nkb4)] = (uint8_t)sb;
     else
@@ -196,8 +196,8 @@ FP4_DEV void quantize_body(const QuantArgs &a)
     }
     const bool hinted = FMT == FP4_NVFP4 && a.gscale_computed;  // second read of x
     const uint64_t pol = l2_policy_evict_first();
-    __shared__ NvScaleTables tab;  // NVFP4 MSE search only
-    if (MSE && FMT == FP4_NVFP4) {
+    __shared__ NvScaleTables tab;  // NVFP4 only
+    if (FMT == FP4_NVFP4) {
         nv_tables_fill(tab, sg, threadIdx.x, blockDim.x);
         __syncthreads();
     }
@@ -228,7 +228,7 @@ FP4_DEV void quantize_body(const QuantArgs &a)
             if (HK) fwht_unit<HK>(v, a.ck, lane);
             if (!live) continue;
 
-            encode_store_unit<FMT, MSE>(v, u, row[i], col[i], a, sg, six_sg, &tab);
+            encode_store_unit<FMT, MSE>(v, u, row[i], col[i], a, sg, six_sg, FMT == FP4_NVFP4 ? &tab : nullptr);
         }
     }
 }
@@ -282,13 +282,17 @@ FP4_DEV void fetch_units(const QuantArgs &a, int64_t base, int64_t stride, int l
 }
 
 template <int FMT, int HK>
-__global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, unsigned *zero, int nzero)
+__global__ void __launch_bounds__(ACT_THREADS) act_quant_kernel(QuantArgs a, unsigned *zero, int nzero, int early)
 {
     // Launched programmatically after the previous work in the stream.  The
-    // dependent split-K kernel streams W before it waits, so it may only start
-    // once everything before this kernel has finished: trigger after the wait.
+    // dependent split-K kernel streams W before it waits, so by default it may
+    // only start once everything before this kernel has finished: trigger
+    // after the wait.  With `early` (the caller's weights are written by no
+    // kernel that can still be running) it starts at once and streams W while
+    // the previous work, and this kernel, finish.
+    if (early) grid_dep_launch();
     grid_dep_wait();
-    grid_dep_launch();
+    if (!early) grid_dep_launch();
     __shared__ float red[ACT_THREADS / 32];
     __shared__ float cta_max;
     const int lane = threadIdx.x & 31;
@@ -611,7 +615,7 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
 
 
 template <int FMT>
-static void (*act_kernel_for(int hk))(QuantArgs, unsigned *, int)
+static void (*act_kernel_for(int hk))(QuantArgs, unsigned *, int, int)
 {
     switch (hk) {
     case 0: return act_quant_kernel<FMT, 0>;
@@ -626,7 +630,7 @@ static void (*act_kernel_for(int hk))(QuantArgs, unsigned *, int)
 // Cluster size of the activation quantizer: ACT_CTAS (a non-portable size)
 // where the device schedules such clusters, else the portable ACT_CTAS_PORTABLE.
 // Decided once per kernel instance.
-static int act_cluster_size(void (*k)(QuantArgs, unsigned *, int))
+static int act_cluster_size(void (*k)(QuantArgs, unsigned *, int, int))
 {
     static std::mutex mu;
     static std::map<const void *, int> sizes;
@@ -660,10 +664,12 @@ static int act_cluster_size(void (*k)(QuantArgs, unsigned *, int))
 }
 
 // Single-launch quantization of a small activation tensor (see
-// act_quant_kernel); scale padding is left unwritten.
+// act_quant_kernel).  Only the NVFP4 tensor maximum needs the CTAs to form a
+// cluster; without it the CTAs are scheduled one by one, which a device
+// still busy with the previous kernel can do sooner.
 cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt, int hk, float ck,
                                 int round_away, int mx_floor, int gscale_given, uint8_t *q, uint8_t *s, float *gscale,
-                                unsigned *zero, int nzero, cudaStream_t st)
+                                unsigned *zero, int nzero, int early, cudaStream_t st)
 {
     QuantArgs a;
     a.x = x;
@@ -682,26 +688,27 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     a.round_away = round_away;
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
-    void (*k)(QuantArgs, unsigned *, int) = (fmt == FP4_MXFP4) ? act_kernel_for<FP4_MXFP4>(hk) : act_kernel_for<FP4_NVFP4>(hk);
+    void (*k)(QuantArgs, unsigned *, int, int) = (fmt == FP4_MXFP4) ? act_kernel_for<FP4_MXFP4>(hk) : act_kernel_for<FP4_NVFP4>(hk);
     if (!k) return cudaErrorInvalidValue;
-    const int ctas = act_cluster_size(k);
+    const bool cluster = a.gscale_computed != 0;
+    const int ctas = cluster ? act_cluster_size(k) : ACT_CTAS;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas);
     cfg.blockDim = dim3(ACT_THREADS);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = ctas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
     // May start while the previous kernel drains (its launch latency is then
     // hidden); the kernel waits for it before touching memory.
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = ctas;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = cluster ? 2 : 1;
     count_launches(1);
-    return cudaLaunchKernelEx(&cfg, k, a, zero, nzero);
+    return cudaLaunchKernelEx(&cfg, k, a, zero, nzero, early);
 }
 
 template <int FMT, int BF>

@@ -91,6 +91,13 @@ typedef struct {
     int gscale_given;   /* NVFP4: 1 = *gscale holds s_g on entry (offline
                            scale); 0 = s_g is computed from the tensor.       */
     int scale_search;   /* fp4_scale_search                                   */
+    int weights_static; /* fp4_linear, M <= 16: 1 = W, its scales and gW are
+                           written by no kernel that may still be running when
+                           the call's kernels start (weights prepared once and
+                           read-only, as in inference).  The decode kernel then
+                           streams W while the work before it in the stream
+                           finishes; activations and C stay ordered after it.
+                           0 (default): W is read only after that work.      */
 } fp4_opts;
 
 /* Human-readable name of a status code (static string). */

@@ -360,3 +360,36 @@ def test_linear_decode_fused_reduction_matches_gemm(fp4, orc, fmt, M, N, K, hk):
     cb = fp4.linear(xd, W, fmt, hadamard_k=hk, out_dtype=1)
     torch.cuda.synchronize()
     assert torch.equal(cb, c1.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_linear_static_weights_chain(fp4, orc, fmt):
+    """weights_static lets the decode kernel stream W while the previous
+    kernel in the stream finishes; activations and outputs stay ordered.  A
+    chain of dependent decode layers (each output is the next layer's input,
+    N = K) with a different weight per layer, issued back to back without a
+    synchronisation, equals the same chain without the option bit for bit."""
+    import torch
+    M, D, L = 4, 4096, 6
+    rng = np.random.default_rng(17 + fmt)
+    Ws = []
+    for i in range(L):
+        w = inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (D, D)).astype(np.float32))
+        Ws.append(fp4.quantize(to_dev_bf16(w), fmt))
+    x0 = to_dev_bf16(inputs.f32_to_bf16_bits(rng.laplace(0, 1, (M, D)).astype(np.float32)))
+    ws = torch.empty((fp4.linear_workspace_size(M, D, D, fmt),), dtype=torch.uint8, device="cuda")
+
+    def chain(static):
+        outs, x = [], x0
+        for i in range(L):
+            x = fp4.linear(x, Ws[i], fmt, out_dtype=1, workspace=ws, weights_static=static)
+            outs.append(x)
+        torch.cuda.synchronize()
+        fp4.check_device_status()
+        return outs
+
+    ref = chain(False)
+    for _ in range(3):
+        got = chain(True)
+        for i in range(L):
+            assert torch.equal(got[i], ref[i]), f"layer {i} differs"
