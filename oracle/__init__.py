@@ -18,6 +18,9 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   quantize / dequantize   pinned: worked examples, power-of-two invariants,
                           Eq.(2) norm identity
   gemm reference          pinned: numpy fp64 matmul
+  MXFP4 -> NVFP4 scales  pinned: dequantized elements unchanged (exact)
+                          within 17 binades, E4M3 rounding past them,
+                          closed-form s_g (tests/test_oracle_pins.py)
   MSE block-scale search  pinned: hand-derived blocks, exhaustive numpy search
                           over every representable scale, nearest-element
                           property (tests/test_oracle_mse_pins.py)
@@ -91,6 +94,8 @@ def lib():
         L.fp4o_scales_to_atoms.argtypes = [vp, i64, i64, vp]
         L.fp4o_scales_from_atoms.argtypes = [vp, i64, i64, vp]
         L.fp4o_gemm_ref.argtypes = [vp, vp, i64, i64, i64, vp, vp]
+        L.fp4o_mx_scales_to_nv.argtypes = [vp, i64, i64, vp, vp]
+        L.fp4o_mx_scales_to_nv.restype = i32
         L.fp4o_num_threads.restype = i32
         _lib = L
     return _lib
@@ -210,6 +215,18 @@ def scales_from_atoms(s_atoms: np.ndarray, rows: int, nkb: int) -> np.ndarray:
     out = np.zeros((rows, nkb), np.uint8)
     lib().fp4o_scales_from_atoms(_ptr(a), rows, nkb, _ptr(out))
     return out
+
+
+def mx_scales_to_nv(s_mx_logical: np.ndarray):
+    """MXFP4 scales (rows, nkb) -> (NVFP4 scales (rows, 2 nkb), s_g) with the
+    same dequantized elements (late binding of an MXFP4 weight to NVFP4)."""
+    s = np.ascontiguousarray(s_mx_logical, dtype=np.uint8)
+    rows, nkb = s.shape
+    out = np.zeros((rows, 2 * nkb), np.uint8)
+    g = np.zeros(1, np.float32)
+    if lib().fp4o_mx_scales_to_nv(_ptr(s), rows, nkb, _ptr(out), _ptr(g)) != 0:
+        raise ValueError("oracle mx_scales_to_nv: invalid arguments")
+    return out, float(g[0])
 
 
 def gemm_ref(a_hat: np.ndarray, w_hat: np.ndarray):

@@ -427,6 +427,39 @@ int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
 }
 
 /* ------------------------------------------------------------------------ */
+/* MXFP4 -> NVFP4 scale repacking ([TransFP4] §2.5 and §3.4: a logical       */
+/* artifact is bound late to the backend's native format; "NVFP4 activations */
+/* with MXFP4 weights" needs the weights in the NVFP4 scale form).  The      */
+/* E2M1 elements are kept; each 32-block power-of-two scale 2^e becomes two  */
+/* 16-block E4M3 scales 2^(e - E) under the tensor scale s_g = 2^E, so that  */
+/* s_g * s_b = 2^e and every element dequantizes to the same value          */
+/* ([Guide] §4.1).  E = max(e_max - 8, -126): the largest block scale lands  */
+/* on 2^8, the largest power of two E4M3 holds, and s_g stays a normal       */
+/* float.  Blocks more than 17 binades below the largest (2^(e-E) below the  */
+/* smallest E4M3 subnormal 2^-9) take the E4M3 rounding of 2^(e-E): 0.       */
+/* E8M0 NaN (0xFF) maps to E4M3 NaN (0x7F).                                   */
+/* ------------------------------------------------------------------------ */
+int fp4o_mx_scales_to_nv(const uint8_t *s_mx, int64_t rows, int64_t nkb, uint8_t *s_nv,
+                         float *gscale)
+{
+    if (rows < 0 || nkb < 0) return -1;
+    int e_max = -1000;
+    for (int64_t i = 0; i < rows * nkb; i++)
+        if (s_mx[i] != 0xFF && (int)s_mx[i] - 127 > e_max) e_max = (int)s_mx[i] - 127;
+    int E = e_max - 8;
+    if (E < -126) E = -126;
+    *gscale = ldexpf(1.0f, E);
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t kb = 0; kb < nkb; kb++) {
+            uint8_t b = s_mx[r * nkb + kb];
+            uint8_t nv = (b == 0xFF) ? 0x7F : (uint8_t)fp4o_e4m3_encode(ldexpf(1.0f, (int)b - 127 - E));
+            s_nv[r * 2 * nkb + 2 * kb] = nv;
+            s_nv[r * 2 * nkb + 2 * kb + 1] = nv;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Scale tile layout consumed by the block-scaled tensor-core MMA: 512-byte   */
 /* atoms of 128 rows x 4 scale columns; atoms ordered row-block major, then  */
 /* scale-column block.  Inside an atom, row r and column j sit at byte       */

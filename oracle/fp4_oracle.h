@@ -68,6 +68,12 @@ int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
                     int64_t rows, int64_t cols, int fmt, int block,
                     int hadamard_k, float *out);
 
+/* MXFP4 scales (logical, rows x nkb, E8M0) -> NVFP4 scales (logical,
+ * rows x 2*nkb, E4M3) and the tensor scale s_g = 2^E that keep every
+ * element's dequantized value (see the function's comment). */
+int fp4o_mx_scales_to_nv(const uint8_t *s_mx, int64_t rows, int64_t nkb, uint8_t *s_nv,
+                         float *gscale);
+
 /* logical scales (rows x nkb) -> tcgen05 scale-atom layout
  * (pad128(rows) x pad4(nkb) bytes, padding bytes 0), and back. */
 void fp4o_scales_to_atoms(const uint8_t *s_logical, int64_t rows, int64_t nkb,

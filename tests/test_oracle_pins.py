@@ -480,3 +480,42 @@ def test_quantize_f32_brute_force_nearest(orc, tie):
         codes[:, 1::2] = q >> 4
         assert np.array_equal(codes, want), fmt
         assert np.all(s == (127 if fmt == 0 else 0x38))
+
+
+# ----------------------------------------------------- MXFP4 -> NVFP4 scales ----
+def test_mx_to_nv_scales_keep_every_element(orc):
+    """Late binding of an MXFP4 weight to the NVFP4 scale form ("Portable FP4
+    quantization (TransFP4)" §2.5): the same E2M1 codes dequantize to the same
+    values, bit for bit, for weights whose block scales span <= 17 binades."""
+    for seed, fmt_rows in ((0, (64, 512)), (1, (37, 1024)), (2, (128, 4096))):
+        rows, cols = fmt_rows
+        rng = np.random.default_rng(seed)
+        w = inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (rows, cols)).astype(np.float32))
+        q, s_mx, _ = orc.quantize(w, orc.MXFP4)
+        s_nv, g = orc.mx_scales_to_nv(s_mx)
+        assert s_nv.shape == (rows, cols // 16)
+        a = orc.dequantize(q, s_mx, 1.0, orc.MXFP4)
+        b = orc.dequantize(q, s_nv, g, orc.NVFP4)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_mx_to_nv_scales_closed_form(orc):
+    """s_g = 2^(e_max - 8); each 2^e becomes 2^(e - E) in E4M3: normal codes
+    (exponent field e - E + 7, mantissa 0), subnormals 2^-7, 2^-8, 2^-9 as
+    mantissa 4, 2, 1, and 2^-10 (a tie with 0) and below as 0."""
+    e_max = 13
+    E = e_max - 8
+    es = [e_max, 0, e_max - 14, e_max - 15, e_max - 16, e_max - 17, e_max - 18, e_max - 40]
+    want = [0x78, ((0 - E) + 7) << 3, 0x08, 0x04, 0x02, 0x01, 0x00, 0x00]
+    s_mx = np.array([[e + 127 for e in es]], np.uint8)
+    s_nv, g = orc.mx_scales_to_nv(s_mx)
+    assert g == 2.0 ** E
+    assert s_nv[0, 0::2].tolist() == want and s_nv[0, 1::2].tolist() == want
+    for e, b in zip(es, want):
+        if b:
+            assert orc.e4m3_decode(b) * g == 2.0 ** e
+    # NaN scale, and a tensor of zero blocks (s_g clamped to the smallest normal float)
+    s_nv, g = orc.mx_scales_to_nv(np.array([[0xFF, 127]], np.uint8))
+    assert s_nv[0, :2].tolist() == [0x7F, 0x7F]
+    s_nv, g = orc.mx_scales_to_nv(np.zeros((2, 4), np.uint8))
+    assert g == 2.0 ** -126 and (s_nv == 0x30).all()
