@@ -143,8 +143,13 @@ def bench_decode(torch, fp4, inputs, dev, reps: int):
         _, w = inputs.decode_linear(1, N, K)
         wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
         del w
-        for fmt, name in ((fp4.FP4_NVFP4, "nvfp4"), (fp4.FP4_MXFP4, "mxfp4")):
-            W0 = fp4.quantize(wd, fmt)
+        # the third case is the workload's literal reading: NVFP4 activations
+        # against MXFP4 weights, bound once to the NVFP4 scale form
+        for fmt, name, wfmt in ((fp4.FP4_NVFP4, "nvfp4", fp4.FP4_NVFP4), (fp4.FP4_MXFP4, "mxfp4", fp4.FP4_MXFP4),
+                                (fp4.FP4_NVFP4, "nvfp4act_mxfp4w", fp4.FP4_MXFP4)):
+            W0 = fp4.quantize(wd, wfmt)
+            if wfmt != fmt:
+                W0 = fp4.mx_to_nv(W0)
             wbytes = W0[0].numel() + W0[1].numel()
             copies = max(2, int(2 * 126e6 // wbytes) + 1)
             Ws = [tuple(t.clone() for t in W0) for _ in range(copies)]

@@ -158,6 +158,21 @@ def gemm_quantized(a, w, M: int, N: int, K: int, fmt, out_fmt, gscale=None, roun
     return Cq, Cs, gC
 
 
+def mx_to_nv(w):
+    """An MXFP4 tensor w = (q, s, g) in the NVFP4 scale form (q, s_nv, s_g)
+    with the same dequantized elements (see fp4_mx_to_nv_scales); q is shared."""
+    import torch
+
+    q, s, _ = w
+    rows, cols = q.shape[0], q.shape[1] * 2
+    _, sb = quantize_sizes(rows, cols, FP4_NVFP4)
+    s_nv = torch.empty((sb,), dtype=torch.uint8, device=q.device)
+    g = torch.empty((1,), dtype=torch.float32, device=q.device)
+    _lib.check("fp4_mx_to_nv_scales", _lib.lib().fp4_mx_to_nv_scales(
+        s.data_ptr(), rows, cols, s_nv.data_ptr(), g.data_ptr(), _stream_handle(torch, q.device)))
+    return q, s_nv, g
+
+
 def linear_workspace_size(M: int, N: int, K: int, fmt) -> int:
     b = ctypes.c_size_t()
     _lib.check("fp4_linear_workspace_size",

@@ -38,6 +38,7 @@ SIGNATURES = {
     "fp4_gemm_workspace_size": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_sz)]),
     "fp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _i64,
                         _vp, _sz, _vp]),
+    "fp4_mx_to_nv_scales": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "fp4_gemm_quantized": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp,
                                   _vp, _vp]),
     "fp4_check_device_status": (_int, [_vp]),

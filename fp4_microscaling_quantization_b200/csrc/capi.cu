@@ -28,6 +28,8 @@ cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const fl
                                   const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K, int fmt,
                                   int out_fmt, int round_away, int mx_floor, const float *gC, uint8_t *Cq, uint8_t *Cs,
                                   int sms, cudaStream_t st);
+cudaError_t launch_mx_to_nv_scales(const uint8_t *s_mx, int64_t rows, int64_t cols, uint8_t *s_nv, float *gscale,
+                                   int sms, cudaStream_t st);
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -280,6 +282,19 @@ fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float 
     cudaError_t e = fp4::launch_gemm_quantized(Aq, As, gA, Wq, Ws, gW, M, N, K, fmt, out_fmt,
                                                o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
                                                gC, Cq, Cs, sm_count(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status fp4_mx_to_nv_scales(const uint8_t *s_mx, int64_t rows, int64_t cols, uint8_t *s_nv, float *gscale,
+                               void *stream)
+{
+    if (rows < 0 || cols < 0 || !gscale) return FP4_ERR_INVALID_ARG;
+    if (cols % 32) return FP4_ERR_UNSUPPORTED;
+    if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
+    if (rows > 0 && cols > 0 && (!s_mx || !s_nv)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(gscale, 4)) return FP4_ERR_ALIGNMENT;
+    cudaError_t e = fp4::launch_mx_to_nv_scales(s_mx, rows, cols, s_nv, gscale, sm_count(),
+                                                static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 

@@ -15,6 +15,7 @@
 // the last butterfly stages exchange values with shuffles.  Warps walk the
 // tensor in a grid-stride loop of 32 consecutive units, so neighbouring
 // lanes read and write neighbouring memory.
+#include <algorithm>
 #include <map>
 #include <mutex>
 
@@ -722,6 +723,94 @@ static void (*deq_kernel_for(int hk))(DequantArgs)
     case 128: return dequantize_kernel<FMT, 128, BF>;
     }
     return nullptr;
+}
+
+// ---------------------------------------------------------------------------
+// MXFP4 -> NVFP4 scale repacking ("Portable FP4 quantization (TransFP4)"
+// §2.5, §3.4: an artifact is bound late to the backend's native format).  The
+// E2M1 elements stay; each 32-block scale 2^e becomes two 16-block E4M3
+// scales 2^(e - E) under s_g = 2^E, E = max(e_max - 8, -126), so that
+// s_g * s_b = 2^e: the largest block scale lands on 2^8, the largest power of
+// two E4M3 holds.  Blocks more than 17 binades below it take the E4M3
+// rounding of 2^(e - E) (0 from 2^-10 down).  E8M0 NaN becomes E4M3 NaN.
+
+// Position (row, scale column) of byte i of a scale tile layout with nkb4
+// 4-column groups (the inverse of scale_offset).
+FP4_DEV void scale_position(int64_t i, int64_t nkb4, int64_t &r, int64_t &kb)
+{
+    const int64_t atom = i >> 9, o = i & 511;
+    r = (atom / nkb4) * 128 + ((o & 15) >> 2) * 32 + (o >> 4);
+    kb = (atom % nkb4) * 4 + (o & 3);
+}
+
+__global__ void set_word_kernel(float *g, float v)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    *g = v;
+}
+
+// *g = max(*g, 2^(e_max - 8)) over the real MXFP4 scale bytes, as an integer
+// max of the float bits (positive floats order like their bits).  2^(b - 135)
+// has the bits (b - 8) << 23 for a byte b >= 9; smaller bytes fall under the
+// 2^-126 that *g starts from.
+__global__ void mx_scale_max_kernel(const uint8_t *s, int64_t rows, int64_t nkb, int64_t nkb4, float *g)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    uint32_t best = 0;
+    const int64_t n = (rows + 127) / 128 * 128 * nkb4 * 4;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r, kb;
+        scale_position(i, nkb4, r, kb);
+        const uint32_t b = s[i];
+        if (r < rows && kb < nkb && b != 0xFFu && b >= 9u) best = max(best, (b - 8u) << 23);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xFFFFFFFFu, best, o));
+    if ((threadIdx.x & 31) == 0 && best) atomicMax(reinterpret_cast<unsigned int *>(g), best);
+}
+
+// Writes every byte of the NVFP4 scale layout: the repacked scale of real
+// positions, 0 in the padding.
+__global__ void mx_to_nv_scale_kernel(const uint8_t *s_mx, int64_t rows, int64_t nkb, int64_t nkb4_mx, int64_t nkb4_nv,
+                                      const float *g, uint8_t *s_nv)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    const int E = (int)((__float_as_uint(*g) >> 23) & 0xFF) - 127;
+    const int64_t n = (rows + 127) / 128 * 128 * nkb4_nv * 4;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r, kb16;
+        scale_position(i, nkb4_nv, r, kb16);
+        uint32_t v = 0;
+        if (r < rows && kb16 < 2 * nkb) {
+            const uint32_t b = s_mx[scale_offset(r, kb16 >> 1, nkb4_mx)];
+            if (b == 0xFFu) {
+                v = 0x7Fu;
+            } else {
+                const int d = (int)b - 127 - E;
+                v = e4m3_rn(exp2i(d < -127 ? -127 : d));
+            }
+        }
+        s_nv[i] = (uint8_t)v;
+    }
+}
+
+cudaError_t launch_mx_to_nv_scales(const uint8_t *s_mx, int64_t rows, int64_t cols, uint8_t *s_nv, float *gscale,
+                                   int sms, cudaStream_t st)
+{
+    const int64_t nkb = cols / 32, nkb4_mx = (nkb + 3) / 4, nkb4_nv = (2 * nkb + 3) / 4;
+    cudaError_t e = launch_k(set_word_kernel, dim3(1), dim3(1), 0, st, true, gscale, 1.17549435082228750797e-38f);
+    if (e != cudaSuccess || rows == 0 || nkb == 0) return e;
+    const int64_t n_mx = (rows + 127) / 128 * 128 * nkb4_mx * 4, n_nv = (rows + 127) / 128 * 128 * nkb4_nv * 4;
+    const int g1 = (int)std::min<int64_t>((n_mx + 255) / 256, (int64_t)sms * 4);
+    const int g2 = (int)std::min<int64_t>((n_nv + 255) / 256, (int64_t)sms * 4);
+    if ((e = launch_k(mx_scale_max_kernel, dim3(g1), dim3(256), 0, st, true, s_mx, rows, nkb, nkb4_mx, gscale)) !=
+        cudaSuccess)
+        return e;
+    return launch_k(mx_to_nv_scale_kernel, dim3(g2), dim3(256), 0, st, true, s_mx, rows, nkb, nkb4_mx, nkb4_nv,
+                    (const float *)gscale, s_nv);
 }
 
 cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,

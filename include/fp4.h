@@ -207,6 +207,26 @@ fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float 
                               uint8_t *Cs, void *stream);
 
 
+/*
+ * fp4_mx_to_nv_scales — late binding of an MXFP4 tensor to the NVFP4 scale
+ * form ("Portable FP4 quantization (TransFP4)" §2.5, §3.4), so that NVFP4
+ * activations can meet MXFP4 weights in the NVFP4 tensor-core product
+ * (fp4_linear / fp4_gemm with fmt = FP4_NVFP4 and the same packed elements).
+ * Each 32-block scale 2^e becomes two 16-block E4M3 scales 2^(e - E) under
+ * the tensor scale s_g = 2^E, E = max(e_max - 8, -126) (e_max: the largest
+ * block exponent), so s_g * s_b = 2^e and every element dequantizes to the
+ * same value.  Blocks more than 17 binades below the largest take the E4M3
+ * rounding of 2^(e - E), which is 0 from 2^-10 down; E8M0 NaN becomes E4M3
+ * NaN.  Three small launches; meant to run once per weight.
+ *   s_mx    MXFP4 scales of a rows x cols tensor in the tile layout, as
+ *           fp4_quantize writes them (cols multiple of 32).
+ *   s_nv    output: fp4_quantize_sizes(rows, cols, FP4_NVFP4, 16) scale
+ *           bytes in the tile layout, padding written 0.
+ *   gscale  output: s_g, one device fp32 (4-byte aligned).
+ */
+fp4_status fp4_mx_to_nv_scales(const uint8_t *s_mx, int64_t rows, int64_t cols, uint8_t *s_nv,
+                               float *gscale, void *stream);
+
 /* Bytes of device scratch fp4_linear needs (quantized activations, their
  * scales and tensor scale, and the GEMM workspace).  Host-only. */
 fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes);
