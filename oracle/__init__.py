@@ -21,6 +21,9 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   MXFP4 -> NVFP4 scales  pinned: dequantized elements unchanged (exact)
                           within 17 binades, E4M3 rounding past them,
                           closed-form s_g (tests/test_oracle_pins.py)
+  sparse residual lane    pinned: FP4 stream equals the plain quantizer on the
+                          zeroed values, bf16 RNE against torch, one-value
+                          units exact, NMSE below the plain quantizer
   MSE block-scale search  pinned: hand-derived blocks, exhaustive numpy search
                           over every representable scale, nearest-element
                           property (tests/test_oracle_mse_pins.py)
@@ -95,6 +98,10 @@ def lib():
         L.fp4o_scales_from_atoms.argtypes = [vp, i64, i64, vp]
         L.fp4o_gemm_ref.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.fp4o_mx_scales_to_nv.argtypes = [vp, i64, i64, vp, vp]
+        L.fp4o_quantize_residual.argtypes = [vp, i64, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.fp4o_quantize_residual.restype = i32
+        L.fp4o_dequantize_residual.argtypes = [vp, vp, f32, vp, i64, i64, i32, i32, i32, vp]
+        L.fp4o_dequantize_residual.restype = i32
         L.fp4o_mx_scales_to_nv.restype = i32
         L.fp4o_num_threads.restype = i32
         _lib = L
@@ -214,6 +221,38 @@ def scales_from_atoms(s_atoms: np.ndarray, rows: int, nkb: int) -> np.ndarray:
     a = np.ascontiguousarray(s_atoms, dtype=np.uint8)
     out = np.zeros((rows, nkb), np.uint8)
     lib().fp4o_scales_from_atoms(_ptr(a), rows, nkb, _ptr(out))
+    return out
+
+
+def quantize_residual(x_bf16: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_EVEN,
+                      mx_rule: int = MX_CEIL, gscale: float | None = None):
+    """quantize() with the sparse residual lane (TransFP4 Eq.(3), one value
+    per 32): returns (q, s_logical, s_g, res), res (rows, cols/32) uint32
+    words = bf16 bits | index << 16."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    block = block_of(fmt)
+    q = np.zeros((rows, cols // 2), np.uint8)
+    s = np.zeros((rows, cols // block), np.uint8)
+    res = np.zeros((rows, cols // 32), np.uint32)
+    g = np.array([gscale if gscale is not None else 0.0], np.float32)
+    rc = lib().fp4o_quantize_residual(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie, mx_rule,
+                                      int(gscale is not None), _ptr(g), _ptr(q), _ptr(s), _ptr(res))
+    if rc != 0:
+        raise ValueError("oracle quantize_residual: invalid arguments")
+    return q, s, (float(g[0]) if fmt == NVFP4 else 1.0), res
+
+
+def dequantize_residual(q, s_logical, gscale, res, fmt, hadamard_k: int = 0):
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s_logical, dtype=np.uint8)
+    r = np.ascontiguousarray(res, dtype=np.uint32)
+    rows, half = q.shape
+    cols = half * 2
+    out = np.zeros((rows, cols), np.float32)
+    if lib().fp4o_dequantize_residual(_ptr(q), _ptr(s), float(gscale), _ptr(r), rows, cols, fmt,
+                                      block_of(fmt), hadamard_k, _ptr(out)) != 0:
+        raise ValueError("oracle dequantize_residual: invalid arguments")
     return out
 
 

@@ -221,6 +221,34 @@ static float nv_global_scale(float amax_t)
     return 1.0f;
 }
 
+/* bf16 bit pattern of an fp32 value, rounded to nearest, ties to even (the
+ * precision of the residual lane). */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x7FFFFFu)) return (uint16_t)((u >> 16) | 0x40);  /* NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    return (uint16_t)((u + 0x7FFFu + lsb) >> 16);
+}
+
+/* Sparse residual lane ([TransFP4] §2.3 Eq.(3), r = 1 per 32 values): in
+ * every 32-value unit of the rotated row y, the value of largest magnitude
+ * (the first of equal ones) leaves the FP4 stream: it is kept as a bf16 value
+ * with its 5-bit position (word = bf16 bits | index << 16) and zeroed in y,
+ * which is then quantized as usual. */
+static void extract_residuals(float *y, int64_t cols, uint32_t *res_row)
+{
+    for (int64_t u = 0; u < cols / 32; u++) {
+        float *v = y + u * 32;
+        int best = 0;
+        for (int i = 1; i < 32; i++)
+            if (fabsf(v[i]) > fabsf(v[best])) best = i;
+        if (res_row) res_row[u] = (uint32_t)f32_to_bf16_rne(v[best]) | ((uint32_t)best << 16);
+        v[best] = 0.0f;
+    }
+}
+
 /* The absmax scale byte of one block ([TransFP4] §3.1): MX the E8M0 byte of
  * fp4o_mx_scale_exponent(amax, rule); NV the E4M3 code of t = amax / (6 s_g). */
 static int absmax_scale_byte(const float *blk, int block, int fmt, int mx_rule, float sg)
@@ -316,7 +344,7 @@ static int mse_scale_byte(const float *blk, int block, int fmt, float sg, int ti
 static int quantize_rows(const uint16_t *xb, const float *xf, int64_t rows, int64_t cols,
                          int64_t ld, int fmt, int block, int hadamard_k, int tie,
                          int mx_rule, int search, int gscale_given, float *gscale, uint8_t *q,
-                         uint8_t *s_logical)
+                         uint8_t *s_logical, uint32_t *res)
 {
     if (!valid_shape(fmt, block, hadamard_k, rows, cols) || ld < cols) return -1;
     if (search != FP4O_SCALE_ABSMAX && search != FP4O_SCALE_MSE) return -1;
@@ -335,6 +363,7 @@ static int quantize_rows(const uint16_t *xb, const float *xf, int64_t rows, int6
 #pragma omp for schedule(static)
                 for (int64_t r = 0; r < rows; r++) {
                     load_row(xb, xf, ld, r, cols, hadamard_k, y);
+                    if (res) extract_residuals(y, cols, NULL);  /* s_g of the FP4 stream */
                     for (int64_t c = 0; c < cols; c++) {
                         float a = fabsf(y[c]);
                         if (a > local) local = a;
@@ -355,6 +384,7 @@ static int quantize_rows(const uint16_t *xb, const float *xf, int64_t rows, int6
 #pragma omp for schedule(static)
         for (int64_t r = 0; r < rows; r++) {
             load_row(xb, xf, ld, r, cols, hadamard_k, y);
+            if (res) extract_residuals(y, cols, res + r * (cols / 32));
             uint8_t *qrow = q + r * (cols / 2);
             memset(qrow, 0, (size_t)(cols / 2));
             for (int64_t kb = 0; kb < nkb; kb++) {
@@ -385,7 +415,17 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                   uint8_t *q, uint8_t *s_logical)
 {
     return quantize_rows(x, NULL, rows, cols, ld, fmt, block, hadamard_k, tie, mx_rule,
-                         search, gscale_given, gscale, q, s_logical);
+                         search, gscale_given, gscale, q, s_logical, NULL);
+}
+
+int fp4o_quantize_residual(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                           int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                           int gscale_given, float *gscale, uint8_t *q, uint8_t *s_logical,
+                           uint32_t *res)
+{
+    if (!res) return -1;
+    return quantize_rows(x, NULL, rows, cols, ld, fmt, block, hadamard_k, tie, mx_rule,
+                         FP4O_SCALE_ABSMAX, gscale_given, gscale, q, s_logical, res);
 }
 
 int fp4o_quantize_f32(const float *x, int64_t rows, int64_t cols, int64_t ld,
@@ -394,15 +434,15 @@ int fp4o_quantize_f32(const float *x, int64_t rows, int64_t cols, int64_t ld,
                       uint8_t *q, uint8_t *s_logical)
 {
     return quantize_rows(NULL, x, rows, cols, ld, fmt, block, hadamard_k, tie, mx_rule,
-                         search, gscale_given, gscale, q, s_logical);
+                         search, gscale_given, gscale, q, s_logical, NULL);
 }
 
 /* ------------------------------------------------------------------------ */
 /* Dequantize ([TransFP4] Eq.(1); [Guide] §4.1 x^ = s_tensor * s_block * q)  */
 /* ------------------------------------------------------------------------ */
-int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
-                    int64_t rows, int64_t cols, int fmt, int block,
-                    int hadamard_k, float *out)
+static int dequantize_rows(const uint8_t *q, const uint8_t *s_logical, float gscale,
+                           const uint32_t *res, int64_t rows, int64_t cols, int fmt, int block,
+                           int hadamard_k, float *out)
 {
     if (!valid_shape(fmt, block, hadamard_k, rows, cols)) return -1;
     const int64_t nkb = cols / block;
@@ -420,10 +460,30 @@ int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
                 o[c] = d * qv;
             }
         }
+        if (res)  /* [TransFP4] Eq.(3): the FP4 stream plus the residual lane */
+            for (int64_t u = 0; u < cols / 32; u++) {
+                uint32_t w = res[r * (cols / 32) + u];
+                o[u * 32 + ((w >> 16) & 31)] += bf16_to_f32((uint16_t)(w & 0xFFFFu));
+            }
         if (hadamard_k)
             for (int64_t c = 0; c < cols; c += hadamard_k) fp4o_fwht(o + c, hadamard_k);
     }
     return 0;
+}
+
+int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
+                    int64_t rows, int64_t cols, int fmt, int block,
+                    int hadamard_k, float *out)
+{
+    return dequantize_rows(q, s_logical, gscale, NULL, rows, cols, fmt, block, hadamard_k, out);
+}
+
+int fp4o_dequantize_residual(const uint8_t *q, const uint8_t *s_logical, float gscale,
+                             const uint32_t *res, int64_t rows, int64_t cols, int fmt, int block,
+                             int hadamard_k, float *out)
+{
+    if (!res) return -1;
+    return dequantize_rows(q, s_logical, gscale, res, rows, cols, fmt, block, hadamard_k, out);
 }
 
 /* ------------------------------------------------------------------------ */

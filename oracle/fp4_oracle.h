@@ -62,6 +62,22 @@ int fp4o_quantize_f32(const float *x, int64_t rows, int64_t cols, int64_t ld,
                       int gscale_given, float *gscale,
                       uint8_t *q, uint8_t *s_logical);
 
+/* Quantization with the sparse residual lane ([TransFP4] §2.3 Eq.(3),
+ * r = 1 per 32 values): res receives rows x cols/32 words (bf16 bits |
+ * index << 16) of the largest-magnitude rotated value of every 32-value
+ * unit, which is zeroed before the FP4 quantization (and before the NVFP4
+ * tensor maximum).  Absmax block scales. */
+int fp4o_quantize_residual(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                           int fmt, int block, int hadamard_k, int tie, int mx_rule,
+                           int gscale_given, float *gscale, uint8_t *q, uint8_t *s_logical,
+                           uint32_t *res);
+
+/* Dequantization of the FP4 stream plus the residual lane, then the inverse
+ * rotation. */
+int fp4o_dequantize_residual(const uint8_t *q, const uint8_t *s_logical, float gscale,
+                             const uint32_t *res, int64_t rows, int64_t cols, int fmt, int block,
+                             int hadamard_k, float *out);
+
 /* out: rows x cols fp32.  hadamard_k > 0 applies the (self-inverse)
  * rotation again to return to the original domain. */
 int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
