@@ -126,6 +126,17 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int):
             ms = time_graph(torch, call_mse, 3, reps * 8)
             gbs = n * bpe / (ms * 1e-3) / 1e9
             res["cases"][f"{name}_mse_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
+        # the sparse residual lane (TransFP4 Eq.(3)): 4 more bytes per 32 elements
+        for k in (0, 32):
+            it = [0]
+
+            def call_res():
+                fp4.quantize_residual(copies[it[0] % 8], fmt, hadamard_k=k)
+                it[0] += 1
+
+            ms = time_graph(torch, call_res, 3, reps * 8)
+            gbs = n * (bpe + 4 / 32) / (ms * 1e-3) / 1e9
+            res["cases"][f"{name}_residual_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
     del copies, xd
     torch.cuda.empty_cache()
     return res

@@ -158,6 +158,47 @@ def gemm_quantized(a, w, M: int, N: int, K: int, fmt, out_fmt, gscale=None, roun
     return Cq, Cs, gC
 
 
+def quantize_residual(x, fmt, hadamard_k: int = 0, round: int = FP4_ROUND_EVEN,
+                      mx_scale_rule: int = FP4_MX_SCALE_CEIL, gscale=None):
+    """:func:`quantize` with the sparse residual lane (TransFP4 Eq.(3), one
+    value per 32): returns (q, s, g, res), res (rows, cols/32) int32 words =
+    bf16 bits | index << 16."""
+    import torch
+
+    fmt = _fmt(fmt)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 CUDA tensor, contiguous along its last axis")
+    rows, cols = x.shape
+    _, sb = quantize_sizes(rows, cols, fmt)
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    s = torch.empty((sb,), dtype=torch.uint8, device=x.device)
+    g = torch.ones((1,), dtype=torch.float32, device=x.device)
+    res = torch.empty((rows, cols // 32), dtype=torch.int32, device=x.device)
+    given = gscale is not None
+    if given:
+        g.copy_(gscale.reshape(1).to(torch.float32))
+    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(given), 0, 0)
+    _lib.check("fp4_quantize_residual", _lib.lib().fp4_quantize_residual(
+        x.data_ptr(), rows, cols, x.stride(0), fmt, block_of(fmt), int(hadamard_k), ctypes.byref(opts),
+        q.data_ptr(), s.data_ptr(), g.data_ptr() if fmt == FP4_NVFP4 else None, res.data_ptr(),
+        _stream_handle(torch, x.device)))
+    return q, s, g, res
+
+
+def dequantize_residual(q, s, g, res, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_F32):
+    """Inverse of :func:`quantize_residual`."""
+    import torch
+
+    fmt = _fmt(fmt)
+    rows, cols = q.shape[0], q.shape[1] * 2
+    out = torch.empty((rows, cols), dtype=torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16,
+                      device=q.device)
+    _lib.check("fp4_dequantize_residual", _lib.lib().fp4_dequantize_residual(
+        q.data_ptr(), s.data_ptr(), g.data_ptr() if fmt == FP4_NVFP4 else None, res.data_ptr(), rows, cols, fmt,
+        block_of(fmt), int(hadamard_k), int(out_dtype), out.data_ptr(), _stream_handle(torch, q.device)))
+    return out
+
+
 def mx_to_nv(w):
     """An MXFP4 tensor w = (q, s, g) in the NVFP4 scale form (q, s_nv, s_g)
     with the same dequantized elements (see fp4_mx_to_nv_scales); q is shared."""

@@ -11,10 +11,11 @@
 namespace fp4 {
 cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
                             int hk, float ck, int round_away, int mx_floor, int mse, int gscale_given,
-                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl);
+                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl,
+                            uint32_t *res);
 cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
                               int64_t cols, int fmt, int hk, float ck, int bf16out, void *out,
-                              int sms, cudaStream_t st);
+                              int sms, cudaStream_t st, const uint32_t *res);
 cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const uint8_t *Wq,
                         const uint8_t *Ws, const float *gW, int64_t M, int64_t N, int64_t K,
                         int fmt, int bf16out, void *C, int64_t ldc, void *ws, size_t ws_bytes,
@@ -91,9 +92,9 @@ fp4_status fp4_quantize_sizes(int64_t rows, int64_t cols, int fmt, int block, si
     return FP4_OK;
 }
 
-fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int fmt, int block,
-                        int hadamard_k, const fp4_opts *opts, uint8_t *q, uint8_t *s, float *gscale,
-                        void *stream)
+static fp4_status quantize_impl(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int fmt, int block,
+                                int hadamard_k, const fp4_opts *opts, uint8_t *q, uint8_t *s, float *gscale,
+                                uint32_t *res, bool with_res, void *stream)
 {
     fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
     if (opts) o = *opts;
@@ -102,26 +103,41 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR)
         return FP4_ERR_INVALID_ARG;
     if (o.scale_search != FP4_SCALE_ABSMAX && o.scale_search != FP4_SCALE_MSE) return FP4_ERR_INVALID_ARG;
+    if (with_res && o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;
     if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
     const bool empty = rows == 0 || cols == 0;
     if (fmt == FP4_NVFP4 && !gscale) return FP4_ERR_INVALID_ARG;
-    if (!empty && (!x || !q || !s)) return FP4_ERR_INVALID_ARG;
+    if (!empty && (!x || !q || !s || (with_res && !res))) return FP4_ERR_INVALID_ARG;
     if (!aligned(x, 16) || (ld_x % 8) || !aligned(q, 16) || !aligned(s, 16)) return FP4_ERR_ALIGNMENT;
-    if (gscale && !aligned(gscale, 4)) return FP4_ERR_ALIGNMENT;
+    if ((gscale && !aligned(gscale, 4)) || (res && !aligned(res, 4))) return FP4_ERR_ALIGNMENT;
     if (empty && fmt == FP4_MXFP4) return FP4_OK;
     cudaError_t e = fp4::launch_quantize(static_cast<const uint16_t *>(x), rows, cols, ld_x, fmt,
                                          hadamard_k, hadamard_constant(hadamard_k),
                                          o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
                                          o.scale_search == FP4_SCALE_MSE, o.gscale_given, q, s, gscale, sm_count(),
-                                         static_cast<cudaStream_t>(stream), true);
+                                         static_cast<cudaStream_t>(stream), true, with_res ? res : nullptr);
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
-fp4_status fp4_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
-                          int64_t cols, int fmt, int block, int hadamard_k, int out_dtype, void *out,
-                          void *stream)
+fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int fmt, int block,
+                        int hadamard_k, const fp4_opts *opts, uint8_t *q, uint8_t *s, float *gscale,
+                        void *stream)
+{
+    return quantize_impl(x, rows, cols, ld_x, fmt, block, hadamard_k, opts, q, s, gscale, nullptr, false, stream);
+}
+
+fp4_status fp4_quantize_residual(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int fmt, int block,
+                                 int hadamard_k, const fp4_opts *opts, uint8_t *q, uint8_t *s, float *gscale,
+                                 uint32_t *res, void *stream)
+{
+    return quantize_impl(x, rows, cols, ld_x, fmt, block, hadamard_k, opts, q, s, gscale, res, true, stream);
+}
+
+static fp4_status dequantize_impl(const uint8_t *q, const uint8_t *s, const float *gscale, const uint32_t *res,
+                                  bool with_res, int64_t rows, int64_t cols, int fmt, int block, int hadamard_k,
+                                  int out_dtype, void *out, void *stream)
 {
     if (rows < 0 || cols < 0) return FP4_ERR_INVALID_ARG;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
@@ -129,12 +145,29 @@ fp4_status fp4_dequantize(const uint8_t *q, const uint8_t *s, const float *gscal
     if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
     if (rows == 0 || cols == 0) return FP4_OK;
-    if (!q || !s || !out || (fmt == FP4_NVFP4 && !gscale)) return FP4_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(s, 16) || !aligned(out, 16)) return FP4_ERR_ALIGNMENT;
+    if (!q || !s || !out || (fmt == FP4_NVFP4 && !gscale) || (with_res && !res)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(s, 16) || !aligned(out, 16) || (res && !aligned(res, 4)))
+        return FP4_ERR_ALIGNMENT;
     cudaError_t e = fp4::launch_dequantize(q, s, gscale, rows, cols, fmt, hadamard_k,
                                            hadamard_constant(hadamard_k), out_dtype == FP4_OUT_BF16,
-                                           out, sm_count(), static_cast<cudaStream_t>(stream));
+                                           out, sm_count(), static_cast<cudaStream_t>(stream),
+                                           with_res ? res : nullptr);
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status fp4_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
+                          int64_t cols, int fmt, int block, int hadamard_k, int out_dtype, void *out,
+                          void *stream)
+{
+    return dequantize_impl(q, s, gscale, nullptr, false, rows, cols, fmt, block, hadamard_k, out_dtype, out,
+                           stream);
+}
+
+fp4_status fp4_dequantize_residual(const uint8_t *q, const uint8_t *s, const float *gscale, const uint32_t *res,
+                                   int64_t rows, int64_t cols, int fmt, int block, int hadamard_k, int out_dtype,
+                                   void *out, void *stream)
+{
+    return dequantize_impl(q, s, gscale, res, true, rows, cols, fmt, block, hadamard_k, out_dtype, out, stream);
 }
 
 fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes)
@@ -247,7 +280,8 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     } else {
         e = fp4::launch_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
                                  hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
-                                 o.mx_scale_rule == FP4_MX_SCALE_FLOOR, 0, gA != nullptr, aq, as, ga, sms, st, true);
+                                 o.mx_scale_rule == FP4_MX_SCALE_FLOOR, 0, gA != nullptr, aq, as, ga, sms, st, true,
+                                 nullptr);
     }
     if (e != cudaSuccess) return FP4_ERR_CUDA;
     int bad = 0;

@@ -39,7 +39,35 @@ struct QuantArgs {
     int round_away;         // E2M1 ties to the larger magnitude
     int mx_floor;           // MX scale: floor rule
     int gscale_computed;    // NVFP4: *gscale was set by the amax pass (see amax_kernel)
+    uint32_t *res;          // sparse residual lane (one word per unit), or null
 };
+
+// Sparse residual lane ("Portable FP4 quantization (TransFP4)" §2.3 Eq.(3),
+// one value per 32): the value of largest magnitude in the rotated unit v
+// (the first of equal ones) leaves the FP4 stream: it is zeroed in v and
+// returned as a word holding its bf16 rounding (RNE) and its index << 16.
+FP4_DEV uint32_t extract_residual(float *v)
+{
+    int best = 0;
+    float bm = fabsf(v[0]);
+#pragma unroll
+    for (int i = 1; i < 32; i++) {
+        const float m = fabsf(v[i]);
+        if (m > bm) {
+            bm = m;
+            best = i;
+        }
+    }
+    float top = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        if (i == best) {
+            top = v[i];
+            v[i] = 0.0f;
+        }
+    }
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(top)) | ((uint32_t)best << 16);
+}
 
 // Units processed per thread and loop trip: their loads are all issued
 // before any is consumed, so each thread keeps UNITS x 64 bytes in flight.
@@ -126,7 +154,7 @@ FP4_DEV void encode_store_unit(float *v, int64_t u, uint32_t row, uint32_t j, co
 // into *gscale with an integer atomicMax (the bits of a non-negative float
 // order like the float; *gscale must be 0 on entry).  The result is s_g =
 // RN(amax / (6 * 448)) itself, or 0 for an all-zero tensor.
-template <int HK>
+template <int HK, bool RES>
 __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
 {
     grid_dep_launch();
@@ -155,6 +183,7 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
             float v[32];
             unpack_unit(raw[i], v);
             if (HK) fwht_unit<HK>(v, a.ck, lane);
+            if (RES) extract_residual(v);  // the tensor scale of the FP4 stream
             m = fmaxf(m, absmax_tree<32>(v));
         }
     }
@@ -181,7 +210,7 @@ __global__ void zero_word_kernel(float *g)
 }
 
 // ---------------------------------------------------------------------------
-template <int FMT, int HK, bool MSE>
+template <int FMT, int HK, bool MSE, bool RES = false>
 FP4_DEV void quantize_body(const QuantArgs &a)
 {
     grid_dep_launch();
@@ -228,6 +257,7 @@ FP4_DEV void quantize_body(const QuantArgs &a)
             unpack_unit(raw[i], v);
             if (HK) fwht_unit<HK>(v, a.ck, lane);
             if (!live) continue;
+            if (RES) a.res[u] = extract_residual(v);
 
             encode_store_unit<FMT, MSE>(v, u, row[i], col[i], a, sg, six_sg, FMT == FP4_NVFP4 ? &tab : nullptr);
         }
@@ -238,6 +268,13 @@ template <int FMT, int HK>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantArgs a)
 {
     quantize_body<FMT, HK, false>(a);
+}
+
+// With the sparse residual lane.
+template <int FMT, int HK>
+__global__ void __launch_bounds__(256) quantize_res_kernel(QuantArgs a)
+{
+    quantize_body<FMT, HK, false, true>(a);
 }
 
 // The MSE scale search: arithmetic-bound, so sized for three CTAs per SM.
@@ -425,9 +462,10 @@ struct DequantArgs {
     int64_t cols;
     void *out;
     float ck;
+    const uint32_t *res;    // sparse residual lane, or null
 };
 
-template <int FMT, int HK, int BF16OUT>
+template <int FMT, int HK, int BF16OUT, bool RES = false>
 __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
 {
     grid_dep_launch();
@@ -441,13 +479,15 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
 
     for (int64_t base = warp * 32 * DUNITS; base < a.total_units; base += nwarps * 32 * DUNITS) {
         uint4 raw[DUNITS];
-        uint32_t sraw[DUNITS];
+        uint32_t sraw[DUNITS], rres[DUNITS];
 #pragma unroll
         for (int i = 0; i < DUNITS; i++) {
             const int64_t u = base + i * 32 + lane;
             raw[i] = make_uint4(0, 0, 0, 0);
             sraw[i] = 0;
+            rres[i] = 0;
             if (u < a.total_units) {
+                if (RES) rres[i] = __ldg(a.res + u);
                 uint32_t row, j;
                 unit_rc(u, a.upr_div, row, j);
                 raw[i] = __ldg(reinterpret_cast<const uint4 *>(a.q + u * 16));
@@ -483,6 +523,14 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
                         v[8 * c + 2 * b] = __fmul_rn(d, lo);
                         v[8 * c + 2 * b + 1] = __fmul_rn(d, hi);
                     }
+                }
+                if (RES) {
+                    // TransFP4 Eq.(3): the FP4 stream plus the residual lane
+                    const int idx = (int)((rres[i] >> 16) & 31u);
+                    const float r = __uint_as_float((rres[i] & 0xFFFFu) << 16);
+#pragma unroll
+                    for (int e = 0; e < 32; e++)
+                        if (e == idx) v[e] = __fadd_rn(v[e], r);
                 }
             } else {
 #pragma unroll
@@ -551,14 +599,28 @@ static void (*quant_kernel_for(int hk))(QuantArgs)
     return nullptr;
 }
 
+template <int FMT>
+static void (*quant_res_kernel_for(int hk))(QuantArgs)
+{
+    switch (hk) {
+    case 0: return quantize_res_kernel<FMT, 0>;
+    case 16: return quantize_res_kernel<FMT, 16>;
+    case 32: return quantize_res_kernel<FMT, 32>;
+    case 64: return quantize_res_kernel<FMT, 64>;
+    case 128: return quantize_res_kernel<FMT, 128>;
+    }
+    return nullptr;
+}
+
+template <bool RES>
 static void (*amax_kernel_for(int hk))(QuantArgs)
 {
     switch (hk) {
-    case 0: return amax_kernel<0>;
-    case 16: return amax_kernel<16>;
-    case 32: return amax_kernel<32>;
-    case 64: return amax_kernel<64>;
-    case 128: return amax_kernel<128>;
+    case 0: return amax_kernel<0, RES>;
+    case 16: return amax_kernel<16, RES>;
+    case 32: return amax_kernel<32, RES>;
+    case 64: return amax_kernel<64, RES>;
+    case 128: return amax_kernel<128, RES>;
     }
     return nullptr;
 }
@@ -566,7 +628,7 @@ static void (*amax_kernel_for(int hk))(QuantArgs)
 // Quantize launch sequence (see the note on `pdl` below).
 cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int fmt,
                             int hk, float ck, int round_away, int mx_floor, int mse, int gscale_given,
-                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl)
+                            uint8_t *q, uint8_t *s, float *gscale, int sms, cudaStream_t st, bool pdl, uint32_t *res)
 {
     QuantArgs a;
     a.x = x;
@@ -585,12 +647,15 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     a.round_away = round_away;
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
+    a.res = res;
     const int grid = grid_for(a.total_units, sms, QUNITS);
-    void (*qk)(QuantArgs) = (fmt == FP4_MXFP4) ? (mse ? quant_kernel_for<FP4_MXFP4, true>(hk)
+    void (*qk)(QuantArgs) = res ? ((fmt == FP4_MXFP4) ? quant_res_kernel_for<FP4_MXFP4>(hk)
+                                                      : quant_res_kernel_for<FP4_NVFP4>(hk))
+                          : (fmt == FP4_MXFP4) ? (mse ? quant_kernel_for<FP4_MXFP4, true>(hk)
                                                       : quant_kernel_for<FP4_MXFP4, false>(hk))
                                                : (mse ? quant_kernel_for<FP4_NVFP4, true>(hk)
                                                       : quant_kernel_for<FP4_NVFP4, false>(hk));
-    void (*ak)(QuantArgs) = amax_kernel_for(hk);
+    void (*ak)(QuantArgs) = res ? amax_kernel_for<true>(hk) : amax_kernel_for<false>(hk);
     if (!qk || !ak) return cudaErrorInvalidValue;
     cudaError_t err = cudaSuccess;
     // With `pdl` every launch, the first included, may start while its
@@ -689,6 +754,7 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     a.round_away = round_away;
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
+    a.res = nullptr;
     void (*k)(QuantArgs, unsigned *, int, int) = (fmt == FP4_MXFP4) ? act_kernel_for<FP4_MXFP4>(hk) : act_kernel_for<FP4_NVFP4>(hk);
     if (!k) return cudaErrorInvalidValue;
     const bool cluster = a.gscale_computed != 0;
@@ -712,15 +778,15 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     return cudaLaunchKernelEx(&cfg, k, a, zero, nzero, early);
 }
 
-template <int FMT, int BF>
+template <int FMT, int BF, bool RES>
 static void (*deq_kernel_for(int hk))(DequantArgs)
 {
     switch (hk) {
-    case 0: return dequantize_kernel<FMT, 0, BF>;
-    case 16: return dequantize_kernel<FMT, 16, BF>;
-    case 32: return dequantize_kernel<FMT, 32, BF>;
-    case 64: return dequantize_kernel<FMT, 64, BF>;
-    case 128: return dequantize_kernel<FMT, 128, BF>;
+    case 0: return dequantize_kernel<FMT, 0, BF, RES>;
+    case 16: return dequantize_kernel<FMT, 16, BF, RES>;
+    case 32: return dequantize_kernel<FMT, 32, BF, RES>;
+    case 64: return dequantize_kernel<FMT, 64, BF, RES>;
+    case 128: return dequantize_kernel<FMT, 128, BF, RES>;
     }
     return nullptr;
 }
@@ -815,7 +881,7 @@ cudaError_t launch_mx_to_nv_scales(const uint8_t *s_mx, int64_t rows, int64_t co
 
 cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *gscale, int64_t rows,
                               int64_t cols, int fmt, int hk, float ck, int bf16out, void *out,
-                              int sms, cudaStream_t st)
+                              int sms, cudaStream_t st, const uint32_t *res)
 {
     DequantArgs a;
     a.q = q;
@@ -831,11 +897,16 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
     a.cols = cols;
     a.out = out;
     a.ck = ck;
+    a.res = res;
     if (a.total_units == 0) return cudaSuccess;
     const int grid = grid_for(a.total_units, sms, DUNITS);
-    void (*k)(DequantArgs) = (fmt == FP4_MXFP4)
-                                 ? (bf16out ? deq_kernel_for<FP4_MXFP4, 1>(hk) : deq_kernel_for<FP4_MXFP4, 0>(hk))
-                                 : (bf16out ? deq_kernel_for<FP4_NVFP4, 1>(hk) : deq_kernel_for<FP4_NVFP4, 0>(hk));
+    void (*k)(DequantArgs) =
+        res ? ((fmt == FP4_MXFP4)
+                   ? (bf16out ? deq_kernel_for<FP4_MXFP4, 1, true>(hk) : deq_kernel_for<FP4_MXFP4, 0, true>(hk))
+                   : (bf16out ? deq_kernel_for<FP4_NVFP4, 1, true>(hk) : deq_kernel_for<FP4_NVFP4, 0, true>(hk)))
+            : ((fmt == FP4_MXFP4)
+                   ? (bf16out ? deq_kernel_for<FP4_MXFP4, 1, false>(hk) : deq_kernel_for<FP4_MXFP4, 0, false>(hk))
+                   : (bf16out ? deq_kernel_for<FP4_NVFP4, 1, false>(hk) : deq_kernel_for<FP4_NVFP4, 0, false>(hk)));
     if (!k) return cudaErrorInvalidValue;
     // programmatic launch: the kernel waits for its predecessor before touching memory
     return launch_k(k, dim3(grid), dim3(256), 0, st, true, a);

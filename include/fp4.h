@@ -148,6 +148,28 @@ fp4_status fp4_dequantize(const uint8_t *q, const uint8_t *s, const float *gscal
                           int64_t rows, int64_t cols, int fmt, int block,
                           int hadamard_k, int out_dtype, void *out, void *stream);
 
+/*
+ * fp4_quantize_residual — fp4_quantize with the sparse residual lane of
+ * "Portable FP4 quantization (TransFP4)" §2.3 Eq.(3), one value per 32:
+ *   x^ = H^T Q_f(H x - P H x) + H^T P H x,
+ * P selecting, in every 32-value unit of the rotated row H x, the value of
+ * largest magnitude (the first of equal ones).  That value is zeroed before
+ * the FP4 quantization (the NVFP4 tensor scale is that of the FP4 stream) and
+ * kept in `res`: rows x cols/32 uint32 words, row-major, each holding the
+ * value's bf16 bits (round to nearest even) in bits 15:0 and its index in the
+ * unit in bits 20:16.  Other arguments as fp4_quantize; absmax scales only
+ * (FP4_SCALE_MSE: FP4_ERR_UNSUPPORTED).  res 4-byte aligned.
+ */
+fp4_status fp4_quantize_residual(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                                 int fmt, int block, int hadamard_k, const fp4_opts *opts,
+                                 uint8_t *q, uint8_t *s, float *gscale, uint32_t *res, void *stream);
+
+/* fp4_dequantize_residual — the inverse: the FP4 stream dequantized, the
+ * residual value added at its index in fp32, then H^T as in fp4_dequantize. */
+fp4_status fp4_dequantize_residual(const uint8_t *q, const uint8_t *s, const float *gscale,
+                                   const uint32_t *res, int64_t rows, int64_t cols, int fmt,
+                                   int block, int hadamard_k, int out_dtype, void *out, void *stream);
+
 /* Bytes of scratch fp4_gemm needs for this shape (0 when none). Host-only. */
 fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt,
                                    size_t *bytes);

@@ -123,6 +123,16 @@ def test_gemm_quantized_rejects_on_host(L):
     assert g(F, F, F, F, F, F, 256, 256, 256, 0, 0, ctypes.byref(o), None, F, F, None) == 1
 
 
+def test_residual_rejects_on_host(L):
+    F = FAKE
+    o = _lib.Fp4Opts(0, 0, 0, _lib.FP4_SCALE_MSE, 0)
+    assert L.fp4_quantize_residual(F, 4, 64, 64, 0, 32, 0, ctypes.byref(o), F, F, F, F, None) == 2
+    assert L.fp4_quantize_residual(F, 4, 64, 64, 0, 32, 0, None, F, F, F, None, None) == 1  # res
+    assert L.fp4_quantize_residual(F, 4, 64, 64, 0, 32, 0, None, F, F, F, F + 2, None) == 3
+    assert L.fp4_dequantize_residual(F, F, F, None, 4, 64, 0, 32, 0, 0, F, None) == 1
+    assert L.fp4_dequantize_residual(F, F, F, F, 4, 48, 0, 32, 0, 0, F, None) == 2
+
+
 def test_empty_mx_is_noop(L):
     assert L.fp4_quantize(None, 0, 64, 64, 0, 32, 0, None, None, None, None, None) == 0
     assert L.fp4_dequantize(None, None, None, 0, 64, 0, 32, 0, 0, None, None) == 0
