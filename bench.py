@@ -34,7 +34,7 @@ ROWS, COLS = 1024, 131072
 # from the ncu capture summarised in profiles/quantize_kernel_mx_512x131072_full.md
 # (512-row capture scaled by rows).  Set to None whenever that kernel changes,
 # until it is captured again.
-QUANT_MX_TRAFFIC_BYTES = 305.8e6
+QUANT_MX_TRAFFIC_BYTES = 304.1e6
 WORKLOAD = "quantize sweep 1024x131072 bf16 Student-t(3)+1% outliers x20: MXFP4 + NVFP4 quantize and dequantize"
 METRIC = "FP4 quantize GB/s (% HBM peak)"
 
