@@ -409,8 +409,6 @@ constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation sca
 constexpr int MAX_CLUSTER = 8;               // portable cluster size
 
 struct Params {
-    const uint8_t *Ws;   // W scales (N rows)
-    const uint8_t *As;   // activation scales (M rows, padded to 128)
     float *ws;           // partials: [G][maxseg][128][16]
     // Fused reduction (counters != nullptr): per-tile arrival counters, zero
     // on entry; the last CTA to finish a tile sums its partials and stores C.
@@ -426,7 +424,6 @@ struct Params {
     int ntiles;          // ceil(N / 128)
     int G;               // CTAs
     int maxseg;
-    int nkb4;
     int csize;           // > 1: the CTAs of a tile form a cluster of csize and reduce through DSMEM
     // Stream W before waiting for the preceding kernel.  Only when that
     // kernel triggers its dependents after its own wait (the decode
@@ -1044,8 +1041,6 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
             !make_sf_map(&tsw, Ws, nkb4, (N + 127) / 128, KA) || !make_sf_map(&tsa, As, nkb4, 1, KA))
             return cudaErrorInvalidValue;
         decode::Params dp;
-        dp.Ws = Ws;
-        dp.As = As;
         dp.ws = static_cast<float *>(ws);
         dp.N = (int)N;
         dp.M = (int)M;
@@ -1056,7 +1051,6 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.maxseg = pl.maxseg;
         dp.csize = pl.csize;
         dp.w_before_wait = (pdl && w_before_wait) ? 1 : 0;
-        dp.nkb4 = (int)nkb4;
         dp.counters = counters;
         dp.budget_ns = budget;
         dp.stall = stall;
