@@ -24,6 +24,9 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   sparse residual lane    pinned: FP4 stream equals the plain quantizer on the
                           zeroed values, bf16 RNE against torch, one-value
                           units exact, NMSE below the plain quantizer
+  NVFP4 s_g refinement    pinned: least-squares optimality of each step,
+                          error never above the absmax s_g's, closed-form
+                          one-block case (tests/test_oracle_mse_pins.py)
   MSE block-scale search  pinned: hand-derived blocks, exhaustive numpy search
                           over every representable scale, nearest-element
                           property (tests/test_oracle_mse_pins.py)
@@ -102,6 +105,8 @@ def lib():
         L.fp4o_quantize_residual.restype = i32
         L.fp4o_dequantize_residual.argtypes = [vp, vp, f32, vp, i64, i64, i32, i32, i32, vp]
         L.fp4o_dequantize_residual.restype = i32
+        L.fp4o_nv_refine_gscale.argtypes = [vp, i64, i64, i64, i32, i32, i32, vp, vp]
+        L.fp4o_nv_refine_gscale.restype = i32
         L.fp4o_mx_scales_to_nv.restype = i32
         L.fp4o_num_threads.restype = i32
         _lib = L
@@ -254,6 +259,18 @@ def dequantize_residual(q, s_logical, gscale, res, fmt, hadamard_k: int = 0):
                                       block_of(fmt), hadamard_k, _ptr(out)) != 0:
         raise ValueError("oracle dequantize_residual: invalid arguments")
     return out
+
+
+def nv_refine_gscale(x_bf16: np.ndarray, hadamard_k: int = 0, tie: int = TIE_EVEN, rounds: int = 4):
+    """Alternating refinement of the NVFP4 tensor scale: (s_g, its squared
+    error) after `rounds` MSE-group / least-squares-global rounds."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    g = np.zeros(1, np.float32)
+    e = np.zeros(1, np.float64)
+    if lib().fp4o_nv_refine_gscale(_ptr(x), rows, cols, cols, hadamard_k, tie, rounds, _ptr(g), _ptr(e)) != 0:
+        raise ValueError("oracle nv_refine_gscale: invalid arguments")
+    return float(g[0]), float(e[0])
 
 
 def mx_scales_to_nv(s_mx_logical: np.ndarray):

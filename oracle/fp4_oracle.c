@@ -418,6 +418,93 @@ int fp4o_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                          search, gscale_given, gscale, q, s_logical, NULL);
 }
 
+/* Alternating refinement of the NVFP4 tensor scale ([MR-GPTQ] §3.2.1: the
+ * group scales and the tensor scale are optimised in turn for the smallest
+ * sum ||Y^_i - X_i||^2).  Starting from the absmax s_g, each round
+ *   (group step)  quantizes the rotated tensor with the MSE block-scale
+ *                 search under the current s_g;
+ *   (evaluation)  E = sum (x_i - y_i)^2 over the rotated values x_i and
+ *                 their reconstructions y_i = RN(RN(s_g dec(s_b)) dec(q_i));
+ *   (global step) s_g <- RN_fp32(sum x_i u_i / sum u_i^2), u_i = dec(s_b)
+ *                 dec(q_i): the least-squares tensor scale for the codes
+ *                 just chosen (kept when the sum of u_i^2 is 0 or the
+ *                 quotient is not a positive finite float).
+ * After `rounds` evaluations the s_g with the smallest E (the first of equal
+ * ones) is returned, with E.  Sums are fp64 in a fixed order: over the 32
+ * values of a unit in index order, over a row's units in order, then over
+ * the rows in order; products x_i u_i and u_i^2 are exact in fp64. */
+int fp4o_nv_refine_gscale(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                          int hadamard_k, int tie, int rounds, float *gscale, double *err)
+{
+    if (!valid_shape(FP4O_NVFP4, 16, hadamard_k, rows, cols) || ld < cols || rounds < 1) return -1;
+    const int64_t nkb = cols / 16, units = cols / 32;
+    uint8_t *q = (uint8_t *)calloc((size_t)(rows * (cols / 2) + 1), 1);
+    uint8_t *s = (uint8_t *)calloc((size_t)(rows * nkb + 1), 1);
+    float *y = (float *)malloc(sizeof(float) * (size_t)(cols ? cols : 1));
+    double *row_xu = (double *)malloc(sizeof(double) * (size_t)(rows ? rows : 1));
+    double *row_uu = (double *)malloc(sizeof(double) * (size_t)(rows ? rows : 1));
+    double *row_ee = (double *)malloc(sizeof(double) * (size_t)(rows ? rows : 1));
+    float sg = 0.0f;
+    /* the absmax s_g, as fp4o_quantize computes it */
+    quantize_rows(x, NULL, rows, cols, ld, FP4O_NVFP4, 16, hadamard_k, tie, FP4O_MX_CEIL,
+                  FP4O_SCALE_ABSMAX, 0, &sg, q, s, NULL);
+    float best_sg = sg;
+    double best_e = 0.0;
+    for (int t = 0; t < rounds; t++) {
+        float cur = sg;
+        quantize_rows(x, NULL, rows, cols, ld, FP4O_NVFP4, 16, hadamard_k, tie, FP4O_MX_CEIL,
+                      FP4O_SCALE_MSE, 1, &cur, q, s, NULL);
+        for (int64_t r = 0; r < rows; r++) {
+            load_row(x, NULL, ld, r, cols, hadamard_k, y);
+            double rxu = 0.0, ruu = 0.0, ree = 0.0;
+            for (int64_t u = 0; u < units; u++) {
+                double uxu = 0.0, uuu = 0.0, uee = 0.0;
+                for (int i = 0; i < 32; i++) {
+                    int64_t c = u * 32 + i;
+                    int code = (q[r * (cols / 2) + c / 2] >> ((c & 1) ? 4 : 0)) & 0xF;
+                    int sb = s[r * nkb + c / 16];
+                    double ui = fp4o_e4m3_decode(sb) * fp4o_e2m1_decode(code);
+                    float d = sg * (float)fp4o_e4m3_decode(sb);
+                    float yi = d * (float)fp4o_e2m1_decode(code);
+                    double e = (double)y[c] - (double)yi;
+                    uxu = uxu + (double)y[c] * ui;
+                    uuu = uuu + ui * ui;
+                    uee = uee + e * e;
+                }
+                rxu = rxu + uxu;
+                ruu = ruu + uuu;
+                ree = ree + uee;
+            }
+            row_xu[r] = rxu;
+            row_uu[r] = ruu;
+            row_ee[r] = ree;
+        }
+        double sxu = 0.0, suu = 0.0, see = 0.0;
+        for (int64_t r = 0; r < rows; r++) {
+            sxu = sxu + row_xu[r];
+            suu = suu + row_uu[r];
+            see = see + row_ee[r];
+        }
+        if (t == 0 || see < best_e) {
+            best_e = see;
+            best_sg = sg;
+        }
+        if (suu > 0.0) {
+            float nxt = (float)(sxu / suu);
+            if (nxt > 0.0f && nxt <= FLT_MAX) sg = nxt;
+        }
+    }
+    *gscale = best_sg;
+    if (err) *err = best_e;
+    free(q);
+    free(s);
+    free(y);
+    free(row_xu);
+    free(row_uu);
+    free(row_ee);
+    return 0;
+}
+
 int fp4o_quantize_residual(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                            int fmt, int block, int hadamard_k, int tie, int mx_rule,
                            int gscale_given, float *gscale, uint8_t *q, uint8_t *s_logical,

@@ -72,6 +72,12 @@ int fp4o_quantize_residual(const uint16_t *x, int64_t rows, int64_t cols, int64_
                            int gscale_given, float *gscale, uint8_t *q, uint8_t *s_logical,
                            uint32_t *res);
 
+/* Alternating refinement of the NVFP4 tensor scale (MSE group step, least-
+ * squares global step), `rounds` evaluations from the absmax s_g; returns
+ * the best s_g and its fp64 squared error (see the function's comment). */
+int fp4o_nv_refine_gscale(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                          int hadamard_k, int tie, int rounds, float *gscale, double *err);
+
 /* Dequantization of the FP4 stream plus the residual lane, then the inverse
  * rotation. */
 int fp4o_dequantize_residual(const uint8_t *q, const uint8_t *s_logical, float gscale,

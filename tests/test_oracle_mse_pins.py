@@ -252,3 +252,43 @@ def test_with_rotation_lowers_the_tensor_error(orc, fmt, hk):
 def test_invalid_search_rejected(orc):
     with pytest.raises(ValueError):
         orc.quantize(np.zeros((1, 32), np.uint16), 0, search=2)
+
+
+# --------------------------------------------- NVFP4 tensor-scale refinement ----
+def _nv_codes_u(orc, q, s, cols):
+    """u_i = dec(s_b) dec(q_i) for every element (fp64)."""
+    codes = codes_of(q, cols).astype(np.int64)
+    mag = GRID[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    sb = np.repeat(np.vectorize(orc.e4m3_decode)(s.astype(np.int64)), 16, axis=1)
+    return sb * mag
+
+
+@pytest.mark.parametrize("gen", ["table5_weight", "table5_activation"])
+def test_refined_tensor_scale_is_a_least_squares_step(orc, gen):
+    """"FP4 quantization analysis" §3.2.1 alternates group and global scales.
+    One round returns the absmax s_g with the MSE quantization's error; two
+    rounds return the better (by an independent fp64 sum) of that s_g and the
+    least-squares scale of its codes, sum x u / sum u^2; more rounds never
+    return a larger error."""
+    x = inputs.f32_to_bf16_bits(getattr(inputs, gen)(32 * 1024, seed=5).reshape(32, 1024))
+    xf = inputs.bf16_bits_to_f32(x).astype(np.float64)
+    _, _, g0 = orc.quantize(x, orc.NVFP4)
+    g1r, e1 = orc.nv_refine_gscale(x, rounds=1)
+    assert g1r == g0
+    q, s, _ = orc.quantize(x, orc.NVFP4, gscale=g0, search=orc.SCALE_MSE)
+    y = orc.dequantize(q, s, g0, orc.NVFP4).astype(np.float64)
+    assert np.isclose(e1, ((xf - y) ** 2).sum(), rtol=1e-12)
+    u = _nv_codes_u(orc, q, s, 1024)
+    g_ls = float(np.float32((xf * u).sum() / (u * u).sum()))
+    q2, s2, _ = orc.quantize(x, orc.NVFP4, gscale=g_ls, search=orc.SCALE_MSE)
+    e_ls = ((xf - orc.dequantize(q2, s2, g_ls, orc.NVFP4)) ** 2).sum()
+    g2r, e2 = orc.nv_refine_gscale(x, rounds=2)
+    assert g2r == (g_ls if e_ls < e1 else g0)
+    errs = [orc.nv_refine_gscale(x, rounds=r)[1] for r in (1, 2, 3, 4, 6)]
+    assert all(b <= a for a, b in zip(errs, errs[1:]))
+    assert errs[-1] <= e1
+
+
+def test_refined_tensor_scale_all_zero(orc):
+    g, e = orc.nv_refine_gscale(np.zeros((2, 64), np.uint16), rounds=3)
+    assert g == 1.0 and e == 0.0
