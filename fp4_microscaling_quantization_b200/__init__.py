@@ -199,6 +199,31 @@ def dequantize_residual(q, s, g, res, fmt, hadamard_k: int = 0, out_dtype: int =
     return out
 
 
+def nv_refine_gscale(x, hadamard_k: int = 0, rounds: int = 4, round: int = FP4_ROUND_EVEN):
+    """The NVFP4 tensor scale of x refined by alternating MSE group steps and
+    least-squares global steps (see fp4_nv_refine_gscale); returns a
+    1-element fp32 tensor for ``quantize(..., gscale=...,
+    scale_search=FP4_SCALE_MSE)``."""
+    import torch
+
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 CUDA tensor, contiguous along its last axis")
+    rows, cols = x.shape
+    qb, sb = quantize_sizes(rows, cols, FP4_NVFP4)
+    q = torch.empty((max(qb, 16),), dtype=torch.uint8, device=x.device)
+    s = torch.empty((max(sb, 16),), dtype=torch.uint8, device=x.device)
+    nb = ctypes.c_size_t()
+    _lib.check("fp4_nv_refine_gscale_workspace_size",
+               _lib.lib().fp4_nv_refine_gscale_workspace_size(rows, cols, ctypes.byref(nb)))
+    ws = torch.empty((nb.value,), dtype=torch.uint8, device=x.device)
+    g = torch.empty((1,), dtype=torch.float32, device=x.device)
+    opts = _lib.Fp4Opts(int(round), 0, 0, 0, 0)
+    _lib.check("fp4_nv_refine_gscale", _lib.lib().fp4_nv_refine_gscale(
+        x.data_ptr(), rows, cols, x.stride(0), int(hadamard_k), ctypes.byref(opts), int(rounds), q.data_ptr(),
+        s.data_ptr(), ws.data_ptr(), nb.value, g.data_ptr(), _stream_handle(torch, x.device)))
+    return g
+
+
 def mx_to_nv(w):
     """An MXFP4 tensor w = (q, s, g) in the NVFP4 scale form (q, s_nv, s_g)
     with the same dequantized elements (see fp4_mx_to_nv_scales); q is shared."""

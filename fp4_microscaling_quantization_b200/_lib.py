@@ -41,6 +41,8 @@ SIGNATURES = {
     "fp4_mx_to_nv_scales": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "fp4_quantize_residual": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fp4_dequantize_residual": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _int, _int, _vp, _vp]),
+    "fp4_nv_refine_gscale_workspace_size": (_int, [_i64, _i64, _vp]),
+    "fp4_nv_refine_gscale": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _int, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp]),
     "fp4_gemm_quantized": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp,
                                   _vp, _vp]),
     "fp4_check_device_status": (_int, [_vp]),

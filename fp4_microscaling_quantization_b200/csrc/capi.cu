@@ -31,6 +31,10 @@ cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const fl
                                   int sms, cudaStream_t st);
 cudaError_t launch_mx_to_nv_scales(const uint8_t *s_mx, int64_t rows, int64_t cols, uint8_t *s_nv, float *gscale,
                                    int sms, cudaStream_t st);
+size_t nv_refine_workspace_bytes(int64_t rows, int64_t cols);
+cudaError_t launch_nv_refine(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int hk, float ck,
+                             int round_away, int rounds, uint8_t *q, uint8_t *s, void *ws, float *gscale, int sms,
+                             cudaStream_t st);
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -329,6 +333,37 @@ fp4_status fp4_mx_to_nv_scales(const uint8_t *s_mx, int64_t rows, int64_t cols, 
     if (!aligned(gscale, 4)) return FP4_ERR_ALIGNMENT;
     cudaError_t e = fp4::launch_mx_to_nv_scales(s_mx, rows, cols, s_nv, gscale, sm_count(),
                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status fp4_nv_refine_gscale_workspace_size(int64_t rows, int64_t cols, size_t *bytes)
+{
+    if (rows < 0 || cols < 0 || !bytes) return FP4_ERR_INVALID_ARG;
+    if (cols % 32) return FP4_ERR_UNSUPPORTED;
+    *bytes = fp4::nv_refine_workspace_bytes(rows, cols);
+    return FP4_OK;
+}
+
+fp4_status fp4_nv_refine_gscale(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard_k,
+                                const fp4_opts *opts, int rounds, uint8_t *q, uint8_t *s, void *workspace,
+                                size_t ws_bytes, float *gscale, void *stream)
+{
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
+    if (opts) o = *opts;
+    if (rows < 0 || cols < 0 || ld_x < cols || rounds < 1 || rounds > 64) return FP4_ERR_INVALID_ARG;
+    if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
+    if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
+    if (!gscale || !workspace) return FP4_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0 && (!x || !q || !s)) return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || (ld_x % 8) || !aligned(q, 16) || !aligned(s, 16) || !aligned(workspace, 256) ||
+        !aligned(gscale, 4))
+        return FP4_ERR_ALIGNMENT;
+    if (ws_bytes < fp4::nv_refine_workspace_bytes(rows, cols)) return FP4_ERR_INVALID_ARG;
+    cudaError_t e = fp4::launch_nv_refine(static_cast<const uint16_t *>(x), rows, cols, ld_x, hadamard_k,
+                                          hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY, rounds, q, s,
+                                          workspace, gscale, sm_count(), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 

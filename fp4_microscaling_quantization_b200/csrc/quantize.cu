@@ -792,6 +792,192 @@ static void (*deq_kernel_for(int hk))(DequantArgs)
 }
 
 // ---------------------------------------------------------------------------
+// Alternating refinement of the NVFP4 tensor scale ("FP4 quantization
+// analysis: MXFP4 vs NVFP4" §3.2.1: group and global scales optimised in
+// turn).  From the absmax s_g, each round quantizes with the MSE block-scale
+// search under the current s_g, measures E = sum (x_i - y_i)^2 over the
+// rotated values and their reconstructions, and moves s_g to the least-
+// squares scale of the chosen codes, sum x_i u_i / sum u_i^2 with u_i =
+// dec(s_b) dec(q_i); the s_g of the smallest E is kept.  All sums are fp64
+// in a fixed order (a unit's 32 values, a row's units, the rows), so the
+// result does not depend on the launch shape.
+struct RefineState {
+    double best_err;
+    float cur_sg;   // the s_g the current round quantizes with
+    float best_sg;
+};
+
+// Per unit: (sum x u, sum u u, sum e e) of the current round, in value order.
+template <int HK>
+__global__ void __launch_bounds__(256) nv_unit_stats_kernel(QuantArgs a, const RefineState *st, double *stats)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    const float sg = st->cur_sg;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t base = warp * 32; base < a.total_units; base += nwarps * 32) {
+        const int64_t u = base + lane;
+        const bool live = u < a.total_units;
+        uint4 raw[4];
+        uint32_t row = 0, j = 0;
+        if (live) {
+            unit_rc(u, a.upr_div, row, j);
+            fetch_unit(a.x, a.ld, row, j, raw);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; c++) raw[c] = make_uint4(0, 0, 0, 0);
+        }
+        float v[32];
+        unpack_unit(raw, v);
+        if (HK) fwht_unit<HK>(v, a.ck, lane);  // the whole warp takes part
+        if (!live) continue;
+        const uint4 qw = *reinterpret_cast<const uint4 *>(a.q + u * 16);
+        const uint32_t sb2 = *reinterpret_cast<const uint16_t *>(a.s + scale_offset(row, 2 * j, a.nkb4));
+        const uint32_t words[4] = {qw.x, qw.y, qw.z, qw.w};
+        double sxu = 0.0, suu = 0.0, see = 0.0;
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const float dsb = e4m3_to_f32((sb2 >> (8 * h)) & 0xFF);
+            const float d = __fmul_rn(sg, dsb);
+#pragma unroll
+            for (int b = 0; b < 8; b++) {
+                const int i0 = 16 * h + 2 * b;
+                float q0, q1;
+                e2m1x2_to_f32((words[i0 >> 3] >> (4 * (i0 & 7))) & 0xFF, q0, q1);
+                const float qv[2] = {q0, q1};
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                    const double ui = __dmul_rn((double)dsb, (double)qv[e]);
+                    const float yi = __fmul_rn(d, qv[e]);
+                    const double xi = (double)v[i0 + e];
+                    const double er = __dsub_rn(xi, (double)yi);
+                    sxu = __dadd_rn(sxu, __dmul_rn(xi, ui));
+                    suu = __dadd_rn(suu, __dmul_rn(ui, ui));
+                    see = __dadd_rn(see, __dmul_rn(er, er));
+                }
+            }
+        }
+        stats[u * 3 + 0] = sxu;
+        stats[u * 3 + 1] = suu;
+        stats[u * 3 + 2] = see;
+    }
+}
+
+// Per row: the row's unit sums in unit order.
+__global__ void nv_row_stats_kernel(const double *stats, int64_t rows, int64_t upr, double *row_stats)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows; r += (int64_t)gridDim.x * blockDim.x) {
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0;
+        for (int64_t u = 0; u < upr; u++) {
+            const double *p = stats + (r * upr + u) * 3;
+            a0 = __dadd_rn(a0, p[0]);
+            a1 = __dadd_rn(a1, p[1]);
+            a2 = __dadd_rn(a2, p[2]);
+        }
+        row_stats[r * 3 + 0] = a0;
+        row_stats[r * 3 + 1] = a1;
+        row_stats[r * 3 + 2] = a2;
+    }
+}
+
+// One thread: the round's totals in row order, the best s_g so far (also
+// written to `out`), and the next round's s_g.
+__global__ void nv_refine_step_kernel(const double *row_stats, int64_t rows, int round, RefineState *st, float *out)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    double sxu = 0.0, suu = 0.0, see = 0.0;
+    for (int64_t r = 0; r < rows; r++) {
+        sxu = __dadd_rn(sxu, row_stats[r * 3 + 0]);
+        suu = __dadd_rn(suu, row_stats[r * 3 + 1]);
+        see = __dadd_rn(see, row_stats[r * 3 + 2]);
+    }
+    if (round == 0 || see < st->best_err) {
+        st->best_err = see;
+        st->best_sg = st->cur_sg;
+    }
+    if (suu > 0.0) {
+        const float nxt = __double2float_rn(__ddiv_rn(sxu, suu));
+        if (nxt > 0.0f && nxt <= kFltMax) st->cur_sg = nxt;
+    }
+    *out = st->best_sg;
+}
+
+template <int HK>
+static void (*unit_stats_kernel_for_k())(QuantArgs, const RefineState *, double *)
+{
+    return nv_unit_stats_kernel<HK>;
+}
+
+size_t nv_refine_workspace_bytes(int64_t rows, int64_t cols)
+{
+    const int64_t units = rows * (cols / 32);
+    return 256 + (size_t)((units * 3 * 8 + 255) / 256 * 256) + (size_t)((rows * 3 * 8 + 255) / 256 * 256);
+}
+
+cudaError_t launch_nv_refine(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int hk, float ck,
+                             int round_away, int rounds, uint8_t *q, uint8_t *s, void *ws, float *gscale, int sms,
+                             cudaStream_t st)
+{
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    RefineState *state = reinterpret_cast<RefineState *>(base);
+    const int64_t units = rows * (cols / 32);
+    double *ustats = reinterpret_cast<double *>(base + 256);
+    double *rstats = reinterpret_cast<double *>(base + 256 + (units * 3 * 8 + 255) / 256 * 256);
+    // the absmax s_g, computed into state->cur_sg
+    cudaError_t e = launch_quantize(x, rows, cols, ld, FP4_NVFP4, hk, ck, round_away, 0, 0, 0, q, s, &state->cur_sg,
+                                    sms, st, true, nullptr);
+    if (e != cudaSuccess) return e;
+    QuantArgs a;
+    a.x = x;
+    a.ld = ld;
+    a.units_per_row = cols / 32;
+    a.total_units = units;
+    a.upr_div = make_fastdiv((uint32_t)(a.units_per_row > 0 ? a.units_per_row : 1));
+    a.nkb4 = (cols / 16 + 3) / 4;
+    a.q_row_bytes = cols / 2;
+    a.q = q;
+    a.s = s;
+    a.gscale = &state->cur_sg;
+    a.ck = ck;
+    a.round_away = round_away;
+    a.mx_floor = 0;
+    a.gscale_computed = 0;
+    a.res = nullptr;
+    void (*uk)(QuantArgs, const RefineState *, double *) = nullptr;
+    switch (hk) {
+    case 0: uk = unit_stats_kernel_for_k<0>(); break;
+    case 16: uk = unit_stats_kernel_for_k<16>(); break;
+    case 32: uk = unit_stats_kernel_for_k<32>(); break;
+    case 64: uk = unit_stats_kernel_for_k<64>(); break;
+    case 128: uk = unit_stats_kernel_for_k<128>(); break;
+    }
+    if (!uk) return cudaErrorInvalidValue;
+    const int g_units = grid_for(units, sms, 1);
+    const int g_rows = (int)std::min<int64_t>((rows + 127) / 128, (int64_t)sms * 4);
+    for (int r = 0; r < rounds; r++) {
+        if ((e = launch_quantize(x, rows, cols, ld, FP4_NVFP4, hk, ck, round_away, 0, 1, 1, q, s, &state->cur_sg, sms,
+                                 st, true, nullptr)) != cudaSuccess)
+            return e;
+        if ((e = launch_k(uk, dim3(g_units), dim3(256), 0, st, true, a, (const RefineState *)state, ustats)) !=
+            cudaSuccess)
+            return e;
+        if ((e = launch_k(nv_row_stats_kernel, dim3(g_rows > 0 ? g_rows : 1), dim3(128), 0, st, true,
+                          (const double *)ustats, rows, (int64_t)(cols / 32), rstats)) != cudaSuccess)
+            return e;
+        if ((e = launch_k(nv_refine_step_kernel, dim3(1), dim3(32), 0, st, true, (const double *)rstats, rows, r,
+                          state, gscale)) != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
 // MXFP4 -> NVFP4 scale repacking ("Portable FP4 quantization (TransFP4)"
 // §2.5, §3.4: an artifact is bound late to the backend's native format).  The
 // E2M1 elements stay; each 32-block scale 2^e becomes two 16-block E4M3

@@ -230,6 +230,34 @@ fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float 
 
 
 /*
+ * fp4_nv_refine_gscale — the NVFP4 tensor scale s_g refined by alternating
+ * group and global steps ("FP4 quantization analysis: MXFP4 vs NVFP4"
+ * §3.2.1), for an offline (weight) quantization that then runs
+ * fp4_quantize with scale_search = FP4_SCALE_MSE and gscale_given = 1.
+ * From the absmax s_g, each of `rounds` rounds (1..64) quantizes x (with
+ * H_k when hadamard_k > 0) by the MSE block-scale search under the current
+ * s_g, measures E = sum (x_i - y_i)^2 over the rotated values and their
+ * reconstructions, and moves s_g to the least-squares scale of the chosen
+ * codes, sum x_i u_i / sum u_i^2 with u_i = s_b q_i (kept if that is 0 or
+ * not a positive finite float).  *gscale receives the evaluated s_g with the
+ * smallest E (the first of equal ones; rounds = 1 gives the absmax s_g).
+ * Sums are fp64 in a fixed order (a unit's 32 values, a row's units, the
+ * rows), so the result is reproducible.
+ *   x, rows, cols, ld_x, hadamard_k, opts (round)   as fp4_quantize.
+ *   q, s       scratch of fp4_quantize_sizes(rows, cols, FP4_NVFP4, 16)
+ *              bytes; they end holding the last round's quantization.
+ *   workspace  fp4_nv_refine_gscale_workspace_size() bytes, 256-byte
+ *              aligned.
+ *   gscale     output, one device fp32.
+ * About 5 launches per round; meant to run once per weight.
+ */
+fp4_status fp4_nv_refine_gscale_workspace_size(int64_t rows, int64_t cols, size_t *bytes);
+fp4_status fp4_nv_refine_gscale(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                                int hadamard_k, const fp4_opts *opts, int rounds, uint8_t *q,
+                                uint8_t *s, void *workspace, size_t ws_bytes, float *gscale,
+                                void *stream);
+
+/*
  * fp4_mx_to_nv_scales — late binding of an MXFP4 tensor to the NVFP4 scale
  * form ("Portable FP4 quantization (TransFP4)" §2.5, §3.4), so that NVFP4
  * activations can meet MXFP4 weights in the NVFP4 tensor-core product

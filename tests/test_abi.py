@@ -133,6 +133,16 @@ def test_residual_rejects_on_host(L):
     assert L.fp4_dequantize_residual(F, F, F, F, 4, 48, 0, 32, 0, 0, F, None) == 2
 
 
+def test_refine_rejects_on_host(L):
+    F = FAKE
+    g = L.fp4_nv_refine_gscale
+    assert g(F, 4, 64, 64, 0, None, 0, F, F, F, 1 << 20, F, None) == 1       # rounds < 1
+    assert g(F, 4, 64, 64, 0, None, 65, F, F, F, 1 << 20, F, None) == 1      # rounds > 64
+    assert g(F, 4, 48, 64, 0, None, 2, F, F, F, 1 << 20, F, None) == 2       # cols % 32
+    assert g(F, 4, 64, 64, 0, None, 2, F, F, F, 16, F, None) == 1            # workspace too small
+    assert g(F, 4, 64, 64, 0, None, 2, F, F, F + 16, 1 << 20, F, None) == 3  # workspace alignment
+
+
 def test_empty_mx_is_noop(L):
     assert L.fp4_quantize(None, 0, 64, 64, 0, 32, 0, None, None, None, None, None) == 0
     assert L.fp4_dequantize(None, None, None, 0, 64, 0, 32, 0, 0, None, None) == 0

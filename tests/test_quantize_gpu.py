@@ -258,3 +258,28 @@ def test_mse_full_size_quant_sweep(fp4, orc, fmt):
     n_abs = orc.nmse(xf, orc.dequantize(aq, as_, ag, fmt))
     n_mse = orc.nmse(xf, orc.dequantize(oq[:64], os_[:64], og, fmt))
     assert n_mse < n_abs
+
+
+# ------------------------------------------------ NVFP4 tensor-scale refinement ----
+@pytest.mark.parametrize("shape,hk,tie,rounds", [((64, 1024), 0, 0, 1), ((64, 1024), 0, 0, 4), ((37, 3104), 32, 0, 3),
+                                                 ((130, 512), 128, 1, 2), ((8, 4096), 16, 0, 5)])
+def test_nv_refined_tensor_scale_matches_oracle(fp4, orc, shape, hk, tie, rounds):
+    """Alternating MSE-group / least-squares-global refinement ("FP4
+    quantization analysis" §3.2.1): the GPU's s_g equals the oracle's bit for
+    bit (fixed-order fp64 sums on both sides), and so does the MSE
+    quantization under it."""
+    import torch
+    rows, cols = shape
+    x = inputs.f32_to_bf16_bits(inputs.table5_weight(rows * cols, seed=rows + hk).reshape(rows, cols))
+    g = fp4.nv_refine_gscale(to_dev_bf16(x), hadamard_k=hk, rounds=rounds, round=tie)
+    torch.cuda.synchronize()
+    want, _ = orc.nv_refine_gscale(x, hadamard_k=hk, tie=tie, rounds=rounds)
+    assert np.float32(to_np(g)[0]) == np.float32(want)
+    check_quantize(fp4, orc, x, 1, hk=hk, tie=tie, gscale=want, search=1)
+
+
+def test_nv_refined_tensor_scale_all_zero(fp4, orc):
+    import torch
+    g = fp4.nv_refine_gscale(to_dev_bf16(np.zeros((3, 64), np.uint16)), rounds=3)
+    torch.cuda.synchronize()
+    assert to_np(g)[0] == 1.0
