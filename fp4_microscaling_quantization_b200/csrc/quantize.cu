@@ -48,16 +48,13 @@ struct QuantArgs {
 // returned as a word holding its bf16 rounding (RNE) and its index << 16.
 FP4_DEV uint32_t extract_residual(float *v)
 {
-    int best = 0;
-    float bm = fabsf(v[0]);
+    // the maximum by a balanced tree, then the first index that reaches it:
+    // a short dependency chain instead of a 32-step running search
+    const float amax = absmax_tree<32>(v);
+    uint32_t hit = 0;
 #pragma unroll
-    for (int i = 1; i < 32; i++) {
-        const float m = fabsf(v[i]);
-        if (m > bm) {
-            bm = m;
-            best = i;
-        }
-    }
+    for (int i = 0; i < 32; i++) hit |= (fabsf(v[i]) == amax ? 1u : 0u) << i;
+    const int best = __ffs(hit) - 1;
     float top = 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; i++) {
