@@ -10,8 +10,11 @@
 //
 // Prefill (M > 16): a persistent kernel over 128*CG x 256 output tiles, CG = 2
 // (CTA pairs sharing one 2-SM MMA) once A spans more than 128 rows; see
-// pgemm_kernel.  Decode (M <= 16): a weight-streaming split-K kernel with a
-// deterministic reduction; see decode_kernel.
+// pgemm_kernel.  Its epilogue stores FP32, BF16, or C quantized again to
+// MXFP4 / NVFP4 for the next layer (the QuTLASS-style fused epilogue of the
+// same page, §3.3).  Decode (M <= 16): a weight-streaming split-K kernel with
+// four MMA-issuing warps and a deterministic reduction; see decode_kernel.
+// K is any multiple of 32: the last 256-wide K step of a tail reads zeros.
 // Every wait is bounded (%globaltimer); a wait that gives up sets the device
 // error word, the kernel stops issuing work, frees its TMEM and returns
 // without storing.
@@ -380,7 +383,8 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 // Decode kernel (M <= 16): the weight stream dominates, so the roles swap: a
 // 128-row W tile is the MMA's M operand and the (up to 16) activation rows
 // are N = 16.  Work is cut into (W tile, 256-wide K step) units, and each CTA
-// accumulates the units it owns in TMEM (two buffers, alternating per tile).
+// accumulates the units it owns in TMEM (two buffers, alternating per tile;
+// within a buffer one accumulator per issuing warp, added in warp order).
 // Three ways to spread the tiles over the SMs (plan()):
 //   * whole tiles (ntiles <= SMs, no spare SMs for a split): one CTA per
 //     tile, C stored straight from the accumulator;

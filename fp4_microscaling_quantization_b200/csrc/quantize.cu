@@ -15,6 +15,12 @@
 // the last butterfly stages exchange values with shuffles.  Warps walk the
 // tensor in a grid-stride loop of 32 consecutive units, so neighbouring
 // lanes read and write neighbouring memory.
+//
+// Variants of the same loop: the MSE block-scale search (quantize_mse_kernel,
+// §3.2.1 and §3.3 of the same page), the sparse residual lane
+// (quantize_res_kernel, TransFP4 §2.3 Eq.(3)), the decode activation
+// quantizer (act_quant_kernel, one cluster), and the offline helpers: the
+// NVFP4 tensor-scale refinement and the MXFP4 -> NVFP4 scale binding.
 #include <algorithm>
 #include <map>
 #include <mutex>
