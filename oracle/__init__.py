@@ -10,7 +10,8 @@ a time, fp64 for the GEMM reference).  This module only builds that file and
 marshals numpy arrays into it.
 
 Parity status of each function (what pins it, see tests/test_oracle_pins.py):
-  e2m1 encode/decode      pinned: page magnitude set, brute-force argmin
+  e2m1 encode/decode      pinned: page magnitude set, brute-force argmin over
+                          every fp32 value (tests/test_oracle_exhaustive.py)
   e4m3 encode/decode      pinned: page bit patterns, torch float8_e4m3fn cast
   mx scale exponent       pinned: closed form from the exponent bits, worked
                           example, brute force over all 254 E8M0 scales
