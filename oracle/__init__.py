@@ -19,15 +19,17 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   quantize / dequantize   pinned: worked examples, power-of-two invariants,
                           Eq.(2) norm identity
   gemm reference          pinned: numpy fp64 matmul
-  MXFP4 -> NVFP4 scales  pinned: dequantized elements unchanged (exact)
+  MXFP4 -> NVFP4 scales   pinned: dequantized elements unchanged (exact)
                           within 17 binades, E4M3 rounding past them,
                           closed-form s_g (tests/test_oracle_pins.py)
   sparse residual lane    pinned: FP4 stream equals the plain quantizer on the
                           zeroed values, bf16 RNE against torch, one-value
                           units exact, NMSE below the plain quantizer
-  NVFP4 s_g refinement    pinned: least-squares optimality of each step,
-                          error never above the absmax s_g's, closed-form
-                          one-block case (tests/test_oracle_mse_pins.py)
+  NVFP4 s_g refinement    pinned: one round = the absmax s_g with an
+                          independently summed error, the second round's
+                          least-squares step recomputed in numpy, errors
+                          non-increasing, all-zero tensor
+                          (tests/test_oracle_mse_pins.py)
   MSE block-scale search  pinned: hand-derived blocks, exhaustive numpy search
                           over every representable scale, nearest-element
                           property (tests/test_oracle_mse_pins.py)
