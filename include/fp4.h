@@ -330,7 +330,8 @@ fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *As, const f
 uint64_t fp4_kernel_launches(void);
 
 /* Failure-detection test hook.  With stall != 0 the next GEMM launch
- * (fp4_gemm, fp4_linear or fp4_gemm_decode_noalloc) issues no operand loads,
+ * (fp4_gemm, fp4_gemm_quantized, fp4_linear or fp4_gemm_decode_noalloc)
+ * issues no operand loads,
  * so its MMA warp's bounded wait gives up after budget_ns nanoseconds
  * (0 = the default of 2 s): the kernel sets the device error word, stores
  * nothing, frees its tensor memory and returns, and fp4_check_device_status()
