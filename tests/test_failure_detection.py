@@ -52,3 +52,30 @@ def test_bounded_wait_reports_timeout_and_recovers(fp4, M, N, K):
     torch.cuda.synchronize()
     fp4.check_device_status()  # cleared, and the new call is clean
     assert torch.equal(again, ref)
+
+
+@pytest.mark.parametrize("M,out_fmt", [(128, 0), (256, 1)])
+def test_quantizing_epilogue_times_out_and_recovers(fp4, M, out_fmt):
+    """The same for the GEMM whose epilogue quantizes C (fp4_gemm_quantized)."""
+    import torch
+    from fp4_microscaling_quantization_b200 import _lib
+    N, K = 256, 512
+    rng = np.random.default_rng(M + 7)
+    a = inputs.f32_to_bf16_bits(rng.laplace(0, 1, (M, K)).astype(np.float32))
+    w = inputs.f32_to_bf16_bits(rng.laplace(0, 0.02, (N, K)).astype(np.float32))
+    A = fp4.quantize(to_dev_bf16(a), 0)
+    W = fp4.quantize(to_dev_bf16(w), 0)
+    gC = torch.tensor([0.01], dtype=torch.float32, device="cuda")
+    ref = fp4.gemm_quantized(A, W, M, N, K, 0, out_fmt, gscale=gC if out_fmt else None)
+    torch.cuda.synchronize()
+    fp4.check_device_status()
+    assert _lib.lib().fp4_test_inject_stall(1, 50_000_000) == 0
+    fp4.gemm_quantized(A, W, M, N, K, 0, out_fmt, gscale=gC if out_fmt else None)
+    torch.cuda.synchronize()
+    with pytest.raises(fp4.Fp4Error) as ei:
+        fp4.check_device_status()
+    assert ei.value.code == 5
+    again = fp4.gemm_quantized(A, W, M, N, K, 0, out_fmt, gscale=gC if out_fmt else None)
+    torch.cuda.synchronize()
+    fp4.check_device_status()
+    assert torch.equal(again[0], ref[0]) and torch.equal(again[1], ref[1])
