@@ -166,18 +166,16 @@ FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, i
 // its absmax scale and keeps the one whose reconstruction has the smallest
 // squared error; of equal ones the first tried.
 
-// The E2M1 grid value nearest to s (magnitude saturating at 6, sign of s),
-// ties as the encoder breaks them: the value the hardware conversion's code
-// decodes to, computed in fp32 without a conversion.  The grid step is 1/2
-// below 2, 1 up to 4 and 2 from 4 to 6.  Adding and then subtracting
-// M = 1.5 * 2^22, 2^23 or 2^24 rounds |s| to a multiple of that step, ties to
-// even (a + M lies in the binade whose ulp is the step; the subtraction is
-// exact); the even multiple is the even code in every step.  Magnitudes past
-// 6 saturate.  Ties away: a value exactly half a step above its even
-// rounding goes up one step.
-FP4_DEV float e2m1_grid_value(float s, int round_away)
+// The E2M1 grid value nearest to a >= 0 (saturating at 6), ties as the
+// encoder breaks them: the magnitude the hardware conversion's code decodes
+// to, computed in fp32 without a conversion.  The grid step is 1/2 below 2,
+// 1 up to 4 and 2 from 4 to 6.  Adding and then subtracting M = 1.5 * 2^22,
+// 2^23 or 2^24 rounds a to a multiple of that step, ties to even (a + M lies
+// in the binade whose ulp is the step; the subtraction is exact); the even
+// multiple is the even code in every step.  Magnitudes past 6 saturate.
+// Ties away: a value exactly half a step above its even rounding goes up.
+FP4_DEV float e2m1_grid_magnitude(float a, int round_away)
 {
-    const float a = fabsf(s);
     const bool lo = a < 2.0f, mid = a < 4.0f;
     const float m = lo ? 6291456.0f : (mid ? 12582912.0f : 25165824.0f);
     float r = __fsub_rn(__fadd_rn(a, m), m);
@@ -185,24 +183,27 @@ FP4_DEV float e2m1_grid_value(float s, int round_away)
         const float h = lo ? 0.25f : (mid ? 0.5f : 1.0f);
         if (__fsub_rn(a, r) == h) r = __fadd_rn(r, __fadd_rn(h, h));
     }
-    return copysignf(fminf(r, 6.0f), s);
+    return fminf(r, 6.0f);
 }
 
 // Squared reconstruction error of N values x under the block scale with
 // decode factor d and encode factor r (x_i * r is what the encoder rounds):
 // y_i = RN(q_i * d), e_i = RN(x_i - y_i), each e_i^2 rounded, then summed
 // as a fixed pairwise tree: adjacent pairs first, then the first half of
-// the partial sums plus the second half until one value remains.
+// the partial sums plus the second half until one value remains.  Computed
+// on magnitudes: y_i has the sign of x_i (r, d > 0) and rounding is
+// symmetric, so RN(|x_i| - |y_i|) is e_i up to its sign and squares alike.
 template <int N>
 FP4_DEV float block_sq_error(const float *x, float r, float d, int round_away)
 {
     float t[N / 2];
 #pragma unroll
     for (int i = 0; i < N / 2; i++) {
-        const float y0 = __fmul_rn(e2m1_grid_value(__fmul_rn(x[2 * i], r), round_away), d);
-        const float y1 = __fmul_rn(e2m1_grid_value(__fmul_rn(x[2 * i + 1], r), round_away), d);
-        const float e0 = __fsub_rn(x[2 * i], y0);
-        const float e1 = __fsub_rn(x[2 * i + 1], y1);
+        const float a0 = fabsf(x[2 * i]), a1 = fabsf(x[2 * i + 1]);
+        const float y0 = __fmul_rn(e2m1_grid_magnitude(__fmul_rn(a0, r), round_away), d);
+        const float y1 = __fmul_rn(e2m1_grid_magnitude(__fmul_rn(a1, r), round_away), d);
+        const float e0 = __fsub_rn(a0, y0);
+        const float e1 = __fsub_rn(a1, y1);
         t[i] = __fadd_rn(__fmul_rn(e0, e0), __fmul_rn(e1, e1));
     }
 #pragma unroll
