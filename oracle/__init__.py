@@ -33,6 +33,13 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
   MSE block-scale search  pinned: hand-derived blocks, exhaustive numpy search
                           over every representable scale, nearest-element
                           property (tests/test_oracle_mse_pins.py)
+  MXFP4 on 16-element     pinned: scale bytes by a brute-force search over the
+  blocks (MXFP4_16)       E8M0 scales per 16-block, elements by brute-force
+                          nearest grid point, every element's error at most
+                          the 32-block MXFP4 error (the finer grid contains the
+                          coarse one below the block max), equal to MXFP4
+                          where a unit's halves share its exponent
+                          (tests/test_oracle_mx16_pins.py)
   NMSE vs the page's table   directional only (the page's generator is unknown)
 """
 from __future__ import annotations
@@ -48,6 +55,9 @@ _SRC = os.path.join(_HERE, "fp4_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 MXFP4, NVFP4 = 0, 1
+# MXFP4 elements and E8M0 scales on 16-element blocks (the C oracle's MXFP4
+# with block 16); the tag matches the CUDA library's format code.
+MXFP4_16 = 2
 TIE_EVEN, TIE_AWAY = 0, 1
 MX_CEIL, MX_FLOOR = 0, 1
 SCALE_ABSMAX, SCALE_MSE = 0, 1
@@ -125,6 +135,11 @@ def block_of(fmt: int) -> int:
     return 32 if fmt == MXFP4 else 16
 
 
+def _cfmt(fmt: int) -> int:
+    """The C oracle's format code: MXFP4_16 is MXFP4 with block 16."""
+    return MXFP4 if fmt == MXFP4_16 else fmt
+
+
 # ---- scalar codecs --------------------------------------------------------
 def e2m1_encode(v: float, tie: int = TIE_EVEN) -> int:
     return lib().fp4o_e2m1_encode(float(v), tie)
@@ -180,7 +195,7 @@ def quantize(x_bf16: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_E
     q = np.zeros((rows, cols // 2), np.uint8)
     s = np.zeros((rows, cols // block), np.uint8)
     g = np.array([gscale if gscale is not None else 0.0], np.float32)
-    rc = lib().fp4o_quantize(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie,
+    rc = lib().fp4o_quantize(_ptr(x), rows, cols, cols, _cfmt(fmt), block, hadamard_k, tie,
                              mx_rule, search, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
     if rc != 0:
         raise ValueError("oracle quantize: invalid arguments")
@@ -196,7 +211,7 @@ def quantize_f32(x: np.ndarray, fmt: int, hadamard_k: int = 0, tie: int = TIE_EV
     q = np.zeros((rows, cols // 2), np.uint8)
     s = np.zeros((rows, cols // block), np.uint8)
     g = np.array([gscale if gscale is not None else 0.0], np.float32)
-    rc = lib().fp4o_quantize_f32(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie,
+    rc = lib().fp4o_quantize_f32(_ptr(x), rows, cols, cols, _cfmt(fmt), block, hadamard_k, tie,
                                  mx_rule, search, int(gscale is not None), _ptr(g), _ptr(q), _ptr(s))
     if rc != 0:
         raise ValueError("oracle quantize: invalid arguments")
@@ -210,7 +225,7 @@ def dequantize(q: np.ndarray, s_logical: np.ndarray, gscale: float, fmt: int,
     rows, half = q.shape
     cols = half * 2
     out = np.zeros((rows, cols), np.float32)
-    rc = lib().fp4o_dequantize(_ptr(q), _ptr(s), float(gscale), rows, cols, fmt,
+    rc = lib().fp4o_dequantize(_ptr(q), _ptr(s), float(gscale), rows, cols, _cfmt(fmt),
                                block_of(fmt), hadamard_k, _ptr(out))
     if rc != 0:
         raise ValueError("oracle dequantize: invalid arguments")
@@ -244,7 +259,7 @@ def quantize_residual(x_bf16: np.ndarray, fmt: int, hadamard_k: int = 0, tie: in
     s = np.zeros((rows, cols // block), np.uint8)
     res = np.zeros((rows, cols // 32), np.uint32)
     g = np.array([gscale if gscale is not None else 0.0], np.float32)
-    rc = lib().fp4o_quantize_residual(_ptr(x), rows, cols, cols, fmt, block, hadamard_k, tie, mx_rule,
+    rc = lib().fp4o_quantize_residual(_ptr(x), rows, cols, cols, _cfmt(fmt), block, hadamard_k, tie, mx_rule,
                                       int(gscale is not None), _ptr(g), _ptr(q), _ptr(s), _ptr(res))
     if rc != 0:
         raise ValueError("oracle quantize_residual: invalid arguments")
@@ -258,7 +273,7 @@ def dequantize_residual(q, s_logical, gscale, res, fmt, hadamard_k: int = 0):
     rows, half = q.shape
     cols = half * 2
     out = np.zeros((rows, cols), np.float32)
-    if lib().fp4o_dequantize_residual(_ptr(q), _ptr(s), float(gscale), _ptr(r), rows, cols, fmt,
+    if lib().fp4o_dequantize_residual(_ptr(q), _ptr(s), float(gscale), _ptr(r), rows, cols, _cfmt(fmt),
                                       block_of(fmt), hadamard_k, _ptr(out)) != 0:
         raise ValueError("oracle dequantize_residual: invalid arguments")
     return out

@@ -189,7 +189,11 @@ static float bf16_to_f32(uint16_t b)
 static int valid_shape(int fmt, int block, int hk, int64_t rows, int64_t cols)
 {
     if (rows < 0 || cols < 0) return 0;
-    if (fmt == FP4O_MXFP4 && block != 32) return 0;
+    /* MXFP4 also on 16-element blocks: the microscaling form of [TransFP4]
+     * §1.1 leaves the block size G open, and E8M0 scales on 16-element blocks
+     * separate the block-size effect from the scale-precision effect that
+     * tell MXFP4 and NVFP4 apart ([Guide] §3.3). */
+    if (fmt == FP4O_MXFP4 && block != 32 && block != 16) return 0;
     if (fmt == FP4O_NVFP4 && block != 16) return 0;
     if (fmt != FP4O_MXFP4 && fmt != FP4O_NVFP4) return 0;
     if (!(hk == 0 || hk == 16 || hk == 32 || hk == 64 || hk == 128)) return 0;

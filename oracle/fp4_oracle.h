@@ -13,6 +13,8 @@
  *     operation is fused or reassociated).  Subnormals are kept.
  *   - Elements are bf16 bit patterns (uint16_t), rows x cols, row stride ld
  *     (in elements).  The quantization / contraction axis is cols (K).
+ *   - fmt/block: FP4O_MXFP4 with block 32 or 16 (E8M0 scales), FP4O_NVFP4
+ *     with block 16 (E4M3 scales under an fp32 tensor scale).
  *   - Scales are returned in LOGICAL layout: s[row * (cols/block) + kb].
  *     The hardware tile layout is produced by fp4o_scales_to_atoms().
  *   - Packed elements: byte (row, j) holds element 2j in bits [3:0] and
