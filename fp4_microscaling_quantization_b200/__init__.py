@@ -10,25 +10,26 @@ from __future__ import annotations
 import ctypes
 
 from . import _lib
-from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_NVFP4, FP4_OUT_BF16,
+from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_MXFP4_16, FP4_NVFP4, FP4_OUT_BF16,
                    FP4_OUT_F32, FP4_ROUND_AWAY, FP4_ROUND_EVEN, FP4_SCALE_ABSMAX, FP4_SCALE_MSE, Fp4Error)
 
 __all__ = [
     "quantize", "dequantize", "gemm", "gemm_quantized", "linear", "linear_workspace_size", "quantize_sizes",
     "gemm_workspace_size", "check_device_status",
-    "FP4_MXFP4", "FP4_NVFP4", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
+    "FP4_MXFP4", "FP4_NVFP4", "FP4_MXFP4_16", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
     "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "FP4_SCALE_ABSMAX", "FP4_SCALE_MSE",
     "Fp4Error", "block_of",
 ]
 
 
 def block_of(fmt: int) -> int:
+    """Elements per block: 32 for MXFP4, 16 for NVFP4 and MXFP4_16."""
     return 32 if fmt == FP4_MXFP4 else 16
 
 
 def _fmt(fmt) -> int:
     if isinstance(fmt, str):
-        return {"mxfp4": FP4_MXFP4, "nvfp4": FP4_NVFP4}[fmt.lower()]
+        return {"mxfp4": FP4_MXFP4, "nvfp4": FP4_NVFP4, "mxfp4_16": FP4_MXFP4_16}[fmt.lower()]
     return int(fmt)
 
 

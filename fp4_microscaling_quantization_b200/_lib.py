@@ -13,7 +13,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfp4.so")
 
-FP4_MXFP4, FP4_NVFP4 = 0, 1
+FP4_MXFP4, FP4_NVFP4, FP4_MXFP4_16 = 0, 1, 2
 FP4_ROUND_EVEN, FP4_ROUND_AWAY = 0, 1
 FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR = 0, 1
 FP4_OUT_F32, FP4_OUT_BF16 = 0, 1

@@ -51,10 +51,18 @@ int sm_count()
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Format and block pairs of the quantizer; FP4_MXFP4 with block 16 is
+// FP4_MXFP4_16 (norm_fmt).
 bool valid_fmt(int fmt, int block)
 {
-    return (fmt == FP4_MXFP4 && block == 32) || (fmt == FP4_NVFP4 && block == 16);
+    return (fmt == FP4_MXFP4 && (block == 32 || block == 16)) || (fmt == FP4_NVFP4 && block == 16) ||
+           (fmt == FP4_MXFP4_16 && block == 16);
 }
+
+int norm_fmt(int fmt, int block) { return (fmt == FP4_MXFP4 && block == 16) ? FP4_MXFP4_16 : fmt; }
+
+// Formats of the product (the block size follows from the format).
+bool valid_gemm_fmt(int fmt) { return fmt == FP4_MXFP4 || fmt == FP4_NVFP4 || fmt == FP4_MXFP4_16; }
 
 bool valid_k(int k) { return k == 0 || k == 16 || k == 32 || k == 64 || k == 128; }
 
@@ -109,6 +117,7 @@ static fp4_status quantize_impl(const void *x, int64_t rows, int64_t cols, int64
     if (o.scale_search != FP4_SCALE_ABSMAX && o.scale_search != FP4_SCALE_MSE) return FP4_ERR_INVALID_ARG;
     if (with_res && o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;
     if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    fmt = norm_fmt(fmt, block);
     if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
     const bool empty = rows == 0 || cols == 0;
@@ -116,7 +125,7 @@ static fp4_status quantize_impl(const void *x, int64_t rows, int64_t cols, int64
     if (!empty && (!x || !q || !s || (with_res && !res))) return FP4_ERR_INVALID_ARG;
     if (!aligned(x, 16) || (ld_x % 8) || !aligned(q, 16) || !aligned(s, 16)) return FP4_ERR_ALIGNMENT;
     if ((gscale && !aligned(gscale, 4)) || (res && !aligned(res, 4))) return FP4_ERR_ALIGNMENT;
-    if (empty && fmt == FP4_MXFP4) return FP4_OK;
+    if (empty && fmt != FP4_NVFP4) return FP4_OK;
     cudaError_t e = fp4::launch_quantize(static_cast<const uint16_t *>(x), rows, cols, ld_x, fmt,
                                          hadamard_k, hadamard_constant(hadamard_k),
                                          o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR,
@@ -146,6 +155,7 @@ static fp4_status dequantize_impl(const uint8_t *q, const uint8_t *s, const floa
     if (rows < 0 || cols < 0) return FP4_ERR_INVALID_ARG;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
     if (!valid_fmt(fmt, block) || !valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    fmt = norm_fmt(fmt, block);
     if (cols % 32 || (hadamard_k && cols % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(rows, cols)) return FP4_ERR_UNSUPPORTED;
     if (rows == 0 || cols == 0) return FP4_OK;
@@ -177,7 +187,7 @@ fp4_status fp4_dequantize_residual(const uint8_t *q, const uint8_t *s, const flo
 fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes)
 {
     if (M < 0 || N < 0 || K < 0 || !bytes) return FP4_ERR_INVALID_ARG;
-    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
     *bytes = fp4::gemm_workspace_bytes(M, N, K, fmt, sm_count());
     return FP4_OK;
 }
@@ -187,7 +197,7 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, const
                     int out_dtype, void *C, int64_t ldc, void *workspace, size_t ws_bytes, void *stream)
 {
     if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
-    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
     if (K % 32) return FP4_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return FP4_OK;
@@ -236,7 +246,7 @@ extern "C" {
 fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, size_t *bytes)
 {
     if (M < 0 || N < 0 || K < 0 || !bytes) return FP4_ERR_INVALID_ARG;
-    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
     *bytes = linear_layout(M, N, K, fmt, sm_count()).total;
     return FP4_OK;
 }
@@ -249,7 +259,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
     if (opts) o = *opts;
     if (M < 0 || N < 0 || K < 0 || ld_x < K || ldc < N) return FP4_ERR_INVALID_ARG;
-    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
@@ -303,7 +313,7 @@ fp4_status fp4_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const float 
     fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
     if (opts) o = *opts;
     if (M < 0 || N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
-    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
     if (out_fmt != FP4_MXFP4 && out_fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
     if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
     if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;

@@ -164,6 +164,9 @@ FP4_DEV float exp2i(int e)
     return (e >= -126) ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
+// E8M0 scale byte -> 2^(byte - 127); 0xFF is NaN.
+FP4_DEV float e8m0_to_f32(uint32_t byte) { return (byte == 0xFF) ? __uint_as_float(0x7FC00000u) : exp2i((int)byte - 127); }
+
 // MXFP4 shared exponent from the block max (exact, from the exponent and
 // mantissa bits).  amax = m * 2^E with m in [1, 2):
 //   ceil rule : smallest e with amax <= 6 * 2^e  ->  E - 2 + (m > 1.5)

@@ -6,7 +6,8 @@
 // block scales and nearest rounding; the NVFP4 two-level scale ("4.5 FP8 and
 // NVFP4/MXFP4" §4.1); the block-diagonal Hadamard rotation H_k ("FP4
 // quantization analysis: MXFP4 vs NVFP4" §3.2.3).  A unit is 32 consecutive
-// elements of a row: one MXFP4 block or two NVFP4 blocks.
+// elements of a row: one MXFP4 block, or two 16-element blocks (NVFP4, or
+// MXFP4 on 16-element blocks: E8M0 scales at NVFP4's block size).
 #pragma once
 
 #include "common.cuh"
@@ -129,7 +130,8 @@ FP4_DEV void e2m1_pack_unit(const float *v, int round_away, uint4 &out)
 // Eq.(1): MXFP4 power-of-two scale; NVFP4 E4M3 block scale under the tensor
 // scale sg).  v is scaled in place; the 32 E2M1 codes come back as 16 bytes
 // of nibbles (even element in the low nibble) and the return value holds the
-// scale byte (MXFP4) or the two block-scale bytes, first block low (NVFP4).
+// scale byte (MXFP4) or the two block-scale bytes, first block low (NVFP4,
+// MXFP4_16).
 template <int FMT>
 FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, int mx_floor, uint4 &out,
                              const NvScaleTables *tab = nullptr)
@@ -142,6 +144,16 @@ FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, i
 #pragma unroll
         for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
         sbytes = (uint32_t)(e + 127);
+    } else if (FMT == FP4_MXFP4_16) {
+        sbytes = 0;
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            const int e = mx_exponent(absmax_tree<16>(v + 16 * b), mx_floor);
+            const float inv = exp2i(-e);
+#pragma unroll
+            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], inv);
+            sbytes |= (uint32_t)(e + 127) << (8 * b);
+        }
     } else {
         sbytes = 0;
 #pragma unroll
@@ -214,9 +226,23 @@ FP4_DEV float block_sq_error(const float *x, float r, float d, int round_away)
     return t[0];
 }
 
+// The MSE choice between the CEIL exponent e of an E8M0-scaled block of N
+// values and e - 1 (not below -127): e - 1 only if its error is smaller.
+template <int N>
+FP4_DEV int mx_mse_exponent(const float *x, int round_away)
+{
+    int e = mx_exponent(absmax_tree<N>(x), 0);
+    if (e > -127) {
+        const float e0 = block_sq_error<N>(x, exp2i(-e), exp2i(e), round_away);
+        const float e1 = block_sq_error<N>(x, exp2i(1 - e), exp2i(e - 1), round_away);
+        if (e1 < e0) e -= 1;
+    }
+    return e;
+}
+
 // encode_unit with the MSE method.  Candidates, in the order tried:
-//   MXFP4: e_c (the CEIL exponent), then e_c - 1 unless e_c = -127; the
-//          FLOOR rule's exponent is always one of the two.
+//   MXFP4, MXFP4_16: e_c (the CEIL exponent), then e_c - 1 unless
+//          e_c = -127; the FLOOR rule's exponent is always one of the two.
 //   NVFP4: t0 (the absmax E4M3 code), then t0 - 2, t0 - 1, t0 + 1 .. t0 + 6,
 //          each only within 1 .. 0x7E: scales that put the block max between
 //          about 3.6 and 7.3 on the grid.  Decode and encode factors come
@@ -226,16 +252,21 @@ FP4_DEV uint32_t encode_unit_mse(float *v, float six_sg, int round_away, const N
 {
     uint32_t sbytes;
     if (FMT == FP4_MXFP4) {
-        int e = mx_exponent(absmax_tree<32>(v), 0);
-        if (e > -127) {
-            const float e0 = block_sq_error<32>(v, exp2i(-e), exp2i(e), round_away);
-            const float e1 = block_sq_error<32>(v, exp2i(1 - e), exp2i(e - 1), round_away);
-            if (e1 < e0) e -= 1;
-        }
+        const int e = mx_mse_exponent<32>(v, round_away);
         const float inv = exp2i(-e);
 #pragma unroll
         for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
         sbytes = (uint32_t)(e + 127);
+    } else if (FMT == FP4_MXFP4_16) {
+        sbytes = 0;
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            const int e = mx_mse_exponent<16>(v + 16 * b, round_away);
+            const float inv = exp2i(-e);
+#pragma unroll
+            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], inv);
+            sbytes |= (uint32_t)(e + 127) << (8 * b);
+        }
     } else {
         sbytes = 0;
 #pragma unroll

@@ -6,7 +6,9 @@
 //
 // Operands come straight from fp4_quantize: packed E2M1 rows (K-major) and
 // scales already in the 128x4 atom layout the MMA reads, so no re-layout
-// pass exists.  alpha = s_gA * s_gW for NVFP4, 1 for MXFP4.
+// pass exists.  alpha = s_gA * s_gW for NVFP4, 1 for MXFP4.  MXFP4 on
+// 16-element blocks runs the NVFP4 (16-element block) instantiations with
+// the MMA's scale type switched to E8M0 at run time (sf_e8m0) and alpha = 1.
 //
 // Prefill (M > 16): a persistent kernel over 128*CG x 256 output tiles, CG = 2
 // (CTA pairs sharing one 2-SM MMA) once A spans more than 128 rows; see
@@ -91,6 +93,7 @@ struct PParams {
     int M, N, K;
     int nkb4;
     int num_m_tiles, num_n_tiles;
+    int sf_e8m0;         // FMT == NVFP4 only: E8M0 block scales (MXFP4 on 16-element blocks), alpha = 1
     uint64_t budget_ns;  // limit of every mbarrier wait
     int stall;           // failure-detection test: the producer issues no loads
 };
@@ -212,7 +215,7 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                         const uint64_t bd = bdesc0 + so + 2 * kk;
                         const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
                         const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
-                        const uint32_t idesc = idesc_blockscaled(Cfg::BM * CG, Cfg::BN, FMT == FP4_MXFP4, sfid, sfid);
+                        const uint32_t idesc = idesc_blockscaled(Cfg::BM * CG, Cfg::BN, FMT == FP4_MXFP4 || p.sf_e8m0, sfid, sfid);
                         tc_mma_blockscaled_cg<FMT, CG>(tmem, ad, bd, idesc, (tsfa + 4 * atom) | (sfid << 30),
                                                        (tsfb + 8 * atom) | (sfid << 30), (ks | kk) ? 1u : 0u);
                     }
@@ -297,7 +300,7 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 if (CG == 1) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce) : "memory");
                 else mbar_arrive_cluster(acce_lead);
             }
-            const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
+            const float alpha = (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
             const int m = (mt * CG + (int)rank) * Cfg::BM + quarter * 32 + lane;
             const int n0 = nt * Cfg::BN + half * 128;
             if (OUT >= OUT_MXFP4) {
@@ -421,6 +424,7 @@ struct Params {
     void *C;
     int64_t ldc;
     int bf16out;
+    int sf_e8m0;         // FMT == NVFP4 only: E8M0 block scales (MXFP4 on 16-element blocks), alpha = 1
     uint64_t budget_ns;  // limit of every mbarrier wait
     int stall;           // failure-detection test: the producer issues no loads
     int N, M, K;
@@ -629,7 +633,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                         const uint64_t ad = adesc0 + so + 2 * kk;
                         const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
                         const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
-                        const uint32_t idesc = idesc_blockscaled(BMW, BNA, FMT == FP4_MXFP4, sfid, sfid);
+                        const uint32_t idesc = idesc_blockscaled(BMW, BNA, FMT == FP4_MXFP4 || p.sf_e8m0, sfid, sfid);
                         tc_mma_blockscaled<FMT>(acc, wd, ad, idesc, (tsfw + 4 * atom) | (sfid << 30),
                                                 (tsfa + 4 * atom) | (sfid << 30), (i == first && kk == 0) ? 0u : 1u);
                     }
@@ -650,7 +654,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     // warp w may only read TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
     grid_dep_wait();
-    const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
+    const float alpha = (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
     for (int seg = 0; seg < nseg; seg++) {
         const int b = seg & 1;
         bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error, p.budget_ns);
@@ -763,7 +767,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                     acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
                 }
             }
-            if (n < p.N && !*abort_flag) store_row(p, n, acc, (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
+            if (n < p.N && !*abort_flag) store_row(p, n, acc, (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
         }
         cluster_sync();
     }
@@ -784,7 +788,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(Params p)
     grid_dep_wait();
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     if (n >= p.N) return;
-    const float alpha = (FMT == FP4_NVFP4) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
+    const float alpha = (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
     const int t = n / BMW, r = n % BMW;
     const int64_t U = (int64_t)p.ntiles * p.nk;
     const int c_lo = unit_owner((int64_t)t * p.nk, U, p.G), c_hi = unit_owner((int64_t)(t + 1) * p.nk - 1, U, p.G);
@@ -1063,6 +1067,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.C = C;
         dp.ldc = ldc;
         dp.bf16out = bf16out;
+        dp.sf_e8m0 = fmt == FP4_MXFP4_16;
         return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl)
                                 : launch_decode<FP4_NVFP4>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl);
     }
@@ -1080,6 +1085,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         pp.N = (int)N;
         pp.K = (int)K;
         pp.nkb4 = (int)((K / (fmt == FP4_MXFP4 ? 32 : 16) + 3) / 4);
+        pp.sf_e8m0 = fmt == FP4_MXFP4_16;
         pp.budget_ns = budget;
         pp.stall = stall;
         const int cg = pgemm_cta_group(M);
@@ -1112,6 +1118,7 @@ cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const fl
     pp.N = (int)N;
     pp.K = (int)K;
     pp.nkb4 = (int)((K / (fmt == FP4_MXFP4 ? 32 : 16) + 3) / 4);
+    pp.sf_e8m0 = fmt == FP4_MXFP4_16;
     uint64_t budget = g_inject_budget.exchange(0);
     pp.budget_ns = budget ? budget : kWaitBudgetNs;
     pp.stall = g_inject_stall.exchange(0);
@@ -1191,7 +1198,7 @@ extern "C" fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *
                                               void *C, int64_t ldc, void *stream)
 {
     if (M < 0 || N < 0 || K < 0 || ldc < N) return FP4_ERR_INVALID_ARG;
-    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_UNSUPPORTED;
+    if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4 && fmt != FP4_MXFP4_16) return FP4_ERR_UNSUPPORTED;
     if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
     if (K % 32 || M > fp4::kDecodeMaxM) return FP4_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return FP4_OK;

@@ -509,8 +509,10 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantArgs a)
                 const uint32_t words[4] = {w.x, w.y, w.z, w.w};
                 float d0, d1;
                 if (FMT == FP4_MXFP4) {
-                    const uint32_t sb = sraw[i];
-                    d0 = d1 = (sb == 0xFF) ? __uint_as_float(0x7FC00000u) : exp2i((int)sb - 127);
+                    d0 = d1 = e8m0_to_f32(sraw[i]);
+                } else if (FMT == FP4_MXFP4_16) {
+                    d0 = e8m0_to_f32(sraw[i] & 0xFF);
+                    d1 = e8m0_to_f32(sraw[i] >> 8);
                 } else {
                     const uint32_t sb2 = sraw[i];
                     d0 = __fmul_rn(sg, e4m3_to_f32(sb2 & 0xFF));
@@ -615,6 +617,12 @@ static void (*quant_res_kernel_for(int hk))(QuantArgs)
     return nullptr;
 }
 
+template <int FMT>
+static void (*quant_kernel_pick(int hk, int mse, bool res))(QuantArgs)
+{
+    return res ? quant_res_kernel_for<FMT>(hk) : mse ? quant_kernel_for<FMT, true>(hk) : quant_kernel_for<FMT, false>(hk);
+}
+
 template <bool RES>
 static void (*amax_kernel_for(int hk))(QuantArgs)
 {
@@ -652,12 +660,9 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
     a.res = res;
     const int grid = grid_for(a.total_units, sms, QUNITS);
-    void (*qk)(QuantArgs) = res ? ((fmt == FP4_MXFP4) ? quant_res_kernel_for<FP4_MXFP4>(hk)
-                                                      : quant_res_kernel_for<FP4_NVFP4>(hk))
-                          : (fmt == FP4_MXFP4) ? (mse ? quant_kernel_for<FP4_MXFP4, true>(hk)
-                                                      : quant_kernel_for<FP4_MXFP4, false>(hk))
-                                               : (mse ? quant_kernel_for<FP4_NVFP4, true>(hk)
-                                                      : quant_kernel_for<FP4_NVFP4, false>(hk));
+    void (*qk)(QuantArgs) = fmt == FP4_MXFP4   ? quant_kernel_pick<FP4_MXFP4>(hk, mse, res != nullptr)
+                            : fmt == FP4_NVFP4 ? quant_kernel_pick<FP4_NVFP4>(hk, mse, res != nullptr)
+                                               : quant_kernel_pick<FP4_MXFP4_16>(hk, mse, res != nullptr);
     void (*ak)(QuantArgs) = res ? amax_kernel_for<true>(hk) : amax_kernel_for<false>(hk);
     if (!qk || !ak) return cudaErrorInvalidValue;
     cudaError_t err = cudaSuccess;
@@ -758,7 +763,9 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
     a.res = nullptr;
-    void (*k)(QuantArgs, unsigned *, int, int) = (fmt == FP4_MXFP4) ? act_kernel_for<FP4_MXFP4>(hk) : act_kernel_for<FP4_NVFP4>(hk);
+    void (*k)(QuantArgs, unsigned *, int, int) = fmt == FP4_MXFP4   ? act_kernel_for<FP4_MXFP4>(hk)
+                                                 : fmt == FP4_NVFP4 ? act_kernel_for<FP4_NVFP4>(hk)
+                                                                    : act_kernel_for<FP4_MXFP4_16>(hk);
     if (!k) return cudaErrorInvalidValue;
     const bool cluster = a.gscale_computed != 0;
     const int ctas = cluster ? act_cluster_size(k) : ACT_CTAS;
@@ -792,6 +799,13 @@ static void (*deq_kernel_for(int hk))(DequantArgs)
     case 128: return dequantize_kernel<FMT, 128, BF, RES>;
     }
     return nullptr;
+}
+
+template <int FMT>
+static void (*deq_kernel_pick(int hk, int bf16out, bool res))(DequantArgs)
+{
+    return res ? (bf16out ? deq_kernel_for<FMT, 1, true>(hk) : deq_kernel_for<FMT, 0, true>(hk))
+               : (bf16out ? deq_kernel_for<FMT, 1, false>(hk) : deq_kernel_for<FMT, 0, false>(hk));
 }
 
 // ---------------------------------------------------------------------------
@@ -1089,13 +1103,9 @@ cudaError_t launch_dequantize(const uint8_t *q, const uint8_t *s, const float *g
     a.res = res;
     if (a.total_units == 0) return cudaSuccess;
     const int grid = grid_for(a.total_units, sms, DUNITS);
-    void (*k)(DequantArgs) =
-        res ? ((fmt == FP4_MXFP4)
-                   ? (bf16out ? deq_kernel_for<FP4_MXFP4, 1, true>(hk) : deq_kernel_for<FP4_MXFP4, 0, true>(hk))
-                   : (bf16out ? deq_kernel_for<FP4_NVFP4, 1, true>(hk) : deq_kernel_for<FP4_NVFP4, 0, true>(hk)))
-            : ((fmt == FP4_MXFP4)
-                   ? (bf16out ? deq_kernel_for<FP4_MXFP4, 1, false>(hk) : deq_kernel_for<FP4_MXFP4, 0, false>(hk))
-                   : (bf16out ? deq_kernel_for<FP4_NVFP4, 1, false>(hk) : deq_kernel_for<FP4_NVFP4, 0, false>(hk)));
+    void (*k)(DequantArgs) = fmt == FP4_MXFP4   ? deq_kernel_pick<FP4_MXFP4>(hk, bf16out, res != nullptr)
+                             : fmt == FP4_NVFP4 ? deq_kernel_pick<FP4_NVFP4>(hk, bf16out, res != nullptr)
+                                                : deq_kernel_pick<FP4_MXFP4_16>(hk, bf16out, res != nullptr);
     if (!k) return cudaErrorInvalidValue;
     // programmatic launch: the kernel waits for its predecessor before touching memory
     return launch_k(k, dim3(grid), dim3(256), 0, st, true, a);

@@ -5,6 +5,12 @@
  *   MXFP4  32-element blocks along K, one E8M0 (power-of-two) scale per block.
  *   NVFP4  16-element blocks along K, one unsigned E4M3 scale per block, and
  *          one FP32 tensor-level scale s_g.
+ *   MXFP4_16  16-element blocks along K, one E8M0 scale per block: the
+ *          microscaling form with block size G = 16 (TransFP4 §1.1 leaves G
+ *          open) and the 16-element scale vector the block-scaled MMA also
+ *          takes with E8M0 scales.  It keeps MXFP4's scale encoding at
+ *          NVFP4's block size, so the two effects that tell MXFP4 and NVFP4
+ *          apart can be taken one at a time.
  * Sources: "Portable FP4 quantization (TransFP4)" §1.1 Eq.(1)
  * (x^_i = s_g s_b Q_f(x_i / (s_g s_b))) and Table 1; "4.5 FP8 and
  * NVFP4/MXFP4" §3.1 (E2M1 magnitudes), §3.3 and §4.1 (scale formats, the
@@ -57,7 +63,7 @@ typedef enum {
     FP4_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait           */
 } fp4_status;
 
-typedef enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1 } fp4_fmt;
+typedef enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1, FP4_MXFP4_16 = 2 } fp4_fmt;
 
 /* E2M1 tie rule at exact midpoints: even code (IEEE style, default) or the
  * larger magnitude (reproduces the gpt-oss article's worked example). */
@@ -75,7 +81,7 @@ typedef enum { FP4_MX_SCALE_CEIL = 0, FP4_MX_SCALE_FLOOR = 1 } fp4_mx_scale_rule
  * scales around the absmax one and keeps the one with the smallest fp32
  * squared reconstruction error, summed in a fixed pairwise order; of equal
  * ones the first tried.  Windows, in the order tried:
- *   MXFP4: e_c (the CEIL exponent), e_c - 1 (unless e_c = -127);
+ *   MXFP4, MXFP4_16: e_c (the CEIL exponent), e_c - 1 (unless e_c = -127);
  *          mx_scale_rule is not used;
  *   NVFP4: t0 (the absmax E4M3 code), t0-2, t0-1, t0+1, ..., t0+6, within
  *          1 .. 0x7E.  The tensor scale s_g stays the absmax one.
@@ -105,7 +111,9 @@ const char *fp4_status_string(fp4_status st);
 
 /* Sizes of the packed-element and scale buffers for a rows x cols tensor.
  * q_bytes = rows*cols/2; s_bytes = pad128(rows) * pad4(cols/block).
- * Host-only; block must be 32 for MXFP4 and 16 for NVFP4. */
+ * Host-only; block must be 32 for MXFP4 and 16 for NVFP4 and MXFP4_16
+ * (fmt = FP4_MXFP4 with block = 16 is taken as FP4_MXFP4_16, here and in
+ * fp4_quantize, fp4_dequantize and their residual forms). */
 fp4_status fp4_quantize_sizes(int64_t rows, int64_t cols, int fmt, int block,
                               size_t *q_bytes, size_t *s_bytes);
 
@@ -116,14 +124,16 @@ fp4_status fp4_quantize_sizes(int64_t rows, int64_t cols, int fmt, int block,
  *
  *   x       bf16 input, rows x cols, row stride ld_x elements.  16-byte
  *           aligned; ld_x a multiple of 8.
- *   fmt     FP4_MXFP4 (block 32) or FP4_NVFP4 (block 16).
+ *   fmt     FP4_MXFP4 (block 32), FP4_NVFP4 (block 16) or FP4_MXFP4_16
+ *           (block 16).
  *   hadamard_k  0 (no rotation) or 16, 32, 64, 128; cols % k == 0.  The
  *           rotation is the normalised Sylvester Walsh-Hadamard transform
  *           (stages h = 1, 2, ..., k/2, then x RN(1/sqrt(k))) in fp32.
  *   opts    may be NULL (= round even, CEIL, s_g computed).
  *   q       output, packed elements (layout above), 16-byte aligned.
  *   s       output, scales in the tile layout above (padding written 0).
- *   gscale  NVFP4 only (ignored for MXFP4, may be NULL): one device fp32.
+ *   gscale  NVFP4 only (ignored for the E8M0 formats, may be NULL): one
+ *           device fp32.
  *           gscale_given: read as s_g.  Otherwise written with
  *           s_g = amax(|H_k x|) / (6*448), or 1 for an all-zero tensor.
  * cols must be a multiple of 32 (also for NVFP4).  rows == 0 is a no-op.
@@ -140,7 +150,8 @@ fp4_status fp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
  * MXFP4 s_g = 1 and s_b = 2^(byte-127)), NVFP4 computed as
  * RN(RN(s_g*s_b) * q).  hadamard_k > 0 applies H_k again (it is its own
  * inverse) to return to the unrotated domain; 0 leaves values rotated.
- *   q, s, gscale   as produced by fp4_quantize (gscale ignored for MXFP4).
+ *   q, s, gscale   as produced by fp4_quantize (gscale ignored for MXFP4
+ *                  and MXFP4_16).
  *   out_dtype      FP4_OUT_F32 or FP4_OUT_BF16 (round to nearest even).
  *   out            rows x cols, row stride cols, 16-byte aligned.
  */
@@ -179,7 +190,7 @@ fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt,
  * ("4.5 FP8 and NVFP4/MXFP4" §5: both operands in FP4 on the Blackwell
  * tensor cores), A: M x K, W: N x K, both quantized along K in the same
  * format by fp4_quantize (Aq/As, Wq/Ws).  alpha = s_gA * s_gW for NVFP4
- * (gA, gW device fp32), 1 for MXFP4 (gA, gW ignored).
+ * (gA, gW device fp32), 1 for MXFP4 and MXFP4_16 (gA, gW ignored).
  *   K          multiple of 32 ("Portable FP4 quantization (TransFP4)" Table 3:
  *              the GEMM's K alignment is 32).  The tensor cores step K by
  *              256 per stage; the last step of a tail multiplies zeros read
@@ -208,7 +219,8 @@ fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA,
  * the per-unit encoding of fp4_quantize (TransFP4 §1.1 Eq.(1)) applied to
  * the FP32 values alpha * acc.
  *   Aq/As/gA, Wq/Ws/gW, fmt   as for fp4_gemm.
- *   out_fmt   FP4_MXFP4 or FP4_NVFP4 (may differ from fmt).
+ *   out_fmt   FP4_MXFP4 or FP4_NVFP4 (may differ from fmt; FP4_MXFP4_16
+ *             output: FP4_ERR_UNSUPPORTED).
  *   opts      round and mx_scale_rule as for fp4_quantize; may be NULL.
  *   gC        NVFP4 output: the tensor scale s_g of C, one device fp32, given
  *             (a whole-tensor maximum is not known until every tile is done,
@@ -268,7 +280,8 @@ fp4_status fp4_nv_refine_gscale(const void *x, int64_t rows, int64_t cols, int64
  * same value.  Blocks more than 17 binades below the largest take the E4M3
  * rounding of 2^(e - E), which is 0 from 2^-10 down; E8M0 NaN becomes E4M3
  * NaN.  Three small launches; meant to run once per weight.
- *   s_mx    MXFP4 scales of a rows x cols tensor in the tile layout, as
+ *   s_mx    MXFP4 (32-element block) scales of a rows x cols tensor in the
+ *           tile layout, as
  *           fp4_quantize writes them (cols multiple of 32).
  *   s_nv    output: fp4_quantize_sizes(rows, cols, FP4_NVFP4, 16) scale
  *           bytes in the tile layout, padding written 0.
@@ -290,7 +303,8 @@ fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, s
  * quantized with the same hadamard_k), then C = alpha * x_q W_q^T as in
  * fp4_gemm.  M <= 16 is the decode case the weight stream dominates.
  *   gA      NVFP4 activation tensor scale: NULL = computed from x (dynamic),
- *           else a device fp32 holding a static s_g.  Ignored for MXFP4.
+ *           else a device fp32 holding a static s_g.  Ignored for MXFP4 and
+ *           MXFP4_16.
  *   opts    rounding options for the activation quantization (may be NULL;
  *           gscale_given is ignored, gA decides).
  *   workspace  at least fp4_linear_workspace_size() bytes, 256-byte aligned;

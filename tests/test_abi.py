@@ -46,7 +46,13 @@ def test_quantize_sizes(L):
     assert q.value == 200 * 160 and s.value == 256 * 12
     assert L.fp4_quantize_sizes(200, 320, 1, 16, ctypes.byref(q), ctypes.byref(s)) == 0
     assert s.value == 256 * 20
-    assert L.fp4_quantize_sizes(4, 64, 0, 16, ctypes.byref(q), ctypes.byref(s)) == 2  # MX needs 32
+    # MXFP4 with block 16 is MXFP4_16: 16-element blocks, E8M0 scales
+    assert L.fp4_quantize_sizes(200, 320, 0, 16, ctypes.byref(q), ctypes.byref(s)) == 0
+    assert q.value == 200 * 160 and s.value == 256 * 20
+    assert L.fp4_quantize_sizes(200, 320, 2, 16, ctypes.byref(q), ctypes.byref(s)) == 0
+    assert s.value == 256 * 20
+    assert L.fp4_quantize_sizes(4, 64, 2, 32, ctypes.byref(q), ctypes.byref(s)) == 2  # MXFP4_16 is 16
+    assert L.fp4_quantize_sizes(4, 64, 0, 8, ctypes.byref(q), ctypes.byref(s)) == 2
     assert L.fp4_quantize_sizes(-1, 64, 0, 32, ctypes.byref(q), ctypes.byref(s)) == 1
 
 
@@ -55,8 +61,10 @@ FAKE = 0x10000  # an aligned pointer value never dereferenced: validation fails 
 
 @pytest.mark.parametrize("args,code", [
     (dict(rows=-1), 1),
-    (dict(fmt=0, block=16), 2),
+    (dict(fmt=0, block=8), 2),
     (dict(fmt=1, block=32), 2),
+    (dict(fmt=2, block=32), 2),
+    (dict(fmt=3, block=16), 2),
     (dict(hadamard_k=8), 2),
     (dict(cols=48), 2),
     (dict(cols=64, hadamard_k=128), 2),
@@ -115,6 +123,7 @@ def test_gemm_quantized_rejects_on_host(L):
     assert g(F, F, F, F, F, F, 256, 192, 256, 0, 0, None, None, F, F, None) == 2     # N % 128
     assert g(F, F, F, F, F, F, 256, 256, 112, 0, 0, None, None, F, F, None) == 2     # K % 32
     assert g(F, F, F, F, F, F, 256, 256, 256, 0, 3, None, None, F, F, None) == 2     # output format
+    assert g(F, F, F, F, F, F, 256, 256, 256, 0, 2, None, None, F, F, None) == 2     # no MXFP4_16 output
     assert g(F, F, F, F, F, F, 256, 256, 256, 0, 1, None, None, F, F, None) == 1     # NVFP4 out needs gC
     assert g(F, F, None, F, F, F, 256, 256, 256, 1, 0, None, None, F, F, None) == 1  # NVFP4 in needs gA
     assert g(F, F, F, F, F, F, 256, 256, 256, 0, 0, None, None, None, F, None) == 1  # Cq
