@@ -91,19 +91,23 @@ def time_graph(torch, fn, warmup: int, reps: int):
     return e0.elapsed_time(e1) / reps
 
 
-def bench_rotate(torch, fp4, inputs, dev, reps: int):
+def bench_rotate(torch, fp4, inputs, dev, reps: int, fmts=None):
     """Fused rotate + quantize of 8192x4096 bf16 activations (Laplace(0,1), 1%
-    outlier channels x50), k in {0,16,32,64,128}, MXFP4 and NVFP4.  Eight input
-    copies (537 MB) are rotated so every call reads x from HBM (one fits in L2).
-    Bytes per element: read 2 + nibbles 0.5 + scales 1/32 (MX) or 1/16 (NV);
-    the NVFP4 amax pass re-reads x from L2 and is not counted."""
+    outlier channels x50), k in {0,16,32,64,128}, MXFP4, NVFP4 and MXFP4 on
+    16-element blocks.  Eight input copies (537 MB) are rotated so every call
+    reads x from HBM (one fits in L2).  Bytes per element: read 2 + nibbles
+    0.5 + scales 1/32 (MX) or 1/16 (NV, MX16); the NVFP4 amax pass re-reads x
+    from L2 and is not counted."""
     hbm, kind = peaks()
     x = inputs.rotate_acts()
     xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
     copies = [xd.clone() for _ in range(8)]
     n = xd.numel()
     res = {"peak_gbs": hbm, "peak_kind": kind, "workload": "rotate+quantize 8192x4096 bf16", "cases": {}}
-    for fmt, name, bpe in ((fp4.FP4_MXFP4, "mxfp4", 2 + 0.5 + 1 / 32), (fp4.FP4_NVFP4, "nvfp4", 2 + 0.5 + 1 / 16)):
+    for fmt, name, bpe in ((fp4.FP4_MXFP4, "mxfp4", 2 + 0.5 + 1 / 32), (fp4.FP4_NVFP4, "nvfp4", 2 + 0.5 + 1 / 16),
+                           (fp4.FP4_MXFP4_16, "mxfp4_16", 2 + 0.5 + 1 / 16)):
+        if fmts is not None and name not in fmts:
+            continue
         outs = fp4.quantize(xd, fmt)
         for k in (0, 16, 32, 64, 128):
             it = [0]
@@ -142,7 +146,7 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int):
     return res
 
 
-def bench_decode(torch, fp4, inputs, dev, reps: int):
+def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None):
     """Decode shapes: M in {1,4,16} bf16 activations quantized online inside
     the timed call (fp4_linear), W 14336x4096 and 4096x14336 pre-quantized,
     BF16 out.  W copies are rotated so the weight stream comes from HBM.  The
@@ -157,7 +161,10 @@ def bench_decode(torch, fp4, inputs, dev, reps: int):
         # the third case is the workload's literal reading: NVFP4 activations
         # against MXFP4 weights, bound once to the NVFP4 scale form
         for fmt, name, wfmt in ((fp4.FP4_NVFP4, "nvfp4", fp4.FP4_NVFP4), (fp4.FP4_MXFP4, "mxfp4", fp4.FP4_MXFP4),
-                                (fp4.FP4_NVFP4, "nvfp4act_mxfp4w", fp4.FP4_MXFP4)):
+                                (fp4.FP4_NVFP4, "nvfp4act_mxfp4w", fp4.FP4_MXFP4),
+                                (fp4.FP4_MXFP4_16, "mxfp4_16", fp4.FP4_MXFP4_16)):
+            if fmts is not None and name not in fmts:
+                continue
             W0 = fp4.quantize(wd, wfmt)
             if wfmt != fmt:
                 W0 = fp4.mx_to_nv(W0)
@@ -197,7 +204,7 @@ def bench_prefill(torch, fp4, inputs, dev, reps: int, M: int = 8192, fmts=None):
     peak, kind = fp4_tensor_peak()
     out = {"workload": f"prefill W4A4 linear M={M} N={N} K={K}, BF16 out", "peak_tflops": peak, "peak_kind": kind}
     C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    for fmt, name in ((fp4.FP4_NVFP4, "nvfp4"), (fp4.FP4_MXFP4, "mxfp4")):
+    for fmt, name in ((fp4.FP4_NVFP4, "nvfp4"), (fp4.FP4_MXFP4, "mxfp4"), (fp4.FP4_MXFP4_16, "mxfp4_16")):
         if fmts is not None and name not in fmts:
             continue
         A = fp4.quantize(ad, fmt)
@@ -209,13 +216,15 @@ def bench_prefill(torch, fp4, inputs, dev, reps: int, M: int = 8192, fmts=None):
         out[name]["act_quantize_ms"] = q_ms
         out[name]["tflops_incl_act_quantize"] = 2.0 * M * N * K / ((ms + q_ms) * 1e-3) / 1e12
         # C quantized for the next layer in the GEMM epilogue (NVFP4 with a
-        # given tensor scale), against BF16 C followed by a quantize pass.
+        # given tensor scale; MXFP4 for MXFP4_16 operands), against BF16 C
+        # followed by a quantize pass.
+        ofmt = fp4.FP4_MXFP4 if fmt == fp4.FP4_MXFP4_16 else fmt
         gC = torch.full((1,), 0.05, dtype=torch.float32, device=dev)
-        Cq = fp4.gemm_quantized(A, W, M, N, K, fmt, fmt, gscale=gC if fmt == fp4.FP4_NVFP4 else None)
-        fq_ms = time_graph(torch, lambda: fp4.gemm_quantized(A, W, M, N, K, fmt, fmt, out=Cq), 3, reps)
-        gs = gC if fmt == fp4.FP4_NVFP4 else None
-        Cb = fp4.quantize(C, fmt, gscale=gs)
-        cq_ms = time_graph(torch, lambda: fp4.quantize(C, fmt, gscale=gs, out=Cb), 3, reps)
+        Cq = fp4.gemm_quantized(A, W, M, N, K, fmt, ofmt, gscale=gC if ofmt == fp4.FP4_NVFP4 else None)
+        fq_ms = time_graph(torch, lambda: fp4.gemm_quantized(A, W, M, N, K, fmt, ofmt, out=Cq), 3, reps)
+        gs = gC if ofmt == fp4.FP4_NVFP4 else None
+        Cb = fp4.quantize(C, ofmt, gscale=gs)
+        cq_ms = time_graph(torch, lambda: fp4.quantize(C, ofmt, gscale=gs, out=Cb), 3, reps)
         out[name]["quantized_out"] = {"ms": fq_ms, "tflops": 2.0 * M * N * K / (fq_ms * 1e-3) / 1e12,
                                       "frac": 2.0 * M * N * K / (fq_ms * 1e-3) / 1e12 / peak,
                                       "unfused_bf16_then_quantize_ms": ms + cq_ms}
@@ -367,9 +376,9 @@ def run_ours(args):
         if args.only == "prefill":
             r = bench_prefill(torch, fp4, inputs, dev, reps=args.steps, M=args.prefill_m, fmts=args.fmts)
         elif args.only == "rotate":
-            r = bench_rotate(torch, fp4, inputs, dev, reps=args.steps)
+            r = bench_rotate(torch, fp4, inputs, dev, reps=args.steps, fmts=args.fmts)
         else:
-            r = bench_decode(torch, fp4, inputs, dev, reps=args.steps)
+            r = bench_decode(torch, fp4, inputs, dev, reps=args.steps, fmts=args.fmts)
         print(json.dumps({"only": args.only, "result": r}), flush=True)
         return 0
 
