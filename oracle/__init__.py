@@ -40,7 +40,16 @@ Parity status of each function (what pins it, see tests/test_oracle_pins.py):
                           coarse one below the block max), equal to MXFP4
                           where a unit's halves share its exponent
                           (tests/test_oracle_mx16_pins.py)
-  NMSE vs the page's table   directional only (the page's generator is unknown)
+  INT4 group baseline     pinned: every element at a nearest level of its
+                          group's grid s*{-7..7}, s = amax/7, the group max at
+                          +-7; Table 5's INT4 NMSE reproduced within 5 %
+                          (tests/test_oracle_transfp4_pins.py)
+  TransFP4 (rotation +    pinned: with the INT4 candidate off it equals the
+  residual + NV/INT4      NVFP4 residual-lane round trip bit for bit; each
+  choice per unit)        unit's choice has the smaller error; Table 5's
+                          TransFP4 NMSE reproduced within 6 %
+  NMSE vs the page's table   directional only for MXFP4 / NVFP4 / rotated
+                          MXFP4 (the page's generator is unknown) (the page's generator is unknown)
 """
 from __future__ import annotations
 
@@ -121,6 +130,12 @@ def lib():
         L.fp4o_nv_refine_gscale.argtypes = [vp, i64, i64, i64, i32, i32, i32, vp, vp]
         L.fp4o_nv_refine_gscale.restype = i32
         L.fp4o_mx_scales_to_nv.restype = i32
+        L.fp4o_int4_quantize_f32.argtypes = [vp, i64, i64, i32, vp, vp]
+        L.fp4o_int4_quantize_f32.restype = i32
+        L.fp4o_int4_dequantize.argtypes = [vp, vp, i64, i64, i32, vp]
+        L.fp4o_int4_dequantize.restype = i32
+        L.fp4o_transfp4_f32.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp]
+        L.fp4o_transfp4_f32.restype = i32
         L.fp4o_num_threads.restype = i32
         _lib = L
     return _lib
@@ -301,6 +316,42 @@ def mx_scales_to_nv(s_mx_logical: np.ndarray):
     if lib().fp4o_mx_scales_to_nv(_ptr(s), rows, nkb, _ptr(out), _ptr(g)) != 0:
         raise ValueError("oracle mx_scales_to_nv: invalid arguments")
     return out, float(g[0])
+
+
+def int4_quantize(x: np.ndarray, group: int = 32):
+    """INT4 group quantization of fp32 rows (Table 5's INT4 baseline):
+    returns (q int8 (rows, cols), scales fp32 (rows, cols/group))."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    q = np.zeros((rows, cols), np.int8)
+    s = np.zeros((rows, cols // group if group else 0), np.float32)
+    if lib().fp4o_int4_quantize_f32(_ptr(x), rows, cols, group, _ptr(q), _ptr(s)) != 0:
+        raise ValueError("oracle int4_quantize: invalid arguments")
+    return q, s
+
+
+def int4_dequantize(q: np.ndarray, s: np.ndarray, group: int = 32) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    rows, cols = q.shape
+    out = np.zeros((rows, cols), np.float32)
+    if lib().fp4o_int4_dequantize(_ptr(q), _ptr(s), rows, cols, group, _ptr(out)) != 0:
+        raise ValueError("oracle int4_dequantize: invalid arguments")
+    return out
+
+
+def transfp4(x: np.ndarray, hadamard_k: int = 32, tie: int = TIE_EVEN, allow_int4: bool = True):
+    """The TransFP4 method of the page's Table 5 on fp32 rows (rotation,
+    residual lane, per-unit NVFP4 / INT4 choice): returns (x_hat fp32
+    (rows, cols), choice uint8 (rows, cols/32), 1 = INT4)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    out = np.zeros((rows, cols), np.float32)
+    choice = np.zeros((rows, cols // 32), np.uint8)
+    if lib().fp4o_transfp4_f32(_ptr(x), rows, cols, hadamard_k, tie, int(bool(allow_int4)), _ptr(out),
+                               _ptr(choice)) != 0:
+        raise ValueError("oracle transfp4: invalid arguments")
+    return out, choice
 
 
 def gemm_ref(a_hat: np.ndarray, w_hat: np.ndarray):

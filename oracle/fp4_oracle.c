@@ -611,6 +611,118 @@ int fp4o_mx_scales_to_nv(const uint8_t *s_mx, int64_t rows, int64_t nkb, uint8_t
 }
 
 /* ------------------------------------------------------------------------ */
+/* INT4 group quantization, the INT4 baseline of [TransFP4] Table 5 (§3.1:   */
+/* every method uses per-block absmax scales and nearest rounding).  A group */
+/* of G consecutive values takes the fp32 scale s = amax / 7 and the integer */
+/* codes q_i = x_i / s rounded to nearest (ties to even), clamped to         */
+/* [-7, 7]; an all-zero group has s = 0 and codes 0.  x^_i = q_i * s.         */
+/* ------------------------------------------------------------------------ */
+static float int4_group(const float *x, int G, int8_t *q)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < G; i++)
+        if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+    float s = amax / 7.0f;
+    for (int i = 0; i < G; i++) {
+        float v = (s == 0.0f) ? 0.0f : nearbyintf(x[i] / s);
+        if (v > 7.0f) v = 7.0f;
+        if (v < -7.0f) v = -7.0f;
+        q[i] = (int8_t)v;
+    }
+    return s;
+}
+
+int fp4o_int4_quantize_f32(const float *x, int64_t rows, int64_t cols, int group, int8_t *q,
+                           float *scales)
+{
+    if (rows < 0 || cols < 0 || group < 2 || cols % group) return -1;
+    const int64_t ng = cols / group;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t g = 0; g < ng; g++)
+            scales[r * ng + g] = int4_group(x + r * cols + g * group, group, q + r * cols + g * group);
+    return 0;
+}
+
+int fp4o_int4_dequantize(const int8_t *q, const float *scales, int64_t rows, int64_t cols, int group,
+                         float *out)
+{
+    if (rows < 0 || cols < 0 || group < 2 || cols % group) return -1;
+    const int64_t ng = cols / group;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) out[r * cols + c] = (float)q[r * cols + c] * scales[r * ng + c / group];
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The TransFP4 method as the page's numerical experiment runs it ([TransFP4] */
+/* §2.3 Eq.(2)-(3), §3.1): rotate every k-chunk (H_k; the page uses k = 32),  */
+/* take the largest-magnitude value of each 32-value unit out as the bf16     */
+/* residual lane, and quantize each unit with the better of two candidates   */
+/* by its block error: NVFP4 (two 16-blocks, absmax E4M3 scales under the    */
+/* tensor scale s_g of the remaining values) or INT4 (one 32-value group).   */
+/* Per unit: e_c = sum (y_i - y^_i)^2 in fp64 over the unit's rotated values  */
+/* y (the residual position zeroed); INT4 only if its e is strictly smaller  */
+/* (NVFP4 always with allow_int4 = 0).  x^ = the chosen reconstruction plus  */
+/* the residual value at its position, rotated back.  choice[u] = 0 NVFP4,    */
+/* 1 INT4.  The per-unit 2-bit format tag of the page's IR is this choice.    */
+/* ------------------------------------------------------------------------ */
+int fp4o_transfp4_f32(const float *x, int64_t rows, int64_t cols, int hadamard_k, int tie,
+                      int allow_int4, float *out, uint8_t *choice)
+{
+    if (!valid_shape(FP4O_NVFP4, 16, hadamard_k, rows, cols) || cols % 32) return -1;
+    float *y = (float *)malloc(sizeof(float) * (size_t)(cols ? cols : 1));
+    uint32_t *res = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)(cols / 32 + 1));
+    if (!y || !res) {
+        free(y);
+        free(res);
+        return -1;
+    }
+    /* s_g of the FP4 stream: the maximum over the values left after the
+     * residual lane */
+    float amax_t = 0.0f;
+    for (int64_t r = 0; r < rows; r++) {
+        load_row(NULL, x, cols, r, cols, hadamard_k, y);
+        extract_residuals(y, cols, NULL);
+        for (int64_t c = 0; c < cols; c++)
+            if (fabsf(y[c]) > amax_t) amax_t = fabsf(y[c]);
+    }
+    const float sg = nv_global_scale(amax_t);
+    for (int64_t r = 0; r < rows; r++) {
+        load_row(NULL, x, cols, r, cols, hadamard_k, y);
+        extract_residuals(y, cols, res);
+        float *o = out + r * cols;
+        for (int64_t u = 0; u < cols / 32; u++) {
+            const float *v = y + u * 32;
+            float nv[32], i4[32];
+            for (int b = 0; b < 2; b++) {
+                int codes[16];
+                const int sb = absmax_scale_byte(v + 16 * b, 16, FP4O_NVFP4, FP4O_MX_CEIL, sg);
+                encode_block(v + 16 * b, 16, FP4O_NVFP4, sb, sg, tie, codes);
+                const float d = sg * (float)fp4o_e4m3_decode(sb);
+                for (int i = 0; i < 16; i++) nv[16 * b + i] = d * (float)fp4o_e2m1_decode(codes[i]);
+            }
+            int8_t q4[32];
+            const float s4 = int4_group(v, 32, q4);
+            for (int i = 0; i < 32; i++) i4[i] = (float)q4[i] * s4;
+            double e_nv = 0.0, e_i4 = 0.0;
+            for (int i = 0; i < 32; i++) {
+                e_nv += ((double)v[i] - nv[i]) * ((double)v[i] - nv[i]);
+                e_i4 += ((double)v[i] - i4[i]) * ((double)v[i] - i4[i]);
+            }
+            const int pick = allow_int4 && e_i4 < e_nv;
+            choice[r * (cols / 32) + u] = (uint8_t)pick;
+            for (int i = 0; i < 32; i++) o[u * 32 + i] = pick ? i4[i] : nv[i];
+            o[u * 32 + ((res[u] >> 16) & 31)] += bf16_to_f32((uint16_t)(res[u] & 0xFFFFu));
+        }
+        if (hadamard_k)
+            for (int64_t c = 0; c < cols; c += hadamard_k) fp4o_fwht(o + c, hadamard_k);
+    }
+    free(y);
+    free(res);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Scale tile layout consumed by the block-scaled tensor-core MMA: 512-byte   */
 /* atoms of 128 rows x 4 scale columns; atoms ordered row-block major, then  */
 /* scale-column block.  Inside an atom, row r and column j sit at byte       */

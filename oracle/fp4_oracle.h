@@ -98,7 +98,23 @@ int fp4o_dequantize(const uint8_t *q, const uint8_t *s_logical, float gscale,
 int fp4o_mx_scales_to_nv(const uint8_t *s_mx, int64_t rows, int64_t nkb, uint8_t *s_nv,
                          float *gscale);
 
-/* logical scales (rows x nkb) -> tcgen05 scale-atom layout
+/* INT4 group quantization (Table 5's INT4 baseline): per group of `group`
+ * values, fp32 scale amax / 7 and codes round(x / s) in [-7, 7] (ties to
+ * even); q is rows x cols int8, scales rows x cols/group fp32. */
+int fp4o_int4_quantize_f32(const float *x, int64_t rows, int64_t cols, int group, int8_t *q,
+                           float *scales);
+int fp4o_int4_dequantize(const int8_t *q, const float *scales, int64_t rows, int64_t cols, int group,
+                         float *out);
+
+/* The TransFP4 method of the page's Table 5 on fp32 rows: H_k, the residual
+ * lane (one value per 32), and per 32-value unit the better of an NVFP4 and
+ * an INT4 candidate by squared error (see the function's comment).  out:
+ * rows x cols fp32 reconstruction in the original domain; choice: rows x
+ * cols/32 bytes, 0 = NVFP4, 1 = INT4. */
+int fp4o_transfp4_f32(const float *x, int64_t rows, int64_t cols, int hadamard_k, int tie,
+                      int allow_int4, float *out, uint8_t *choice);
+
+/* logical scales (rows x nkb) -> tcgen05 scale-atom layout/* logical scales (rows x nkb) -> tcgen05 scale-atom layout
  * (pad128(rows) x pad4(nkb) bytes, padding bytes 0), and back. */
 void fp4o_scales_to_atoms(const uint8_t *s_logical, int64_t rows, int64_t nkb,
                           uint8_t *s_atoms);
