@@ -429,7 +429,8 @@ def test_table5_nmse_directional(orc):
             q, s, sg = orc.quantize(x, fmt, hadamard_k=k)
             got[name] = orc.nmse(xb, orc.dequantize(q, s, sg, fmt, hadamard_k=k))
         assert got["nvfp4"] < got["rot_mxfp4"] < got["mxfp4"]
-        for m, v in want.items():
+        for m in got:  # the INT4 / TransFP4 rows are pinned in test_oracle_transfp4_pins.py
+            v = want[m]
             assert v / 2 < got[m] < v * 2, (key, m, got[m], v)
 
 

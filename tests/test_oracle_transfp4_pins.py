@@ -15,10 +15,25 @@ oracle here, apart from its own arithmetic:
     round trip, bit for bit;
   - the method ordering of Table 5 for both tensors.
 """
+import os
+
 import numpy as np
 import pytest
 
 from fp4_microscaling_quantization_b200 import inputs
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def printed_table5():
+    """(tensor, method) -> NMSE as printed in Table 5 (tests/golden/table5_nmse.txt)."""
+    out = {}
+    with open(os.path.join(GOLD, "table5_nmse.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                key, method, v = line.split()
+                out[(key, method)] = float(v)
+    return out
 
 
 def _x(rows, cols, seed):
@@ -72,11 +87,10 @@ def _table5_means(orc, gen, seeds):
     return float(np.mean(i4)), float(np.mean(t4))
 
 
-@pytest.mark.parametrize("kind,printed_int4,printed_transfp4", [
-    ("activation", 0.02690, 0.00460),   # Table 5: activations, 1 % outliers
-    ("weight", 0.01864, 0.00519),       # Table 5: weights, 0.3 % outliers
-])
-def test_table5_int4_and_transfp4(orc, kind, printed_int4, printed_transfp4):
+@pytest.mark.parametrize("kind,key", [("activation", "act_1pct"), ("weight", "w_0.3pct")])
+def test_table5_int4_and_transfp4(orc, kind, key):
+    printed = printed_table5()
+    printed_int4, printed_transfp4 = printed[(key, "int4")], printed[(key, "transfp4")]
     gen = inputs.table5_activation if kind == "activation" else inputs.table5_weight
     i4, t4 = _table5_means(orc, gen, range(500, 504))
     assert abs(i4 / printed_int4 - 1) < 0.05, i4
