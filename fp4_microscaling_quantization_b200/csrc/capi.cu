@@ -98,7 +98,11 @@ fp4_status fp4_quantize_sizes(int64_t rows, int64_t cols, int fmt, int block, si
     if (rows < 0 || cols < 0 || !q_bytes || !s_bytes) return FP4_ERR_INVALID_ARG;
     if (!valid_fmt(fmt, block)) return FP4_ERR_UNSUPPORTED;
     if (cols % block) return FP4_ERR_UNSUPPORTED;
+    // byte counts must fit in 63 bits: rows * cols/2 and the padded scale tile
+    if (rows > 0 && cols / 2 > (INT64_MAX - 127) / rows) return FP4_ERR_INVALID_ARG;
     const int64_t nkb = cols / block;
+    if ((rows + 127) / 128 * 128 > 0 && (nkb + 3) / 4 * 4 > INT64_MAX / ((rows + 127) / 128 * 128))
+        return FP4_ERR_INVALID_ARG;
     *q_bytes = (size_t)(rows * (cols / 2));
     *s_bytes = (size_t)(((rows + 127) / 128 * 128) * ((nkb + 3) / 4 * 4));
     return FP4_OK;
@@ -188,6 +192,7 @@ fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, siz
 {
     if (M < 0 || N < 0 || K < 0 || !bytes) return FP4_ERR_INVALID_ARG;
     if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP4_ERR_UNSUPPORTED;  // as fp4_gemm
     *bytes = fp4::gemm_workspace_bytes(M, N, K, fmt, sm_count());
     return FP4_OK;
 }
@@ -247,6 +252,7 @@ fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, s
 {
     if (M < 0 || N < 0 || K < 0 || !bytes) return FP4_ERR_INVALID_ARG;
     if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP4_ERR_UNSUPPORTED;  // as fp4_gemm
     *bytes = linear_layout(M, N, K, fmt, sm_count()).total;
     return FP4_OK;
 }
@@ -268,6 +274,7 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (K % 32 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
     if (too_many_units(M, K)) return FP4_ERR_UNSUPPORTED;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return FP4_ERR_UNSUPPORTED;  // as fp4_gemm
     if (M == 0 || N == 0) return FP4_OK;
     if (!x || !Wq || !Ws || !C || !workspace) return FP4_ERR_INVALID_ARG;
     if (fmt == FP4_NVFP4 && !gW) return FP4_ERR_INVALID_ARG;

@@ -202,7 +202,8 @@ fp4_status fp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int fmt,
  * Rotated operands: quantize both A and W with the same hadamard_k;
  * (X H)(W H)^T = X W^T, so C needs no correction.
  * M <= 16 runs the decode (weight-streaming, split-K) kernel; larger M the
- * tiled tensor-core kernel.
+ * tiled tensor-core kernel.  M, N and K above 2^30 return FP4_ERR_UNSUPPORTED
+ * (also from the workspace-size queries and fp4_linear).
  */
 fp4_status fp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA,
                     const uint8_t *Wq, const uint8_t *Ws, const float *gW,

@@ -54,6 +54,10 @@ def test_quantize_sizes(L):
     assert L.fp4_quantize_sizes(4, 64, 2, 32, ctypes.byref(q), ctypes.byref(s)) == 2  # MXFP4_16 is 16
     assert L.fp4_quantize_sizes(4, 64, 0, 8, ctypes.byref(q), ctypes.byref(s)) == 2
     assert L.fp4_quantize_sizes(-1, 64, 0, 32, ctypes.byref(q), ctypes.byref(s)) == 1
+    # byte counts that do not fit in 63 bits are rejected, not wrapped
+    assert L.fp4_quantize_sizes(1 << 40, 1 << 30, 0, 32, ctypes.byref(q), ctypes.byref(s)) == 1
+    assert L.fp4_quantize_sizes(1 << 31, 1 << 32, 1, 16, ctypes.byref(q), ctypes.byref(s)) == 0
+    assert q.value == (1 << 31) * (1 << 31) and s.value == (1 << 31) * (1 << 28)
 
 
 FAKE = 0x10000  # an aligned pointer value never dereferenced: validation fails first
@@ -114,6 +118,15 @@ def test_gemm_rejects_on_host(L):
     assert g(None, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 8, None, 0, None) == 1
     assert g(FAKE, FAKE, None, FAKE, FAKE, FAKE, 4, 8, 256, 1, 1, FAKE, 8, None, 0, None) == 1
     assert g(FAKE + 2, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 256, 0, 1, FAKE, 8, None, 0, None) == 3
+
+
+def test_sizes_beyond_2_30_rejected(L):
+    b = ctypes.c_size_t()
+    assert L.fp4_gemm_workspace_size(4, (1 << 30) + 1, 256, 0, ctypes.byref(b)) == 2
+    assert L.fp4_linear_workspace_size(4, 256, (1 << 31), 1, ctypes.byref(b)) == 2
+    assert L.fp4_linear_workspace_size(4, 256, 1024, 2, ctypes.byref(b)) == 0 and b.value > 0
+    F = FAKE
+    assert L.fp4_linear(F, 4, 1 << 31, 1 << 31, 0, 0, None, None, F, F, F, 8, 1, F, 8, F, 1 << 20, None) == 2
 
 
 def test_gemm_quantized_rejects_on_host(L):
