@@ -37,6 +37,46 @@ def _stream_handle(torch, device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _dev(t, name: str, device, dtype=None, min_bytes: int = 0, contiguous: bool = True):
+    """Checks a tensor whose device pointer goes to the library: a CUDA tensor
+    on `device`, of `dtype`, contiguous, holding at least `min_bytes` bytes.
+    The library sees only the pointer, so a host tensor or a short buffer
+    would otherwise be read or written out of bounds on the device."""
+    import torch
+
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() * t.element_size() < min_bytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, {min_bytes} needed")
+    return t
+
+
+def _operand(t3, rows: int, cols: int, fmt: int, name: str, device):
+    """A quantized operand (q, s, g) of a rows x cols tensor in format fmt."""
+    import torch
+
+    q, s, g = t3
+    qb, sb = quantize_sizes(rows, cols, fmt)
+    _dev(q, name + " elements", device, torch.uint8, qb)
+    _dev(s, name + " scales", device, torch.uint8, sb)
+    _dev(g, name + " tensor scale", device, torch.float32, 4)
+    return q, s, g
+
+
+def _out2d(out, rows: int, cols: int, dtype, name: str, device):
+    """A row-major output of at least rows x cols (its row stride is passed on)."""
+    _dev(out, name, device, dtype, contiguous=False)
+    if out.dim() != 2 or out.shape[0] < rows or out.shape[1] < cols or (out.numel() and out.stride(1) != 1):
+        raise ValueError(f"{name} must be a 2-D tensor of at least {rows} x {cols}, contiguous along its rows")
+    return out
+
+
 def quantize_sizes(rows: int, cols: int, fmt) -> tuple[int, int]:
     fmt = _fmt(fmt)
     qb, sb = ctypes.c_size_t(), ctypes.c_size_t()
@@ -71,6 +111,9 @@ def quantize(x, fmt, hadamard_k: int = 0, round: int = FP4_ROUND_EVEN,
         g = torch.ones((1,), dtype=torch.float32, device=x.device)
     else:
         q, s, g = out
+        _dev(q, "q", x.device, torch.uint8, qb)
+        _dev(s, "s", x.device, torch.uint8, sb)
+        _dev(g, "g", x.device, torch.float32, 4)
     given = gscale is not None
     if given:
         g.copy_(gscale.reshape(1).to(torch.float32))
@@ -90,8 +133,10 @@ def dequantize(q, s, g, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_F32, 
     rows, half = q.shape
     cols = half * 2
     dt = torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16
+    _operand((q, s, g), rows, cols, fmt, "x", q.device)
     if out is None:
         out = torch.empty((rows, cols), dtype=dt, device=q.device)
+    _dev(out, "out", q.device, dt, rows * cols * (4 if dt == torch.float32 else 2))
     gp = g.data_ptr() if fmt == FP4_NVFP4 else None
     _lib.check("fp4_dequantize", _lib.lib().fp4_dequantize(
         q.data_ptr(), s.data_ptr(), gp, rows, cols, fmt, block_of(fmt), int(hadamard_k), int(out_dtype),
@@ -111,14 +156,18 @@ def gemm(a, w, M: int, N: int, K: int, fmt, out_dtype: int = FP4_OUT_BF16, out=N
     import torch
 
     fmt = _fmt(fmt)
-    Aq, As, gA = a
-    Wq, Ws, gW = w
+    dev = a[0].device
+    Aq, As, gA = _operand(a, M, K, fmt, "A", dev)
+    Wq, Ws, gW = _operand(w, N, K, fmt, "W", dev)
     dt = torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16
     if out is None:
         out = torch.empty((M, N), dtype=dt, device=Aq.device)
+    _out2d(out, M, N, dt, "out", dev)
     need = gemm_workspace_size(M, N, K, fmt)
     if need and workspace is None:
         workspace = torch.empty((need,), dtype=torch.uint8, device=Aq.device)
+    if workspace is not None:
+        _dev(workspace, "workspace", dev, torch.uint8)
     wp = workspace.data_ptr() if workspace is not None else None
     wb = workspace.numel() if workspace is not None else 0
     _lib.check("fp4_gemm", _lib.lib().fp4_gemm(
@@ -140,8 +189,9 @@ def gemm_quantized(a, w, M: int, N: int, K: int, fmt, out_fmt, gscale=None, roun
     import torch
 
     fmt, out_fmt = _fmt(fmt), _fmt(out_fmt)
-    Aq, As, gA = a
-    Wq, Ws, gW = w
+    dev = a[0].device
+    Aq, As, gA = _operand(a, M, K, fmt, "A", dev)
+    Wq, Ws, gW = _operand(w, N, K, fmt, "W", dev)
     qb, sb = quantize_sizes(M, N, out_fmt)
     if out is None:
         Cq = torch.empty((M, N // 2), dtype=torch.uint8, device=Aq.device)
@@ -149,6 +199,7 @@ def gemm_quantized(a, w, M: int, N: int, K: int, fmt, out_fmt, gscale=None, roun
         gC = torch.ones((1,), dtype=torch.float32, device=Aq.device)
     else:
         Cq, Cs, gC = out
+        _operand(out, M, N, out_fmt, "C", dev)
     if gscale is not None:
         gC.copy_(gscale.reshape(1).to(torch.float32))
     opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(gscale is not None))
@@ -192,6 +243,8 @@ def dequantize_residual(q, s, g, res, fmt, hadamard_k: int = 0, out_dtype: int =
 
     fmt = _fmt(fmt)
     rows, cols = q.shape[0], q.shape[1] * 2
+    _operand((q, s, g), rows, cols, fmt, "x", q.device)
+    _dev(res, "res", q.device, None, rows * (cols // 32) * 4)
     out = torch.empty((rows, cols), dtype=torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16,
                       device=q.device)
     _lib.check("fp4_dequantize_residual", _lib.lib().fp4_dequantize_residual(
@@ -232,6 +285,7 @@ def mx_to_nv(w):
 
     q, s, _ = w
     rows, cols = q.shape[0], q.shape[1] * 2
+    _dev(s, "MXFP4 scales", q.device, torch.uint8, quantize_sizes(rows, cols, FP4_MXFP4)[1])
     _, sb = quantize_sizes(rows, cols, FP4_NVFP4)
     s_nv = torch.empty((sb,), dtype=torch.uint8, device=q.device)
     g = torch.empty((1,), dtype=torch.float32, device=q.device)
@@ -259,14 +313,19 @@ def linear(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale
     fmt = _fmt(fmt)
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be a 2-D bf16 tensor, contiguous along K")
-    Wq, Ws, gW = w
+    _dev(x, "x", None, torch.bfloat16, contiguous=False)
     M, K = x.shape
-    N = Wq.shape[0]
+    N = w[0].shape[0]
+    Wq, Ws, gW = _operand(w, N, K, fmt, "W", x.device)
+    if gscale is not None:
+        _dev(gscale, "gscale", x.device, torch.float32, 4)
     dt = torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16
     if out is None:
         out = torch.empty((M, N), dtype=dt, device=x.device)
+    _out2d(out, M, N, dt, "out", x.device)
     if workspace is None:
         workspace = torch.empty((linear_workspace_size(M, N, K, fmt),), dtype=torch.uint8, device=x.device)
+    _dev(workspace, "workspace", x.device, torch.uint8)
     opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), 0, 0, int(bool(weights_static)))
     _lib.check("fp4_linear", _lib.lib().fp4_linear(
         x.data_ptr(), M, K, x.stride(0), fmt, int(hadamard_k), ctypes.byref(opts),

@@ -168,3 +168,29 @@ def test_refine_rejects_on_host(L):
 def test_empty_mx_is_noop(L):
     assert L.fp4_quantize(None, 0, 64, 64, 0, 32, 0, None, None, None, None, None) == 0
     assert L.fp4_dequantize(None, None, None, 0, 64, 0, 32, 0, 0, None, None) == 0
+
+
+def test_binding_refuses_host_tensors():
+    """The Python binding passes raw device pointers: a host tensor (or a short
+    buffer) is refused before anything reaches the library."""
+    import torch
+    import fp4_microscaling_quantization_b200 as fp4
+    M, N, K = 4, 256, 512
+    qa = torch.zeros((M, K // 2), dtype=torch.uint8)
+    sa = torch.zeros((fp4.quantize_sizes(M, K, 0)[1],), dtype=torch.uint8)
+    qw = torch.zeros((N, K // 2), dtype=torch.uint8)
+    sw = torch.zeros((fp4.quantize_sizes(N, K, 0)[1],), dtype=torch.uint8)
+    g = torch.ones((1,), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fp4.gemm((qa, sa, g), (qw, sw, g), M, N, K, 0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fp4.gemm_quantized((qa, sa, g), (qw, sw, g), M, N, K, 0, 0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fp4.dequantize(qa, sa, g, 0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fp4.linear(torch.zeros((M, K), dtype=torch.bfloat16), (qw, sw, g), 0)
+    with pytest.raises(ValueError):
+        fp4.quantize(torch.zeros((M, K), dtype=torch.bfloat16), 0)
+    # shapes the library rejects are refused while sizing the operands
+    with pytest.raises(fp4.Fp4Error):
+        fp4.gemm((qa, sa, g), (qw, sw, g), M, N, 100, 0)
