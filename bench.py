@@ -30,10 +30,10 @@ sys.path.insert(0, ROOT)
 
 ROWS, COLS = 1024, 131072
 
-# DRAM bytes (read + write) per launch of the roofline kernel at 1024 x 131072,
-# from the ncu capture summarised in profiles/quantize_kernel_mx_512x131072_full.md
-# (512-row capture scaled by rows).  Set to None whenever that kernel changes,
-# until it is captured again.
+# DRAM bytes (read + write) per launch of the roofline kernel at 1024 x 131072:
+# dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of the MXFP4
+# quantize kernel on 512 rows of this workload, scaled by rows.  Set to None
+# whenever that kernel changes, until it is captured again.
 QUANT_MX_TRAFFIC_BYTES = 304.1e6
 WORKLOAD = "quantize sweep 1024x131072 bf16 Student-t(3)+1% outliers x20: MXFP4 + NVFP4 quantize and dequantize"
 METRIC = "FP4 quantize GB/s (% HBM peak)"

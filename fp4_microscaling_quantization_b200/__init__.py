@@ -37,6 +37,17 @@ def _stream_handle(torch, device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _run(name: str, device, *args) -> None:
+    """Calls entry point `name` of the library with `device` current.  The
+    library launches on the current device and takes the SM count and the
+    scratch it uses from it, so that must be the device whose memory and
+    stream the call is given."""
+    import torch
+
+    with torch.cuda.device(device):
+        _lib.check(name, getattr(_lib.lib(), name)(*args))
+
+
 def _dev(t, name: str, device, dtype=None, min_bytes: int = 0, contiguous: bool = True):
     """Checks a tensor whose device pointer goes to the library: a CUDA tensor
     on `device`, of `dtype`, contiguous, holding at least `min_bytes` bytes.
@@ -119,9 +130,9 @@ def quantize(x, fmt, hadamard_k: int = 0, round: int = FP4_ROUND_EVEN,
         g.copy_(gscale.reshape(1).to(torch.float32))
     opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(given), int(scale_search))
     gp = g.data_ptr() if fmt == FP4_NVFP4 else None
-    _lib.check("fp4_quantize", _lib.lib().fp4_quantize(
+    _run("fp4_quantize", x.device,
         x.data_ptr(), rows, cols, x.stride(0), fmt, block_of(fmt), int(hadamard_k), ctypes.byref(opts),
-        q.data_ptr(), s.data_ptr(), gp, _stream_handle(torch, x.device)))
+        q.data_ptr(), s.data_ptr(), gp, _stream_handle(torch, x.device))
     return q, s, g
 
 
@@ -138,9 +149,9 @@ def dequantize(q, s, g, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_F32, 
         out = torch.empty((rows, cols), dtype=dt, device=q.device)
     _dev(out, "out", q.device, dt, rows * cols * (4 if dt == torch.float32 else 2))
     gp = g.data_ptr() if fmt == FP4_NVFP4 else None
-    _lib.check("fp4_dequantize", _lib.lib().fp4_dequantize(
+    _run("fp4_dequantize", q.device,
         q.data_ptr(), s.data_ptr(), gp, rows, cols, fmt, block_of(fmt), int(hadamard_k), int(out_dtype),
-        out.data_ptr(), _stream_handle(torch, q.device)))
+        out.data_ptr(), _stream_handle(torch, q.device))
     return out
 
 
@@ -170,10 +181,10 @@ def gemm(a, w, M: int, N: int, K: int, fmt, out_dtype: int = FP4_OUT_BF16, out=N
         _dev(workspace, "workspace", dev, torch.uint8)
     wp = workspace.data_ptr() if workspace is not None else None
     wb = workspace.numel() if workspace is not None else 0
-    _lib.check("fp4_gemm", _lib.lib().fp4_gemm(
+    _run("fp4_gemm", Aq.device,
         Aq.data_ptr(), As.data_ptr(), gA.data_ptr(), Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(),
         M, N, K, fmt, int(out_dtype), out.data_ptr(), out.stride(0), wp, wb,
-        _stream_handle(torch, Aq.device)))
+        _stream_handle(torch, Aq.device))
     return out
 
 
@@ -203,10 +214,10 @@ def gemm_quantized(a, w, M: int, N: int, K: int, fmt, out_fmt, gscale=None, roun
     if gscale is not None:
         gC.copy_(gscale.reshape(1).to(torch.float32))
     opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(gscale is not None))
-    _lib.check("fp4_gemm_quantized", _lib.lib().fp4_gemm_quantized(
+    _run("fp4_gemm_quantized", Aq.device,
         Aq.data_ptr(), As.data_ptr(), gA.data_ptr(), Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(),
         M, N, K, fmt, out_fmt, ctypes.byref(opts), gC.data_ptr() if out_fmt == FP4_NVFP4 else None,
-        Cq.data_ptr(), Cs.data_ptr(), _stream_handle(torch, Aq.device)))
+        Cq.data_ptr(), Cs.data_ptr(), _stream_handle(torch, Aq.device))
     return Cq, Cs, gC
 
 
@@ -230,10 +241,10 @@ def quantize_residual(x, fmt, hadamard_k: int = 0, round: int = FP4_ROUND_EVEN,
     if given:
         g.copy_(gscale.reshape(1).to(torch.float32))
     opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), int(given), 0, 0)
-    _lib.check("fp4_quantize_residual", _lib.lib().fp4_quantize_residual(
+    _run("fp4_quantize_residual", x.device,
         x.data_ptr(), rows, cols, x.stride(0), fmt, block_of(fmt), int(hadamard_k), ctypes.byref(opts),
         q.data_ptr(), s.data_ptr(), g.data_ptr() if fmt == FP4_NVFP4 else None, res.data_ptr(),
-        _stream_handle(torch, x.device)))
+        _stream_handle(torch, x.device))
     return q, s, g, res
 
 
@@ -247,9 +258,9 @@ def dequantize_residual(q, s, g, res, fmt, hadamard_k: int = 0, out_dtype: int =
     _dev(res, "res", q.device, None, rows * (cols // 32) * 4)
     out = torch.empty((rows, cols), dtype=torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16,
                       device=q.device)
-    _lib.check("fp4_dequantize_residual", _lib.lib().fp4_dequantize_residual(
+    _run("fp4_dequantize_residual", q.device,
         q.data_ptr(), s.data_ptr(), g.data_ptr() if fmt == FP4_NVFP4 else None, res.data_ptr(), rows, cols, fmt,
-        block_of(fmt), int(hadamard_k), int(out_dtype), out.data_ptr(), _stream_handle(torch, q.device)))
+        block_of(fmt), int(hadamard_k), int(out_dtype), out.data_ptr(), _stream_handle(torch, q.device))
     return out
 
 
@@ -272,9 +283,9 @@ def nv_refine_gscale(x, hadamard_k: int = 0, rounds: int = 4, round: int = FP4_R
     ws = torch.empty((nb.value,), dtype=torch.uint8, device=x.device)
     g = torch.empty((1,), dtype=torch.float32, device=x.device)
     opts = _lib.Fp4Opts(int(round), 0, 0, 0, 0)
-    _lib.check("fp4_nv_refine_gscale", _lib.lib().fp4_nv_refine_gscale(
+    _run("fp4_nv_refine_gscale", x.device,
         x.data_ptr(), rows, cols, x.stride(0), int(hadamard_k), ctypes.byref(opts), int(rounds), q.data_ptr(),
-        s.data_ptr(), ws.data_ptr(), nb.value, g.data_ptr(), _stream_handle(torch, x.device)))
+        s.data_ptr(), ws.data_ptr(), nb.value, g.data_ptr(), _stream_handle(torch, x.device))
     return g
 
 
@@ -289,8 +300,8 @@ def mx_to_nv(w):
     _, sb = quantize_sizes(rows, cols, FP4_NVFP4)
     s_nv = torch.empty((sb,), dtype=torch.uint8, device=q.device)
     g = torch.empty((1,), dtype=torch.float32, device=q.device)
-    _lib.check("fp4_mx_to_nv_scales", _lib.lib().fp4_mx_to_nv_scales(
-        s.data_ptr(), rows, cols, s_nv.data_ptr(), g.data_ptr(), _stream_handle(torch, q.device)))
+    _run("fp4_mx_to_nv_scales", q.device,
+        s.data_ptr(), rows, cols, s_nv.data_ptr(), g.data_ptr(), _stream_handle(torch, q.device))
     return q, s_nv, g
 
 
@@ -327,11 +338,11 @@ def linear(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale
         workspace = torch.empty((linear_workspace_size(M, N, K, fmt),), dtype=torch.uint8, device=x.device)
     _dev(workspace, "workspace", x.device, torch.uint8)
     opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), 0, 0, int(bool(weights_static)))
-    _lib.check("fp4_linear", _lib.lib().fp4_linear(
+    _run("fp4_linear", x.device,
         x.data_ptr(), M, K, x.stride(0), fmt, int(hadamard_k), ctypes.byref(opts),
         gscale.data_ptr() if gscale is not None else None, Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(), N,
         int(out_dtype), out.data_ptr(), out.stride(0), workspace.data_ptr(), workspace.numel(),
-        _stream_handle(torch, x.device)))
+        _stream_handle(torch, x.device))
     return out
 
 

@@ -24,6 +24,8 @@
 
 #include <atomic>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "encode.cuh"
 #include "sm100.cuh"
@@ -909,6 +911,23 @@ static bool make_sf_map(CUtensorMap *m, const void *base, int64_t nkb4, int64_t 
     return r == CUDA_SUCCESS;
 }
 
+// Raises a kernel's dynamic shared-memory limit on the current device.  The
+// attribute belongs to the device's context, so it is set once per (kernel,
+// device) pair; the set of pairs done is guarded for calls from several host
+// threads.
+static cudaError_t set_smem_limit(const void *kern, int bytes)
+{
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kern, dev})) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert({kern, dev});
+    return e;
+}
+
 template <int FMT, int OUT, int CG>
 static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Wq, const uint8_t *Ws,
                                 const PParams &p, int sms, cudaStream_t st, bool pdl)
@@ -921,12 +940,8 @@ static cudaError_t launch_pgemm(const uint8_t *Aq, const uint8_t *As, const uint
         !make_sf_map(&tsa, As, p.nkb4, nrb_a, KA) || !make_sf_map(&tsb, Ws, p.nkb4, nrb_w, KA))
         return cudaErrorInvalidValue;
     auto kern = pgemm_kernel<FMT, OUT, CG>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    if (cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), Cfg::SMEM_BYTES); e != cudaSuccess)
+        return e;
     const int tiles = p.num_m_tiles * p.num_n_tiles;
     const int groups = tiles < sms / CG ? tiles : sms / CG;
     cudaLaunchConfig_t cfg = {};
@@ -990,12 +1005,8 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
                                  const CUtensorMap &tsa, const decode::Params &p, bool any_cut, cudaStream_t st, bool pdl)
 {
     auto kern = decode::decode_kernel<FMT>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, decode::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    if (cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), decode::SMEM_BYTES); e != cudaSuccess)
+        return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
     cfg.blockDim = dim3(decode::DECODE_THREADS);

@@ -703,13 +703,20 @@ static void (*act_kernel_for(int hk))(QuantArgs, unsigned *, int, int)
 
 // Cluster size of the activation quantizer: ACT_CTAS (a non-portable size)
 // where the device schedules such clusters, else the portable ACT_CTAS_PORTABLE.
-// Decided once per kernel instance.
+// Decided once per kernel instance and device (the attribute it sets belongs
+// to the current device's context).
 static int act_cluster_size(void (*k)(QuantArgs, unsigned *, int, int))
 {
     static std::mutex mu;
-    static std::map<const void *, int> sizes;
+    static std::map<std::pair<const void *, int>, int> sizes;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return ACT_CTAS_PORTABLE;
+    }
+    const std::pair<const void *, int> key(reinterpret_cast<const void *>(k), dev);
     std::lock_guard<std::mutex> lock(mu);
-    auto it = sizes.find(reinterpret_cast<const void *>(k));
+    auto it = sizes.find(key);
     if (it != sizes.end()) return it->second;
     int n = ACT_CTAS_PORTABLE;
     bool refused = false;  // a refused call leaves its error for cudaGetLastError: clear only ours
@@ -733,7 +740,7 @@ static int act_cluster_size(void (*k)(QuantArgs, unsigned *, int, int))
             n = ACT_CTAS;
     }
     if (refused) cudaGetLastError();
-    sizes[reinterpret_cast<const void *>(k)] = n;
+    sizes[key] = n;
     return n;
 }
 

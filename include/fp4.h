@@ -328,8 +328,11 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
  *   FP4_ERR_UNSUPPORTED (nothing launched).
  *   The array is a device variable: every GPU that loads the library holds
  *   4 MiB for it until the process exits.  The first call on a device looks
- *   up the array's device address (with that device current); make that first
- *   call before any stream capture.  All calls share the array: calls whose
+ *   up the array's device address (with that device current) and keeps it
+ *   for the life of the process; make that first call before any stream
+ *   capture.  A cudaDeviceReset (or any other teardown of the device's
+ *   primary context) makes the kept address stale: after one, this entry
+ *   point must not be called again in the same process.  All calls share the array: calls whose
  *   kernels overlap on the GPU (different streams without ordering) race and
  *   give wrong results.  Nothing in it needs to start at zero; it keeps the
  *   last call's partial sums.
@@ -344,7 +347,10 @@ fp4_status fp4_gemm_decode_noalloc(const uint8_t *Aq, const uint8_t *As, const f
  * (host-side counter; diagnostics and launch accounting). */
 uint64_t fp4_kernel_launches(void);
 
-/* Failure-detection test hook.  With stall != 0 the next GEMM launch
+/* Failure-detection test hook: for tests only, not for production use, and
+ * not thread-safe.  The setting is one process-wide value that the next GEMM
+ * launch from any host thread consumes, so use it only while a single thread
+ * launches GEMMs.  With stall != 0 the next GEMM launch
  * (fp4_gemm, fp4_gemm_quantized, fp4_linear or fp4_gemm_decode_noalloc)
  * issues no operand loads,
  * so its MMA warp's bounded wait gives up after budget_ns nanoseconds
@@ -352,7 +358,7 @@ uint64_t fp4_kernel_launches(void);
  * nothing, frees its tensor memory and returns, and fp4_check_device_status()
  * then reports FP4_ERR_TIMEOUT.  The context stays usable.  A nonzero
  * budget_ns with stall == 0 only shortens the waits of the next launch.
- * Host-side, applies to one launch; not for production use. */
+ * Host-side, applies to one launch. */
 fp4_status fp4_test_inject_stall(int stall, uint64_t budget_ns);
 
 /* Reads and clears the device-side error word that kernels set when a

@@ -37,27 +37,54 @@ def noalloc_fn(fp4):
     return f
 
 
-@pytest.mark.parametrize("fmt,M,N,K", [(1, 16, 14336, 4096), (0, 4, 4096, 1024), (1, 1, 300, 512)])
-def test_noalloc_matches_workspace_entry_point(fp4, fmt, M, N, K):
+# (fmt, M, N, K, uses the array): the last case takes whole tiles and needs no
+# partial sums; the others cut tiles between CTAs (a few tiles split over many
+# CTAs, or stream-K over more tiles than SMs), so their partials go through
+# the library's array.
+CASES = [(1, 1, 300, 512, True), (0, 16, 1000, 4096, True), (2, 4, 128 * 200, 512, True),
+         (1, 16, 14336, 4096, False)]
+
+
+def operands(fp4, fmt, M, N, K, seed):
     import torch
-    f = noalloc_fn(fp4)
-    a, w = inputs.decode_linear(M, N, K, seed=M + N)
+    a, w = inputs.decode_linear(M, N, K, seed=seed)
     A = fp4.quantize(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda(), fmt)
     W = fp4.quantize(torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).cuda(), fmt)
-    ref = fp4.gemm(A, W, M, N, K, fmt, out_dtype=fp4.FP4_OUT_F32).cpu().numpy().astype(np.float64)
+    return A, W
+
+
+@pytest.mark.parametrize("fmt,M,N,K,uses_array", CASES)
+def test_noalloc_matches_workspace_entry_point(fp4, fmt, M, N, K, uses_array):
+    import torch
+    f = noalloc_fn(fp4)
+    assert (fp4.gemm_workspace_size(M, N, K, fmt) > 0) == uses_array
+    A, W = operands(fp4, fmt, M, N, K, seed=M + N)
+    # other operands of the same shape: a call with them leaves different
+    # partial sums in the shared array, so a partial that a later call failed
+    # to write would show up as a wrong result
+    A2, W2 = operands(fp4, fmt, M, N, K, seed=M + N + 7)
     # the GEMM tolerance: 1e-5 * sum_k |a_k||w_k| over the dequantized operands
     ah = fp4.dequantize(*A, fmt).cpu().numpy()
     wh = fp4.dequantize(*W, fmt).cpu().numpy()
     bound = np.abs(ah).astype(np.float64) @ np.abs(wh).astype(np.float64).T
     stream = torch.cuda.current_stream().cuda_stream
-    for call in range(2):
-        C = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
-        rc = f(A[0].data_ptr(), A[1].data_ptr(), A[2].data_ptr(), W[0].data_ptr(), W[1].data_ptr(),
-               W[2].data_ptr(), M, N, K, fmt, fp4.FP4_OUT_F32, C.data_ptr(), N, stream)
-        assert rc == 0, f"call {call}: status {rc}"
-        torch.cuda.synchronize()
-        got = C.cpu().numpy().astype(np.float64)
-        assert np.all(np.abs(got - ref) <= 1e-5 * bound), f"call {call} differs from fp4_gemm"
+
+    def call(Aop, Wop, out_dtype, C):
+        return f(Aop[0].data_ptr(), Aop[1].data_ptr(), Aop[2].data_ptr(), Wop[0].data_ptr(), Wop[1].data_ptr(),
+                 Wop[2].data_ptr(), M, N, K, fmt, out_dtype, C.data_ptr(), N, stream)
+
+    for out_dtype, dt in ((fp4.FP4_OUT_F32, torch.float32), (fp4.FP4_OUT_BF16, torch.bfloat16)):
+        ref = fp4.gemm(A, W, M, N, K, fmt, out_dtype=out_dtype).float().cpu().numpy().astype(np.float64)
+        tol = 1e-5 * bound + (2.0 ** -8 * np.abs(ref) if out_dtype == fp4.FP4_OUT_BF16 else 0.0)
+        dirty = torch.empty((M, N), dtype=dt, device="cuda")
+        assert call(A2, W2, out_dtype, dirty) == 0
+        for n in range(2):
+            C = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+            rc = call(A, W, out_dtype, C)
+            assert rc == 0, f"call {n}: status {rc}"
+            torch.cuda.synchronize()
+            got = C.float().cpu().numpy().astype(np.float64)
+            assert np.all(np.abs(got - ref) <= tol), f"call {n} ({dt}) differs from fp4_gemm"
 
 
 def test_noalloc_rejects_what_it_cannot_hold(fp4):
