@@ -15,7 +15,7 @@ from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_MXFP4_1
 
 __all__ = [
     "quantize", "dequantize", "gemm", "gemm_quantized", "linear", "linear_workspace_size", "quantize_sizes",
-    "gemm_workspace_size", "check_device_status",
+    "gemm_workspace_size", "check_device_status", "kernel_launches",
     "FP4_MXFP4", "FP4_NVFP4", "FP4_MXFP4_16", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
     "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "FP4_SCALE_ABSMAX", "FP4_SCALE_MSE",
     "Fp4Error", "block_of",
@@ -344,6 +344,11 @@ def linear(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale
         int(out_dtype), out.data_ptr(), out.stride(0), workspace.data_ptr(), workspace.numel(),
         _stream_handle(torch, x.device))
     return out
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(_lib.lib().fp4_kernel_launches())
 
 
 def check_device_status() -> None:

@@ -35,6 +35,10 @@ size_t nv_refine_workspace_bytes(int64_t rows, int64_t cols);
 cudaError_t launch_nv_refine(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int hk, float ck,
                              int round_away, int rounds, uint8_t *q, uint8_t *s, void *ws, float *gscale, int sms,
                              cudaStream_t st);
+cudaError_t launch_linear_fused(const uint16_t *x, int64_t ldx, int64_t M, int64_t K, int fmt, int hk, float ck,
+                                int round_away, int mx_floor, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
+                                const float *gW, int64_t N, int bf16out, void *C, int64_t ldc, int sms, cudaStream_t st,
+                                bool w_before_wait, bool *taken);
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -292,8 +296,17 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     unsigned *counters = decode ? reinterpret_cast<unsigned *>(base + L.counters) : nullptr;
     cudaError_t e;
     if (decode) {
-        // two launches: one cluster quantizes the activations (and zeroes the
-        // tile counters); the split-K kernel streams W meanwhile and reduces.
+        // one launch: the decode kernel quantizes the activations itself
+        // (whole-tile and cluster work splits)
+        bool taken = false;
+        e = fp4::launch_linear_fused(static_cast<const uint16_t *>(x), ld_x, M, K, fmt, hadamard_k,
+                                     hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
+                                     o.mx_scale_rule == FP4_MX_SCALE_FLOOR, fmt == FP4_NVFP4 ? gA : nullptr, Wq, Ws, gW,
+                                     N, out_dtype == FP4_OUT_BF16, C, ldc, sms, st, o.weights_static != 0, &taken);
+        if (taken) return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+        // otherwise two launches: one cluster quantizes the activations (and
+        // zeroes the tile counters); the split-K kernel streams W meanwhile
+        // and reduces.
         e = fp4::launch_act_quantize(static_cast<const uint16_t *>(x), M, K, ld_x, fmt, hadamard_k,
                                      hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
                                      o.mx_scale_rule == FP4_MX_SCALE_FLOOR, gA != nullptr, aq, as, ga, counters,

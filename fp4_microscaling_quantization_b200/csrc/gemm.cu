@@ -410,7 +410,7 @@ constexpr int A_BYTES = BNA * BK / 2;        // 2 KB
 constexpr int SFW_BYTES = 4 * 512;
 constexpr int SFA_BYTES = 4 * 512;
 constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;  // 22528 = 22 KB
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
 constexpr int TMEM_COLS = 512;
 constexpr int NI = 4;                        // MMA issuer warps
 constexpr int SF_COL0 = 2 * NI * 16;         // accumulators: buffer b, issuer j at columns 16 (NI b + j)
@@ -437,9 +437,15 @@ struct Params {
     int csize;           // > 1: the CTAs of a tile form a cluster of csize and reduce through DSMEM
     // Stream W before waiting for the preceding kernel.  Only when that
     // kernel triggers its dependents after its own wait (the decode
-    // activation quantizer), so every earlier kernel, whatever wrote W,
-    // has finished.
+    // activation quantizer, or the fused kernel of an earlier fp4_linear), so
+    // every earlier kernel, whatever wrote W, has finished.
     int w_before_wait;
+    // Fused activation quantization (fp4_linear): bf16 x, M x K, row stride
+    // ldx elements; gA null = the NVFP4 tensor scale is computed from x.
+    const uint16_t *x;
+    int64_t ldx;
+    float ck;            // RN(1/sqrt(k)) of the rotation
+    int round_away, mx_floor;
 };
 
 __host__ __device__ inline int64_t unit_begin(int c, int64_t U, int G) { return (int64_t)c * U / G; }
@@ -461,30 +467,203 @@ FP4_DEV void store_row(const Params &p, int n, const float *acc, float alpha)
 }
 
 // Threads: warp 0 loads, warps 1, 6, 7, 8 issue MMAs, warps 2-5 drain the
-// accumulators (warp w may read TMEM lanes 32 (w % 4) .. + 31).
-constexpr int DECODE_THREADS = 32 * (6 + NI - 1);
+// accumulators (warp w may read TMEM lanes 32 (w % 4) .. + 31).  The fused
+// variant (fp4_linear) adds warps 9-12: with warps 2-5 they quantize the
+// activations into the stages before the accumulators are drained.
+constexpr int NQ_EXTRA = 4;                  // warps 9 .. 12 of the fused variant
+constexpr int NQ = 4 + NQ_EXTRA;             // activation quantizer warps of the fused variant
+__host__ __device__ constexpr int decode_threads(bool fused) { return 32 * (6 + NI - 1 + (fused ? NQ_EXTRA : 0)); }
 static_assert(STAGES % NI == 0, "a stage is always issued by the same warp");
 static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "TMEM budget");
 
-template <int FMT>
-__global__ void __launch_bounds__(DECODE_THREADS, 1)
+// Quantizer warp index of warp w (fused variant): warps 2-5 -> 0-3, 9-12 -> 4-7.
+FP4_DEV int quantizer_index(int warp) { return warp <= 5 ? warp - 2 : warp - 5; }
+
+// Named barrier over the NQ quantizer warps (id 2; id 1 is the epilogue's).
+FP4_DEV void quantizers_sync() { asm volatile("bar.sync 2, %0;" ::"n"(NQ * 32) : "memory"); }
+
+// Makes this thread's generic-proxy shared-memory writes visible to the
+// tensor cores' (async-proxy) reads that follow a barrier.
+FP4_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+FP4_DEV void mbar_arrive_local(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Arrive on a barrier of another CTA of the cluster, ordering this thread's
+// earlier shared::cluster stores before it (release at cluster scope).
+FP4_DEV void mbar_arrive_remote_release(uint32_t bar_cluster)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// Bounded wait with acquire at cluster scope (sees the stores that remote
+// arrivals released).
+FP4_DEV bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity, volatile uint32_t *abort, unsigned int *err_word,
+                                       uint64_t budget_ns)
+{
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > budget_ns) {
+            *abort = 1u;
+            atomicOr(err_word, 1u);
+            return false;
+        }
+    }
+}
+
+FP4_DEV void st_shared_cluster_f32(uint32_t addr_cluster, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr_cluster), "f"(v) : "memory");
+}
+
+// Raw bf16 bytes of unit column j of activation row m (zeros for a row at or
+// past M, or a column at or past K: they quantize to zero codes and zero
+// scales, finite as the product's K tail needs).
+FP4_DEV void fetch_act_unit(const Params &p, int m, int j, uint4 *raw)
+{
+    if (m < p.M && j < p.K / 32) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (int64_t)m * p.ldx + (int64_t)j * 32);
+#pragma unroll
+        for (int c = 0; c < 4; c++) raw[c] = __ldg(src + c);
+    } else {
+#pragma unroll
+        for (int c = 0; c < 4; c++) raw[c] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// max |H_k x| over the unit columns [j0, j1) of every activation row,
+// reduced over the NQ quantizer warps (all of them call it; every one gets
+// the result).  j0 and j1 are multiples of k / 32, and consecutive lanes hold
+// consecutive units of a row, so a rotation chunk lies in neighbouring lanes.
+template <int HK>
+FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float *red)
+{
+    const int ncols = j1 - j0;
+    const int total = p.M * ncols;
+    constexpr int U = 2;  // units per lane and trip, loads issued together
+    float mx = 0.0f;
+    for (int base = qw * 32 * U; base < total; base += NQ * 32 * U) {
+        uint4 raw[U][4];
+#pragma unroll
+        for (int i = 0; i < U; i++) {
+            const int u = base + i * 32 + lane;
+            const int m = u < total ? u / ncols : p.M;
+            fetch_act_unit(p, m, j0 + (u < total ? u - m * ncols : 0), raw[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < U; i++) {
+            float v[32];
+            unpack_unit(raw[i], v);
+            if (HK) fwht_unit<HK>(v, p.ck, lane);
+            mx = fmaxf(mx, absmax_tree<32>(v));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 0) red[qw] = mx;
+    quantizers_sync();
+    float t = red[0];
+#pragma unroll
+    for (int w = 1; w < NQ; w++) t = fmaxf(t, red[w]);
+    return t;
+}
+
+// The fused activation quantizer, one warp: for every unit i = qw (mod NQ)
+// of this CTA (its K step; a CTA's units may run over into the next tile),
+// once the stage's previous MMAs are done,
+// encodes the M x 256 activation slice of that K step into stage i % STAGES
+// exactly as the TMA would have placed fp4_quantize's output there (nibble
+// rows of 128 bytes in the 128-byte swizzle; scales in the tile layout's
+// atoms), then arrives on the stage's activation barrier.  Rows past M keep the
+// zeros written at kernel start.  Returns false after an abort.
+template <int QFMT, int HK>
+FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready0, uint32_t empty0, int n_units,
+                                 int t_first, int ks_first, int qw, int lane, float sg, volatile uint32_t *abort_flag)
+{
+    const float six_sg = __fmul_rn(6.0f, sg);
+    const int nwork = p.M * 8;  // units of one K step: (row m, column cu = 0..7)
+    for (int i = qw; i < n_units; i += NQ) {
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)((i / STAGES) & 1);
+        if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) return false;
+        uint8_t *st = smem + s * STAGE_BYTES;
+        uint8_t *sa = st + W_BYTES;
+        uint8_t *sfa = st + W_BYTES + A_BYTES + SFW_BYTES;
+        const int j0 = (int)(((int64_t)t_first * p.nk + ks_first + i) % p.nk) * 8;  // K step of unit i
+        uint4 raw[BNA * 8 / 32][4];
+#pragma unroll
+        for (int r = 0; r < BNA * 8 / 32; r++) {
+            const int w = r * 32 + lane;
+            if (r * 32 < nwork) fetch_act_unit(p, w < nwork ? w >> 3 : p.M, j0 + (w & 7), raw[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < BNA * 8 / 32; r++) {
+            if (r * 32 >= nwork) break;  // warp-uniform
+            const int w = r * 32 + lane;
+            const int m = w >> 3, cu = w & 7;
+            float v[32];
+            unpack_unit(raw[r], v);
+            if (HK) fwht_unit<HK>(v, p.ck, lane);
+            uint4 nib;
+            const uint32_t sb = encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib);
+            if (w < nwork) {
+                *reinterpret_cast<uint4 *>(sa + m * 128 + ((cu ^ (m & 7)) << 4)) = nib;
+                if (QFMT == FP4_MXFP4)
+                    sfa[(cu >> 2) * 512 + m * 16 + (cu & 3)] = (uint8_t)sb;
+                else
+                    *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + m * 16 + 2 * (cu & 1)) = (uint16_t)sb;
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(aready0 + 8 * s);
+    }
+    return true;
+}
+
+// QFMT: the operands' format (MXFP4_16 runs the 16-element block-scaled MMA,
+// FMT below, with E8M0 scales).  FUSED: fp4_linear's single-launch form,
+// which quantizes the activations itself (HK: their rotation) and needs a
+// whole-tile or cluster work split; otherwise A comes quantized (fp4_gemm).
+template <int QFMT, int HK, bool FUSED>
+__global__ void __launch_bounds__(decode_threads(FUSED), 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
               const __grid_constant__ CUtensorMap tmSW, const __grid_constant__ CUtensorMap tmSA, Params p)
 {
+    constexpr int FMT = QFMT == FP4_MXFP4 ? FP4_MXFP4 : FP4_NVFP4;
     constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    // bars: full[S], empty[S], accfull[2], accempty[2], drain
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    // bars: full[S] (TMA bytes), empty[S], aready[S] (fused: the stage's
+    // activations written), accfull[2], accempty[2], drain, amax (fused)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 6);
     __shared__ volatile unsigned s_last;
+    __shared__ float s_red[NQ];             // fused: per-warp maxima
+    __shared__ float s_amax[MAX_CLUSTER];   // fused: the cluster CTAs' maxima, by rank
+    __shared__ float s_sg;                  // fused: the activation tensor scale
     volatile uint32_t *abort_flag = tmem_slot + 1;
     // cluster split: this CTA's 128 x 16 partial, [4][128][4] floats (16-byte
     // groups of one row's columns 4q..4q+3), in stage 0's W buffer, which no
     // load or MMA touches once the accumulator is complete
     float4 *part = reinterpret_cast<float4 *>(smem);
 
-    grid_dep_launch();
+    // The fused kernel lets the next launch start only after its own wait
+    // (below): by then every kernel before this one has finished, so the next
+    // one may stream static weights at once.
+    if (!FUSED) grid_dep_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
     const int64_t U = (int64_t)p.ntiles * p.nk;
@@ -495,10 +674,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const int t_first = (int)(u0 / p.nk);
     const int ks_first = (int)(u0 - (int64_t)t_first * p.nk);
     const int nseg = (int)((u1 - 1) / p.nk) - t_first + 1;
-    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
-    const uint32_t accf0 = smem_u32(bars + 2 * STAGES), acce0 = smem_u32(bars + 2 * STAGES + 2);
-    const uint32_t drainb = smem_u32(bars + 2 * STAGES + 4);
-    const uint32_t tx = W_BYTES + A_BYTES + 2 * KA * 512;
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES), aready0 = smem_u32(bars + 2 * STAGES);
+    const uint32_t accf0 = smem_u32(bars + 3 * STAGES), acce0 = smem_u32(bars + 3 * STAGES + 2);
+    const uint32_t drainb = smem_u32(bars + 3 * STAGES + 4);
+    const uint32_t amaxb = smem_u32(bars + 3 * STAGES + 5);
+    const uint32_t tx = FUSED ? W_BYTES + KA * 512 : W_BYTES + A_BYTES + 2 * KA * 512;
     const int npre = n_units < STAGES ? n_units : STAGES;
     const uint32_t smem0 = smem_u32(smem);
     // NI issuers: a tcgen05 instruction costs its issuing thread tens of
@@ -531,18 +711,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         for (int s = 0; s < STAGES; s++) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
+            mbar_init(aready0 + 8 * s, 1);  // fused: the stage's quantizer warp
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(accf0 + 8 * b, NI);
             mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
         }
         mbar_init(drainb, NI);
+        mbar_init(amaxb, p.csize);  // fused, computed s_g: one arrival per CTA of the cluster
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch_desc(&tmW);
-        tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmSW);
-        tma_prefetch_desc(&tmSA);
+        if (!FUSED) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmSA);
+        }
         // The weight stream depends on no earlier kernel (the one before may
         // still be quantizing the activations): start it at once, while warp
         // 1 allocates tensor memory.
@@ -560,8 +744,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
         tmem_relinquish();
     }
+    if (FUSED) {
+        // activation rows past M are never written by the quantizers: zero
+        // every stage's activation tile and scale atoms once
+        for (int s = 0; s < STAGES; s++) {
+            uint4 *a4 = reinterpret_cast<uint4 *>(smem + s * STAGE_BYTES + W_BYTES);
+            uint4 *sf4 = reinterpret_cast<uint4 *>(smem + s * STAGE_BYTES + W_BYTES + A_BYTES + SFW_BYTES);
+            for (int i = threadIdx.x; i < A_BYTES / 16; i += blockDim.x) a4[i] = make_uint4(0, 0, 0, 0);
+            for (int i = threadIdx.x; i < SFA_BYTES / 16; i += blockDim.x) sf4[i] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
-    __syncthreads();
+    // fused cluster split: the amax barriers of every CTA are initialised
+    // before any CTA arrives on a peer's
+    if (FUSED && p.csize > 1) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -569,9 +766,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         if (lane == 0 && !p.stall) {
             grid_dep_wait();
             int t = t_first, ks = ks_first;
-            for (int i = 0; i < npre; i++) {
-                load_a(ks, i);
-                advance(t, ks);
+            if (!FUSED) {
+                for (int i = 0; i < npre; i++) {
+                    load_a(ks, i);
+                    advance(t, ks);
+                }
+            } else {
+                for (int i = 0; i < npre; i++) advance(t, ks);
             }
             int issued = npre;
             for (int i = npre; i < n_units; i++) {
@@ -580,17 +781,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) break;
                 mbar_arrive_expect_tx(full0 + 8 * s, tx);
                 load_w(t, ks, s);
-                load_a(ks, s);
+                if (!FUSED) load_a(ks, s);
                 advance(t, ks);
                 issued = i + 1;
             }
+            // wait (bounded) for the copies still in flight before leaving
             for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++) {
                 volatile uint32_t no_abort = 0;
                 mbar_wait_bounded(full0 + 8 * (i % STAGES), (uint32_t)((i / STAGES) & 1), &no_abort, &g_gemm_error, p.budget_ns);
             }
         }
         __syncwarp();
-    } else if (warp == 1 || warp >= 6) {
+    } else if (warp == 1 || (warp >= 6 && warp <= 8)) {
         const int j = warp == 1 ? 0 : warp - 5;  // issuer index
         if (lane == 0) {
             // Descriptors of stage 0: a stage, atom or K step only moves the
@@ -616,7 +818,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 for (int i = first; i < i0 + len; i += NI) {
                     const int s = i % STAGES;
                     const uint32_t ph = (uint32_t)((i / STAGES) & 1);
-                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns)) {
+                    if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns) ||
+                        (FUSED && !mbar_wait_bounded(aready0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns))) {
                         stop = true;
                         break;
                     }
@@ -652,11 +855,44 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         }
         __syncwarp();
     } else {
+    // ---------------- warps 2-5 (and 9-12 when fused) ----------------
+    grid_dep_wait();
+    float sg = 1.0f;  // the activations' NVFP4 tensor scale (fused)
+    if (FUSED) {
+        grid_dep_launch();
+        const int qw = quantizer_index(warp);
+        if (QFMT == FP4_NVFP4) {
+            if (p.gA) {
+                sg = *p.gA;
+            } else {
+                // s_g from max |H_k x|: over the whole tensor (whole tiles), or
+                // over this CTA's K slice, combined across the cluster, whose
+                // slices cover K
+                const int K32 = p.K / 32;
+                const int j0 = p.csize > 1 ? ks_first * 8 : 0;
+                const int j1 = p.csize > 1 ? min((ks_first + n_units) * 8, K32) : K32;
+                float mx = act_amax<HK>(p, j0, j1, qw, lane, s_red);
+                if (p.csize > 1) {
+                    if (qw == 0 && lane < p.csize) {
+                        const uint32_t rk = cluster_ctarank();
+                        st_shared_cluster_f32(mapa_shared(smem_u32(&s_amax[rk]), (uint32_t)lane), mx);
+                        mbar_arrive_remote_release(mapa_shared(amaxb, (uint32_t)lane));
+                    }
+                    mbar_wait_cluster_bounded(amaxb, 0, abort_flag, &g_gemm_error, p.budget_ns);
+                    mx = 0.0f;
+                    for (int r = 0; r < p.csize; r++) mx = fmaxf(mx, s_amax[r]);
+                }
+                sg = nv_global_from_amax(mx);
+            }
+        }
+        if (warp == 2 && lane == 0) s_sg = sg;
+        quantize_act_stages<QFMT, HK>(p, smem, aready0, empty0, n_units, t_first, ks_first, qw, lane, sg, abort_flag);
+    }
+    if (!FUSED || warp <= 5) {  // warps 9-12 only quantize
     // ---------------- epilogue warps 2-5: one result per tile segment ----------------
     // warp w may only read TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
-    grid_dep_wait();
-    const float alpha = (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(*p.gA, *p.gW) : 1.0f;
+    const float alpha = (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(FUSED ? sg : *p.gA, *p.gW) : 1.0f;
     for (int seg = 0; seg < nseg; seg++) {
         const int b = seg & 1;
         bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error, p.budget_ns);
@@ -698,8 +934,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             continue;
         }
         const int c_lo = unit_owner((int64_t)t * p.nk, U, p.G), c_hi = unit_owner((int64_t)(t + 1) * p.nk - 1, U, p.G);
-        if (c_lo == c_hi) {
-            // the whole K range of this tile is ours: store C directly
+        if (FUSED || c_lo == c_hi) {
+            // the whole K range of this tile is ours (the fused kernel runs
+            // whole-tile and cluster splits only): store C directly
             float acc[BNA];
 #pragma unroll
             for (int m = 0; m < BNA; m++) acc[m] = __fadd_rn(0.0f, __uint_as_float(r[m]));
@@ -725,8 +962,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
 #pragma unroll
                 for (int m = 0; m < BNA; m++) acc[m] = 0.0f;
                 for (int cc = c_lo; cc <= c_hi; cc++) {
-                    const int sg = t - (int)(unit_begin(cc, U, p.G) / p.nk);
-                    const float4 *src = reinterpret_cast<const float4 *>(p.ws + (((int64_t)cc * p.maxseg + sg) * 128 + row) * 16);
+                    const int sg2 = t - (int)(unit_begin(cc, U, p.G) / p.nk);
+                    const float4 *src = reinterpret_cast<const float4 *>(p.ws + (((int64_t)cc * p.maxseg + sg2) * 128 + row) * 16);
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
                         const float4 v = __ldcg(src + q);
@@ -741,6 +978,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");  // s_last is reused by the next segment
         }
+    }
     }
     }
     tc_fence_before();
@@ -769,7 +1007,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                     acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
                 }
             }
-            if (n < p.N && !*abort_flag) store_row(p, n, acc, (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(*p.gA, *p.gW) : 1.0f);
+            const float sgA = FUSED ? s_sg : (FMT == FP4_NVFP4 && !p.sf_e8m0 ? *p.gA : 1.0f);
+            if (n < p.N && !*abort_flag) store_row(p, n, acc, (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(sgA, *p.gW) : 1.0f);
         }
         cluster_sync();
     }
@@ -1000,16 +1239,17 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
     return decode::plan(M, N, K, sms).ws_bytes;
 }
 
-template <int FMT>
+template <int QFMT, int HK, bool FUSED>
 static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const CUtensorMap &tsw,
                                  const CUtensorMap &tsa, const decode::Params &p, bool any_cut, cudaStream_t st, bool pdl)
 {
-    auto kern = decode::decode_kernel<FMT>;
+    constexpr int FMT = QFMT == FP4_MXFP4 ? FP4_MXFP4 : FP4_NVFP4;
+    auto kern = decode::decode_kernel<QFMT, HK, FUSED>;
     if (cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), decode::SMEM_BYTES); e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
-    cfg.blockDim = dim3(decode::DECODE_THREADS);
+    cfg.blockDim = dim3(decode::decode_threads(FUSED));
     cfg.dynamicSmemBytes = decode::SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -1030,7 +1270,7 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
     cfg.numAttrs = na;
     count_launches(1);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, ta, tsw, tsa, p);
-    if (e != cudaSuccess || p.counters || !any_cut) return e;
+    if (e != cudaSuccess || FUSED || p.counters || !any_cut) return e;
     // the reduction waits for the split-K kernel inside (grid_dep_wait)
     return launch_k(decode::reduce_kernel<FMT>, dim3((p.N + 127) / 128), dim3(128), 0, st, true, p);
 }
@@ -1079,8 +1319,12 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.ldc = ldc;
         dp.bf16out = bf16out;
         dp.sf_e8m0 = fmt == FP4_MXFP4_16;
-        return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl)
-                                : launch_decode<FP4_NVFP4>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl);
+        dp.x = nullptr;
+        dp.ldx = 0;
+        dp.ck = 1.0f;
+        dp.round_away = dp.mx_floor = 0;
+        return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4, 0, false>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl)
+                                : launch_decode<FP4_NVFP4, 0, false>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl);
     }
     {
         PParams pp;
@@ -1139,6 +1383,75 @@ cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const fl
     const int out = out_fmt == FP4_MXFP4 ? OUT_MXFP4 : OUT_NVFP4;
     return cg == 2 ? launch_pgemm_fmt<2>(fmt, out, Aq, As, Wq, Ws, pp, sms, st, true)
                    : launch_pgemm_fmt<1>(fmt, out, Aq, As, Wq, Ws, pp, sms, st, true);
+}
+
+template <int QFMT>
+static cudaError_t launch_linear_fused_k(int hk, const CUtensorMap &tw, const CUtensorMap &tsw, const decode::Params &p,
+                                         cudaStream_t st)
+{
+    switch (hk) {
+    case 0: return launch_decode<QFMT, 0, true>(tw, tw, tsw, tsw, p, false, st, true);
+    case 16: return launch_decode<QFMT, 16, true>(tw, tw, tsw, tsw, p, false, st, true);
+    case 32: return launch_decode<QFMT, 32, true>(tw, tw, tsw, tsw, p, false, st, true);
+    case 64: return launch_decode<QFMT, 64, true>(tw, tw, tsw, tsw, p, false, st, true);
+    case 128: return launch_decode<QFMT, 128, true>(tw, tw, tsw, tsw, p, false, st, true);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// fp4_linear for M <= 16 in one launch: the decode kernel quantizes the bf16
+// activations itself (decode_kernel<..., FUSED>).  Work splits that cut a
+// tile between CTAs outside a cluster (very few tiles, or stream-K) are left
+// to the two-launch path: *taken = false, nothing launched.
+cudaError_t launch_linear_fused(const uint16_t *x, int64_t ldx, int64_t M, int64_t K, int fmt, int hk, float ck,
+                                int round_away, int mx_floor, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
+                                const float *gW, int64_t N, int bf16out, void *C, int64_t ldc, int sms, cudaStream_t st,
+                                bool w_before_wait, bool *taken)
+{
+    *taken = false;
+    if (M < 1 || M > kDecodeMaxM || N > (1 << 30) || K > (1 << 30)) return cudaSuccess;
+    const decode::Plan pl = decode::plan(M, N, K, sms);
+    if (pl.any_cut) return cudaSuccess;
+    *taken = true;
+    const int stall = g_inject_stall.exchange(0);
+    uint64_t budget = g_inject_budget.exchange(0);
+    if (budget == 0) budget = kWaitBudgetNs;
+    const int64_t nkb4 = (K / (fmt == FP4_MXFP4 ? 32 : 16) + 3) / 4;
+    const int KA = fmt == FP4_MXFP4 ? 2 : 4;
+    CUtensorMap tw, tsw;
+    if (!make_fp4_map(&tw, Wq, N, K, decode::BMW) || !make_sf_map(&tsw, Ws, nkb4, (N + 127) / 128, KA))
+        return cudaErrorInvalidValue;
+    decode::Params dp;
+    dp.ws = nullptr;
+    dp.counters = nullptr;
+    dp.N = (int)N;
+    dp.M = (int)M;
+    dp.K = (int)K;
+    dp.nk = pl.nk;
+    dp.ntiles = pl.ntiles;
+    dp.G = pl.G;
+    dp.maxseg = pl.maxseg;
+    dp.csize = pl.csize;
+    dp.w_before_wait = w_before_wait ? 1 : 0;
+    dp.budget_ns = budget;
+    dp.stall = stall;
+    dp.gA = fmt == FP4_NVFP4 ? gA : nullptr;
+    dp.gW = gW;
+    dp.C = C;
+    dp.ldc = ldc;
+    dp.bf16out = bf16out;
+    dp.sf_e8m0 = fmt == FP4_MXFP4_16;
+    dp.x = x;
+    dp.ldx = ldx;
+    dp.ck = ck;
+    dp.round_away = round_away;
+    dp.mx_floor = mx_floor;
+    switch (fmt) {
+    case FP4_MXFP4: return launch_linear_fused_k<FP4_MXFP4>(hk, tw, tsw, dp, st);
+    case FP4_NVFP4: return launch_linear_fused_k<FP4_NVFP4>(hk, tw, tsw, dp, st);
+    case FP4_MXFP4_16: return launch_linear_fused_k<FP4_MXFP4_16>(hk, tw, tsw, dp, st);
+    }
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err)
