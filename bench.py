@@ -35,6 +35,11 @@ ROWS, COLS = 1024, 131072
 # quantize kernel on 512 rows of this workload, scaled by rows.  Set to None
 # whenever that kernel changes, until it is captured again.
 QUANT_MX_TRAFFIC_BYTES = 304.1e6
+# Nominal B200 figures the fractions are also given against ("frac_spec"):
+# ~8 TB/s HBM3e and ~9 PFLOP/s dense FP4 (the gpt-oss MXFP4 article's B200
+# paragraph).  "frac" is always against the measured peaks.
+SPEC_HBM_GBS = 8000.0
+SPEC_FP4_TFLOPS = 9000.0
 WORKLOAD = "quantize sweep 1024x131072 bf16 Student-t(3)+1% outliers x20: MXFP4 + NVFP4 quantize and dequantize"
 METRIC = "FP4 quantize GB/s (% HBM peak)"
 
@@ -118,7 +123,8 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int, fmts=None):
 
             ms = time_graph(torch, call, 3, reps * 8)
             gbs = n * bpe / (ms * 1e-3) / 1e9
-            res["cases"][f"{name}_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
+            res["cases"][f"{name}_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm,
+                                            "frac_spec": gbs / SPEC_HBM_GBS}
         # the MSE block-scale search (same bytes, more arithmetic per block)
         for k in (0, 128):
             it = [0]
@@ -129,7 +135,8 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int, fmts=None):
 
             ms = time_graph(torch, call_mse, 3, reps * 8)
             gbs = n * bpe / (ms * 1e-3) / 1e9
-            res["cases"][f"{name}_mse_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
+            res["cases"][f"{name}_mse_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm,
+                                                "frac_spec": gbs / SPEC_HBM_GBS}
         # the sparse residual lane (TransFP4 Eq.(3)): 4 more bytes per 32 elements
         for k in (0, 32):
             it = [0]
@@ -140,7 +147,8 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int, fmts=None):
 
             ms = time_graph(torch, call_res, 3, reps * 8)
             gbs = n * (bpe + 4 / 32) / (ms * 1e-3) / 1e9
-            res["cases"][f"{name}_residual_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm}
+            res["cases"][f"{name}_residual_k{k}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm,
+                                                     "frac_spec": gbs / SPEC_HBM_GBS}
     del copies, xd
     torch.cuda.empty_cache()
     return res
@@ -186,8 +194,9 @@ def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None):
 
                 ms = time_graph(torch, call, 3, reps * copies)
                 b = wbytes + M * K * 2 + M * N * 2
-                res["cases"][f"{name}_M{M}_N{N}_K{K}"] = {"us": ms * 1e3, "gbs": b / (ms * 1e-3) / 1e9,
-                                                          "frac": b / (ms * 1e-3) / 1e9 / hbm}
+                gbs = b / (ms * 1e-3) / 1e9
+                res["cases"][f"{name}_M{M}_N{N}_K{K}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm,
+                                                          "frac_spec": gbs / SPEC_HBM_GBS}
             del Ws, W0
         del wd
     torch.cuda.empty_cache()
@@ -211,7 +220,7 @@ def bench_prefill(torch, fp4, inputs, dev, reps: int, M: int = 8192, fmts=None):
         W = fp4.quantize(wd, fmt)
         ms = time_graph(torch, lambda: fp4.gemm(A, W, M, N, K, fmt, out=C), 3, reps)
         tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
-        out[name] = {"ms": ms, "tflops": tf, "frac": tf / peak}
+        out[name] = {"ms": ms, "tflops": tf, "frac": tf / peak, "frac_spec": tf / SPEC_FP4_TFLOPS}
         q_ms = time_graph(torch, lambda: fp4.quantize(ad, fmt, out=A), 3, reps)
         out[name]["act_quantize_ms"] = q_ms
         out[name]["tflops_incl_act_quantize"] = 2.0 * M * N * K / ((ms + q_ms) * 1e-3) / 1e12
@@ -227,6 +236,7 @@ def bench_prefill(torch, fp4, inputs, dev, reps: int, M: int = 8192, fmts=None):
         cq_ms = time_graph(torch, lambda: fp4.quantize(C, ofmt, gscale=gs, out=Cb), 3, reps)
         out[name]["quantized_out"] = {"ms": fq_ms, "tflops": 2.0 * M * N * K / (fq_ms * 1e-3) / 1e12,
                                       "frac": 2.0 * M * N * K / (fq_ms * 1e-3) / 1e12 / peak,
+                                      "frac_spec": 2.0 * M * N * K / (fq_ms * 1e-3) / 1e12 / SPEC_FP4_TFLOPS,
                                       "unfused_bf16_then_quantize_ms": ms + cq_ms}
         del A, W, Cq, Cb
     del ad, wd, C
@@ -472,6 +482,7 @@ def run_ours(args):
     achieved = sb[dom] / (dom_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "quantize_kernel<MXFP4,k=0>", "achieved": achieved, "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                "frac_spec": achieved / SPEC_HBM_GBS, "peak_spec": SPEC_HBM_GBS,
                 "traffic": QUANT_MX_TRAFFIC_BYTES if rows == ROWS else None,
                 "launch_ms": dom_ms,
                 "per_call_ms": per,
@@ -596,6 +607,7 @@ def run_ours(args):
                    "l2": "inputs larger than L2 (268 MB bf16 tensor), no flush",
                    "step_bytes": sum(sb.values())},
         "frac_of_hbm_peak": value / ws / peak,
+        "frac_of_hbm_spec": value / ws / SPEC_HBM_GBS,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
