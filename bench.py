@@ -154,7 +154,8 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int, fmts=None):
     return res
 
 
-def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None):
+def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None, m_list=(1, 4, 16),
+                 shapes=((14336, 4096), (4096, 14336))):
     """Decode shapes: M in {1,4,16} bf16 activations quantized online inside
     the timed call (fp4_linear), W 14336x4096 and 4096x14336 pre-quantized,
     BF16 out.  W copies are rotated so the weight stream comes from HBM.  The
@@ -162,7 +163,7 @@ def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None):
     decode kernel streams its W while the previous call finishes."""
     hbm, kind = peaks()
     res = {"peak_gbs": hbm, "peak_kind": kind, "copies": 0, "cases": {}}
-    for (N, K) in ((14336, 4096), (4096, 14336)):
+    for (N, K) in shapes:
         _, w = inputs.decode_linear(1, N, K)
         wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
         del w
@@ -180,7 +181,7 @@ def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None):
             copies = max(2, int(2 * 126e6 // wbytes) + 1)
             Ws = [tuple(t.clone() for t in W0) for _ in range(copies)]
             res["copies"] = copies
-            for M in (1, 4, 16):
+            for M in m_list:
                 a, _ = inputs.decode_linear(M, 8, K)
                 x = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
                 C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -388,7 +389,12 @@ def run_ours(args):
         elif args.only == "rotate":
             r = bench_rotate(torch, fp4, inputs, dev, reps=args.steps, fmts=args.fmts)
         else:
-            r = bench_decode(torch, fp4, inputs, dev, reps=args.steps, fmts=args.fmts)
+            kw = {}
+            if args.decode_m:
+                kw["m_list"] = tuple(args.decode_m)
+            if args.decode_nk:
+                kw["shapes"] = tuple(tuple(int(v) for v in nk.split("x")) for nk in args.decode_nk)
+            r = bench_decode(torch, fp4, inputs, dev, reps=args.steps, fmts=args.fmts, **kw)
         print(json.dumps({"only": args.only, "result": r}), flush=True)
         return 0
 
@@ -634,6 +640,8 @@ def main():
                     help="profiling helper: run one GEMM leg alone")
     ap.add_argument("--prefill-m", type=int, default=8192)
     ap.add_argument("--fmts", nargs="*", default=None)
+    ap.add_argument("--decode-m", type=int, nargs="*", default=None, help="--only decode: activation rows")
+    ap.add_argument("--decode-nk", nargs="*", default=None, help="--only decode: weight shapes NxK, e.g. 14336x4096")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -14,7 +14,8 @@ from ._lib import (FP4_MX_SCALE_CEIL, FP4_MX_SCALE_FLOOR, FP4_MXFP4, FP4_MXFP4_1
                    FP4_OUT_F32, FP4_ROUND_AWAY, FP4_ROUND_EVEN, FP4_SCALE_ABSMAX, FP4_SCALE_MSE, Fp4Error)
 
 __all__ = [
-    "quantize", "dequantize", "gemm", "gemm_quantized", "linear", "linear_workspace_size", "quantize_sizes",
+    "quantize", "dequantize", "gemm", "gemm_quantized", "linear", "linear_residual", "linear_workspace_size",
+    "quantize_sizes",
     "gemm_workspace_size", "check_device_status", "kernel_launches",
     "FP4_MXFP4", "FP4_NVFP4", "FP4_MXFP4_16", "FP4_ROUND_EVEN", "FP4_ROUND_AWAY", "FP4_MX_SCALE_CEIL",
     "FP4_MX_SCALE_FLOOR", "FP4_OUT_F32", "FP4_OUT_BF16", "FP4_SCALE_ABSMAX", "FP4_SCALE_MSE",
@@ -343,6 +344,37 @@ def linear(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale
         gscale.data_ptr() if gscale is not None else None, Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(), N,
         int(out_dtype), out.data_ptr(), out.stride(0), workspace.data_ptr(), workspace.numel(),
         _stream_handle(torch, x.device))
+    return out
+
+
+def linear_residual(x, w, fmt, hadamard_k: int = 0, out_dtype: int = FP4_OUT_BF16, gscale=None,
+                    round: int = FP4_ROUND_EVEN, mx_scale_rule: int = FP4_MX_SCALE_CEIL, out=None,
+                    weights_static: bool = False):
+    """The decode linear (M <= 16) with the sparse residual lane of TransFP4
+    Eq.(3) in the activations (see fp4_linear_residual): each 32-value unit's
+    largest rotated value (bf16) stays out of the FP4 stream and its product
+    with W is added in the same launch.  w = (Wq, Ws, gW) as for
+    :func:`linear`; no workspace."""
+    import torch
+
+    fmt = _fmt(fmt)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor, contiguous along K")
+    _dev(x, "x", None, torch.bfloat16, contiguous=False)
+    M, K = x.shape
+    N = w[0].shape[0]
+    Wq, Ws, gW = _operand(w, N, K, fmt, "W", x.device)
+    if gscale is not None:
+        _dev(gscale, "gscale", x.device, torch.float32, 4)
+    dt = torch.float32 if out_dtype == FP4_OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, N), dtype=dt, device=x.device)
+    _out2d(out, M, N, dt, "out", x.device)
+    opts = _lib.Fp4Opts(int(round), int(mx_scale_rule), 0, 0, int(bool(weights_static)))
+    _run("fp4_linear_residual", x.device,
+         x.data_ptr(), M, K, x.stride(0), fmt, int(hadamard_k), ctypes.byref(opts),
+         gscale.data_ptr() if gscale is not None else None, Wq.data_ptr(), Ws.data_ptr(), gW.data_ptr(), N,
+         int(out_dtype), out.data_ptr(), out.stride(0), _stream_handle(torch, x.device))
     return out
 
 

@@ -49,6 +49,8 @@ SIGNATURES = {
     "fp4_linear_workspace_size": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_sz)]),
     "fp4_linear": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _int, _vp, _i64,
                           _vp, _sz, _vp]),
+    "fp4_linear_residual": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _int, _vp, _i64,
+                                   _vp]),
     "fp4_kernel_launches": (ctypes.c_uint64, []),
     "fp4_test_inject_stall": (_int, [_int, ctypes.c_uint64]),
 }

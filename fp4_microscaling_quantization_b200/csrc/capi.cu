@@ -38,7 +38,7 @@ cudaError_t launch_nv_refine(const uint16_t *x, int64_t rows, int64_t cols, int6
 cudaError_t launch_linear_fused(const uint16_t *x, int64_t ldx, int64_t M, int64_t K, int fmt, int hk, float ck,
                                 int round_away, int mx_floor, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
                                 const float *gW, int64_t N, int bf16out, void *C, int64_t ldc, int sms, cudaStream_t st,
-                                bool w_before_wait, bool *taken);
+                                bool w_before_wait, bool residual, bool *taken);
 cudaError_t read_and_clear_device_errors(cudaStream_t st, unsigned int *err);
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -302,7 +302,8 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
         e = fp4::launch_linear_fused(static_cast<const uint16_t *>(x), ld_x, M, K, fmt, hadamard_k,
                                      hadamard_constant(hadamard_k), o.round == FP4_ROUND_AWAY,
                                      o.mx_scale_rule == FP4_MX_SCALE_FLOOR, fmt == FP4_NVFP4 ? gA : nullptr, Wq, Ws, gW,
-                                     N, out_dtype == FP4_OUT_BF16, C, ldc, sms, st, o.weights_static != 0, &taken);
+                                     N, out_dtype == FP4_OUT_BF16, C, ldc, sms, st, o.weights_static != 0, false,
+                                     &taken);
         if (taken) return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
         // otherwise two launches: one cluster quantizes the activations (and
         // zeroes the tile counters); the split-K kernel streams W meanwhile
@@ -322,6 +323,39 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
     e = fp4::launch_gemm(aq, as, ga, Wq, Ws, gW, M, N, K, fmt, out_dtype == FP4_OUT_BF16, C, ldc, base + L.gemm,
                          L.counters - L.gemm, sms, st, &bad, true, counters, decode);
     if (bad) return FP4_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+fp4_status fp4_linear_residual(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt, int hadamard_k,
+                               const fp4_opts *opts, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
+                               const float *gW, int64_t N, int out_dtype, void *C, int64_t ldc, void *stream)
+{
+    fp4_opts o = {FP4_ROUND_EVEN, FP4_MX_SCALE_CEIL, 0, FP4_SCALE_ABSMAX, 0};
+    if (opts) o = *opts;
+    if (M < 0 || N < 0 || K < 0 || ld_x < K || ldc < N) return FP4_ERR_INVALID_ARG;
+    if (!valid_gemm_fmt(fmt)) return FP4_ERR_UNSUPPORTED;
+    if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+    if (o.round != FP4_ROUND_EVEN && o.round != FP4_ROUND_AWAY) return FP4_ERR_INVALID_ARG;
+    if (o.mx_scale_rule != FP4_MX_SCALE_CEIL && o.mx_scale_rule != FP4_MX_SCALE_FLOOR) return FP4_ERR_INVALID_ARG;
+    if (o.scale_search != FP4_SCALE_ABSMAX) return FP4_ERR_UNSUPPORTED;
+    if (o.weights_static != 0 && o.weights_static != 1) return FP4_ERR_INVALID_ARG;
+    if (!valid_k(hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (K % 32 || (hadamard_k && K % hadamard_k)) return FP4_ERR_UNSUPPORTED;
+    if (M > 16 || N > (1 << 30) || K > (1 << 30)) return FP4_ERR_UNSUPPORTED;  // the decode product only
+    if (M == 0 || N == 0) return FP4_OK;
+    if (K == 0) return FP4_ERR_UNSUPPORTED;
+    if (!x || !Wq || !Ws || !C) return FP4_ERR_INVALID_ARG;
+    if (fmt == FP4_NVFP4 && !gW) return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || (ld_x % 8) || !aligned(Wq, 16) || !aligned(Ws, 16) || !aligned(C, 16))
+        return FP4_ERR_ALIGNMENT;
+    if (gA && !aligned(gA, 4)) return FP4_ERR_ALIGNMENT;
+    bool taken = false;
+    const cudaError_t e = fp4::launch_linear_fused(
+        static_cast<const uint16_t *>(x), ld_x, M, K, fmt, hadamard_k, hadamard_constant(hadamard_k),
+        o.round == FP4_ROUND_AWAY, o.mx_scale_rule == FP4_MX_SCALE_FLOOR, fmt == FP4_NVFP4 ? gA : nullptr, Wq, Ws, gW,
+        N, out_dtype == FP4_OUT_BF16, C, ldc, sm_count(), static_cast<cudaStream_t>(stream), o.weights_static != 0, true,
+        &taken);
+    if (!taken) return FP4_ERR_UNSUPPORTED;
     return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 

@@ -86,6 +86,30 @@ FP4_DEV float absmax_tree(const float *v)
     return t[0];
 }
 
+// Sparse residual lane ("Portable FP4 quantization (TransFP4)" §2.3 Eq.(3),
+// one value per 32): the value of largest magnitude in the rotated unit v
+// (the first of equal ones) leaves the FP4 stream: it is zeroed in v and
+// returned as a word holding its bf16 rounding (RNE) and its index << 16.
+FP4_DEV uint32_t extract_residual(float *v)
+{
+    // the maximum by a balanced tree, then the first index that reaches it:
+    // a short dependency chain instead of a 32-step running search
+    const float amax = absmax_tree<32>(v);
+    uint32_t hit = 0;
+#pragma unroll
+    for (int i = 0; i < 32; i++) hit |= (fabsf(v[i]) == amax ? 1u : 0u) << i;
+    const int best = __ffs(hit) - 1;
+    float top = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        if (i == best) {
+            top = v[i];
+            v[i] = 0.0f;
+        }
+    }
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(top)) | ((uint32_t)best << 16);
+}
+
 // NVFP4 encode factor of a block scale with decode factor d: RN(1/d),
 // clamped to the largest float; 0 for d = 0 (the block encodes as zeros).
 FP4_DEV float nv_encode_factor(float d) { return (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), kFltMax); }

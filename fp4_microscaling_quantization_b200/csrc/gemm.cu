@@ -25,6 +25,7 @@
 #include <atomic>
 #include <mutex>
 #include <set>
+#include <type_traits>
 #include <utility>
 
 #include "encode.cuh"
@@ -404,19 +405,43 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 namespace decode {
 
 constexpr int BMW = 128, BNA = 16, BK = 256;
-constexpr int STAGES = 8;
 constexpr int W_BYTES = BMW * BK / 2;        // 16 KB
-constexpr int A_BYTES = BNA * BK / 2;        // 2 KB
 constexpr int SFW_BYTES = 4 * 512;
 constexpr int SFA_BYTES = 4 * 512;
-constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;  // 22528 = 22 KB
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
 constexpr int TMEM_COLS = 512;
 constexpr int NI = 4;                        // MMA issuer warps
-constexpr int SF_COL0 = 2 * NI * 16;         // accumulators: buffer b, issuer j at columns 16 (NI b + j)
 constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation scales 16 cols
 constexpr int MAX_CLUSTER = 8;               // portable cluster size
 
+// Stage and tensor-memory layout of a decode_kernel variant.  A stage holds
+// [W tile 128 x 256 | activation rows NB x 256 | W scale atoms | activation
+// scale atoms], the rows 128 bytes each in the 128-byte swizzle.  NB = 16
+// (1 + ND): the residual variant's ND groups of 16 more rows carry the
+// sparse residual lane's values, split into terms the block-scaled MMA
+// multiplies exactly, through the same MMA as the activations.  Tensor
+// memory: NBUF accumulator buffers of NI issuers x NB columns, then STAGES x
+// 32 columns of scales.
+template <int ND, int NSTAGES>
+struct DCfg {
+    static constexpr int STAGES = NSTAGES;
+    static constexpr int NB = BNA * (1 + ND);
+    static constexpr int A_BYTES = NB * BK / 2;
+    static constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;
+    static constexpr int NBUF = ND ? 1 : 2;  // the residual variant runs one tile segment per CTA
+    static constexpr int SF_COL0 = NBUF * NI * NB;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
+    static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the 128-byte swizzle");
+    static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+    static_assert(NB <= 128, "one 128-row scale atom covers the activation rows");
+};
+// fp4_gemm's and fp4_linear's decode kernels: 8 stages of 22 KB
+using DPlain = DCfg<0, 8>;
+// the residual lane (fp4_linear_residual): E8M0-scaled terms have two
+// significant bits, so a bf16 value takes up to 4 (MXFP4, MXFP4_16); E4M3-scaled
+// terms have four, so 2 (NVFP4)
+template <int QFMT>
+using DRes = DCfg<QFMT == FP4_NVFP4 ? 2 : 4, QFMT == FP4_NVFP4 ? 8 : 6>;
 struct Params {
     float *ws;           // partials: [G][maxseg][128][16]
     // Fused reduction (counters != nullptr): per-tile arrival counters, zero
@@ -468,15 +493,14 @@ FP4_DEV void store_row(const Params &p, int n, const float *acc, float alpha)
 
 // Threads: warp 0 loads, warps 1, 6, 7, 8 issue MMAs, warps 2-5 drain the
 // accumulators (warp w may read TMEM lanes 32 (w % 4) .. + 31).  The fused
-// variant (fp4_linear) adds warps 9-12: with warps 2-5 they quantize the
-// activations into the stages before the accumulators are drained.
-constexpr int NQ_EXTRA = 4;                  // warps 9 .. 12 of the fused variant
-constexpr int NQ = 4 + NQ_EXTRA;             // activation quantizer warps of the fused variant
+// variants (fp4_linear, fp4_linear_residual) add warps 9-12: with warps 2-5
+// they quantize the activations into the stages before the accumulators
+// are drained.
+constexpr int NQ_EXTRA = 4;                  // warps 9 .. 12 of the fused variants
+constexpr int NQ = 4 + NQ_EXTRA;             // activation quantizer warps of the fused variants
 __host__ __device__ constexpr int decode_threads(bool fused) { return 32 * (6 + NI - 1 + (fused ? NQ_EXTRA : 0)); }
-static_assert(STAGES % NI == 0, "a stage is always issued by the same warp");
-static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "TMEM budget");
 
-// Quantizer warp index of warp w (fused variant): warps 2-5 -> 0-3, 9-12 -> 4-7.
+// Quantizer warp index of warp w (fused variants): warps 2-5 -> 0-3, 9-12 -> 4-7.
 FP4_DEV int quantizer_index(int warp) { return warp <= 5 ? warp - 2 : warp - 5; }
 
 // Named barrier over the NQ quantizer warps (id 2; id 1 is the epilogue's).
@@ -530,25 +554,92 @@ FP4_DEV void st_shared_cluster_f32(uint32_t addr_cluster, float v)
 
 // Raw bf16 bytes of unit column j of activation row m (zeros for a row at or
 // past M, or a column at or past K: they quantize to zero codes and zero
-// scales, finite as the product's K tail needs).
+// scales, finite as the product's K tail needs).  Read through L2 only: x
+// may be the output of the kernel this one overlapped.
 FP4_DEV void fetch_act_unit(const Params &p, int m, int j, uint4 *raw)
 {
     if (m < p.M && j < p.K / 32) {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (int64_t)m * p.ldx + (int64_t)j * 32);
 #pragma unroll
-        for (int c = 0; c < 4; c++) raw[c] = __ldg(src + c);
+        for (int c = 0; c < 4; c++) raw[c] = __ldcg(src + c);
     } else {
 #pragma unroll
         for (int c = 0; c < 4; c++) raw[c] = make_uint4(0, 0, 0, 0);
     }
 }
 
+// ---- the sparse residual lane in the product ----------------------------------
+// "Portable FP4 quantization (TransFP4)" §2.3 Eq.(3): with both operands
+// rotated by the same H, C = Q(A - R) Q_W^T + R Q_W^T, R holding one value per
+// 32-element unit of a row (its largest rotated value, as bf16).  The second
+// term rides on the tensor cores: each residual r is split into ND terms
+// that the block-scaled MMA represents exactly (one nonzero element in its
+// block, whose scale carries the magnitude), placed at the residual's K
+// position in ND extra groups of 16 activation rows, so one MMA with
+// N = 16 (1 + ND) multiplies the weight tile with the activations and with
+// every term.  The epilogue adds the term rows to the residual sum.
+
+// E8M0-scaled terms (MXFP4, MXFP4_16): r as at most 4 terms sign * {1, 1.5}
+// * 2^e, each the next two significant bits of what is left (E2M1 codes 2 and
+// 3 under the E8M0 scale byte e + 127); bf16 has 8 significant bits, so 4
+// terms leave nothing.  Terms below 2^-126 (fp32 subnormal) are dropped.
+FP4_DEV void residual_terms_e8m0(float r, uint32_t *code, uint32_t *sbyte)
+{
+    float rem = r;
+#pragma unroll
+    for (int d = 0; d < 4; d++) {
+        const uint32_t u = __float_as_uint(rem);
+        const uint32_t ef = (u >> 23) & 0xFFu;
+        if (ef == 0) {
+            code[d] = 0;
+            sbyte[d] = 0;
+            continue;
+        }
+        const float t = __uint_as_float(u & 0xFFC00000u);  // sign, exponent, first mantissa bit
+        rem = __fsub_rn(rem, t);                             // exact: t is a prefix of rem
+        code[d] = (((u >> 22) & 1u) ? 3u : 2u) | ((u >> 28) & 8u);
+        sbyte[d] = ef;  // 2^(ef - 127): the term's exponent as an E8M0 byte
+    }
+}
+
+// E4M3-scaled terms (NVFP4): u = r / 2^E as at most 2 E4M3 values, the
+// nearest one, then the nearest to what is left (which has at most 4
+// significant bits: the rounding error of an 8-bit value at 4 bits), each an
+// element +-1 (E2M1 code 2) under that block scale.  Exact while the terms
+// stay within E4M3's range (see the row exponent below).
+FP4_DEV void residual_terms_e4m3(float u, uint32_t *code, uint32_t *sbyte)
+{
+#pragma unroll
+    for (int d = 0; d < 2; d++) {
+        const uint32_t b = e4m3_rn(fabsf(u));
+        const float v = e4m3_to_f32(b);
+        sbyte[d] = b;
+        code[d] = b ? (2u | ((__float_as_uint(u) >> 28) & 8u)) : 0u;
+        u = __fsub_rn(u, copysignf(v, u));  // exact: both are multiples of u's last bit
+    }
+}
+
+// Row exponent E of the NVFP4 terms: with e the exponent of the row's
+// largest residual magnitude, E = e - 7 puts every u = r / 2^E below 256
+// (inside E4M3's 448) and keeps the terms exact for residuals down to 2^(e-9)
+// (the second term's last bit then sits at E4M3's smallest step, 2^-9).
+FP4_DEV int residual_row_exponent(float rowmax)
+{
+    if (!(rowmax > 0.0f)) return 0;
+    int e = (int)((__float_as_uint(rowmax) >> 23) & 0xFF) - 127;
+    e -= 7;
+    return e < -126 ? -126 : (e > 126 ? 126 : e);
+}
+
 // max |H_k x| over the unit columns [j0, j1) of every activation row,
 // reduced over the NQ quantizer warps (all of them call it; every one gets
 // the result).  j0 and j1 are multiples of k / 32, and consecutive lanes hold
 // consecutive units of a row, so a rotation chunk lies in neighbouring lanes.
-template <int HK>
-FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float *red)
+// RES: the maximum is that of the FP4 stream (each unit's residual value
+// removed), and rowmax[m] (shared, zero on entry, float bits) receives the
+// largest residual magnitude of row m.
+template <int HK, bool RES>
+FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float *red, unsigned *rowmax)
 {
     const int ncols = j1 - j0;
     const int total = p.M * ncols;
@@ -556,17 +647,22 @@ FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float 
     float mx = 0.0f;
     for (int base = qw * 32 * U; base < total; base += NQ * 32 * U) {
         uint4 raw[U][4];
+        int mrow[U];
 #pragma unroll
         for (int i = 0; i < U; i++) {
             const int u = base + i * 32 + lane;
-            const int m = u < total ? u / ncols : p.M;
-            fetch_act_unit(p, m, j0 + (u < total ? u - m * ncols : 0), raw[i]);
+            mrow[i] = u < total ? u / ncols : p.M;
+            fetch_act_unit(p, mrow[i], j0 + (u < total ? u - mrow[i] * ncols : 0), raw[i]);
         }
 #pragma unroll
         for (int i = 0; i < U; i++) {
             float v[32];
             unpack_unit(raw[i], v);
             if (HK) fwht_unit<HK>(v, p.ck, lane);
+            if (RES) {
+                const uint32_t w = extract_residual(v);
+                if (mrow[i] < p.M) atomicMax(rowmax + mrow[i], __float_as_uint(fabsf(bf16lo(w))));
+            }
             mx = fmaxf(mx, absmax_tree<32>(v));
         }
     }
@@ -582,25 +678,30 @@ FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float 
 
 // The fused activation quantizer, one warp: for every unit i = qw (mod NQ)
 // of this CTA (its K step; a CTA's units may run over into the next tile),
-// once the stage's previous MMAs are done,
-// encodes the M x 256 activation slice of that K step into stage i % STAGES
-// exactly as the TMA would have placed fp4_quantize's output there (nibble
-// rows of 128 bytes in the 128-byte swizzle; scales in the tile layout's
-// atoms), then arrives on the stage's activation barrier.  Rows past M keep the
-// zeros written at kernel start.  Returns false after an abort.
-template <int QFMT, int HK>
+// once the stage's previous MMAs are done, encodes the M x 256 activation
+// slice of that K step into stage i % STAGES exactly as the TMA would have
+// placed fp4_quantize's output there (nibble rows of 128 bytes in the
+// 128-byte swizzle; scales in the tile layout's atoms), then arrives on the
+// stage's activation barrier.  Rows past M keep the zeros written at kernel
+// start.  RES: each unit's residual value leaves the FP4 stream (as
+// fp4_quantize_residual takes it) and its terms go to rows 16 d + m,
+// d = 1 .. ND, at the residual's position (rexp[m]: the NVFP4 row exponent).
+// Returns false after an abort.
+template <int QFMT, int HK, bool RES, typename Cfg>
 FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready0, uint32_t empty0, int n_units,
-                                 int t_first, int ks_first, int qw, int lane, float sg, volatile uint32_t *abort_flag)
+                                 int t_first, int ks_first, int qw, int lane, float sg, const int *rexp,
+                                 volatile uint32_t *abort_flag)
 {
+    constexpr int ND = Cfg::NB / BNA - 1;
     const float six_sg = __fmul_rn(6.0f, sg);
     const int nwork = p.M * 8;  // units of one K step: (row m, column cu = 0..7)
     for (int i = qw; i < n_units; i += NQ) {
-        const int s = i % STAGES;
-        const uint32_t ph = (uint32_t)((i / STAGES) & 1);
+        const int s = i % Cfg::STAGES;
+        const uint32_t ph = (uint32_t)((i / Cfg::STAGES) & 1);
         if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) return false;
-        uint8_t *st = smem + s * STAGE_BYTES;
+        uint8_t *st = smem + s * Cfg::STAGE_BYTES;
         uint8_t *sa = st + W_BYTES;
-        uint8_t *sfa = st + W_BYTES + A_BYTES + SFW_BYTES;
+        uint8_t *sfa = st + W_BYTES + Cfg::A_BYTES + SFW_BYTES;
         const int j0 = (int)(((int64_t)t_first * p.nk + ks_first + i) % p.nk) * 8;  // K step of unit i
         uint4 raw[BNA * 8 / 32][4];
 #pragma unroll
@@ -616,6 +717,8 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
             float v[32];
             unpack_unit(raw[r], v);
             if (HK) fwht_unit<HK>(v, p.ck, lane);
+            uint32_t rw = 0;
+            if (RES) rw = extract_residual(v);
             uint4 nib;
             const uint32_t sb = encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib);
             if (w < nwork) {
@@ -625,6 +728,31 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
                 else
                     *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + m * 16 + 2 * (cu & 1)) = (uint16_t)sb;
             }
+            if (RES && w < nwork) {
+                uint32_t code[ND > 0 ? ND : 1], sbyte[ND > 0 ? ND : 1];
+                const float rv = bf16lo(rw);
+                const int idx = (int)((rw >> 16) & 31u);
+                if (QFMT == FP4_NVFP4)
+                    residual_terms_e4m3(__fmul_rn(rv, exp2i(-rexp[m])), code, sbyte);
+                else
+                    residual_terms_e8m0(rv, code, sbyte);
+#pragma unroll
+                for (int d = 0; d < ND; d++) {
+                    const int R = BNA * (d + 1) + m;  // R & 7 == m & 7
+                    uint32_t wds[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int q = 0; q < 4; q++)
+                        if (q == (idx >> 3)) wds[q] = code[d] << (4 * (idx & 7));
+                    *reinterpret_cast<uint4 *>(sa + R * 128 + ((cu ^ (m & 7)) << 4)) =
+                        make_uint4(wds[0], wds[1], wds[2], wds[3]);
+                    const int rb = (R & 31) * 16 + (R >> 5) * 4;  // row's bytes in a scale atom
+                    if (QFMT == FP4_MXFP4)
+                        sfa[(cu >> 2) * 512 + rb + (cu & 3)] = (uint8_t)sbyte[d];
+                    else  // two 16-element blocks: the term's block takes the scale, the other 0
+                        *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + rb + 2 * (cu & 1)) =
+                            (uint16_t)(sbyte[d] << (8 * (idx >> 4)));
+                }
+            }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -633,15 +761,36 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
     return true;
 }
 
+// C[m][n] for the m < M activation rows of one output row n, from the
+// activation sum and the residual lane's sum: RN(alpha acc) + RN(aR[m] racc).
+FP4_DEV void store_row_res(const Params &p, int n, const float *acc, const float *racc, float alpha, const float *aR)
+{
+#pragma unroll
+    for (int m = 0; m < BNA; m++) {
+        if (m >= p.M) break;
+        const float v = __fadd_rn(__fmul_rn(acc[m], alpha), __fmul_rn(racc[m], aR[m]));
+        if (p.bf16out)
+            reinterpret_cast<__nv_bfloat16 *>(p.C)[(int64_t)m * p.ldc + n] = __float2bfloat16_rn(v);
+        else
+            reinterpret_cast<float *>(p.C)[(int64_t)m * p.ldc + n] = v;
+    }
+}
+
 // QFMT: the operands' format (MXFP4_16 runs the 16-element block-scaled MMA,
 // FMT below, with E8M0 scales).  FUSED: fp4_linear's single-launch form,
 // which quantizes the activations itself (HK: their rotation) and needs a
-// whole-tile or cluster work split; otherwise A comes quantized (fp4_gemm).
-template <int QFMT, int HK, bool FUSED>
+// work split without tiles cut between CTAs outside a cluster; otherwise A
+// comes quantized (fp4_gemm).  RES (fused only): the sparse residual lane in
+// the product (fp4_linear_residual), one tile segment per CTA.
+template <int QFMT, int HK, bool FUSED, bool RES>
 __global__ void __launch_bounds__(decode_threads(FUSED), 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
               const __grid_constant__ CUtensorMap tmSW, const __grid_constant__ CUtensorMap tmSA, Params p)
 {
+    static_assert(FUSED || !RES, "the residual lane needs the fused activation quantizer");
+    using Cfg = typename std::conditional<RES, DRes<QFMT>, DPlain>::type;
+    constexpr int STAGES = Cfg::STAGES, STAGE_BYTES = Cfg::STAGE_BYTES, A_BYTES = Cfg::A_BYTES, NB = Cfg::NB;
+    constexpr int ND = NB / BNA - 1;
     constexpr int FMT = QFMT == FP4_MXFP4 ? FP4_MXFP4 : FP4_NVFP4;
     constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -653,14 +802,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     __shared__ volatile unsigned s_last;
     __shared__ float s_red[NQ];             // fused: per-warp maxima
     __shared__ float s_amax[MAX_CLUSTER];   // fused: the cluster CTAs' maxima, by rank
-    __shared__ float s_sg;                  // fused: the activation tensor scale
+    __shared__ float s_sg;                  // fused: the activations' tensor scale
+    __shared__ unsigned s_rowmax[BNA];      // residual lane, NVFP4: largest residual of each row (float bits)
+    __shared__ int s_rexp[BNA];             // ... and its row exponent
     volatile uint32_t *abort_flag = tmem_slot + 1;
     // cluster split: this CTA's 128 x 16 partial, [4][128][4] floats (16-byte
     // groups of one row's columns 4q..4q+3), in stage 0's W buffer, which no
-    // load or MMA touches once the accumulator is complete
+    // load or MMA touches once the accumulator is complete; the residual
+    // variant's residual partial follows it in the same buffer
     float4 *part = reinterpret_cast<float4 *>(smem);
 
-    // The fused kernel lets the next launch start only after its own wait
+    // The fused kernels let the next launch start only after their own wait
     // (below): by then every kernel before this one has finished, so the next
     // one may stream static weights at once.
     if (!FUSED) grid_dep_launch();
@@ -682,7 +834,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const int npre = n_units < STAGES ? n_units : STAGES;
     const uint32_t smem0 = smem_u32(smem);
     // NI issuers: a tcgen05 instruction costs its issuing thread tens of
-    // cycles, far longer than the tensor pipe needs for an N = 16 MMA, so NI
+    // cycles, far longer than the tensor pipe needs for a skinny MMA, so NI
     // warps take the units i = j (mod NI) and accumulate them in their own
     // accumulators, which the epilogue adds in issuer order.  Every issuer
     // commits once per tile segment (also one that owns no unit of it), so
@@ -740,13 +892,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             }
         }
     }
+    if (threadIdx.x < BNA) s_rowmax[threadIdx.x] = 0u;
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
         tmem_relinquish();
     }
     if (FUSED) {
         // activation rows past M are never written by the quantizers: zero
-        // every stage's activation tile and scale atoms once
+        // every stage's activation rows and scale atoms once
         for (int s = 0; s < STAGES; s++) {
             uint4 *a4 = reinterpret_cast<uint4 *>(smem + s * STAGE_BYTES + W_BYTES);
             uint4 *sf4 = reinterpret_cast<uint4 *>(smem + s * STAGE_BYTES + W_BYTES + A_BYTES + SFW_BYTES);
@@ -814,7 +967,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 if (seg >= 2 &&
                     !mbar_wait_bounded(acce0 + 8 * b, (uint32_t)(((seg >> 1) - 1) & 1), abort_flag, &g_gemm_error, p.budget_ns))
                     break;
-                const uint32_t acc = tmem + (uint32_t)(b * NI + j) * BNA;
+                const uint32_t acc = tmem + (uint32_t)((b % Cfg::NBUF) * NI + j) * NB;
                 for (int i = first; i < i0 + len; i += NI) {
                     const int s = i % STAGES;
                     const uint32_t ph = (uint32_t)((i / STAGES) & 1);
@@ -825,7 +978,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                     }
                     tc_fence_after();
                     const uint64_t so = (uint64_t)((s * STAGE_BYTES) >> 4);
-                    const uint32_t tsfw = tmem + SF_COL0 + s * SF_STAGE_COLS;
+                    const uint32_t tsfw = tmem + Cfg::SF_COL0 + s * SF_STAGE_COLS;
                     const uint32_t tsfa = tsfw + 16;
 #pragma unroll
                     for (int a = 0; a < KA; a++) {
@@ -838,7 +991,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                         const uint64_t ad = adesc0 + so + 2 * kk;
                         const int atom = (FMT == FP4_MXFP4) ? (kk >> 1) : kk;
                         const uint32_t sfid = (FMT == FP4_MXFP4) ? (uint32_t)((kk & 1) * 2) : 0u;
-                        const uint32_t idesc = idesc_blockscaled(BMW, BNA, FMT == FP4_MXFP4 || p.sf_e8m0, sfid, sfid);
+                        const uint32_t idesc = idesc_blockscaled(BMW, NB, FMT == FP4_MXFP4 || p.sf_e8m0, sfid, sfid);
                         tc_mma_blockscaled<FMT>(acc, wd, ad, idesc, (tsfw + 4 * atom) | (sfid << 30),
                                                 (tsfa + 4 * atom) | (sfid << 30), (i == first && kk == 0) ? 0u : 1u);
                     }
@@ -861,17 +1014,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     if (FUSED) {
         grid_dep_launch();
         const int qw = quantizer_index(warp);
-        if (QFMT == FP4_NVFP4) {
+        if (QFMT == FP4_NVFP4 && (RES || !p.gA)) {
+            // One pass over x before any encoding: max |H_k x| for a computed
+            // s_g (of the FP4 stream with the residual lane) and, with the
+            // lane, each row's largest residual.  Whole tiles cover all of K;
+            // the CTAs of a cluster split each take their K slice and combine
+            // the tensor maxima through distributed shared memory, whose slices
+            // cover K.  A row exponent is per CTA: its partial is scaled before
+            // the cluster adds them.
+            const int K32 = p.K / 32;
+            const int j0 = p.csize > 1 ? ks_first * 8 : 0;
+            const int j1 = p.csize > 1 ? min((ks_first + n_units) * 8, K32) : K32;
+            float mx = act_amax<HK, RES>(p, j0, j1, qw, lane, s_red, s_rowmax);
             if (p.gA) {
                 sg = *p.gA;
             } else {
-                // s_g from max |H_k x|: over the whole tensor (whole tiles), or
-                // over this CTA's K slice, combined across the cluster, whose
-                // slices cover K
-                const int K32 = p.K / 32;
-                const int j0 = p.csize > 1 ? ks_first * 8 : 0;
-                const int j1 = p.csize > 1 ? min((ks_first + n_units) * 8, K32) : K32;
-                float mx = act_amax<HK>(p, j0, j1, qw, lane, s_red);
                 if (p.csize > 1) {
                     if (qw == 0 && lane < p.csize) {
                         const uint32_t rk = cluster_ctarank();
@@ -884,9 +1041,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 }
                 sg = nv_global_from_amax(mx);
             }
+            if (RES && qw == 0 && lane < BNA) s_rexp[lane] = residual_row_exponent(__uint_as_float(s_rowmax[lane]));
+            quantizers_sync();  // s_rexp
+        } else if (QFMT == FP4_NVFP4) {
+            sg = *p.gA;
         }
         if (warp == 2 && lane == 0) s_sg = sg;
-        quantize_act_stages<QFMT, HK>(p, smem, aready0, empty0, n_units, t_first, ks_first, qw, lane, sg, abort_flag);
+        quantize_act_stages<QFMT, HK, RES, Cfg>(p, smem, aready0, empty0, n_units, t_first, ks_first, qw, lane, sg,
+                                                s_rexp, abort_flag);
     }
     if (!FUSED || warp <= 5) {  // warps 9-12 only quantize
     // ---------------- epilogue warps 2-5: one result per tile segment ----------------
@@ -905,22 +1067,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                                    : ((p.nk < n_units - i0) ? p.nk : n_units - i0);
         uint32_t r[16];
         const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
-        float sum[BNA];
+        float sum[BNA], rsum[BNA];
 #pragma unroll
-        for (int m = 0; m < BNA; m++) sum[m] = 0.0f;
+        for (int m = 0; m < BNA; m++) sum[m] = rsum[m] = 0.0f;
 #pragma unroll
         for (int j = 0; j < NI; j++) {
             if (((j - i0) % NI + NI) % NI >= len) continue;  // issuer j owns no unit of this segment
-            tmem_ld16(tmem + (uint32_t)(b * NI + j) * BNA + lanes, r);
+            const uint32_t accj = tmem + (uint32_t)((b % Cfg::NBUF) * NI + j) * NB + lanes;
+            tmem_ld16(accj, r);
             tmem_ld_wait();
 #pragma unroll
             for (int m = 0; m < BNA; m++) sum[m] = __fadd_rn(sum[m], __uint_as_float(r[m]));
-        }
 #pragma unroll
-        for (int m = 0; m < BNA; m++) r[m] = __float_as_uint(sum[m]);
+            for (int d = 1; d <= ND; d++) {
+                tmem_ld16(accj + BNA * d, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int m = 0; m < BNA; m++) rsum[m] = __fadd_rn(rsum[m], __uint_as_float(r[m]));
+            }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");
+        // the residual sums of NVFP4 rows: back to the row exponent's scale
+        if (RES && QFMT == FP4_NVFP4) {
+#pragma unroll
+            for (int m = 0; m < BNA; m++) rsum[m] = __fmul_rn(rsum[m], exp2i(s_rexp[m]));
+        }
         const int t = t_first + seg;
         const int row = quarter * 32 + lane;  // row of the W tile = output column n
         const int n = t * BMW + row;
@@ -928,26 +1101,36 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             // cluster split (one segment per CTA): leave the partial for the
             // cluster's first CTA
 #pragma unroll
-            for (int q = 0; q < 4; q++)
-                part[q * 128 + row] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                                  __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+            for (int q = 0; q < 4; q++) {
+                part[q * 128 + row] = make_float4(sum[4 * q], sum[4 * q + 1], sum[4 * q + 2], sum[4 * q + 3]);
+                if (RES)
+                    part[512 + q * 128 + row] = make_float4(rsum[4 * q], rsum[4 * q + 1], rsum[4 * q + 2], rsum[4 * q + 3]);
+            }
             continue;
         }
         const int c_lo = unit_owner((int64_t)t * p.nk, U, p.G), c_hi = unit_owner((int64_t)(t + 1) * p.nk - 1, U, p.G);
         if (FUSED || c_lo == c_hi) {
-            // the whole K range of this tile is ours (the fused kernel runs
+            // the whole K range of this tile is ours (the fused kernels run
             // whole-tile and cluster splits only): store C directly
             float acc[BNA];
 #pragma unroll
-            for (int m = 0; m < BNA; m++) acc[m] = __fadd_rn(0.0f, __uint_as_float(r[m]));
-            if (n < p.N) store_row(p, n, acc, alpha);
+            for (int m = 0; m < BNA; m++) acc[m] = __fadd_rn(0.0f, sum[m]);
+            if (n < p.N) {
+                if (RES) {
+                    float aR[BNA];
+                    const float gw = (FMT == FP4_NVFP4 && !p.sf_e8m0) ? *p.gW : 1.0f;
+#pragma unroll
+                    for (int m = 0; m < BNA; m++) aR[m] = gw;
+                    store_row_res(p, n, acc, rsum, alpha, aR);
+                } else {
+                    store_row(p, n, acc, alpha);
+                }
+            }
             continue;
         }
         float4 *dst = reinterpret_cast<float4 *>(p.ws + (((int64_t)c * p.maxseg + seg) * 128 + row) * 16);
 #pragma unroll
-        for (int q = 0; q < 4; q++)
-            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                                 __uint_as_float(r[4 * q + 3]));
+        for (int q = 0; q < 4; q++) dst[q] = make_float4(sum[4 * q], sum[4 * q + 1], sum[4 * q + 2], sum[4 * q + 3]);
         if (p.counters) {
             // Fused reduction: the last of the tile's c_hi - c_lo + 1 CTAs to get
             // here sums every partial in CTA order (the same order as
@@ -994,9 +1177,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             const int row = (warp & 3) * 32 + lane;
             const int t = c / p.csize;
             const int n = t * BMW + row;
-            float acc[BNA];
+            float acc[BNA], racc[BNA];
 #pragma unroll
-            for (int m = 0; m < BNA; m++) acc[m] = 0.0f;
+            for (int m = 0; m < BNA; m++) acc[m] = racc[m] = 0.0f;
             for (int rk = 0; rk < p.csize; rk++) {
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
@@ -1005,10 +1188,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                     acc[4 * q + 1] = __fadd_rn(acc[4 * q + 1], v.y);
                     acc[4 * q + 2] = __fadd_rn(acc[4 * q + 2], v.z);
                     acc[4 * q + 3] = __fadd_rn(acc[4 * q + 3], v.w);
+                    if (RES) {
+                        const float4 u = ld_shared_cluster_f32x4(mapa_shared(smem_u32(part + 512 + q * 128 + row), (uint32_t)rk));
+                        racc[4 * q] = __fadd_rn(racc[4 * q], u.x);
+                        racc[4 * q + 1] = __fadd_rn(racc[4 * q + 1], u.y);
+                        racc[4 * q + 2] = __fadd_rn(racc[4 * q + 2], u.z);
+                        racc[4 * q + 3] = __fadd_rn(racc[4 * q + 3], u.w);
+                    }
                 }
             }
-            const float sgA = FUSED ? s_sg : (FMT == FP4_NVFP4 && !p.sf_e8m0 ? *p.gA : 1.0f);
-            if (n < p.N && !*abort_flag) store_row(p, n, acc, (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(sgA, *p.gW) : 1.0f);
+            const bool nv = FMT == FP4_NVFP4 && !p.sf_e8m0;
+            const float sgA = FUSED ? s_sg : (nv ? *p.gA : 1.0f);
+            if (n < p.N && !*abort_flag) {
+                const float alpha = nv ? __fmul_rn(sgA, *p.gW) : 1.0f;
+                if (RES) {
+                    float aR[BNA];
+                    const float gw = nv ? *p.gW : 1.0f;
+#pragma unroll
+                    for (int m = 0; m < BNA; m++) aR[m] = gw;
+                    store_row_res(p, n, acc, racc, alpha, aR);
+                } else {
+                    store_row(p, n, acc, alpha);
+                }
+            }
         }
         cluster_sync();
     }
@@ -1095,6 +1297,29 @@ inline Plan plan(int64_t M, int64_t N, int64_t K, int sms)
             pl.any_cut = unit_owner((int64_t)t * pl.nk, U, pl.G) != unit_owner((int64_t)(t + 1) * pl.nk - 1, U, pl.G);
     pl.ws_bytes = pl.any_cut ? (size_t)pl.G * pl.maxseg * 128 * BNA * sizeof(float) : 0;
     (void)M;
+    return pl;
+}
+
+// A split without tiles cut between CTAs outside a cluster, one tile segment
+// per CTA (the residual variant's): plan()'s whole tiles or cluster split;
+// instead of its global split, clusters of up to MAX_CLUSTER slices for few
+// tiles, or one CTA per tile, in several waves, for more tiles than SMs.
+inline Plan plan_nocut(int64_t M, int64_t N, int64_t K, int sms)
+{
+    Plan pl = plan(M, N, K, sms);
+    if (!pl.any_cut && pl.maxseg == 1) return pl;
+    if (pl.ntiles > sms) {
+        pl.G = pl.ntiles;
+        pl.csize = 1;
+    } else {
+        int split = 1;
+        while (split * 2 <= MAX_CLUSTER && (int64_t)pl.ntiles * split * 2 <= sms && split * 2 <= pl.nk) split *= 2;
+        pl.G = pl.ntiles * split;
+        pl.csize = split;
+    }
+    pl.maxseg = 1;
+    pl.any_cut = false;
+    pl.ws_bytes = 0;
     return pl;
 }
 
@@ -1239,18 +1464,18 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int, int sms)
     return decode::plan(M, N, K, sms).ws_bytes;
 }
 
-template <int QFMT, int HK, bool FUSED>
+template <int QFMT, int HK, bool FUSED, bool RES = false>
 static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, const CUtensorMap &tsw,
                                  const CUtensorMap &tsa, const decode::Params &p, bool any_cut, cudaStream_t st, bool pdl)
 {
     constexpr int FMT = QFMT == FP4_MXFP4 ? FP4_MXFP4 : FP4_NVFP4;
-    auto kern = decode::decode_kernel<QFMT, HK, FUSED>;
-    if (cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), decode::SMEM_BYTES); e != cudaSuccess)
-        return e;
+    constexpr int smem = RES ? decode::DRes<QFMT>::SMEM_BYTES : decode::DPlain::SMEM_BYTES;
+    auto kern = decode::decode_kernel<QFMT, HK, FUSED, RES>;
+    if (cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), smem); e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
     cfg.blockDim = dim3(decode::decode_threads(FUSED));
-    cfg.dynamicSmemBytes = decode::SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     int na = 0;
@@ -1385,16 +1610,16 @@ cudaError_t launch_gemm_quantized(const uint8_t *Aq, const uint8_t *As, const fl
                    : launch_pgemm_fmt<1>(fmt, out, Aq, As, Wq, Ws, pp, sms, st, true);
 }
 
-template <int QFMT>
+template <int QFMT, bool RES>
 static cudaError_t launch_linear_fused_k(int hk, const CUtensorMap &tw, const CUtensorMap &tsw, const decode::Params &p,
                                          cudaStream_t st)
 {
     switch (hk) {
-    case 0: return launch_decode<QFMT, 0, true>(tw, tw, tsw, tsw, p, false, st, true);
-    case 16: return launch_decode<QFMT, 16, true>(tw, tw, tsw, tsw, p, false, st, true);
-    case 32: return launch_decode<QFMT, 32, true>(tw, tw, tsw, tsw, p, false, st, true);
-    case 64: return launch_decode<QFMT, 64, true>(tw, tw, tsw, tsw, p, false, st, true);
-    case 128: return launch_decode<QFMT, 128, true>(tw, tw, tsw, tsw, p, false, st, true);
+    case 0: return launch_decode<QFMT, 0, true, RES>(tw, tw, tsw, tsw, p, false, st, true);
+    case 16: return launch_decode<QFMT, 16, true, RES>(tw, tw, tsw, tsw, p, false, st, true);
+    case 32: return launch_decode<QFMT, 32, true, RES>(tw, tw, tsw, tsw, p, false, st, true);
+    case 64: return launch_decode<QFMT, 64, true, RES>(tw, tw, tsw, tsw, p, false, st, true);
+    case 128: return launch_decode<QFMT, 128, true, RES>(tw, tw, tsw, tsw, p, false, st, true);
     }
     return cudaErrorInvalidValue;
 }
@@ -1402,15 +1627,19 @@ static cudaError_t launch_linear_fused_k(int hk, const CUtensorMap &tw, const CU
 // fp4_linear for M <= 16 in one launch: the decode kernel quantizes the bf16
 // activations itself (decode_kernel<..., FUSED>).  Work splits that cut a
 // tile between CTAs outside a cluster (very few tiles, or stream-K) are left
-// to the two-launch path: *taken = false, nothing launched.
+// to the two-launch path: *taken = false, nothing launched.  With `residual`
+// (fp4_linear_residual) the sparse residual lane is added to the product and
+// every shape is taken.
 cudaError_t launch_linear_fused(const uint16_t *x, int64_t ldx, int64_t M, int64_t K, int fmt, int hk, float ck,
                                 int round_away, int mx_floor, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
                                 const float *gW, int64_t N, int bf16out, void *C, int64_t ldc, int sms, cudaStream_t st,
-                                bool w_before_wait, bool *taken)
+                                bool w_before_wait, bool residual, bool *taken)
 {
     *taken = false;
-    if (M < 1 || M > kDecodeMaxM || N > (1 << 30) || K > (1 << 30)) return cudaSuccess;
-    const decode::Plan pl = decode::plan(M, N, K, sms);
+    if (M < 1 || M > kDecodeMaxM || N < 1 || K < 32 || N > (1 << 30) || K > (1 << 30)) return cudaSuccess;
+    // fp4_linear keeps the two-launch path for splits that cut tiles; the
+    // residual lane takes a split without cuts for every shape
+    const decode::Plan pl = residual ? decode::plan_nocut(M, N, K, sms) : decode::plan(M, N, K, sms);
     if (pl.any_cut) return cudaSuccess;
     *taken = true;
     const int stall = g_inject_stall.exchange(0);
@@ -1446,10 +1675,18 @@ cudaError_t launch_linear_fused(const uint16_t *x, int64_t ldx, int64_t M, int64
     dp.ck = ck;
     dp.round_away = round_away;
     dp.mx_floor = mx_floor;
+    if (residual) {
+        switch (fmt) {
+        case FP4_MXFP4: return launch_linear_fused_k<FP4_MXFP4, true>(hk, tw, tsw, dp, st);
+        case FP4_NVFP4: return launch_linear_fused_k<FP4_NVFP4, true>(hk, tw, tsw, dp, st);
+        case FP4_MXFP4_16: return launch_linear_fused_k<FP4_MXFP4_16, true>(hk, tw, tsw, dp, st);
+        }
+        return cudaErrorInvalidValue;
+    }
     switch (fmt) {
-    case FP4_MXFP4: return launch_linear_fused_k<FP4_MXFP4>(hk, tw, tsw, dp, st);
-    case FP4_NVFP4: return launch_linear_fused_k<FP4_NVFP4>(hk, tw, tsw, dp, st);
-    case FP4_MXFP4_16: return launch_linear_fused_k<FP4_MXFP4_16>(hk, tw, tsw, dp, st);
+    case FP4_MXFP4: return launch_linear_fused_k<FP4_MXFP4, false>(hk, tw, tsw, dp, st);
+    case FP4_NVFP4: return launch_linear_fused_k<FP4_NVFP4, false>(hk, tw, tsw, dp, st);
+    case FP4_MXFP4_16: return launch_linear_fused_k<FP4_MXFP4_16, false>(hk, tw, tsw, dp, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -317,6 +317,30 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
                       void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * fp4_linear_residual — fp4_linear for the decode case (M <= 16) with the
+ * sparse residual lane of "Portable FP4 quantization (TransFP4)" §2.3
+ * Eq.(3) in the activations: with x rotated by H_k (hadamard_k, as W was),
+ *   C = alpha * Q_f(H x - P H x) W_q^T  +  (P H x) W_q^T,
+ * where P keeps, in every 32-value unit of each rotated activation row, the
+ * value of largest magnitude (the first of equal ones) rounded to bf16, as
+ * fp4_quantize_residual defines it; the FP4 stream's NVFP4 tensor scale is
+ * that of the values left (computed, or the static gA).  One launch: the
+ * lane's product runs on the tensor cores with the activations', each
+ * residual split into terms the block-scaled product represents exactly:
+ * 4 terms under E8M0 scales for MXFP4 and MXFP4_16 (every bf16 value of
+ * magnitude >= 2^-126), 2 terms under E4M3 scales and a power-of-two scale
+ * per activation row for NVFP4 (exact for residuals within a factor 2^9 of
+ * their row's largest; smaller ones are rounded at that row's finest E4M3
+ * step).
+ *   Arguments as fp4_linear, without a workspace (none is needed): W is the
+ *   weight as fp4_quantize wrote it (with the same hadamard_k).  M > 16
+ *   returns FP4_ERR_UNSUPPORTED, as does FP4_SCALE_MSE.
+ */
+fp4_status fp4_linear_residual(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt, int hadamard_k,
+                               const fp4_opts *opts, const float *gA, const uint8_t *Wq, const uint8_t *Ws,
+                               const float *gW, int64_t N, int out_dtype, void *C, int64_t ldc, void *stream);
+
+/*
  * fp4_gemm_decode_noalloc — the decode product of fp4_gemm (M <= 16) for
  * callers that cannot allocate device memory at call time (inside a stream
  * capture that must not add allocations, a plugin given fixed buffers, a
@@ -358,7 +382,7 @@ uint64_t fp4_kernel_launches(void);
  * nothing, frees its tensor memory and returns, and fp4_check_device_status()
  * then reports FP4_ERR_TIMEOUT.  The context stays usable.  A nonzero
  * budget_ns with stall == 0 only shortens the waits of the next launch.
- * Host-side, applies to one launch. */
+ * Host-side, applies to one launch.  fp4_linear_residual is a GEMM launch too. */
 fp4_status fp4_test_inject_stall(int stall, uint64_t budget_ns);
 
 /* Reads and clears the device-side error word that kernels set when a
