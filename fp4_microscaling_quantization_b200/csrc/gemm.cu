@@ -437,11 +437,12 @@ struct DCfg {
 };
 // fp4_gemm's and fp4_linear's decode kernels: 8 stages of 22 KB
 using DPlain = DCfg<0, 8>;
-// the residual lane (fp4_linear_residual): E8M0-scaled terms have two
-// significant bits, so a bf16 value takes up to 4 (MXFP4, MXFP4_16); E4M3-scaled
-// terms have four, so 2 (NVFP4)
+// the residual lane (fp4_linear_residual): 4 groups of term rows, 6 stages.
+// E8M0-scaled terms have two significant bits, so a bf16 value takes up to 4
+// (MXFP4, MXFP4_16); E4M3-scaled terms have four, so 2, in one of two bands
+// of a row's scale (NVFP4)
 template <int QFMT>
-using DRes = DCfg<QFMT == FP4_NVFP4 ? 2 : 4, QFMT == FP4_NVFP4 ? 8 : 6>;
+using DRes = DCfg<4, 6>;
 struct Params {
     float *ws;           // partials: [G][maxseg][128][16]
     // Fused reduction (counters != nullptr): per-tile arrival counters, zero
@@ -619,16 +620,21 @@ FP4_DEV void residual_terms_e4m3(float u, uint32_t *code, uint32_t *sbyte)
     }
 }
 
-// Row exponent E of the NVFP4 terms: with e the exponent of the row's
-// largest residual magnitude, E = e - 7 puts every u = r / 2^E below 256
-// (inside E4M3's 448) and keeps the terms exact for residuals down to 2^(e-9)
-// (the second term's last bit then sits at E4M3's smallest step, 2^-9).
+// Row exponent E0 of the NVFP4 terms: with e the exponent of the row's
+// largest residual magnitude, E0 = e - 7 puts every u = r / 2^E0 below 256
+// (inside E4M3's 448).  Two E4M3 terms of u are exact while the second one's
+// last bit, 2^(e(r) - 7 - E0), stays at or above E4M3's smallest step 2^-9,
+// i.e. for |r| >= 2^(E0 - 2): band 0.  Smaller residuals go to band 1, the
+// same terms of r / 2^(E0 - 10), exact down to 2^(E0 - 12) = 2^(e - 19); below
+// that (19 binades under the row's largest) the terms are E4M3 roundings.
+// E0 is clamped so that both bands' factors stay normal floats.
+constexpr int RES_BAND_SHIFT = 10;
 FP4_DEV int residual_row_exponent(float rowmax)
 {
     if (!(rowmax > 0.0f)) return 0;
     int e = (int)((__float_as_uint(rowmax) >> 23) & 0xFF) - 127;
     e -= 7;
-    return e < -126 ? -126 : (e > 126 ? 126 : e);
+    return e < -126 + RES_BAND_SHIFT ? -126 + RES_BAND_SHIFT : (e > 126 ? 126 : e);
 }
 
 // max |H_k x| over the unit columns [j0, j1) of every activation row,
@@ -732,10 +738,22 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
                 uint32_t code[ND > 0 ? ND : 1], sbyte[ND > 0 ? ND : 1];
                 const float rv = bf16lo(rw);
                 const int idx = (int)((rw >> 16) & 31u);
-                if (QFMT == FP4_NVFP4)
-                    residual_terms_e4m3(__fmul_rn(rv, exp2i(-rexp[m])), code, sbyte);
-                else
+                if (QFMT == FP4_NVFP4) {
+                    // band 0 (rows 16-47) or band 1 (rows 48-79) of the row's scale
+                    const int E0 = rexp[m];
+                    const bool hi = fabsf(rv) >= exp2i(E0 - 2);
+                    uint32_t tc[2], ts[2];
+                    residual_terms_e4m3(__fmul_rn(rv, exp2i(hi ? -E0 : RES_BAND_SHIFT - E0)), tc, ts);
+#pragma unroll
+                    for (int d = 0; d < 2; d++) {
+                        code[d] = hi ? tc[d] : 0u;
+                        sbyte[d] = hi ? ts[d] : 0u;
+                        code[2 + d] = hi ? 0u : tc[d];
+                        sbyte[2 + d] = hi ? 0u : ts[d];
+                    }
+                } else {
                     residual_terms_e8m0(rv, code, sbyte);
+                }
 #pragma unroll
                 for (int d = 0; d < ND; d++) {
                     const int R = BNA * (d + 1) + m;  // R & 7 == m & 7
@@ -1067,9 +1085,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                                    : ((p.nk < n_units - i0) ? p.nk : n_units - i0);
         uint32_t r[16];
         const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
-        float sum[BNA], rsum[BNA];
+        // sum: the activations' accumulators; rsum / rsum1: the residual
+        // lane's term rows (NVFP4: bands 0 and 1)
+        float sum[BNA], rsum[BNA], rsum1[BNA];
 #pragma unroll
-        for (int m = 0; m < BNA; m++) sum[m] = rsum[m] = 0.0f;
+        for (int m = 0; m < BNA; m++) sum[m] = rsum[m] = rsum1[m] = 0.0f;
 #pragma unroll
         for (int j = 0; j < NI; j++) {
             if (((j - i0) % NI + NI) % NI >= len) continue;  // issuer j owns no unit of this segment
@@ -1082,17 +1102,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             for (int d = 1; d <= ND; d++) {
                 tmem_ld16(accj + BNA * d, r);
                 tmem_ld_wait();
+                float *dst = (QFMT == FP4_NVFP4 && d > 2) ? rsum1 : rsum;
 #pragma unroll
-                for (int m = 0; m < BNA; m++) rsum[m] = __fadd_rn(rsum[m], __uint_as_float(r[m]));
+                for (int m = 0; m < BNA; m++) dst[m] = __fadd_rn(dst[m], __uint_as_float(r[m]));
             }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");
-        // the residual sums of NVFP4 rows: back to the row exponent's scale
+        // the residual sums of NVFP4 rows: back to the row's scale, band by band
         if (RES && QFMT == FP4_NVFP4) {
 #pragma unroll
-            for (int m = 0; m < BNA; m++) rsum[m] = __fmul_rn(rsum[m], exp2i(s_rexp[m]));
+            for (int m = 0; m < BNA; m++)
+                rsum[m] = __fadd_rn(__fmul_rn(rsum[m], exp2i(s_rexp[m])),
+                                    __fmul_rn(rsum1[m], exp2i(s_rexp[m] - RES_BAND_SHIFT)));
         }
         const int t = t_first + seg;
         const int row = quarter * 32 + lane;  // row of the W tile = output column n

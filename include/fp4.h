@@ -328,10 +328,10 @@ fp4_status fp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, int fmt
  * lane's product runs on the tensor cores with the activations', each
  * residual split into terms the block-scaled product represents exactly:
  * 4 terms under E8M0 scales for MXFP4 and MXFP4_16 (every bf16 value of
- * magnitude >= 2^-126), 2 terms under E4M3 scales and a power-of-two scale
- * per activation row for NVFP4 (exact for residuals within a factor 2^9 of
- * their row's largest; smaller ones are rounded at that row's finest E4M3
- * step).
+ * magnitude >= 2^-126), 2 terms under E4M3 scales and one of two
+ * power-of-two scales per activation row, 2^10 apart, for NVFP4 (exact for
+ * residuals within a factor 2^19 of their row's largest; smaller ones are
+ * rounded at that row's finest E4M3 step).
  *   Arguments as fp4_linear, without a workspace (none is needed): W is the
  *   weight as fp4_quantize wrote it (with the same hadamard_k).  M > 16
  *   returns FP4_ERR_UNSUPPORTED, as does FP4_SCALE_MSE.
