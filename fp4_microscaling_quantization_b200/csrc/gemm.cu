@@ -409,7 +409,7 @@ constexpr int W_BYTES = BMW * BK / 2;        // 16 KB
 constexpr int SFW_BYTES = 4 * 512;
 constexpr int SFA_BYTES = 4 * 512;
 constexpr int TMEM_COLS = 512;
-constexpr int NI = 4;                        // MMA issuer warps
+constexpr int NI = 4;                        // MMA issuer warps (warps 1, 6, 7, 8) at most
 constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation scales 16 cols
 constexpr int MAX_CLUSTER = 8;               // portable cluster size
 
@@ -419,30 +419,37 @@ constexpr int MAX_CLUSTER = 8;               // portable cluster size
 // (1 + ND): the residual variant's ND groups of 16 more rows carry the
 // sparse residual lane's values, split into terms the block-scaled MMA
 // multiplies exactly, through the same MMA as the activations.  Tensor
-// memory: NBUF accumulator buffers of NI issuers x NB columns, then STAGES x
-// 32 columns of scales.
-template <int ND, int NSTAGES>
+// memory: NBUF accumulator buffers of NIS issuers x NB columns, then STAGES x
+// 32 columns of scales.  Issuer j takes the units i = j (mod NIS); STAGES is
+// a multiple of NIS so that a stage is always consumed by the same issuer:
+// an issuer then waits for every phase of its stages' barriers in turn, which
+// is what their parity waits need (a barrier two phases further than its
+// waiter last saw reads as ready).
+template <int ND, int NSTAGES, int NISSUERS>
 struct DCfg {
     static constexpr int STAGES = NSTAGES;
+    static constexpr int NIS = NISSUERS;
     static constexpr int NB = BNA * (1 + ND);
     static constexpr int A_BYTES = NB * BK / 2;
     static constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;
     static constexpr int NBUF = ND ? 1 : 2;  // the residual variant runs one tile segment per CTA
-    static constexpr int SF_COL0 = NBUF * NI * NB;
+    static constexpr int SF_COL0 = NBUF * NIS * NB;
+    static_assert(STAGES % NIS == 0 && NIS <= NI, "a stage is always consumed by the same issuer");
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
     static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the 128-byte swizzle");
     static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     static_assert(NB <= 128, "one 128-row scale atom covers the activation rows");
 };
-// fp4_gemm's and fp4_linear's decode kernels: 8 stages of 22 KB
-using DPlain = DCfg<0, 8>;
-// the residual lane (fp4_linear_residual): 4 groups of term rows, 6 stages.
+// fp4_gemm's and fp4_linear's decode kernels: 8 stages of 22 KB, 4 issuers
+using DPlain = DCfg<0, 8, 4>;
+// the residual lane (fp4_linear_residual): 4 groups of term rows, 6 stages
+// of 30 KB, 3 issuers (warp 8 stays idle).
 // E8M0-scaled terms have two significant bits, so a bf16 value takes up to 4
 // (MXFP4, MXFP4_16); E4M3-scaled terms have four, so 2, in one of two bands
 // of a row's scale (NVFP4)
 template <int QFMT>
-using DRes = DCfg<4, 6>;
+using DRes = DCfg<4, 6, 3>;
 struct Params {
     float *ws;           // partials: [G][maxseg][128][16]
     // Fused reduction (counters != nullptr): per-tile arrival counters, zero
@@ -808,6 +815,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     static_assert(FUSED || !RES, "the residual lane needs the fused activation quantizer");
     using Cfg = typename std::conditional<RES, DRes<QFMT>, DPlain>::type;
     constexpr int STAGES = Cfg::STAGES, STAGE_BYTES = Cfg::STAGE_BYTES, A_BYTES = Cfg::A_BYTES, NB = Cfg::NB;
+    constexpr int NIS = Cfg::NIS;
     constexpr int ND = NB / BNA - 1;
     constexpr int FMT = QFMT == FP4_MXFP4 ? FP4_MXFP4 : FP4_NVFP4;
     constexpr int KA = (FMT == FP4_MXFP4) ? 2 : 4;
@@ -851,12 +859,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const uint32_t tx = FUSED ? W_BYTES + KA * 512 : W_BYTES + A_BYTES + 2 * KA * 512;
     const int npre = n_units < STAGES ? n_units : STAGES;
     const uint32_t smem0 = smem_u32(smem);
-    // NI issuers: a tcgen05 instruction costs its issuing thread tens of
-    // cycles, far longer than the tensor pipe needs for a skinny MMA, so NI
-    // warps take the units i = j (mod NI) and accumulate them in their own
+    // NIS issuers: a tcgen05 instruction costs its issuing thread tens of
+    // cycles, far longer than the tensor pipe needs for a skinny MMA, so NIS
+    // warps take the units i = j (mod NIS) and accumulate them in their own
     // accumulators, which the epilogue adds in issuer order.  Every issuer
     // commits once per tile segment (also one that owns no unit of it), so
-    // the segment barrier counts NI arrivals.
+    // the segment barrier counts NIS arrivals.
 
     auto advance = [&](int &t, int &ks) {
         if (++ks == p.nk) {
@@ -884,10 +892,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             mbar_init(aready0 + 8 * s, 1);  // fused: the stage's quantizer warp
         }
         for (int b = 0; b < 2; b++) {
-            mbar_init(accf0 + 8 * b, NI);
+            mbar_init(accf0 + 8 * b, NIS);
             mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
         }
-        mbar_init(drainb, NI);
+        mbar_init(drainb, NIS);
         mbar_init(amaxb, p.csize);  // fused, computed s_g: one arrival per CTA of the cluster
         *abort_flag = 0u;
         fence_barrier_init();
@@ -965,7 +973,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         __syncwarp();
     } else if (warp == 1 || (warp >= 6 && warp <= 8)) {
         const int j = warp == 1 ? 0 : warp - 5;  // issuer index
-        if (lane == 0) {
+        if (lane == 0 && j < NIS) {
             // Descriptors of stage 0: a stage, atom or K step only moves the
             // 16-byte-unit start address in the low 14 bits (shared memory
             // offsets stay below 256 KB, so the add never carries out).
@@ -978,15 +986,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             for (int seg = 0; seg < nseg && !stop; seg++) {
                 const int len = (p.nk - ks0 < n_units - i0) ? p.nk - ks0 : n_units - i0;
                 const int b = seg & 1;
-                const int first = i0 + ((j - i0) % NI + NI) % NI;  // this issuer's first unit of the segment
+                const int first = i0 + ((j - i0) % NIS + NIS) % NIS;  // this issuer's first unit of the segment
                 // Buffer b is free once the epilogue has drained segment seg - 2.
                 // Every issuer waits, also one without units here: its commit
                 // below must not count toward the barrier's previous phase.
                 if (seg >= 2 &&
                     !mbar_wait_bounded(acce0 + 8 * b, (uint32_t)(((seg >> 1) - 1) & 1), abort_flag, &g_gemm_error, p.budget_ns))
                     break;
-                const uint32_t acc = tmem + (uint32_t)((b % Cfg::NBUF) * NI + j) * NB;
-                for (int i = first; i < i0 + len; i += NI) {
+                const uint32_t acc = tmem + (uint32_t)((b % Cfg::NBUF) * NIS + j) * NB;
+                for (int i = first; i < i0 + len; i += NIS) {
                     const int s = i % STAGES;
                     const uint32_t ph = (uint32_t)((i / STAGES) & 1);
                     if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns) ||
@@ -1091,9 +1099,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
 #pragma unroll
         for (int m = 0; m < BNA; m++) sum[m] = rsum[m] = rsum1[m] = 0.0f;
 #pragma unroll
-        for (int j = 0; j < NI; j++) {
-            if (((j - i0) % NI + NI) % NI >= len) continue;  // issuer j owns no unit of this segment
-            const uint32_t accj = tmem + (uint32_t)((b % Cfg::NBUF) * NI + j) * NB + lanes;
+        for (int j = 0; j < NIS; j++) {
+            if (((j - i0) % NIS + NIS) % NIS >= len) continue;  // issuer j owns no unit of this segment
+            const uint32_t accj = tmem + (uint32_t)((b % Cfg::NBUF) * NIS + j) * NB + lanes;
             tmem_ld16(accj, r);
             tmem_ld_wait();
 #pragma unroll
