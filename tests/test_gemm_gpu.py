@@ -190,11 +190,12 @@ def test_rotated_operands_preserve_product(fp4, orc, fmt):
         assert errs[128] < errs[0]
 
 
-@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("fmt", [0, 1, 2])
 def test_full_size_prefill_sampled(fp4, orc, fmt):
     """8192 x 8192 activations times a 28672 x 8192 weight (70B MLP shape), in
     the benchmark's launch configuration; 64 x 64 sampled outputs against the
-    oracle's fp64 product of the same quantized bytes."""
+    oracle's fp64 product of the same quantized bytes.  Formats: MXFP4, NVFP4
+    and MXFP4 on 16-element blocks (the benchmark's three prefill rows)."""
     import torch
     M, N, K = 8192, 28672, 8192
     a, w = inputs.prefill_linear()
