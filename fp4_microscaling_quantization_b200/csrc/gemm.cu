@@ -468,9 +468,6 @@ struct Params {
     int G;               // CTAs
     int maxseg;
     int csize;           // > 1: the CTAs of a tile form a cluster of csize and reduce through DSMEM
-    // Fused kernels: tq tiles' CTAs with the same K range share the activation
-    // quantization; the cluster holds csize * tq CTAs, rank = tile * csize + slice.
-    int tq;
     // Stream W before waiting for the preceding kernel.  Only when that
     // kernel triggers its dependents after its own wait (the decode
     // activation quantizer, or the fused kernel of an earlier fp4_linear), so
@@ -563,47 +560,6 @@ FP4_DEV void st_shared_cluster_f32(uint32_t addr_cluster, float v)
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr_cluster), "f"(v) : "memory");
 }
 
-FP4_DEV void st_shared_cluster_v4(uint32_t addr_cluster, uint4 v)
-{
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr_cluster), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
-}
-
-FP4_DEV void st_shared_cluster_b32(uint32_t addr_cluster, uint32_t v)
-{
-    asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
-}
-
-// Orders this thread's generic-proxy stores to any CTA of the cluster before
-// the tensor cores' (async-proxy) reads that follow a release / acquire.
-FP4_DEV void fence_proxy_async_cluster() { asm volatile("fence.proxy.async.shared::cluster;" ::: "memory"); }
-
-// Arrives on the barrier at the same shared offset in every CTA of `mask`
-// once all tcgen05 operations this thread issued so far have completed.
-FP4_DEV void tc_commit_multicast(uint32_t bar, uint16_t mask)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-                 "h"(mask)
-                 : "memory");
-}
-
-// The scale bytes of a K step for one activation row form whole 4-byte
-// words of a scale atom: `sb` of this lane's unit (cu = lane % 8; MXFP4 one
-// byte, otherwise two) gathered with its neighbours' into the word that the
-// lane with cu % 4 == 0 (MXFP4) or even cu holds.  Every lane calls it.
-template <int QFMT>
-FP4_DEV uint32_t gather_scale_word(uint32_t sb)
-{
-    if (QFMT == FP4_MXFP4) {
-        const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1), b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2),
-                       b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
-        return (sb & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
-    }
-    const uint32_t h1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
-    return (sb & 0xFFFFu) | ((h1 & 0xFFFFu) << 16);
-}
-
 // Raw bf16 bytes of unit column j of activation row m (zeros for a row at or
 // past M, or a column at or past K: they quantize to zero codes and zero
 // scales, finite as the product's K tail needs).  Read through L2 only: x
@@ -688,20 +644,18 @@ FP4_DEV int residual_row_exponent(float rowmax)
     return e < -126 + RES_BAND_SHIFT ? -126 + RES_BAND_SHIFT : (e > 126 ? 126 : e);
 }
 
-// max |H_k x| over the units this CTA quantizes (its K steps i = t0, t0 + T,
-// ... below n_units, K step (u0 + i) mod nk, every activation row), reduced
-// over the NQ quantizer warps (all of them call it; every one gets the
-// result).  Consecutive lanes hold consecutive units of a row's K step, so a
-// rotation chunk lies in neighbouring lanes.  RES: the maximum is that of the
-// FP4 stream (each unit's residual value removed), and rowmax[m] (shared,
-// zero on entry, float bits) receives the largest residual magnitude of row m.
+// max |H_k x| over the unit columns [j0, j1) of every activation row,
+// reduced over the NQ quantizer warps (all of them call it; every one gets
+// the result).  j0 and j1 are multiples of k / 32, and consecutive lanes hold
+// consecutive units of a row, so a rotation chunk lies in neighbouring lanes.
+// RES: the maximum is that of the FP4 stream (each unit's residual value
+// removed), and rowmax[m] (shared, zero on entry, float bits) receives the
+// largest residual magnitude of row m.
 template <int HK, bool RES>
-FP4_DEV float act_amax(const Params &p, int64_t u0, int n_units, int t0, int T, int qw, int lane, float *red,
-                       unsigned *rowmax)
+FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float *red, unsigned *rowmax)
 {
-    const int owned = n_units > t0 ? (n_units - t0 + T - 1) / T : 0;
-    const int per = p.M * 8;
-    const int total = owned * per;
+    const int ncols = j1 - j0;
+    const int total = p.M * ncols;
     constexpr int U = 2;  // units per lane and trip, loads issued together
     float mx = 0.0f;
     for (int base = qw * 32 * U; base < total; base += NQ * 32 * U) {
@@ -710,14 +664,8 @@ FP4_DEV float act_amax(const Params &p, int64_t u0, int n_units, int t0, int T, 
 #pragma unroll
         for (int i = 0; i < U; i++) {
             const int u = base + i * 32 + lane;
-            int j = 0;
-            mrow[i] = p.M;
-            if (u < total) {
-                const int st = u / per, rem = u - st * per;
-                mrow[i] = rem >> 3;
-                j = (int)((u0 + t0 + (int64_t)st * T) % p.nk) * 8 + (rem & 7);
-            }
-            fetch_act_unit(p, mrow[i], j, raw[i]);
+            mrow[i] = u < total ? u / ncols : p.M;
+            fetch_act_unit(p, mrow[i], j0 + (u < total ? u - mrow[i] * ncols : 0), raw[i]);
         }
 #pragma unroll
         for (int i = 0; i < U; i++) {
@@ -741,39 +689,39 @@ FP4_DEV float act_amax(const Params &p, int64_t u0, int n_units, int t0, int T, 
     return t;
 }
 
-// The fused activation quantizer, one warp.  The cluster's CTAs whose K
-// ranges are equal (tq of them: this CTA is t0 of T, slice `slice` of S per
-// tile) share the work: this CTA quantizes the units i = t0, t0 + T, ... of
-// the range (its K step (u0 + i) mod nk), the k-th of them taken by quantizer
-// warp k mod NQ.  For each, once every member has consumed the stage's
-// previous contents (aempty: one multicast commit per member), it encodes
-// the M x 256 activation slice into stage i % STAGES of every member, over
-// distributed shared memory, exactly as the TMA would have placed
-// fp4_quantize's output there (nibble rows of 128 bytes in the 128-byte
-// swizzle; scales in the tile layout's atoms, written as whole 4-byte words),
-// and every lane then arrives on each member's aready barrier of the stage
-// (release at cluster scope, after a proxy fence for the tensor cores).
-// Rows past M keep the zeros written at kernel start.  RES: each unit's
-// residual value leaves the FP4 stream (as fp4_quantize_residual takes it) and
-// its terms go to rows 16 d + m, d = 1 .. ND, at the residual's position
-// (rexp[m]: the NVFP4 row exponent).  Returns false after an abort.
+// The fused activation quantizer, one warp: for every unit i of this CTA
+// whose stage s = i % STAGES has s % NQ == qw (its K step; a CTA's units may
+// run over into the next tile), once the stage's previous MMAs are done,
+// encodes the M x 256 activation slice of that K step into stage s exactly
+// as the TMA would have
+// placed fp4_quantize's output there (nibble rows of 128 bytes in the
+// 128-byte swizzle; scales in the tile layout's atoms), then arrives on the
+// stage's activation barrier.  Every use of a stage is written by the same
+// warp, in order, so its wait for the stage's previous use always targets
+// the phase after the last one it saw: a parity wait two phases behind would
+// read as complete (a warp taking units i = qw (mod NQ) with NQ != STAGES
+// waited for use 2 of a stage before use 0 was consumed).  Rows past M keep the zeros written at kernel
+// start.  RES: each unit's residual value leaves the FP4 stream (as
+// fp4_quantize_residual takes it) and its terms go to rows 16 d + m,
+// d = 1 .. ND, at the residual's position (rexp[m]: the NVFP4 row exponent).
+// Returns false after an abort.
 template <int QFMT, int HK, bool RES, typename Cfg>
-FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready0, uint32_t aempty0, int n_units,
-                                 int64_t u0, int t0, int T, int S, int slice, int qw, int lane, float sg,
-                                 const int *rexp, volatile uint32_t *abort_flag)
+FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready0, uint32_t empty0, int n_units,
+                                 int t_first, int ks_first, int qw, int lane, float sg, const int *rexp,
+                                 volatile uint32_t *abort_flag)
 {
     constexpr int ND = Cfg::NB / BNA - 1;
     const float six_sg = __fmul_rn(6.0f, sg);
     const int nwork = p.M * 8;  // units of one K step: (row m, column cu = 0..7)
-    for (int k = qw;; k += NQ) {
-        const int i = t0 + k * T;
-        if (i >= n_units) break;
+    for (int i = 0; i < n_units; i++) {
         const int s = i % Cfg::STAGES;
+        if (s % NQ != qw) continue;
         const uint32_t ph = (uint32_t)((i / Cfg::STAGES) & 1);
-        if (!mbar_wait_bounded(aempty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) return false;
-        const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES + W_BYTES);
-        const uint32_t sfa = sa + Cfg::A_BYTES + SFW_BYTES;
-        const int j0 = (int)((u0 + i) % p.nk) * 8;  // first unit column of the K step
+        if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) return false;
+        uint8_t *st = smem + s * Cfg::STAGE_BYTES;
+        uint8_t *sa = st + W_BYTES;
+        uint8_t *sfa = st + W_BYTES + Cfg::A_BYTES + SFW_BYTES;
+        const int j0 = (int)(((int64_t)t_first * p.nk + ks_first + i) % p.nk) * 8;  // K step of unit i
         uint4 raw[BNA * 8 / 32][4];
 #pragma unroll
         for (int r = 0; r < BNA * 8 / 32; r++) {
@@ -785,30 +733,27 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
             if (r * 32 >= nwork) break;  // warp-uniform
             const int w = r * 32 + lane;
             const int m = w >> 3, cu = w & 7;
-            const bool live = w < nwork;
-            // the lane that writes the 4-byte scale word of its row and atom
-            const bool lead = (QFMT == FP4_MXFP4) ? (cu & 3) == 0 : (cu & 1) == 0;
-            const uint32_t word_off = (uint32_t)((QFMT == FP4_MXFP4 ? (cu >> 2) : (cu >> 1)) * 512);
             float v[32];
             unpack_unit(raw[r], v);
             if (HK) fwht_unit<HK>(v, p.ck, lane);
             uint32_t rw = 0;
             if (RES) rw = extract_residual(v);
             uint4 nib;
-            const uint32_t word = gather_scale_word<QFMT>(encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib));
-            for (int tt = 0; tt < T; tt++) {
-                const uint32_t rk = (uint32_t)(tt * S + slice);
-                const uint32_t sa_r = mapa_shared(sa, rk), sfa_r = mapa_shared(sfa, rk);
-                if (live) st_shared_cluster_v4(sa_r + m * 128 + ((cu ^ (m & 7)) << 4), nib);
-                if (live && lead) st_shared_cluster_b32(sfa_r + word_off + m * 16, word);
+            const uint32_t sb = encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib);
+            if (w < nwork) {
+                *reinterpret_cast<uint4 *>(sa + m * 128 + ((cu ^ (m & 7)) << 4)) = nib;
+                if (QFMT == FP4_MXFP4)
+                    sfa[(cu >> 2) * 512 + m * 16 + (cu & 3)] = (uint8_t)sb;
+                else
+                    *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + m * 16 + 2 * (cu & 1)) = (uint16_t)sb;
             }
-            if (RES) {
+            if (RES && w < nwork) {
                 uint32_t code[ND > 0 ? ND : 1], sbyte[ND > 0 ? ND : 1];
                 const float rv = bf16lo(rw);
                 const int idx = (int)((rw >> 16) & 31u);
                 if (QFMT == FP4_NVFP4) {
                     // band 0 (rows 16-47) or band 1 (rows 48-79) of the row's scale
-                    const int E0 = live ? rexp[m] : 0;
+                    const int E0 = rexp[m];
                     const bool hi = fabsf(rv) >= exp2i(E0 - 2);
                     uint32_t tc[2], ts[2];
                     residual_terms_e4m3(__fmul_rn(rv, exp2i(hi ? -E0 : RES_BAND_SHIFT - E0)), tc, ts);
@@ -829,22 +774,20 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
 #pragma unroll
                     for (int q = 0; q < 4; q++)
                         if (q == (idx >> 3)) wds[q] = code[d] << (4 * (idx & 7));
-                    // the term's block takes the scale, the unit's other 16-element block 0
-                    const uint32_t tsb = (QFMT == FP4_MXFP4) ? sbyte[d] : (sbyte[d] << (8 * (idx >> 4)));
-                    const uint32_t tword = gather_scale_word<QFMT>(tsb);
+                    *reinterpret_cast<uint4 *>(sa + R * 128 + ((cu ^ (m & 7)) << 4)) =
+                        make_uint4(wds[0], wds[1], wds[2], wds[3]);
                     const int rb = (R & 31) * 16 + (R >> 5) * 4;  // row's bytes in a scale atom
-                    for (int tt = 0; tt < T; tt++) {
-                        const uint32_t rk = (uint32_t)(tt * S + slice);
-                        if (live)
-                            st_shared_cluster_v4(mapa_shared(sa, rk) + R * 128 + ((cu ^ (m & 7)) << 4),
-                                                 make_uint4(wds[0], wds[1], wds[2], wds[3]));
-                        if (live && lead) st_shared_cluster_b32(mapa_shared(sfa, rk) + word_off + rb, tword);
-                    }
+                    if (QFMT == FP4_MXFP4)
+                        sfa[(cu >> 2) * 512 + rb + (cu & 3)] = (uint8_t)sbyte[d];
+                    else  // two 16-element blocks: the term's block takes the scale, the other 0
+                        *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + rb + 2 * (cu & 1)) =
+                            (uint16_t)(sbyte[d] << (8 * (idx >> 4)));
                 }
             }
         }
-        fence_proxy_async_cluster();
-        for (int tt = 0; tt < T; tt++) mbar_arrive_remote_release(mapa_shared(aready0 + 8 * s, (uint32_t)(tt * S + slice)));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(aready0 + 8 * s);
     }
     return true;
 }
@@ -886,14 +829,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     // bars: full[S] (TMA bytes), empty[S], aready[S] (fused: the stage's
-    // activations written), aempty[S] (fused: every CTA sharing them has
-    // consumed the stage), accfull[2], accempty[2], drain, amax (fused)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 6);
+    // activations written), accfull[2], accempty[2], drain, amax (fused)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 6);
     __shared__ volatile unsigned s_last;
     __shared__ float s_red[NQ];             // fused: per-warp maxima
-    // fused: the cluster CTAs' tensor maxima and, with the residual lane, row
-    // maxima, by rank
-    __shared__ float s_xchg[MAX_CLUSTER][BNA + 1];
+    __shared__ float s_amax[MAX_CLUSTER];   // fused: the cluster CTAs' maxima, by rank
     __shared__ float s_sg;                  // fused: the activations' tensor scale
     __shared__ unsigned s_rowmax[BNA];      // residual lane, NVFP4: largest residual of each row (float bits)
     __shared__ int s_rexp[BNA];             // ... and its row exponent
@@ -919,17 +859,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const int ks_first = (int)(u0 - (int64_t)t_first * p.nk);
     const int nseg = (int)((u1 - 1) / p.nk) - t_first + 1;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES), aready0 = smem_u32(bars + 2 * STAGES);
-    const uint32_t aempty0 = smem_u32(bars + 3 * STAGES);
-    const uint32_t accf0 = smem_u32(bars + 4 * STAGES), acce0 = smem_u32(bars + 4 * STAGES + 2);
-    const uint32_t drainb = smem_u32(bars + 4 * STAGES + 4);
-    const uint32_t amaxb = smem_u32(bars + 4 * STAGES + 5);
-    // cluster: rank = t0 * S + slice; the tq CTAs with the same slice share
-    // the activation quantization (fused), the S slices of a tile reduce
-    const int S = p.csize, T = FUSED ? p.tq : 1, cdim = S * T;
-    const int rank = cdim > 1 ? (int)cluster_ctarank() : 0;
-    const int slice = rank % S, t0 = rank / S;
-    uint16_t group = 0;  // the ranks sharing this CTA's activation stages
-    for (int tt = 0; tt < T; tt++) group |= (uint16_t)(1u << (tt * S + slice));
+    const uint32_t accf0 = smem_u32(bars + 3 * STAGES), acce0 = smem_u32(bars + 3 * STAGES + 2);
+    const uint32_t drainb = smem_u32(bars + 3 * STAGES + 4);
+    const uint32_t amaxb = smem_u32(bars + 3 * STAGES + 5);
     const uint32_t tx = FUSED ? W_BYTES + KA * 512 : W_BYTES + A_BYTES + 2 * KA * 512;
     const int npre = n_units < STAGES ? n_units : STAGES;
     const uint32_t smem0 = smem_u32(smem);
@@ -963,15 +895,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         for (int s = 0; s < STAGES; s++) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
-            mbar_init(aready0 + 8 * s, 32);  // fused: every lane of the writing quantizer warp
-            mbar_init(aempty0 + 8 * s, T);   // fused: one commit per CTA sharing the stage
+            mbar_init(aready0 + 8 * s, 1);  // fused: the stage's quantizer warp
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(accf0 + 8 * b, NIS);
             mbar_init(acce0 + 8 * b, 4);  // one arrival per epilogue warp
         }
         mbar_init(drainb, NIS);
-        mbar_init(amaxb, cdim);  // fused: one arrival per CTA of the cluster
+        mbar_init(amaxb, p.csize);  // fused, computed s_g: one arrival per CTA of the cluster
         *abort_flag = 0u;
         fence_barrier_init();
         tma_prefetch_desc(&tmW);
@@ -1010,9 +941,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         fence_proxy_async_smem();
     }
     tc_fence_before();
-    // fused: every CTA of the cluster has initialised its barriers and zeroed
-    // its stages before any CTA writes or arrives into a peer
-    if (FUSED && cdim > 1) cluster_sync(); else __syncthreads();
+    // fused cluster split: the amax barriers of every CTA are initialised
+    // before any CTA arrives on a peer's
+    if (FUSED && p.csize > 1) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -1073,7 +1004,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                     const int s = i % STAGES;
                     const uint32_t ph = (uint32_t)((i / STAGES) & 1);
                     if (!mbar_wait_bounded(full0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns) ||
-                        (FUSED && !mbar_wait_cluster_bounded(aready0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns))) {
+                        (FUSED && !mbar_wait_bounded(aready0 + 8 * s, ph, abort_flag, &g_gemm_error, p.budget_ns))) {
                         stop = true;
                         break;
                     }
@@ -1097,7 +1028,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                                                 (tsfa + 4 * atom) | (sfid << 30), (i == first && kk == 0) ? 0u : 1u);
                     }
                     tc_commit(empty0 + 8 * s);
-                    if (FUSED) tc_commit_multicast(aempty0 + 8 * s, group);
                 }
                 if (stop) break;
                 // this issuer's part of the segment is complete (at once if it had none)
@@ -1117,39 +1047,39 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         grid_dep_launch();
         const int qw = quantizer_index(warp);
         if (QFMT == FP4_NVFP4 && (RES || !p.gA)) {
-            // One pass over the units this CTA quantizes, before any encoding:
-            // max |H_k x| for a computed s_g (of the FP4 stream with the
-            // residual lane) and, with the lane, each row's largest residual.
-            // The cluster's CTAs together quantize all of x: each sends its
-            // maxima to every CTA of the cluster (distributed shared memory).
-            float mx = act_amax<HK, RES>(p, u0, n_units, t0, T, qw, lane, s_red, s_rowmax);
-            if (cdim > 1) {
-                if (qw == 0 && lane == 0) {
-                    for (int r = 0; r < cdim; r++) {
-                        const uint32_t dst = mapa_shared(smem_u32(&s_xchg[rank][0]), (uint32_t)r);
-                        st_shared_cluster_f32(dst, mx);
-                        for (int m = 0; m < BNA; m++) st_shared_cluster_f32(dst + 4 * (1 + m), __uint_as_float(s_rowmax[m]));
-                        mbar_arrive_remote_release(mapa_shared(amaxb, (uint32_t)r));
+            // One pass over x before any encoding: max |H_k x| for a computed
+            // s_g (of the FP4 stream with the residual lane) and, with the
+            // lane, each row's largest residual.  Whole tiles cover all of K;
+            // the CTAs of a cluster split each take their K slice and combine
+            // the tensor maxima through distributed shared memory, whose slices
+            // cover K.  A row exponent is per CTA: its partial is scaled before
+            // the cluster adds them.
+            const int K32 = p.K / 32;
+            const int j0 = p.csize > 1 ? ks_first * 8 : 0;
+            const int j1 = p.csize > 1 ? min((ks_first + n_units) * 8, K32) : K32;
+            float mx = act_amax<HK, RES>(p, j0, j1, qw, lane, s_red, s_rowmax);
+            if (p.gA) {
+                sg = *p.gA;
+            } else {
+                if (p.csize > 1) {
+                    if (qw == 0 && lane < p.csize) {
+                        const uint32_t rk = cluster_ctarank();
+                        st_shared_cluster_f32(mapa_shared(smem_u32(&s_amax[rk]), (uint32_t)lane), mx);
+                        mbar_arrive_remote_release(mapa_shared(amaxb, (uint32_t)lane));
                     }
+                    mbar_wait_cluster_bounded(amaxb, 0, abort_flag, &g_gemm_error, p.budget_ns);
+                    mx = 0.0f;
+                    for (int r = 0; r < p.csize; r++) mx = fmaxf(mx, s_amax[r]);
                 }
-                mbar_wait_cluster_bounded(amaxb, 0, abort_flag, &g_gemm_error, p.budget_ns);
-                mx = 0.0f;
-                for (int r = 0; r < cdim; r++) mx = fmaxf(mx, s_xchg[r][0]);
-                if (RES && qw == 0 && lane < BNA) {
-                    float rm = 0.0f;
-                    for (int r = 0; r < cdim; r++) rm = fmaxf(rm, s_xchg[r][1 + lane]);
-                    s_rowmax[lane] = __float_as_uint(rm);
-                }
-                quantizers_sync();  // s_rowmax
+                sg = nv_global_from_amax(mx);
             }
-            sg = p.gA ? *p.gA : nv_global_from_amax(mx);
             if (RES && qw == 0 && lane < BNA) s_rexp[lane] = residual_row_exponent(__uint_as_float(s_rowmax[lane]));
             quantizers_sync();  // s_rexp
         } else if (QFMT == FP4_NVFP4) {
             sg = *p.gA;
         }
         if (warp == 2 && lane == 0) s_sg = sg;
-        quantize_act_stages<QFMT, HK, RES, Cfg>(p, smem, aready0, aempty0, n_units, u0, t0, T, S, slice, qw, lane, sg,
+        quantize_act_stages<QFMT, HK, RES, Cfg>(p, smem, aready0, empty0, n_units, t_first, ks_first, qw, lane, sg,
                                                 s_rexp, abort_flag);
     }
     if (!FUSED || warp <= 5) {  // warps 9-12 only quantize
@@ -1271,30 +1201,23 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     }
     }
     }
-    if (warp == 1) {
-        // every MMA has completed (and with it every commit this CTA sends to
-        // its cluster peers) before the CTA passes the cluster barrier
-        volatile uint32_t no_abort = 0;
-        mbar_wait_bounded(drainb, 0, &no_abort, &g_gemm_error, p.budget_ns);
-    }
     tc_fence_before();
     __syncthreads();
-    if (cdim > 1) {
+    if (p.csize > 1) {
         // Every partial of the cluster is in place once all its CTAs pass
-        // this barrier; each tile's first CTA (slice 0) sums its slices'
-        // partials in slice order (the CTA order of the global reduction) and
-        // stores C.  The second barrier keeps every CTA's shared memory alive
-        // until the others have read it or written into it.  Both are reached
-        // on every path, the abort paths included.
+        // this barrier; the first CTA sums them in rank order (the CTA order
+        // of the global reduction) and stores C.  The second barrier keeps
+        // the other CTAs' shared memory alive until it has read it.  Both are
+        // reached on every path, the abort paths included.
         cluster_sync();
-        if (S > 1 && slice == 0 && warp >= 2 && warp <= 5) {
+        if (cluster_ctarank() == 0 && warp >= 2 && warp <= 5) {
             const int row = (warp & 3) * 32 + lane;
             const int t = c / p.csize;
             const int n = t * BMW + row;
             float acc[BNA], racc[BNA];
 #pragma unroll
             for (int m = 0; m < BNA; m++) acc[m] = racc[m] = 0.0f;
-            for (int rk = rank; rk < rank + S; rk++) {
+            for (int rk = 0; rk < p.csize; rk++) {
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
                     const float4 v = ld_shared_cluster_f32x4(mapa_shared(smem_u32(part + q * 128 + row), (uint32_t)rk));
@@ -1330,7 +1253,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     }
     if (warp == 1) {
         tc_fence_after();
-        // every MMA completed (waited above) before TMEM is released
+        // every MMA has completed before TMEM is released (also on the abort path)
+        volatile uint32_t no_abort = 0;
+        mbar_wait_bounded(drainb, 0, &no_abort, &g_gemm_error, p.budget_ns);
         tmem_dealloc(tmem, TMEM_COLS);
     }
 }
@@ -1433,18 +1358,6 @@ inline Plan plan_nocut(int64_t M, int64_t N, int64_t K, int sms)
     pl.any_cut = false;
     pl.ws_bytes = 0;
     return pl;
-}
-
-// Tiles whose CTAs share the fused activation quantization: the CTAs of tq
-// consecutive tiles with the same K slice form one cluster with the tile's
-// csize slices (csize * tq <= MAX_CLUSTER), tq dividing the tile count; one
-// tile segment per CTA (a CTA running over several tiles shares nothing).
-inline int share_tiles(const Plan &pl)
-{
-    if (pl.maxseg != 1 || pl.any_cut || (int64_t)pl.G != (int64_t)pl.ntiles * pl.csize) return 1;
-    int tq = 1;
-    while (pl.csize * tq * 2 <= MAX_CLUSTER && pl.ntiles % (tq * 2) == 0) tq *= 2;
-    return tq;
 }
 
 }  // namespace decode
@@ -1603,10 +1516,9 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     int na = 0;
-    const int cdim = p.csize * (FUSED ? p.tq : 1);
-    if (cdim > 1) {
+    if (p.csize > 1) {
         attr[na].id = cudaLaunchAttributeClusterDimension;
-        attr[na].val.clusterDim.x = cdim;
+        attr[na].val.clusterDim.x = p.csize;
         attr[na].val.clusterDim.y = 1;
         attr[na].val.clusterDim.z = 1;
         na++;
@@ -1659,7 +1571,6 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.G = pl.G;
         dp.maxseg = pl.maxseg;
         dp.csize = pl.csize;
-        dp.tq = 1;
         dp.w_before_wait = (pdl && w_before_wait) ? 1 : 0;
         dp.counters = counters;
         dp.budget_ns = budget;
@@ -1787,7 +1698,6 @@ cudaError_t launch_linear_fused(const uint16_t *x, int64_t ldx, int64_t M, int64
     dp.G = pl.G;
     dp.maxseg = pl.maxseg;
     dp.csize = pl.csize;
-    dp.tq = decode::share_tiles(pl);
     dp.w_before_wait = w_before_wait ? 1 : 0;
     dp.budget_ns = budget;
     dp.stall = stall;

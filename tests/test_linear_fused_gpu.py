@@ -67,9 +67,11 @@ def gemm_path(fp4, xd, W, fmt, hk, out_dtype, round_, rule, gA=None):
 
 # (M, N, K, hk): whole tiles (N = 12800: 100 tiles), clusters of 8 (16 tiles,
 # K = 2048), of 4 (32 tiles, K = 1024) and of 2 (64 tiles), a K tail (800 =
-# 3 steps + 32) and every rotation size.
+# 3 steps + 32), every rotation size, and whole tiles whose 32 / 25 K steps
+# run through the 8-stage pipeline four times.
 SHAPES = [(1, 12800, 512, 0), (16, 12800, 512, 128), (7, 12800, 800, 32), (16, 2048, 2048, 0), (3, 2048, 2048, 64),
-          (16, 4096, 1024, 16), (4, 4096, 800, 32), (16, 8192, 512, 128), (9, 8192, 4096, 64)]
+          (16, 4096, 1024, 16), (4, 4096, 800, 32), (16, 8192, 512, 128), (9, 8192, 4096, 64),
+          (4, 12800, 8192, 0), (16, 12800, 6400, 32)]
 
 
 @pytest.mark.parametrize("fmt", [MX, NV, MX16])
