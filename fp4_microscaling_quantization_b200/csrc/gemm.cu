@@ -851,13 +851,28 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
     const int64_t U = (int64_t)p.ntiles * p.nk;
-    const int64_t u0 = unit_begin(c, U, p.G), u1 = unit_begin(c + 1, U, p.G);
+    // This CTA's units [u0, u1): 32-bit divisions when the products fit (every
+    // decode shape), 64-bit ones otherwise; the weight stream waits on them.
+    int64_t u0, u1;
+    int t_first, nseg_last;
+    if ((uint64_t)U * (uint64_t)p.G < (1ull << 32)) {
+        const uint32_t Uu = (uint32_t)U, Gu = (uint32_t)p.G, nk = (uint32_t)p.nk;
+        const uint32_t a = (uint32_t)c * Uu / Gu, b = (uint32_t)(c + 1) * Uu / Gu;
+        u0 = a;
+        u1 = b;
+        t_first = (int)(a / nk);
+        nseg_last = (int)((b - 1) / nk);
+    } else {
+        u0 = unit_begin(c, U, p.G);
+        u1 = unit_begin(c + 1, U, p.G);
+        t_first = (int)(u0 / p.nk);
+        nseg_last = (int)((u1 - 1) / p.nk);
+    }
     // The loops below run on single threads, where integer latency is not
     // hidden: positions advance incrementally instead of by division.
     const int n_units = (int)(u1 - u0);
-    const int t_first = (int)(u0 / p.nk);
     const int ks_first = (int)(u0 - (int64_t)t_first * p.nk);
-    const int nseg = (int)((u1 - 1) / p.nk) - t_first + 1;
+    const int nseg = nseg_last - t_first + 1;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES), aready0 = smem_u32(bars + 2 * STAGES);
     const uint32_t accf0 = smem_u32(bars + 3 * STAGES), acce0 = smem_u32(bars + 3 * STAGES + 2);
     const uint32_t drainb = smem_u32(bars + 3 * STAGES + 4);
@@ -892,8 +907,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     };
 
     if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmSW);
+        // the stages' TMA barriers first: with static weights the weight
+        // stream starts before anything else is set up
+        for (int s = 0; s < STAGES; s++) mbar_init(full0 + 8 * s, 1);
+        fence_barrier_init();
+        if (!p.stall && p.w_before_wait) {
+            int t = t_first, ks = ks_first;
+            for (int i = 0; i < npre; i++) {
+                mbar_arrive_expect_tx(full0 + 8 * i, tx);
+                load_w(t, ks, i);
+                advance(t, ks);
+            }
+        }
         for (int s = 0; s < STAGES; s++) {
-            mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
             mbar_init(aready0 + 8 * s, 1);  // fused: the stage's quantizer warp
         }
@@ -905,17 +933,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         mbar_init(amaxb, p.csize);  // fused, computed s_g: one arrival per CTA of the cluster
         *abort_flag = 0u;
         fence_barrier_init();
-        tma_prefetch_desc(&tmW);
-        tma_prefetch_desc(&tmSW);
         if (!FUSED) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmSA);
         }
-        // The weight stream depends on no earlier kernel (the one before may
-        // still be quantizing the activations): start it at once, while warp
-        // 1 allocates tensor memory.
-        if (!p.stall) {
-            if (!p.w_before_wait) grid_dep_wait();
+        // Without the static-weights promise the weight stream starts after
+        // the wait for the preceding kernel (which may have written W), while
+        // warp 1 allocates tensor memory.
+        if (!p.stall && !p.w_before_wait) {
+            grid_dep_wait();
             int t = t_first, ks = ks_first;
             for (int i = 0; i < npre; i++) {
                 mbar_arrive_expect_tx(full0 + 8 * i, tx);
@@ -1310,15 +1336,26 @@ inline Plan plan(int64_t M, int64_t N, int64_t K, int sms)
     pl.ntiles = (int)((N + BMW - 1) / BMW);
     pl.csize = 1;
     const int64_t U = (int64_t)pl.ntiles * pl.nk;
+    // Whole tiles and cluster splits keep to half the SMs, so that the next
+    // launch's CTAs find free SMs at once (they start while this launch runs,
+    // and stream static weights): with one CTA per SM, consecutive calls on
+    // the same SMs would leave the memory idle through each CTA's start-up
+    // and tail.
+    const int half = sms / 2 > 0 ? sms / 2 : 1;
     if (pl.ntiles > sms) {
         pl.G = (int)(U < sms ? U : sms);
     } else if ((int64_t)pl.ntiles * 2 * MAX_CLUSTER <= sms) {
         int64_t split = sms / pl.ntiles;
         if (split > pl.nk) split = pl.nk;
         pl.G = (int)(pl.ntiles * split);
+    } else if (pl.ntiles > half) {
+        // two whole tiles per CTA where that adds up (an even tile count) and
+        // keeps each tile's K steps with the issuers a single tile gives them
+        // (nk a multiple of the issuer count: the same accumulation order)
+        pl.G = (pl.ntiles % 2 == 0 && pl.nk % NI == 0) ? pl.ntiles / 2 : pl.ntiles;
     } else {
         int split = 1;
-        while (split * 2 <= MAX_CLUSTER && (int64_t)pl.ntiles * split * 2 <= sms && split * 2 <= pl.nk) split *= 2;
+        while (split * 2 <= MAX_CLUSTER && (int64_t)pl.ntiles * split * 2 <= half && split * 2 <= pl.nk) split *= 2;
         pl.G = pl.ntiles * split;
         pl.csize = split;
     }
