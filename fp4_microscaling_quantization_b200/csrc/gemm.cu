@@ -711,49 +711,45 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
                                  volatile uint32_t *abort_flag)
 {
     constexpr int ND = Cfg::NB / BNA - 1;
+    constexpr int R = BNA * 8 / 32;  // units per lane of one K step (16 rows x 8 units)
     const float six_sg = __fmul_rn(6.0f, sg);
     const int nwork = p.M * 8;  // units of one K step: (row m, column cu = 0..7)
     for (int i = 0; i < n_units; i++) {
         const int s = i % Cfg::STAGES;
         if (s % NQ != qw) continue;
         const uint32_t ph = (uint32_t)((i / Cfg::STAGES) & 1);
-        if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) return false;
-        uint8_t *st = smem + s * Cfg::STAGE_BYTES;
-        uint8_t *sa = st + W_BYTES;
-        uint8_t *sfa = st + W_BYTES + Cfg::A_BYTES + SFW_BYTES;
         const int j0 = (int)(((int64_t)t_first * p.nk + ks_first + i) % p.nk) * 8;  // K step of unit i
-        uint4 raw[BNA * 8 / 32][4];
+        // Load and encode first, into registers; only the stores wait for the
+        // stage to be free, so the loads' latency overlaps the MMAs of the
+        // stage's previous use.
+        uint4 raw[R][4];
 #pragma unroll
-        for (int r = 0; r < BNA * 8 / 32; r++) {
+        for (int r = 0; r < R; r++) {
             const int w = r * 32 + lane;
             if (r * 32 < nwork) fetch_act_unit(p, w < nwork ? w >> 3 : p.M, j0 + (w & 7), raw[r]);
         }
+        uint4 nib[R];
+        uint32_t sb[R];
+        // residual lane, per unit: the terms' E2M1 codes (4 bits each) and the
+        // residual's index << 16, and the terms' scale bytes (8 bits each)
+        uint32_t tcodes[R], tscales[R];
 #pragma unroll
-        for (int r = 0; r < BNA * 8 / 32; r++) {
+        for (int r = 0; r < R; r++) {
             if (r * 32 >= nwork) break;  // warp-uniform
             const int w = r * 32 + lane;
-            const int m = w >> 3, cu = w & 7;
+            const int m = w >> 3;
             float v[32];
             unpack_unit(raw[r], v);
             if (HK) fwht_unit<HK>(v, p.ck, lane);
             uint32_t rw = 0;
             if (RES) rw = extract_residual(v);
-            uint4 nib;
-            const uint32_t sb = encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib);
-            if (w < nwork) {
-                *reinterpret_cast<uint4 *>(sa + m * 128 + ((cu ^ (m & 7)) << 4)) = nib;
-                if (QFMT == FP4_MXFP4)
-                    sfa[(cu >> 2) * 512 + m * 16 + (cu & 3)] = (uint8_t)sb;
-                else
-                    *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + m * 16 + 2 * (cu & 1)) = (uint16_t)sb;
-            }
-            if (RES && w < nwork) {
-                uint32_t code[ND > 0 ? ND : 1], sbyte[ND > 0 ? ND : 1];
+            sb[r] = encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib[r]);
+            if (RES) {
                 const float rv = bf16lo(rw);
-                const int idx = (int)((rw >> 16) & 31u);
+                uint32_t code[ND > 0 ? ND : 1], sbyte[ND > 0 ? ND : 1];
                 if (QFMT == FP4_NVFP4) {
                     // band 0 (rows 16-47) or band 1 (rows 48-79) of the row's scale
-                    const int E0 = rexp[m];
+                    const int E0 = w < nwork ? rexp[m] : 0;
                     const bool hi = fabsf(rv) >= exp2i(E0 - 2);
                     uint32_t tc[2], ts[2];
                     residual_terms_e4m3(__fmul_rn(rv, exp2i(hi ? -E0 : RES_BAND_SHIFT - E0)), tc, ts);
@@ -767,21 +763,48 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
                 } else {
                     residual_terms_e8m0(rv, code, sbyte);
                 }
+                tcodes[r] = rw & 0x1F0000u;
+                tscales[r] = 0;
 #pragma unroll
                 for (int d = 0; d < ND; d++) {
-                    const int R = BNA * (d + 1) + m;  // R & 7 == m & 7
+                    tcodes[r] |= code[d] << (4 * d);
+                    tscales[r] |= sbyte[d] << (8 * d);
+                }
+            }
+        }
+        if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag, &g_gemm_error, p.budget_ns)) return false;
+        uint8_t *st = smem + s * Cfg::STAGE_BYTES;
+        uint8_t *sa = st + W_BYTES;
+        uint8_t *sfa = st + W_BYTES + Cfg::A_BYTES + SFW_BYTES;
+#pragma unroll
+        for (int r = 0; r < R; r++) {
+            if (r * 32 >= nwork) break;  // warp-uniform
+            const int w = r * 32 + lane;
+            if (w >= nwork) continue;
+            const int m = w >> 3, cu = w & 7;
+            *reinterpret_cast<uint4 *>(sa + m * 128 + ((cu ^ (m & 7)) << 4)) = nib[r];
+            if (QFMT == FP4_MXFP4)
+                sfa[(cu >> 2) * 512 + m * 16 + (cu & 3)] = (uint8_t)sb[r];
+            else
+                *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + m * 16 + 2 * (cu & 1)) = (uint16_t)sb[r];
+            if (RES) {
+                const int idx = (int)(tcodes[r] >> 16);
+#pragma unroll
+                for (int d = 0; d < ND; d++) {
+                    const int Rw = BNA * (d + 1) + m;  // Rw & 7 == m & 7
+                    const uint32_t code = (tcodes[r] >> (4 * d)) & 0xFu, sbyte = (tscales[r] >> (8 * d)) & 0xFFu;
                     uint32_t wds[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                     for (int q = 0; q < 4; q++)
-                        if (q == (idx >> 3)) wds[q] = code[d] << (4 * (idx & 7));
-                    *reinterpret_cast<uint4 *>(sa + R * 128 + ((cu ^ (m & 7)) << 4)) =
+                        if (q == (idx >> 3)) wds[q] = code << (4 * (idx & 7));
+                    *reinterpret_cast<uint4 *>(sa + Rw * 128 + ((cu ^ (m & 7)) << 4)) =
                         make_uint4(wds[0], wds[1], wds[2], wds[3]);
-                    const int rb = (R & 31) * 16 + (R >> 5) * 4;  // row's bytes in a scale atom
+                    const int rb = (Rw & 31) * 16 + (Rw >> 5) * 4;  // row's bytes in a scale atom
                     if (QFMT == FP4_MXFP4)
-                        sfa[(cu >> 2) * 512 + rb + (cu & 3)] = (uint8_t)sbyte[d];
+                        sfa[(cu >> 2) * 512 + rb + (cu & 3)] = (uint8_t)sbyte;
                     else  // two 16-element blocks: the term's block takes the scale, the other 0
                         *reinterpret_cast<uint16_t *>(sfa + (cu >> 1) * 512 + rb + 2 * (cu & 1)) =
-                            (uint16_t)(sbyte[d] << (8 * (idx >> 4)));
+                            (uint16_t)(sbyte << (8 * (idx >> 4)));
                 }
             }
         }

@@ -46,6 +46,7 @@ struct QuantArgs {
     int mx_floor;           // MX scale: floor rule
     int gscale_computed;    // NVFP4: *gscale was set by the amax pass (see amax_kernel)
     uint32_t *res;          // sparse residual lane (one word per unit), or null
+    int wide;               // x and its row stride are 32-byte aligned: 32-byte loads
 };
 
 // Units processed per thread and loop trip: their loads are all issued
@@ -61,9 +62,30 @@ FP4_DEV void unit_rc(int64_t u, const FastDiv &upr, uint32_t &row, uint32_t &j)
 }
 
 // Raw bytes of unit j of row `row` (4 x 16-byte loads, read-only path).
-FP4_DEV void fetch_unit(const uint16_t *x, int64_t ld, uint32_t row, uint32_t j, uint4 *w)
+// 32-byte loads (one full sector per lane) when every unit starts on a
+// 32-byte boundary (x and its row stride 32-byte aligned), else 16-byte ones.
+FP4_DEV void ld_nc_v8(const void *p, uint4 &a, uint4 &b)
+{
+    asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+}
+
+FP4_DEV void ld_nc_v8_hint(const void *p, uint4 &a, uint4 &b, uint64_t pol)
+{
+    asm volatile("ld.global.nc.L2::cache_hint.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], %9;"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p), "l"(pol));
+}
+
+FP4_DEV void fetch_unit(const uint16_t *x, int64_t ld, uint32_t row, uint32_t j, uint4 *w, bool wide = false)
 {
     const uint4 *p = reinterpret_cast<const uint4 *>(x + (int64_t)row * ld + (int64_t)j * 32);
+    if (wide) {
+        ld_nc_v8(p, w[0], w[1]);
+        ld_nc_v8(p + 2, w[2], w[3]);
+        return;
+    }
 #pragma unroll
     for (int c = 0; c < 4; c++) w[c] = __ldg(p + c);
 }
@@ -85,9 +107,15 @@ FP4_DEV uint64_t l2_policy_evict_first()
     return pol;
 }
 
-FP4_DEV void fetch_unit_hint(const uint16_t *x, int64_t ld, uint32_t row, uint32_t j, uint4 *w, uint64_t pol)
+FP4_DEV void fetch_unit_hint(const uint16_t *x, int64_t ld, uint32_t row, uint32_t j, uint4 *w, uint64_t pol,
+                             bool wide = false)
 {
     const uint4 *p = reinterpret_cast<const uint4 *>(x + (int64_t)row * ld + (int64_t)j * 32);
+    if (wide) {
+        ld_nc_v8_hint(p, w[0], w[1], pol);
+        ld_nc_v8_hint(p + 2, w[2], w[3], pol);
+        return;
+    }
 #pragma unroll
     for (int c = 0; c < 4; c++)
         asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
@@ -151,7 +179,7 @@ __global__ void __launch_bounds__(256) amax_kernel(QuantArgs a)
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
                 unit_rc(u, a.upr_div, row[i], col[i]);
-                fetch_unit_hint(a.x, a.ld, row[i], col[i], raw[i], pol);
+                fetch_unit_hint(a.x, a.ld, row[i], col[i], raw[i], pol, a.wide);
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -222,7 +250,7 @@ FP4_DEV void quantize_body(const QuantArgs &a)
             const int64_t u = base + i * 32 + lane;
             if (u < a.total_units) {
                 unit_rc(u, a.upr_div, row[i], col[i]);
-                if (hinted) fetch_unit_hint(a.x, a.ld, row[i], col[i], raw[i], pol); else fetch_unit(a.x, a.ld, row[i], col[i], raw[i]);
+                if (hinted) fetch_unit_hint(a.x, a.ld, row[i], col[i], raw[i], pol, a.wide); else fetch_unit(a.x, a.ld, row[i], col[i], raw[i], a.wide);
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; c++) raw[i][c] = make_uint4(0, 0, 0, 0);
@@ -635,6 +663,7 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
     a.res = res;
+    a.wide = ((reinterpret_cast<uintptr_t>(x) & 31) == 0 && (ld * 2) % 32 == 0) ? 1 : 0;
     const int grid = grid_for(a.total_units, sms, QUNITS);
     void (*qk)(QuantArgs) = fmt == FP4_MXFP4   ? quant_kernel_pick<FP4_MXFP4>(hk, mse, res != nullptr)
                             : fmt == FP4_NVFP4 ? quant_kernel_pick<FP4_NVFP4>(hk, mse, res != nullptr)
@@ -746,6 +775,7 @@ cudaError_t launch_act_quantize(const uint16_t *x, int64_t rows, int64_t cols, i
     a.mx_floor = mx_floor;
     a.gscale_computed = (fmt == FP4_NVFP4 && !gscale_given) ? 1 : 0;
     a.res = nullptr;
+    a.wide = 0;
     void (*k)(QuantArgs, unsigned *, int, int) = fmt == FP4_MXFP4   ? act_kernel_for<FP4_MXFP4>(hk)
                                                  : fmt == FP4_NVFP4 ? act_kernel_for<FP4_NVFP4>(hk)
                                                                     : act_kernel_for<FP4_MXFP4_16>(hk);
@@ -949,6 +979,7 @@ cudaError_t launch_nv_refine(const uint16_t *x, int64_t rows, int64_t cols, int6
     a.mx_floor = 0;
     a.gscale_computed = 0;
     a.res = nullptr;
+    a.wide = 0;
     void (*uk)(QuantArgs, const RefineState *, double *) = nullptr;
     switch (hk) {
     case 0: uk = unit_stats_kernel_for_k<0>(); break;
