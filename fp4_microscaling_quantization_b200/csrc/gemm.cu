@@ -477,6 +477,7 @@ struct Params {
     // ldx elements; gA null = the NVFP4 tensor scale is computed from x.
     const uint16_t *x;
     int64_t ldx;
+    int xwide;           // x and its row stride are 32-byte aligned: 32-byte loads
     float ck;            // RN(1/sqrt(k)) of the rotation
     int round_away, mx_floor;
 };
@@ -513,6 +514,21 @@ FP4_DEV int quantizer_index(int warp) { return warp <= 5 ? warp - 2 : warp - 5; 
 
 // Named barrier over the NQ quantizer warps (id 2; id 1 is the epilogue's).
 FP4_DEV void quantizers_sync() { asm volatile("bar.sync 2, %0;" ::"n"(NQ * 32) : "memory"); }
+
+// True for all four epilogue warps (2-5) iff v holds in every one of their
+// threads: one abort decision for warps that then take the same sequence of
+// named barriers (a warp that left the loop alone would strand the others
+// at the reduction's bar.sync).
+FP4_DEV bool epilogue_all(bool v)
+{
+    int r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.s32 q, %1, 0;\n\tbar.red.and.pred p, 1, 128, q;\n\t"
+                 "selp.s32 %0, 1, 0, p;\n\t}"
+                 : "=r"(r)
+                 : "r"(v ? 1 : 0)
+                 : "memory");
+    return r != 0;
+}
 
 // Makes this thread's generic-proxy shared-memory writes visible to the
 // tensor cores' (async-proxy) reads that follow a barrier.
@@ -564,10 +580,22 @@ FP4_DEV void st_shared_cluster_f32(uint32_t addr_cluster, float v)
 // past M, or a column at or past K: they quantize to zero codes and zero
 // scales, finite as the product's K tail needs).  Read through L2 only: x
 // may be the output of the kernel this one overlapped.
+FP4_DEV void ld_cg_v8(const void *ptr, uint4 &a, uint4 &b)
+{
+    asm volatile("ld.global.cg.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(ptr));
+}
+
 FP4_DEV void fetch_act_unit(const Params &p, int m, int j, uint4 *raw)
 {
     if (m < p.M && j < p.K / 32) {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (int64_t)m * p.ldx + (int64_t)j * 32);
+        if (p.xwide) {  // two 32-byte loads: a full sector per lane
+            ld_cg_v8(src, raw[0], raw[1]);
+            ld_cg_v8(src + 2, raw[2], raw[3]);
+            return;
+        }
 #pragma unroll
         for (int c = 0; c < 4; c++) raw[c] = __ldcg(src + c);
     } else {
@@ -656,7 +684,7 @@ FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float 
 {
     const int ncols = j1 - j0;
     const int total = p.M * ncols;
-    constexpr int U = 2;  // units per lane and trip, loads issued together
+    constexpr int U = 4;  // units per lane and trip, loads issued together
     float mx = 0.0f;
     for (int base = qw * 32 * U; base < total; base += NQ * 32 * U) {
         uint4 raw[U][4];
@@ -1138,9 +1166,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     const float alpha = (FMT == FP4_NVFP4 && !p.sf_e8m0) ? __fmul_rn(FUSED ? sg : *p.gA, *p.gW) : 1.0f;
     for (int seg = 0; seg < nseg; seg++) {
         const int b = seg & 1;
-        bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag, &g_gemm_error, p.budget_ns);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) break;
+        const bool ok = !*abort_flag && mbar_wait_bounded(accf0 + 8 * b, (uint32_t)((seg >> 1) & 1), abort_flag,
+                                                          &g_gemm_error, p.budget_ns);
+        if (!epilogue_all(ok)) break;
         tc_fence_after();
         // the segment's units and the issuers that own some of them
         const int i0 = seg == 0 ? 0 : (p.nk - ks_first) + (seg - 1) * p.nk;
@@ -1359,26 +1387,15 @@ inline Plan plan(int64_t M, int64_t N, int64_t K, int sms)
     pl.ntiles = (int)((N + BMW - 1) / BMW);
     pl.csize = 1;
     const int64_t U = (int64_t)pl.ntiles * pl.nk;
-    // Whole tiles and cluster splits keep to half the SMs, so that the next
-    // launch's CTAs find free SMs at once (they start while this launch runs,
-    // and stream static weights): with one CTA per SM, consecutive calls on
-    // the same SMs would leave the memory idle through each CTA's start-up
-    // and tail.
-    const int half = sms / 2 > 0 ? sms / 2 : 1;
     if (pl.ntiles > sms) {
         pl.G = (int)(U < sms ? U : sms);
     } else if ((int64_t)pl.ntiles * 2 * MAX_CLUSTER <= sms) {
         int64_t split = sms / pl.ntiles;
         if (split > pl.nk) split = pl.nk;
         pl.G = (int)(pl.ntiles * split);
-    } else if (pl.ntiles > half) {
-        // two whole tiles per CTA where that adds up (an even tile count) and
-        // keeps each tile's K steps with the issuers a single tile gives them
-        // (nk a multiple of the issuer count: the same accumulation order)
-        pl.G = (pl.ntiles % 2 == 0 && pl.nk % NI == 0) ? pl.ntiles / 2 : pl.ntiles;
     } else {
         int split = 1;
-        while (split * 2 <= MAX_CLUSTER && (int64_t)pl.ntiles * split * 2 <= half && split * 2 <= pl.nk) split *= 2;
+        while (split * 2 <= MAX_CLUSTER && (int64_t)pl.ntiles * split * 2 <= sms && split * 2 <= pl.nk) split *= 2;
         pl.G = pl.ntiles * split;
         pl.csize = split;
     }
@@ -1643,6 +1660,7 @@ cudaError_t launch_gemm(const uint8_t *Aq, const uint8_t *As, const float *gA, c
         dp.sf_e8m0 = fmt == FP4_MXFP4_16;
         dp.x = nullptr;
         dp.ldx = 0;
+        dp.xwide = 0;
         dp.ck = 1.0f;
         dp.round_away = dp.mx_floor = 0;
         return fmt == FP4_MXFP4 ? launch_decode<FP4_MXFP4, 0, false>(tw, ta, tsw, tsa, dp, pl.any_cut, st, pdl)
@@ -1769,6 +1787,7 @@ cudaError_t launch_linear_fused(const uint16_t *x, int64_t ldx, int64_t M, int64
     dp.sf_e8m0 = fmt == FP4_MXFP4_16;
     dp.x = x;
     dp.ldx = ldx;
+    dp.xwide = ((reinterpret_cast<uintptr_t>(x) & 31) == 0 && (ldx * 2) % 32 == 0) ? 1 : 0;
     dp.ck = ck;
     dp.round_away = round_away;
     dp.mx_floor = mx_floor;
