@@ -34,7 +34,7 @@ ROWS, COLS = 1024, 131072
 # dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of the MXFP4
 # quantize kernel on 512 rows of this workload, scaled by rows.  Set to None
 # whenever that kernel changes, until it is captured again.
-QUANT_MX_TRAFFIC_BYTES = None
+QUANT_MX_TRAFFIC_BYTES = 2 * (134_253_312 + 17_516_288)
 # Nominal B200 figures the fractions are also given against ("frac_spec"):
 # ~8 TB/s HBM3e and ~9 PFLOP/s dense FP4 (the gpt-oss MXFP4 article's B200
 # paragraph).  "frac" is always against the measured peaks.
@@ -160,7 +160,9 @@ def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None, m_list=(1, 4, 16
     the timed call (fp4_linear), W 14336x4096 and 4096x14336 pre-quantized,
     BF16 out.  W copies are rotated so the weight stream comes from HBM.  The
     weights are marked static (prepared once, read-only), so each call's
-    decode kernel streams its W while the previous call finishes."""
+    decode kernel streams its W while the previous call finishes.  Each
+    format's weights are also timed with the sparse residual lane
+    (fp4_linear_residual, no rotation), the "_residual_" rows."""
     hbm, kind = peaks()
     res = {"peak_gbs": hbm, "peak_kind": kind, "copies": 0, "cases": {}}
     for (N, K) in shapes:
@@ -198,6 +200,19 @@ def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None, m_list=(1, 4, 16
                 gbs = b / (ms * 1e-3) / 1e9
                 res["cases"][f"{name}_M{M}_N{N}_K{K}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm,
                                                           "frac_spec": gbs / SPEC_HBM_GBS}
+                if wfmt != fmt:
+                    continue
+
+                # the same call with the sparse residual lane (TransFP4 Eq.(3))
+                def call_res():
+                    W = Ws[it[0] % copies]
+                    it[0] += 1
+                    fp4.linear_residual(x, W, fmt, out=C, weights_static=True)
+
+                ms = time_graph(torch, call_res, 3, reps * copies)
+                gbs = b / (ms * 1e-3) / 1e9
+                res["cases"][f"{name}_residual_M{M}_N{N}_K{K}"] = {"us": ms * 1e3, "gbs": gbs, "frac": gbs / hbm,
+                                                                   "frac_spec": gbs / SPEC_HBM_GBS}
             del Ws, W0
         del wd
     torch.cuda.empty_cache()
