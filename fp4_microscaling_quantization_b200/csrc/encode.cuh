@@ -31,21 +31,67 @@ FP4_DEV void unpack_unit(const uint4 *raw, float *v)
     }
 }
 
+// Two-wide fp32 arithmetic (sm_100's packed f32x2 add, sub and multiply):
+// each half is rounded to nearest even exactly as the scalar operation, and
+// subnormals are kept (no .ftz), so results are those of two __fadd_rn /
+// __fsub_rn / __fmul_rn calls, in half the instructions (checked on the B200
+// over random operands of every class).  One hazard: ptxas contracts a packed
+// product that feeds a packed sum or difference into a fused multiply-add
+// (CUDA 12.9, sm_100a, in spite of .rn and -fmad=false), which skips the
+// product's rounding.  So no packed product here feeds an add or subtract:
+// the packed multiplies come last (the rotation's c_k, the block scales),
+// and sums of products stay scalar.
+// (a0, a1), (b0, b1) -> (a0 + b0, a1 + b1), (a0 - b0, a1 - b1)
+FP4_DEV void add_sub_x2(float &a0, float &a1, float &b0, float &b1)
+{
+    asm("{\n\t.reg .b64 pa, pb, ps, pd;\n\t"
+        "mov.b64 pa, {%0, %1};\n\tmov.b64 pb, {%2, %3};\n\t"
+        "add.rn.f32x2 ps, pa, pb;\n\tsub.rn.f32x2 pd, pa, pb;\n\t"
+        "mov.b64 {%0, %1}, ps;\n\tmov.b64 {%2, %3}, pd;\n\t}"
+        : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+
+// (a0, a1) *= (m0, m1)
+FP4_DEV void mul_x2(float &a0, float &a1, float m0, float m1)
+{
+    asm("{\n\t.reg .b64 pa, pm;\n\t"
+        "mov.b64 pa, {%0, %1};\n\tmov.b64 pm, {%2, %3};\n\t"
+        "mul.rn.f32x2 pa, pa, pm;\n\tmov.b64 {%0, %1}, pa;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(m0), "f"(m1));
+}
+
+// v[j] *= m0 and v[j + 16] *= m1 for j < 16: the two 16-element halves of a
+// unit (one scale each for 16-element blocks; m0 = m1 for one scale).
+FP4_DEV void scale_halves(float *v, float m0, float m1)
+{
+#pragma unroll
+    for (int j = 0; j < 16; j++) mul_x2(v[j], v[j + 16], m0, m1);
+}
+
 // Normalised Sylvester Walsh-Hadamard transform of every k-chunk, stages
 // h = 1, 2, ..., k/2 in ascending order: (a, b) -> (a + b, a - b) with a the
 // element whose index has bit h clear; then every value times ck.  Stages
-// with h >= 32 pair this lane with lane ^ (h / 32).
+// with h >= 32 pair this lane with lane ^ (h / 32).  Stages h < 16 run two
+// butterflies per instruction, one in each 16-element half of the unit
+// (elements j and j + 16 share a packed operand).
 template <int HK>
 FP4_DEV void fwht_unit(float *v, float ck, int lane)
 {
 #pragma unroll
-    for (int h = 1; h < (HK < 32 ? HK : 32); h <<= 1) {
+    for (int h = 1; h < (HK < 16 ? HK : 16); h <<= 1) {
 #pragma unroll
-        for (int j = 0; j < 32; j++) {
+        for (int j = 0; j < 16; j++) {
             if (j & h) continue;
-            float a = v[j], b = v[j + h];
+            add_sub_x2(v[j], v[j + 16], v[j + h], v[j + h + 16]);
+        }
+    }
+    if (HK >= 32) {
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+            const float a = v[j], b = v[j + 16];
             v[j] = __fadd_rn(a, b);
-            v[j + h] = __fsub_rn(a, b);
+            v[j + 16] = __fsub_rn(a, b);
         }
     }
 #pragma unroll
@@ -60,8 +106,7 @@ FP4_DEV void fwht_unit(float *v, float ck, int lane)
             v[j] = __fadd_rn(o, __uint_as_float(__float_as_uint(v[j]) ^ flip));
         }
     }
-#pragma unroll
-    for (int j = 0; j < 32; j++) v[j] = __fmul_rn(v[j], ck);
+    scale_halves(v, ck, ck);
 }
 
 FP4_DEV float nv_global_from_amax(float amax)
@@ -165,31 +210,24 @@ FP4_DEV uint32_t encode_unit(float *v, float sg, float six_sg, int round_away, i
         const float amax = absmax_tree<32>(v);
         const int e = mx_exponent(amax, mx_floor);
         const float inv = exp2i(-e);
-#pragma unroll
-        for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
+        scale_halves(v, inv, inv);
         sbytes = (uint32_t)(e + 127);
     } else if (FMT == FP4_MXFP4_16) {
-        sbytes = 0;
-#pragma unroll
-        for (int b = 0; b < 2; b++) {
-            const int e = mx_exponent(absmax_tree<16>(v + 16 * b), mx_floor);
-            const float inv = exp2i(-e);
-#pragma unroll
-            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], inv);
-            sbytes |= (uint32_t)(e + 127) << (8 * b);
-        }
+        const int e0 = mx_exponent(absmax_tree<16>(v), mx_floor);
+        const int e1 = mx_exponent(absmax_tree<16>(v + 16), mx_floor);
+        scale_halves(v, exp2i(-e0), exp2i(-e1));
+        sbytes = (uint32_t)(e0 + 127) | ((uint32_t)(e1 + 127) << 8);
     } else {
+        float r[2];
         sbytes = 0;
 #pragma unroll
         for (int b = 0; b < 2; b++) {
             const float amax = absmax_tree<16>(v + 16 * b);
-            const float t = __fdiv_rn(amax, six_sg);
-            const uint32_t sb = e4m3_rn(t);
-            const float r = tab ? tab->r[sb] : nv_encode_factor(__fmul_rn(sg, e4m3_to_f32(sb)));
-#pragma unroll
-            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], r);
+            const uint32_t sb = e4m3_rn(__fdiv_rn(amax, six_sg));
+            r[b] = tab ? tab->r[sb] : nv_encode_factor(__fmul_rn(sg, e4m3_to_f32(sb)));
             sbytes |= sb << (8 * b);
         }
+        scale_halves(v, r[0], r[1]);
     }
     e2m1_pack_unit(v, round_away, out);
     return sbytes;
@@ -235,6 +273,8 @@ FP4_DEV float block_sq_error(const float *x, float r, float d, int round_away)
     float t[N / 2];
 #pragma unroll
     for (int i = 0; i < N / 2; i++) {
+        // scalar: a packed product here would be contracted into the
+        // following subtraction (see add_sub_x2)
         const float a0 = fabsf(x[2 * i]), a1 = fabsf(x[2 * i + 1]);
         const float y0 = __fmul_rn(e2m1_grid_magnitude(__fmul_rn(a0, r), round_away), d);
         const float y1 = __fmul_rn(e2m1_grid_magnitude(__fmul_rn(a1, r), round_away), d);
@@ -278,19 +318,13 @@ FP4_DEV uint32_t encode_unit_mse(float *v, float six_sg, int round_away, const N
     if (FMT == FP4_MXFP4) {
         const int e = mx_mse_exponent<32>(v, round_away);
         const float inv = exp2i(-e);
-#pragma unroll
-        for (int i = 0; i < 32; i++) v[i] = __fmul_rn(v[i], inv);
+        scale_halves(v, inv, inv);
         sbytes = (uint32_t)(e + 127);
     } else if (FMT == FP4_MXFP4_16) {
-        sbytes = 0;
-#pragma unroll
-        for (int b = 0; b < 2; b++) {
-            const int e = mx_mse_exponent<16>(v + 16 * b, round_away);
-            const float inv = exp2i(-e);
-#pragma unroll
-            for (int i = 0; i < 16; i++) v[16 * b + i] = __fmul_rn(v[16 * b + i], inv);
-            sbytes |= (uint32_t)(e + 127) << (8 * b);
-        }
+        const int e0 = mx_mse_exponent<16>(v, round_away);
+        const int e1 = mx_mse_exponent<16>(v + 16, round_away);
+        scale_halves(v, exp2i(-e0), exp2i(-e1));
+        sbytes = (uint32_t)(e0 + 127) | ((uint32_t)(e1 + 127) << 8);
     } else {
         sbytes = 0;
 #pragma unroll
@@ -309,11 +343,9 @@ FP4_DEV uint32_t encode_unit_mse(float *v, float six_sg, int round_away, const N
                     best_err = err;
                 }
             }
-            const float r = tab->r[best];
-#pragma unroll
-            for (int i = 0; i < 16; i++) x[i] = __fmul_rn(x[i], r);
             sbytes |= (uint32_t)best << (8 * b);
         }
+        scale_halves(v, tab->r[sbytes & 0xFF], tab->r[sbytes >> 8]);
     }
     e2m1_pack_unit(v, round_away, out);
     return sbytes;

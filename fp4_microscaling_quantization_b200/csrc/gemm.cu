@@ -322,7 +322,8 @@ pgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     if (n >= p.N || !in_layout) break;
                     float v[32];
 #pragma unroll
-                    for (int e = 0; e < 32; e++) v[e] = __fmul_rn(__uint_as_float(r[32 * u + e]), alpha);
+                    for (int e = 0; e < 32; e++) v[e] = __uint_as_float(r[32 * u + e]);
+                    scale_halves(v, alpha, alpha);
                     uint4 nib;
                     uint32_t sb = encode_unit<QF>(v, sgc, six_sgc, p.round_away, p.mx_floor, nib);
                     if (m < p.M)
