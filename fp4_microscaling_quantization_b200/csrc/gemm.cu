@@ -413,6 +413,10 @@ constexpr int TMEM_COLS = 512;
 constexpr int NI = 4;                        // MMA issuer warps (warps 1, 6, 7, 8) at most
 constexpr int SF_STAGE_COLS = 32;            // W scales 16 cols, activation scales 16 cols
 constexpr int MAX_CLUSTER = 8;               // portable cluster size
+// A cluster split's CTAs each read all of x for the NVFP4 tensor maximum
+// while x (M x K bf16) is at most this large, instead of exchanging their
+// K slices' maxima (a cross-CTA wait that costs more than the extra reads).
+constexpr int64_t X_LOCAL_AMAX_BYTES = int64_t(64) << 10;
 
 // Stage and tensor-memory layout of a decode_kernel variant.  A stage holds
 // [W tile 128 x 256 | activation rows NB x 256 | W scale atoms | activation
@@ -1019,9 +1023,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         fence_proxy_async_smem();
     }
     tc_fence_before();
-    // fused cluster split: the amax barriers of every CTA are initialised
-    // before any CTA arrives on a peer's
-    if (FUSED && p.csize > 1) cluster_sync(); else __syncthreads();
+    // fused cluster split with the tensor maximum exchanged: the amax
+    // barriers of every CTA are initialised before any CTA arrives on a peer's
+    const bool amax_exchange = FUSED && QFMT == FP4_NVFP4 && p.csize > 1 &&
+                               (RES || (!p.gA && (int64_t)p.M * p.K * 2 > X_LOCAL_AMAX_BYTES));
+    if (amax_exchange) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -1127,19 +1133,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         if (QFMT == FP4_NVFP4 && (RES || !p.gA)) {
             // One pass over x before any encoding: max |H_k x| for a computed
             // s_g (of the FP4 stream with the residual lane) and, with the
-            // lane, each row's largest residual.  Whole tiles cover all of K;
-            // the CTAs of a cluster split each take their K slice and combine
-            // the tensor maxima through distributed shared memory, whose slices
-            // cover K.  A row exponent is per CTA: its partial is scaled before
-            // the cluster adds them.
+            // lane, each row's largest residual.  Whole tiles cover all of K,
+            // and so does every CTA of a cluster split while x is small; with
+            // amax_exchange the CTAs of a cluster split each take their K
+            // slice and combine the tensor maxima through distributed shared
+            // memory, whose slices cover K.  A row exponent is per CTA: its
+            // partial is scaled before the cluster adds them.
             const int K32 = p.K / 32;
-            const int j0 = p.csize > 1 ? ks_first * 8 : 0;
-            const int j1 = p.csize > 1 ? min((ks_first + n_units) * 8, K32) : K32;
+            const bool slice = p.csize > 1 && (RES || amax_exchange);
+            const int j0 = slice ? ks_first * 8 : 0;
+            const int j1 = slice ? min((ks_first + n_units) * 8, K32) : K32;
             float mx = act_amax<HK, RES>(p, j0, j1, qw, lane, s_red, s_rowmax);
             if (p.gA) {
                 sg = *p.gA;
             } else {
-                if (p.csize > 1) {
+                if (amax_exchange) {
                     if (qw == 0 && lane < p.csize) {
                         const uint32_t rk = cluster_ctarank();
                         st_shared_cluster_f32(mapa_shared(smem_u32(&s_amax[rk]), (uint32_t)lane), mx);

@@ -124,12 +124,14 @@ def test_static_activation_scale(fp4, M, N, K):
     assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
 
 
-def test_zero_and_single_outlier_activations(fp4):
+@pytest.mark.parametrize("M,N,K", [(4, 2048, 2048), (16, 2048, 10240)])
+def test_zero_and_single_outlier_activations(fp4, M, N, K):
     """All-zero activations give C = 0 (NVFP4 s_g = 1, zero scales); one
-    nonzero activation in a cluster split sets the tensor maximum of every
-    CTA of the cluster, including those whose K slice holds only zeros."""
+    nonzero activation sets the tensor maximum of every CTA of a cluster
+    split: each CTA reads all of x (16 KB of x), or the CTAs exchange their
+    K slices' maxima (320 KB), including those whose slice holds only
+    zeros."""
     import torch
-    M, N, K = 4, 2048, 2048
     _, w = inputs.decode_linear(1, N, K, seed=5)
     for fmt in (MX, NV, MX16):
         W = fp4.quantize(to_dev_bf16(w), fmt)
