@@ -154,6 +154,34 @@ def bench_rotate(torch, fp4, inputs, dev, reps: int, fmts=None):
     return res
 
 
+def bench_l2_encode(torch, fp4, inputs, dev, reps: int):
+    """The encode pass of NVFP4 with a computed tensor scale, on its own
+    footing: MXFP4 and NVFP4 (a static s_g, so no tensor-maximum pass)
+    quantize of one 8192x4096 bf16 tensor (the rotate workload, k = 0) that
+    stays in L2 (67 MB).  Three untimed calls of each come first, in that
+    order (after one call of each that allocates the outputs): the launches a
+    profiler captures.  Then each is timed in a graph of calls on the same
+    tensor."""
+    hbm, kind = peaks()
+    x = inputs.rotate_acts()
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    g = torch.tensor([0.0123], dtype=torch.float32, device=dev)
+    om = fp4.quantize(xd, fp4.FP4_MXFP4)
+    on = fp4.quantize(xd, fp4.FP4_NVFP4, gscale=g)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        fp4.quantize(xd, fp4.FP4_MXFP4, out=om)
+    for _ in range(3):
+        fp4.quantize(xd, fp4.FP4_NVFP4, gscale=g, out=on)
+    torch.cuda.synchronize()
+    res = {"peak_gbs": hbm, "peak_kind": kind, "workload": "quantize 8192x4096 bf16, x in L2", "cases": {}}
+    for name, fn in (("mxfp4", lambda: fp4.quantize(xd, fp4.FP4_MXFP4, out=om)),
+                     ("nvfp4_static", lambda: fp4.quantize(xd, fp4.FP4_NVFP4, gscale=g, out=on))):
+        ms = time_graph(torch, fn, 3, reps * 8)
+        res["cases"][name] = {"us": ms * 1e3}
+    return res
+
+
 def bench_decode(torch, fp4, inputs, dev, reps: int, fmts=None, m_list=(1, 4, 16),
                  shapes=((14336, 4096), (4096, 14336))):
     """Decode shapes: M in {1,4,16} bf16 activations quantized online inside
@@ -403,6 +431,8 @@ def run_ours(args):
             r = bench_prefill(torch, fp4, inputs, dev, reps=args.steps, M=args.prefill_m, fmts=args.fmts)
         elif args.only == "rotate":
             r = bench_rotate(torch, fp4, inputs, dev, reps=args.steps, fmts=args.fmts)
+        elif args.only == "l2-encode":
+            r = bench_l2_encode(torch, fp4, inputs, dev, reps=args.steps)
         else:
             kw = {}
             if args.decode_m:
@@ -651,8 +681,8 @@ def main():
     ap.add_argument("--rows", type=int, default=ROWS, help="rows of the tensor (profiling runs use fewer)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-gemm", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "rotate"], default=None,
-                    help="profiling helper: run one GEMM leg alone")
+    ap.add_argument("--only", choices=["prefill", "decode", "rotate", "l2-encode"], default=None,
+                    help="profiling helper: run one leg alone")
     ap.add_argument("--prefill-m", type=int, default=8192)
     ap.add_argument("--fmts", nargs="*", default=None)
     ap.add_argument("--decode-m", type=int, nargs="*", default=None, help="--only decode: activation rows")

@@ -505,17 +505,20 @@ FP4_DEV void store_row(const Params &p, int n, const float *acc, float alpha)
     }
 }
 
-// Threads: warp 0 loads, warps 1, 6, 7, 8 issue MMAs, warps 2-5 drain the
-// accumulators (warp w may read TMEM lanes 32 (w % 4) .. + 31).  The fused
-// variants (fp4_linear, fp4_linear_residual) add warps 9-12: with warps 2-5
+// Threads: warp 0 loads, warps 1 and 6 .. 4 + NIS issue MMAs (NIS issuers:
+// 1, 6, 7, 8 for four), warps 2-5 drain the accumulators (warp w may read
+// TMEM lanes 32 (w % 4) .. + 31).  The fused variants (fp4_linear,
+// fp4_linear_residual) add four warps after the issuers: with warps 2-5
 // they quantize the activations into the stages before the accumulators
-// are drained.
-constexpr int NQ_EXTRA = 4;                  // warps 9 .. 12 of the fused variants
+// are drained.  (Thirteen warps cap a thread at 128 registers, as four of
+// them share one SM sub-partition's 16K; twelve allow 168.)
+constexpr int NQ_EXTRA = 4;                  // warps 5 + NIS .. 8 + NIS of the fused variants
 constexpr int NQ = 4 + NQ_EXTRA;             // activation quantizer warps of the fused variants
-__host__ __device__ constexpr int decode_threads(bool fused) { return 32 * (6 + NI - 1 + (fused ? NQ_EXTRA : 0)); }
+__host__ __device__ constexpr int decode_threads(bool fused, int nis) { return 32 * (6 + nis - 1 + (fused ? NQ_EXTRA : 0)); }
 
-// Quantizer warp index of warp w (fused variants): warps 2-5 -> 0-3, 9-12 -> 4-7.
-FP4_DEV int quantizer_index(int warp) { return warp <= 5 ? warp - 2 : warp - 5; }
+// Quantizer warp index of warp w (fused variants): warps 2-5 -> 0-3, the
+// four after the issuers -> 4-7.
+FP4_DEV int quantizer_index(int warp, int nis) { return warp <= 5 ? warp - 2 : warp - nis - 1; }
 
 // Named barrier over the NQ quantizer warps (id 2; id 1 is the epilogue's).
 FP4_DEV void quantizers_sync() { asm volatile("bar.sync 2, %0;" ::"n"(NQ * 32) : "memory"); }
@@ -870,7 +873,7 @@ FP4_DEV void store_row_res(const Params &p, int n, const float *acc, const float
 // comes quantized (fp4_gemm).  RES (fused only): the sparse residual lane in
 // the product (fp4_linear_residual), one tile segment per CTA.
 template <int QFMT, int HK, bool FUSED, bool RES>
-__global__ void __launch_bounds__(decode_threads(FUSED), 1)
+__global__ void __launch_bounds__(decode_threads(FUSED, std::conditional<RES, DRes<QFMT>, DPlain>::type::NIS), 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
               const __grid_constant__ CUtensorMap tmSW, const __grid_constant__ CUtensorMap tmSA, Params p)
 {
@@ -1061,7 +1064,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             }
         }
         __syncwarp();
-    } else if (warp == 1 || (warp >= 6 && warp <= 8)) {
+    } else if (warp == 1 || (warp >= 6 && warp < 5 + NIS)) {
         const int j = warp == 1 ? 0 : warp - 5;  // issuer index
         if (lane == 0 && j < NIS) {
             // Descriptors of stage 0: a stage, atom or K step only moves the
@@ -1129,7 +1132,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     float sg = 1.0f;  // the activations' NVFP4 tensor scale (fused)
     if (FUSED) {
         grid_dep_launch();
-        const int qw = quantizer_index(warp);
+        const int qw = quantizer_index(warp, NIS);
         if (QFMT == FP4_NVFP4 && (RES || !p.gA)) {
             // One pass over x before any encoding: max |H_k x| for a computed
             // s_g (of the FP4 stream with the residual lane) and, with the
@@ -1168,7 +1171,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
         quantize_act_stages<QFMT, HK, RES, Cfg>(p, smem, aready0, empty0, n_units, t_first, ks_first, qw, lane, sg,
                                                 s_rexp, abort_flag);
     }
-    if (!FUSED || warp <= 5) {  // warps 9-12 only quantize
+    if (!FUSED || warp <= 5) {  // the four warps after the issuers only quantize
     // ---------------- epilogue warps 2-5: one result per tile segment ----------------
     // warp w may only read TMEM lanes 32*(w%4) .. 32*(w%4)+31
     const int quarter = warp & 3;
@@ -1597,7 +1600,7 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
     if (cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), smem); e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
-    cfg.blockDim = dim3(decode::decode_threads(FUSED));
+    cfg.blockDim = dim3(decode::decode_threads(FUSED, RES ? decode::DRes<QFMT>::NIS : decode::DPlain::NIS));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];

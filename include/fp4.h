@@ -302,7 +302,12 @@ fp4_status fp4_linear_workspace_size(int64_t M, int64_t N, int64_t K, int fmt, s
  * format, optionally rotated by H_k ("FP4 quantization analysis" §3.2.3:
  * activations rotated online, weights rotated offline — W must have been
  * quantized with the same hadamard_k), then C = alpha * x_q W_q^T as in
- * fp4_gemm.  M <= 16 is the decode case the weight stream dominates.
+ * fp4_gemm.  M <= 16 is the decode case the weight stream dominates: one
+ * kernel launch, whose warps quantize each 256-wide K step of x straight
+ * into the pipeline stage the tensor cores read (bit-identical to
+ * fp4_quantize + fp4_gemm with the same work split).  Splits that cut tiles
+ * between CTAs outside a cluster (very few or very many 128-row W tiles)
+ * take two launches: the activation quantizer, then fp4_gemm's kernel.
  *   gA      NVFP4 activation tensor scale: NULL = computed from x (dynamic),
  *           else a device fp32 holding a static s_g.  Ignored for MXFP4 and
  *           MXFP4_16.
