@@ -430,10 +430,11 @@ constexpr int64_t X_LOCAL_AMAX_BYTES = int64_t(64) << 10;
 // an issuer then waits for every phase of its stages' barriers in turn, which
 // is what their parity waits need (a barrier two phases further than its
 // waiter last saw reads as ready).
-template <int ND, int NSTAGES, int NISSUERS>
+template <int ND, int NSTAGES, int NISSUERS, int NQX>
 struct DCfg {
     static constexpr int STAGES = NSTAGES;
     static constexpr int NIS = NISSUERS;
+    static constexpr int NQ = 4 + NQX;  // fused variants: activation quantizer warps (2-5 and NQX more)
     static constexpr int NB = BNA * (1 + ND);
     static constexpr int A_BYTES = NB * BK / 2;
     static constexpr int STAGE_BYTES = W_BYTES + A_BYTES + SFW_BYTES + SFA_BYTES;
@@ -446,15 +447,18 @@ struct DCfg {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     static_assert(NB <= 128, "one 128-row scale atom covers the activation rows");
 };
-// fp4_gemm's and fp4_linear's decode kernels: 8 stages of 22 KB, 4 issuers
-using DPlain = DCfg<0, 8, 4>;
+// fp4_gemm's and fp4_linear's decode kernels: 8 stages of 22 KB, 4 issuers,
+// 8 quantizer warps (fused: 13 warps in all, one per stage: with 7 quantizers
+// and so 12 warps, the warp writing two stages held M = 16 back by 2.4 to
+// 3.5 us, more than the spills of 13 warps cost)
+using DPlain = DCfg<0, 8, 4, 4>;
 // the residual lane (fp4_linear_residual): 4 groups of term rows, 6 stages
-// of 30 KB, 3 issuers (warp 8 stays idle).
+// of 30 KB, 3 issuers, 8 quantizer warps (12 warps in all).
 // E8M0-scaled terms have two significant bits, so a bf16 value takes up to 4
 // (MXFP4, MXFP4_16); E4M3-scaled terms have four, so 2, in one of two bands
 // of a row's scale (NVFP4)
 template <int QFMT>
-using DRes = DCfg<4, 6, 3>;
+using DRes = DCfg<4, 6, 3, 4>;
 struct Params {
     float *ws;           // partials: [G][maxseg][128][16]
     // Fused reduction (counters != nullptr): per-tile arrival counters, zero
@@ -508,19 +512,22 @@ FP4_DEV void store_row(const Params &p, int n, const float *acc, float alpha)
 // Threads: warp 0 loads, warps 1 and 6 .. 4 + NIS issue MMAs (NIS issuers:
 // 1, 6, 7, 8 for four), warps 2-5 drain the accumulators (warp w may read
 // TMEM lanes 32 (w % 4) .. + 31).  The fused variants (fp4_linear,
-// fp4_linear_residual) add four warps after the issuers: with warps 2-5
-// they quantize the activations into the stages before the accumulators
-// are drained.  (Thirteen warps cap a thread at 128 registers, as four of
-// them share one SM sub-partition's 16K; twelve allow 168.)
-constexpr int NQ_EXTRA = 4;                  // warps 5 + NIS .. 8 + NIS of the fused variants
-constexpr int NQ = 4 + NQ_EXTRA;             // activation quantizer warps of the fused variants
-__host__ __device__ constexpr int decode_threads(bool fused, int nis) { return 32 * (6 + nis - 1 + (fused ? NQ_EXTRA : 0)); }
+// fp4_linear_residual) add NQX warps after the issuers: with warps 2-5 they
+// quantize the activations into the stages before the accumulators are
+// drained.  Thirteen warps cap a thread at 128 registers (four of them
+// share one SM sub-partition's 16K) and the NVFP4 quantizers spill; twelve
+// (the residual variant, one issuer fewer) allow 168.
+__host__ __device__ constexpr int decode_threads(bool fused, int nis, int nqx)
+{
+    return 32 * (6 + nis - 1 + (fused ? nqx : 0));
+}
 
 // Quantizer warp index of warp w (fused variants): warps 2-5 -> 0-3, the
-// four after the issuers -> 4-7.
+// warps after the issuers -> 4, 5, ...
 FP4_DEV int quantizer_index(int warp, int nis) { return warp <= 5 ? warp - 2 : warp - nis - 1; }
 
 // Named barrier over the NQ quantizer warps (id 2; id 1 is the epilogue's).
+template <int NQ>
 FP4_DEV void quantizers_sync() { asm volatile("bar.sync 2, %0;" ::"n"(NQ * 32) : "memory"); }
 
 // True for all four epilogue warps (2-5) iff v holds in every one of their
@@ -687,7 +694,7 @@ FP4_DEV int residual_row_exponent(float rowmax)
 // RES: the maximum is that of the FP4 stream (each unit's residual value
 // removed), and rowmax[m] (shared, zero on entry, float bits) receives the
 // largest residual magnitude of row m.
-template <int HK, bool RES>
+template <int HK, bool RES, int NQ>
 FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float *red, unsigned *rowmax)
 {
     const int ncols = j1 - j0;
@@ -718,7 +725,7 @@ FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float 
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
     if (lane == 0) red[qw] = mx;
-    quantizers_sync();
+    quantizers_sync<NQ>();
     float t = red[0];
 #pragma unroll
     for (int w = 1; w < NQ; w++) t = fmaxf(t, red[w]);
@@ -752,7 +759,7 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
     const int nwork = p.M * 8;  // units of one K step: (row m, column cu = 0..7)
     for (int i = 0; i < n_units; i++) {
         const int s = i % Cfg::STAGES;
-        if (s % NQ != qw) continue;
+        if (s % Cfg::NQ != qw) continue;
         const uint32_t ph = (uint32_t)((i / Cfg::STAGES) & 1);
         const int j0 = (int)(((int64_t)t_first * p.nk + ks_first + i) % p.nk) * 8;  // K step of unit i
         // Load and encode first, into registers; only the stores wait for the
@@ -873,7 +880,9 @@ FP4_DEV void store_row_res(const Params &p, int n, const float *acc, const float
 // comes quantized (fp4_gemm).  RES (fused only): the sparse residual lane in
 // the product (fp4_linear_residual), one tile segment per CTA.
 template <int QFMT, int HK, bool FUSED, bool RES>
-__global__ void __launch_bounds__(decode_threads(FUSED, std::conditional<RES, DRes<QFMT>, DPlain>::type::NIS), 1)
+__global__ void __launch_bounds__(decode_threads(FUSED, std::conditional<RES, DRes<QFMT>, DPlain>::type::NIS,
+                                                 std::conditional<RES, DRes<QFMT>, DPlain>::type::NQ - 4),
+                                  1)
 decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
               const __grid_constant__ CUtensorMap tmSW, const __grid_constant__ CUtensorMap tmSA, Params p)
 {
@@ -891,7 +900,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     // activations written), accfull[2], accempty[2], drain, amax (fused)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 6);
     __shared__ volatile unsigned s_last;
-    __shared__ float s_red[NQ];             // fused: per-warp maxima
+    __shared__ float s_red[Cfg::NQ];        // fused: per-warp maxima
     __shared__ float s_amax[MAX_CLUSTER];   // fused: the cluster CTAs' maxima, by rank
     __shared__ float s_sg;                  // fused: the activations' tensor scale
     __shared__ unsigned s_rowmax[BNA];      // residual lane, NVFP4: largest residual of each row (float bits)
@@ -1146,7 +1155,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             const bool slice = p.csize > 1 && (RES || amax_exchange);
             const int j0 = slice ? ks_first * 8 : 0;
             const int j1 = slice ? min((ks_first + n_units) * 8, K32) : K32;
-            float mx = act_amax<HK, RES>(p, j0, j1, qw, lane, s_red, s_rowmax);
+            float mx = act_amax<HK, RES, Cfg::NQ>(p, j0, j1, qw, lane, s_red, s_rowmax);
             if (p.gA) {
                 sg = *p.gA;
             } else {
@@ -1163,7 +1172,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
                 sg = nv_global_from_amax(mx);
             }
             if (RES && qw == 0 && lane < BNA) s_rexp[lane] = residual_row_exponent(__uint_as_float(s_rowmax[lane]));
-            quantizers_sync();  // s_rexp
+            quantizers_sync<Cfg::NQ>();  // s_rexp
         } else if (QFMT == FP4_NVFP4) {
             sg = *p.gA;
         }
@@ -1600,7 +1609,8 @@ static cudaError_t launch_decode(const CUtensorMap &tw, const CUtensorMap &ta, c
     if (cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), smem); e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
-    cfg.blockDim = dim3(decode::decode_threads(FUSED, RES ? decode::DRes<QFMT>::NIS : decode::DPlain::NIS));
+    using Cfg = typename std::conditional<RES, decode::DRes<QFMT>, decode::DPlain>::type;
+    cfg.blockDim = dim3(decode::decode_threads(FUSED, Cfg::NIS, Cfg::NQ - 4));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
