@@ -751,7 +751,7 @@ FP4_DEV float act_amax(const Params &p, int j0, int j1, int qw, int lane, float 
 template <int QFMT, int HK, bool RES, typename Cfg>
 FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready0, uint32_t empty0, int n_units,
                                  int t_first, int ks_first, int qw, int lane, float sg, const int *rexp,
-                                 volatile uint32_t *abort_flag)
+                                 const NvScaleTables *tab, volatile uint32_t *abort_flag)
 {
     constexpr int ND = Cfg::NB / BNA - 1;
     constexpr int R = BNA * 8 / 32;  // units per lane of one K step (16 rows x 8 units)
@@ -786,7 +786,7 @@ FP4_DEV bool quantize_act_stages(const Params &p, uint8_t *smem, uint32_t aready
             if (HK) fwht_unit<HK>(v, p.ck, lane);
             uint32_t rw = 0;
             if (RES) rw = extract_residual(v);
-            sb[r] = encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib[r]);
+            sb[r] = encode_unit<QFMT>(v, sg, six_sg, p.round_away, p.mx_floor, nib[r], tab);
             if (RES) {
                 const float rv = bf16lo(rw);
                 uint32_t code[ND > 0 ? ND : 1], sbyte[ND > 0 ? ND : 1];
@@ -901,6 +901,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 6);
     __shared__ volatile unsigned s_last;
     __shared__ float s_red[Cfg::NQ];        // fused: per-warp maxima
+    __shared__ NvScaleTables s_tab;         // fused NVFP4: block-scale factors for s_g
     __shared__ float s_amax[MAX_CLUSTER];   // fused: the cluster CTAs' maxima, by rank
     __shared__ float s_sg;                  // fused: the activations' tensor scale
     __shared__ unsigned s_rowmax[BNA];      // residual lane, NVFP4: largest residual of each row (float bits)
@@ -1177,8 +1178,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ C
             sg = *p.gA;
         }
         if (warp == 2 && lane == 0) s_sg = sg;
+        // NVFP4: the block scales' decode and encode factors for this s_g, once
+        // per CTA (the quantize kernels' tables: the same values as computing
+        // each factor per block, without a reciprocal per block)
+        if (QFMT == FP4_NVFP4) {
+            nv_tables_fill(s_tab, sg, qw * 32 + lane, Cfg::NQ * 32);
+            quantizers_sync<Cfg::NQ>();
+        }
         quantize_act_stages<QFMT, HK, RES, Cfg>(p, smem, aready0, empty0, n_units, t_first, ks_first, qw, lane, sg,
-                                                s_rexp, abort_flag);
+                                                s_rexp, QFMT == FP4_NVFP4 ? &s_tab : nullptr, abort_flag);
     }
     if (!FUSED || warp <= 5) {  // the four warps after the issuers only quantize
     // ---------------- epilogue warps 2-5: one result per tile segment ----------------
