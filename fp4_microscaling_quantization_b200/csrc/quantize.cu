@@ -679,7 +679,12 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64
         if ((err = launch_k(ak, dim3(grid), dim3(256), 0, st, pdl, a)) != cudaSuccess) return err;
     }
     if (a.total_units > 0 || a.gscale_computed) {  // an empty NVFP4 tensor still gets s_g = 1
-        if ((err = launch_k(qk, dim3(grid), dim3(256), 0, st, pdl, a)) != cudaSuccess) return err;
+        // NVFP4 (absmax scales, k <= 32): one resident wave (3 CTAs per SM at
+        // its register count), so fewer CTAs build the scale tables; with the
+        // rotation's cross-lane stages or the residual lane the longer grid
+        // balances better
+        const int qgrid = (fmt == FP4_NVFP4 && !mse && !res && hk <= 32 && grid > sms * 3) ? sms * 3 : grid;
+        if ((err = launch_k(qk, dim3(qgrid), dim3(256), 0, st, pdl, a)) != cudaSuccess) return err;
     }
     const int64_t rows_p = (rows + 127) / 128 * 128;
     const int64_t npad = rows * (a.nkb4 * 4 - nkb) + (rows_p - rows) * a.nkb4 * 4;
