@@ -61,6 +61,16 @@ FP4_DEV void mul_x2(float &a0, float &a1, float m0, float m1)
         : "f"(m0), "f"(m1));
 }
 
+// (a0, a1) = (a0 * m0 + c0, a1 * m1 + c1), each rounded once (fused)
+FP4_DEV void fma_x2(float &a0, float &a1, float m0, float m1, float c0, float c1)
+{
+    asm("{\n\t.reg .b64 pa, pm, pc;\n\t"
+        "mov.b64 pa, {%0, %1};\n\tmov.b64 pm, {%2, %3};\n\tmov.b64 pc, {%4, %5};\n\t"
+        "fma.rn.f32x2 pa, pa, pm, pc;\n\tmov.b64 {%0, %1}, pa;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(m0), "f"(m1), "f"(c0), "f"(c1));
+}
+
 // v[j] *= m0 and v[j + 16] *= m1 for j < 16: the two 16-element halves of a
 // unit (one scale each for 16-element blocks; m0 = m1 for one scale).
 FP4_DEV void scale_halves(float *v, float m0, float m1)
@@ -96,14 +106,16 @@ FP4_DEV void fwht_unit(float *v, float ck, int lane)
     }
 #pragma unroll
     for (int lm = 1; lm < HK / 32; lm <<= 1) {
-        // lower lane: a + b; upper lane: b - a, i.e. b + (-a): the same
-        // rounded sum either way, with the operand's sign flipped by bit
-        // (exact) instead of a second add and a select
-        const uint32_t flip = (lane & lm) ? 0x80000000u : 0u;
+        // lower lane: b + a; upper lane: a - b = (-1) * b + a.  One fused
+        // multiply-add with a lane's sign s = +-1: the product v * s is exact,
+        // so v * s + o rounds once to the same sum as o + (+-v), two elements
+        // per instruction, without a select or a sign flip per value.
+        const float s = (lane & lm) ? -1.0f : 1.0f;
 #pragma unroll
-        for (int j = 0; j < 32; j++) {
-            const float o = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
-            v[j] = __fadd_rn(o, __uint_as_float(__float_as_uint(v[j]) ^ flip));
+        for (int j = 0; j < 16; j++) {
+            const float o0 = __shfl_xor_sync(0xFFFFFFFFu, v[j], lm);
+            const float o1 = __shfl_xor_sync(0xFFFFFFFFu, v[j + 16], lm);
+            fma_x2(v[j], v[j + 16], s, s, o0, o1);
         }
     }
     scale_halves(v, ck, ck);
